@@ -1,0 +1,159 @@
+"""Pins of the double-quantization oracle.
+
+Sources: "QLoRA：冻结的 4-bit 权重怎样参与一次微调" §Double Quantization 压缩的是
+Scale (mean offset, block 256, fp32 second-level scale, signed 8-bit dynamic
+codebook, error C_j * delta_a with codes unchanged); "精读笔记 · QLoRA" §3.2.
+The 8-bit codebook's values are this build's own definition (the pages print
+none): its structure is pinned here, its values are not ("parity unpinned").
+"""
+from fractions import Fraction
+
+import numpy as np
+
+from oracle import nf4
+
+
+def test_codebook_structure():
+    t = nf4.dq_codebook()
+    assert t.dtype == np.float32 and t.size == 256
+    assert t[0x00] == 0.0 and t[0x80] == 0.0
+    assert len(set(t.tolist())) == 255
+    assert t[0x7F] == 1.0 and t[0xFF] == -1.0
+    pos = t[1:128]
+    assert np.all(np.diff(pos) > 0)                       # monotone within a sign
+    assert np.all(t[0x81:0x100] == -pos)                  # sign bit mirrors
+    assert np.all(np.abs(t) <= 1.0)
+    # decades: indices 64..127 cover (0.1, 1], 32..63 cover (0.01, 0.1], ...
+    assert np.all((pos[63:] > np.float32(0.1)) & (pos[63:] <= 1))
+    assert np.all((pos[31:63] > np.float32(0.01)) & (pos[31:63] <= np.float32(0.1)))
+    assert t[63] == np.float32(0.1) and t[1] == np.float32(1e-6)
+    # not FP8 E4M3: E4M3's largest finite value is 448, its grid is binary
+    assert np.float32(0.1) in t and np.max(np.abs(t)) != 448.0
+
+
+def _mean_by_fraction(v):
+    s = sum(Fraction(float(x)) for x in v) / len(v)
+    # nearest fp32 by bracketing (independent of the oracle's rounding helper)
+    f = np.float32(float(s))
+    cands = [np.nextafter(f, np.float32(-np.inf)), f, np.nextafter(f, np.float32(np.inf))]
+    d = [abs(Fraction(float(c)) - s) for c in cands]
+    best = min(d)
+    winners = [c for c, dd in zip(cands, d) if dd == best]
+    if len(winners) == 1:
+        return winners[0]
+    even = [c for c in winners if (int(np.array(c).view(np.uint32)) & 1) == 0]
+    return even[0]
+
+
+def test_exact_mean_closed_forms_and_ties():
+    one = np.float32(1.0)
+    ulp = np.float32(2.0 ** -23)
+    assert nf4.exact_mean_f32([one, one + ulp]) == one               # tie -> even
+    assert nf4.exact_mean_f32([one + ulp, one + 2 * ulp]) == one + 2 * ulp
+    assert nf4.exact_mean_f32(np.full(1000, 0.037, np.float32)) == np.float32(0.037)
+    assert nf4.exact_mean_f32([1.0, 2.0, 4.0]) == np.float32(7.0 / 3.0)
+    # a naive fp32 running sum loses the small terms; the exact mean does not
+    v = np.array([2.0 ** 24] + [1.0] * 4095, np.float32)
+    naive = np.float32(0)
+    for x in v:
+        naive = np.float32(naive + x)
+    exact = np.float32((2.0 ** 24 + 4095) / 4096)
+    assert nf4.exact_mean_f32(v) == exact and np.float32(naive / 4096) != exact
+    # subnormals and the largest finite value
+    tiny = np.float32(2.0 ** -149)
+    assert nf4.exact_mean_f32([tiny, tiny, tiny]) == tiny
+    big = np.finfo(np.float32).max
+    assert nf4.exact_mean_f32([big, big]) == big
+
+
+def test_exact_mean_random_against_fractions():
+    rng = np.random.default_rng(5)
+    for n in (1, 2, 3, 17, 300, 1001):
+        v = np.abs(rng.standard_normal(n) * 10.0 ** rng.uniform(-8, 3, n)).astype(np.float32)
+        assert nf4.exact_mean_f32(v) == _mean_by_fraction(v)
+
+
+def _brute_code8(c, s2):
+    table = nf4.dq_codebook()
+    x = Fraction(float(c)) / Fraction(float(s2))
+    best_u, bd, bv = None, None, None
+    for u in range(256):
+        v = Fraction(float(table[u]))
+        d = abs(x - v)
+        # ties -> the smaller value; equal values (the two zeros) -> code 0x00
+        if bd is None or d < bd or (d == bd and (v < bv or (v == bv and u < best_u))):
+            best_u, bd, bv = u, d, v
+    return best_u
+
+
+def test_double_quantize_bruteforce_ragged():
+    rng = np.random.default_rng(6)
+    for n1 in (1, 5, 256, 257, 700):
+        a = np.abs(rng.standard_normal(n1) * 0.02 + 0.05).astype(np.float32)
+        a[rng.random(n1) < 0.05] = 1.0                     # all-zero blocks keep scale 1
+        code8, s2, off = nf4.double_quantize(a)
+        assert s2.size == -(-n1 // 256) and code8.size == n1
+        assert off == nf4.exact_mean_f32(a)
+        c = (a - off).astype(np.float32)
+        for i in range(n1):
+            g = i // 256
+            grp = c[g * 256:(g + 1) * 256]
+            want_s2 = np.max(np.abs(grp)) if np.max(np.abs(grp)) > 0 else np.float32(1)
+            assert s2[g] == want_s2
+            assert code8[i] == _brute_code8(c[i], s2[g]), i
+
+
+def test_double_quantize_exact_midpoint_ties():
+    table = nf4.dq_codebook()
+    vals = sorted(set(table.astype(np.float64).tolist()))
+    # scales whose centred values sit exactly on T8 midpoints (s2 = 1 group)
+    rng = np.random.default_rng(7)
+    picks = rng.choice(len(vals) - 1, size=40, replace=False)
+    mids = []
+    for k in picks:
+        m = (vals[k] + vals[k + 1]) / 2
+        if float(np.float32(m)) == m:
+            mids.append(np.float32(m))
+    assert mids, "need fp32-exact midpoints"
+    # build a = c + offset with offset 0: include +1 and -1 so s2 = 1, mean 0
+    c = np.array([1.0, -1.0] + mids + [-x for x in mids], np.float32)
+    code8, s2, off = nf4.double_quantize(c)
+    assert off == 0.0 and s2[0] == 1.0
+    for i, x in enumerate(c):
+        assert code8[i] == _brute_code8(x, s2[0])
+        if x in mids:       # a tie resolves to the smaller value
+            lo = max(v for v in vals if v < x)
+            assert table[code8[i]] == np.float32(lo)
+
+
+def test_equal_group_decodes_to_offset_and_error_bound():
+    a = np.full(300, 0.0421, np.float32)
+    code8, s2, off = nf4.double_quantize(a)
+    dec = nf4.decode_scales(300, code8=code8, s2=s2, offset=off)
+    assert np.all(code8 == 0) and np.all(s2 == 1.0) and np.all(dec == a)
+    rng = np.random.default_rng(8)
+    a = np.abs(rng.standard_normal(5000) * 0.01 + 0.05).astype(np.float32)
+    code8, s2, off = nf4.double_quantize(a)
+    dec = nf4.decode_scales(5000, code8=code8, s2=s2, offset=off)
+    vals = np.array(sorted(set(nf4.dq_codebook().astype(np.float64).tolist())))
+    half_gap = np.max(np.diff(vals)) / 2
+    g = np.arange(5000) // 256
+    bound = s2[g].astype(np.float64) * half_gap + 4 * np.spacing(np.float32(1.0)) * np.abs(a)
+    assert np.all(np.abs(dec.astype(np.float64) - a) <= bound)
+
+
+def test_codes_independent_of_double_quant_and_zero_block_stays_zero():
+    rng = np.random.default_rng(9)
+    w = (rng.standard_normal(64 * 40) * 0.02).astype(np.float32)
+    w[64 * 3:64 * 4] = 0.0
+    codes, absmax = nf4.quantize_nf4(w)
+    payload, n = nf4.pack_codes(codes)
+    code8, s2, off = nf4.double_quantize(absmax)
+    a_dq = nf4.decode_scales(absmax.size, code8=code8, s2=s2, offset=off)
+    w_dq = nf4.dequantize(payload, n, a_dq)
+    w_plain = nf4.dequantize(payload, n, absmax)
+    assert np.all(w_dq[64 * 3:64 * 4] == 0.0) and np.all(w_plain[64 * 3:64 * 4] == 0.0)
+    # the scale error moves each weight by about C_j * delta_a
+    C = np.array(nf4.NF4)[codes]
+    delta = (a_dq.astype(np.float64) - absmax)[np.arange(w.size) // 64]
+    assert np.all(np.abs((w_dq - w_plain) - C * delta) <= 2 * 2 ** -8 * np.abs(w_plain) + 1e-12)
