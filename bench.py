@@ -1,0 +1,471 @@
+#!/usr/bin/env python
+"""Benchmark of the NF4 frozen-base LoRA linear layer on B200.
+
+One step = the whole hot path on one batch: NF4-quantize the frozen 4096x4096
+weight with double quantization, forward (Zc = c·X·A, Y = X·Ŵ + Zc·B) and
+backward (dZ, dX = dY·Ŵᵀ + dZ·Aᵀ, dA, dB) for M = 4096 tokens, r = 16,
+alpha = 32.  With N > 1 processes (torchrun, one per GPU) every rank runs its
+own batch of 4096 tokens against the same frozen weight (data parallel, weak
+scaling) and dA, dB are summed across ranks with an NCCL all-reduce.
+
+metric : fwd+bwd TFLOP/s = (4MKN + 6Mr(K+N)) per step per rank, summed over
+         ranks, divided by the step time (max over ranks).  The step time
+         includes the per-step quantization.
+Also reported: the live roofline of the dominant kernel (the fused NF4 GEMM),
+the GEMV GB/s sweep (M in 1/4/16 on 4096x11008 and 11008x4096) and the
+quantize GB/s of the 8192x22016 weight, the end-to-end number with host
+buffers, and the CPU oracle on a bounded sample.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "QLoRA NF4 linear fwd+bwd TFLOP/s (M=4096), GEMV GB/s; % of B200 roofline"
+WORKLOAD = "proj-4096x4096-m4096-r16-dq"
+M, K, N, R, ALPHA = 4096, 4096, 4096, 16, 32.0
+ROTATE = 3          # input sets cycled per step: 3 x 96 MB of bf16 inputs > 2 x 126 MB L2
+
+
+def flops_step(Mt=M, Kt=K, Nt=N, r=R):
+    return 4.0 * Mt * Kt * Nt + 6.0 * Mt * r * (Kt + Nt)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm": float(d["hbm_gbs"]), "bf16": float(d["bf16_tflops"]),
+                "bf16_sus": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "src": "measured"}
+    except Exception:
+        return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sus": 1400.0, "src": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+        time.sleep(0.15)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle on a bounded sample (baseline only)
+# ---------------------------------------------------------------------------
+ORACLE_KS, ORACLE_MS = 1024, 256   # rows of W quantized, tokens pushed through fwd+bwd
+
+
+def oracle_sample_inputs():
+    import numpy as np
+    from bit_nf4_quantized_pack_b200 import synthetic as S
+    lin = S.config2(M=ORACLE_MS).linears[0]
+    return (np.ascontiguousarray(lin.W[:ORACLE_KS]), np.ascontiguousarray(lin.X[:, :ORACLE_KS]),
+            np.ascontiguousarray(lin.A[:ORACLE_KS]), lin.B, lin.dY)
+
+
+def oracle_step(inputs):
+    from oracle import nf4
+    from oracle.linear import lora_backward, lora_forward
+    W, X, A, B, G = inputs
+    codes, absmax = nf4.quantize_nf4(W.ravel())
+    payload, n = nf4.pack_codes(codes)
+    code8, s2, off = nf4.double_quantize(absmax)
+    a = nf4.decode_scales(absmax.size, code8=code8, s2=s2, offset=off)
+    w_hat = nf4.dequantize(payload, n, a).reshape(W.shape)
+    c = ALPHA / R
+    lora_forward(X, w_hat, A, B, c)
+    lora_backward(G, X, w_hat, A, B, c)
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def oracle_flops():
+    return flops_step(ORACLE_MS, ORACLE_KS, N, R)
+
+
+SAMPLE_DESC = (f"oracle (NumPy fp64) on a slice: quantize+double-quantize+dequantize "
+               f"W[:{ORACLE_KS}, :{N}], then fwd+bwd for {ORACLE_MS} tokens over K={ORACLE_KS}; "
+               f"TFLOP/s from that slice's 4MKN+6Mr(K+N)")
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    inputs = oracle_sample_inputs()
+    for _ in range(args.warmup):
+        oracle_step(inputs)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(inputs)
+    dt = (time.perf_counter() - t0) / args.steps
+    v = oracle_flops() / dt / 1e12
+    cores = oracle_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample": SAMPLE_DESC},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": SAMPLE_DESC},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def make_sets(torch, dev, nsets):
+    import numpy as np
+    from bit_nf4_quantized_pack_b200 import synthetic as S
+    sets = []
+    for s in range(nsets):
+        lin = S.config2(seed=s).linears[0]
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev).to(torch.bfloat16)
+        sets.append({"W": t(lin.W), "X": t(lin.X), "dY": t(lin.dY), "A": t(lin.A), "B": t(lin.B),
+                     "host": lin if s == 0 else None})
+    return sets
+
+
+def prof_read(q, kind):
+    import ctypes as C
+    ms, n = C.c_double(0), C.c_int64(0)
+    q.lib.qlora_profile_read(kind, C.byref(ms), C.byref(n))
+    return ms.value, n.value
+
+
+def gemv_sweep(torch, q, dev, peaks):
+    """Forward GEMV GB/s for M in {1,4,16} on 4096x11008 and 11008x4096 (DQ,
+    r=16), >= 12 rotated weight copies (> 2x L2), replayed from a CUDA graph."""
+    out = []
+    gen = torch.Generator(device=dev)
+    for (Kg, Ng) in ((4096, 11008), (11008, 4096)):
+        ncopy = 12
+        ws = []
+        for i in range(ncopy):
+            gen.manual_seed(1000 + i)
+            W = (torch.randn((Kg, Ng), generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+            ws.append(q.quantize(W, double_quant=True))
+            del W
+        gen.manual_seed(7)
+        A = (torch.randn((Kg, 16), generator=gen, device=dev) * 0.01).to(torch.bfloat16)
+        B = (torch.randn((16, Ng), generator=gen, device=dev) * 0.01).to(torch.bfloat16)
+        for Mg in (1, 4, 16):
+            X = torch.randn((Mg, Kg), generator=gen, device=dev).to(torch.bfloat16)
+            Y = torch.empty((Mg, Ng), dtype=torch.bfloat16, device=dev)
+            Zc = torch.empty((Mg, 16), dtype=torch.bfloat16, device=dev)
+            for w in ws:                       # warm-up, workspace sizing
+                q.linear_forward(X, w, A, B, 2.0, Y=Y, Zc=Zc)
+            torch.cuda.synchronize()
+            st = q.new_status(dev)
+            s = torch.cuda.Stream(device=dev)
+            g = torch.cuda.CUDAGraph()
+            reps = 4
+            with torch.cuda.stream(s):
+                with torch.cuda.graph(g, stream=s):
+                    for _ in range(reps):
+                        for w in ws:
+                            q.linear_forward(X, w, A, B, 2.0, Y=Y, Zc=Zc, status=st)
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            per = e0.elapsed_time(e1) / (reps * ncopy) * 1e-3
+            n1 = Kg * Ng // 64
+            n2 = (n1 + 255) // 256
+            nbytes = Kg * Ng // 2 + n1 + 4 * n2 + 4 + 2 * Mg * Kg + 2 * 16 * (Kg + Ng) + 2 * Mg * Ng
+            gbs = nbytes / per / 1e9
+            out.append({"M": Mg, "K": Kg, "N": Ng, "us": per * 1e6, "GB/s": gbs,
+                        "frac": gbs / peaks["hbm"]})
+            del g
+        del ws
+    return out
+
+
+def quantize_bench(torch, q, dev, peaks):
+    """Quantize (with DQ) of the 8192x22016 bf16 weight: GB/s of 2P + P/2 + n1 + 4n2 + 4."""
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5)
+    Kq, Nq = 8192, 22016
+    W = (torch.randn((Kq, Nq), generator=gen, device=dev) * 0.015).to(torch.bfloat16)
+    w = q.quantize(W, double_quant=True)
+    st = q.new_status(dev)
+    for _ in range(3):
+        q.quantize(W, double_quant=True, out=w, status=st)
+    q.lib.qlora_profile_reset()
+    q.lib.qlora_profile_enable(1)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 10
+    e0.record()
+    for _ in range(reps):
+        q.quantize(W, double_quant=True, out=w, status=st)
+    e1.record()
+    torch.cuda.synchronize()
+    q.lib.qlora_profile_enable(0)
+    per = e0.elapsed_time(e1) / reps * 1e-3
+    P = Kq * Nq
+    n1 = P // 64
+    n2 = (n1 + 255) // 256
+    nbytes = 2 * P + P // 2 + n1 + 4 * n2 + 4
+    gbs = nbytes / per / 1e9
+    del W
+    return {"shape": [Kq, Nq], "us": per * 1e6, "GB/s": gbs, "frac": gbs / peaks["hbm"]}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--no-extras", action="store_true", help="skip the GEMV and quantize sweeps")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    import bit_nf4_quantized_pack_b200 as q
+    peaks = load_peaks()
+    c = ALPHA / R
+    sets = make_sets(torch, dev, ROTATE)
+    wbuf = q.NF4Weight.empty((K, N), True, dev)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    Zc = torch.empty((M, R), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    dA = torch.empty((K, R), dtype=torch.float32, device=dev)
+    dB = torch.empty((R, N), dtype=torch.float32, device=dev)
+    status = q.new_status(dev)
+
+    def step(i):
+        s = sets[i % ROTATE]
+        q.quantize(s["W"], double_quant=True, out=wbuf, status=status)
+        q.linear_forward(s["X"], wbuf, s["A"], s["B"], c, Y=Y, Zc=Zc, status=status)
+        q.linear_backward(s["dY"], s["X"], Zc, wbuf, s["A"], s["B"], c, dX=dX, dA=dA, dB=dB,
+                          status=status)
+        if world > 1:
+            dist.all_reduce(dA)
+            dist.all_reduce(dB)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    code, mask = q.status_sync(status)
+    if code != 0:
+        raise SystemExit(f"device status {code} (mask {mask}) during warm-up")
+
+    # ---------------- timed region (device time, max over ranks) ----------------
+    sampler = ClockSampler(local) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    q.lib.qlora_profile_reset()
+    q.lib.qlora_profile_enable(1)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    q.lib.qlora_profile_enable(0)
+    clocks = sampler.stop() if sampler else None
+    ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    fwd_ms, fwd_n = prof_read(q, 0)
+    bwd_ms, bwd_n = prof_read(q, 1)
+    _, launches = prof_read(q, -1)
+    code, mask = q.status_sync(status)
+    if code != 0:
+        raise SystemExit(f"device status {code} (mask {mask}) in the timed region")
+    value = world * flops_step() / (ms * 1e-3) / 1e12
+
+    # dominant kernel: the fused NF4 GEMM (forward and dX launches together)
+    f_fwd = 2.0 * M * K * N + 2.0 * M * R * N
+    f_bwd = 2.0 * M * K * N + 2.0 * M * R * K
+    kern_ms = (fwd_ms + bwd_ms) / max(1, fwd_n + bwd_n)
+    kern_flops = (f_fwd * fwd_n + f_bwd * bwd_n) / max(1, fwd_n + bwd_n)
+    achieved = kern_flops / (kern_ms * 1e-3) / 1e12 if kern_ms > 0 else None
+    roofline = {"bound": "tensor", "kernel": "fused_nf4_gemm_kernel (fwd + dX)",
+                "achieved": achieved, "peak": peaks["bf16"], "unit": "TFLOP/s",
+                "frac": (achieved / peaks["bf16"]) if achieved else None, "traffic": None,
+                "peak_src": f"{peaks['src']} bf16 burst",
+                "avg_launch_ms": kern_ms, "flops_per_launch": kern_flops,
+                "fwd_ms": fwd_ms / max(1, fwd_n), "bwd_ms": bwd_ms / max(1, bwd_n)}
+
+    # ---------------- end to end through the public API with host buffers ----------------
+    e2e = None
+    if rank == 0 or world > 1:
+        h = sets[0]["host"]
+        pin = lambda a: torch.from_numpy(a.astype("float32")).to(torch.bfloat16).pin_memory()
+        hW, hX, hG = pin(h.W), pin(h.X), pin(h.dY)
+        hdA = torch.empty((K, R), dtype=torch.float32).pin_memory()
+        hdB = torch.empty((R, N), dtype=torch.float32).pin_memory()
+        dW, dXin, dG = torch.empty_like(sets[0]["W"]), torch.empty_like(sets[0]["X"]), \
+            torch.empty_like(sets[0]["dY"])
+        A_, B_ = sets[0]["A"], sets[0]["B"]
+
+        def e2e_step():
+            dW.copy_(hW, non_blocking=True)
+            dXin.copy_(hX, non_blocking=True)
+            dG.copy_(hG, non_blocking=True)
+            q.quantize(dW, double_quant=True, out=wbuf, status=status)
+            q.linear_forward(dXin, wbuf, A_, B_, c, Y=Y, Zc=Zc, status=status)
+            q.linear_backward(dG, dXin, Zc, wbuf, A_, B_, c, dX=dX, dA=dA, dB=dB, status=status)
+            if world > 1:
+                dist.all_reduce(dA)
+                dist.all_reduce(dB)
+            hdA.copy_(dA, non_blocking=True)
+            hdB.copy_(dB, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        n_e2e = max(3, min(args.steps, 20))
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record()
+        for _ in range(n_e2e):
+            e2e_step()
+        a1.record()
+        torch.cuda.synchronize()
+        ems = a0.elapsed_time(a1) / n_e2e
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        h2d = (hW.numel() + hX.numel() + hG.numel()) * 2
+        d2h = (hdA.numel() + hdB.numel()) * 4
+        e2e = {"value": world * flops_step() / (ems * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": ems, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    extras = {}
+    if rank == 0 and not args.no_extras:
+        extras["gemv"] = gemv_sweep(torch, q, dev, peaks)
+        extras["quantize"] = quantize_bench(torch, q, dev, peaks)
+
+    cpu = None
+    if rank == 0 and world == 1:
+        inputs = oracle_sample_inputs()
+        t0 = time.perf_counter()
+        oracle_step(inputs)
+        dt = time.perf_counter() - t0
+        cpu = {"value": oracle_flops() / dt / 1e12, "unit": "TFLOP/s", "cores": oracle_threads(),
+               "kind": "oracle", "sample": SAMPLE_DESC, "seconds": dt}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "r": R, "alpha": ALPHA,
+                           "double_quant": True, "parallelism": f"dp{world}",
+                           "step": "quantize(W) + fwd + bwd" + (" + allreduce(dA,dB)" if world > 1 else ""),
+                           "l2": f"{ROTATE} rotated input sets (W, X, dY: 96 MB each) > L2"},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": int(launches), "clocks": clocks}
+        line.update(extras)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,230 @@
+"""NF4 frozen-base LoRA linear layer for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/qlora_nf4.h``: PyTorch is used
+for device memory and the current CUDA stream only; every step of the
+computation runs in the library's CUDA kernels.  The calls mirror the C
+entry points:
+
+    quantize(W, double_quant)            -> NF4Weight     (qlora_nf4_quantize)
+    dequantize(w)                        -> bf16 K x N    (qlora_nf4_dequantize)
+    linear_forward(X, w, A, B, c)        -> (Y, Zc)       (qlora_linear_fwd)
+    linear_backward(dY, X, Zc, w, A, B, c) -> (dX, dA, dB) (qlora_linear_bwd)
+
+Page "QLoRA：冻结的 4-bit 权重怎样参与一次微调" defines the method (see the
+header for the section of each call).
+"""
+from __future__ import annotations
+
+import ctypes as C
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import NF4StateC, QLoRAError, check, lib
+
+__all__ = ["NF4Weight", "quantize", "dequantize", "linear_forward", "linear_backward",
+           "status_sync", "status_clear", "new_status", "QLoRAError", "lib"]
+
+BLOCKSIZE = 64
+DQ_BLOCKSIZE = 256
+
+
+def _stream():
+    return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return C.c_void_p(t.data_ptr()) if t is not None else C.c_void_p(0)
+
+
+def n1_of(numel: int) -> int:
+    return int(lib.qlora_nf4_n1(numel))
+
+
+def n2_of(numel: int) -> int:
+    return int(lib.qlora_nf4_n2(numel))
+
+
+@dataclass
+class NF4Weight:
+    """Quantized state of a K x N weight (the caller-owned buffers of
+    ``qlora_nf4_state``)."""
+    shape: tuple
+    double_quant: bool
+    packed: torch.Tensor
+    absmax: torch.Tensor | None = None
+    code8: torch.Tensor | None = None
+    s2: torch.Tensor | None = None
+    offset: torch.Tensor | None = None
+
+    @property
+    def numel(self) -> int:
+        n = 1
+        for s in self.shape:
+            n *= int(s)
+        return n
+
+    def cstruct(self) -> NF4StateC:
+        st = NF4StateC()
+        st.numel = self.numel
+        st.blocksize = BLOCKSIZE
+        st.double_quant = 1 if self.double_quant else 0
+        st.dq_blocksize = DQ_BLOCKSIZE
+        st.reserved = 0
+        st.packed = self.packed.data_ptr()
+        st.absmax = self.absmax.data_ptr() if self.absmax is not None else None
+        st.code8 = self.code8.data_ptr() if self.code8 is not None else None
+        st.s2 = self.s2.data_ptr() if self.s2 is not None else None
+        st.offset = self.offset.data_ptr() if self.offset is not None else None
+        return st
+
+    @staticmethod
+    def empty(shape, double_quant: bool, device="cuda") -> "NF4Weight":
+        numel = 1
+        for s in shape:
+            numel *= int(s)
+        n1, n2 = n1_of(numel), n2_of(numel)
+        u8, f32 = torch.uint8, torch.float32
+        w = NF4Weight(tuple(int(s) for s in shape), bool(double_quant),
+                      torch.empty((numel + 1) // 2, dtype=u8, device=device))
+        if double_quant:
+            w.code8 = torch.empty(n1, dtype=u8, device=device)
+            w.s2 = torch.empty(n2, dtype=f32, device=device)
+            w.offset = torch.empty(1, dtype=f32, device=device)
+        else:
+            w.absmax = torch.empty(n1, dtype=f32, device=device)
+        return w
+
+
+def new_status(device="cuda") -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def status_sync(status: torch.Tensor):
+    """(first error code or 0, raw bit mask); synchronizes the current stream."""
+    mask = C.c_int32(0)
+    code = lib.qlora_status_sync(_ptr(status), _stream(), C.byref(mask))
+    return int(code), int(mask.value)
+
+
+def status_clear(status: torch.Tensor) -> None:
+    check(lib.qlora_status_clear(_ptr(status), _stream()), "qlora_status_clear")
+
+
+class _WorkspaceCache:
+    """Reuses one device buffer per (device, purpose) so repeated calls do not
+    allocate; grows when a larger workspace is needed."""
+
+    def __init__(self):
+        self._bufs = {}
+
+    def get(self, key, nbytes, device):
+        if nbytes == 0:
+            return None
+        buf = self._bufs.get(key)
+        if buf is None or buf.numel() < nbytes or buf.device != torch.device(device):
+            buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+            self._bufs[key] = buf
+        return buf
+
+
+_ws = _WorkspaceCache()
+
+
+def _finish(status, own_status, where):
+    if own_status:
+        code, _ = status_sync(status)
+        check(code, where)
+
+
+def quantize(W: torch.Tensor, double_quant: bool = True, *, out: NF4Weight | None = None,
+             status: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> NF4Weight:
+    """Blockwise NF4 quantization of a contiguous bf16 or fp32 CUDA tensor."""
+    if W.dtype == torch.bfloat16:
+        dt = _lib.QLORA_DTYPE_BF16
+    elif W.dtype == torch.float32:
+        dt = _lib.QLORA_DTYPE_F32
+    else:
+        raise TypeError("W must be bfloat16 or float32")
+    if not W.is_contiguous():
+        raise ValueError("W must be contiguous")
+    w = out if out is not None else NF4Weight.empty(W.shape, double_quant, W.device)
+    st = w.cstruct()
+    need = int(lib.qlora_nf4_quantize_workspace_size(w.numel, st.double_quant))
+    ws = workspace if workspace is not None else _ws.get(("q", W.device), need, W.device)
+    own = status is None
+    status = new_status(W.device) if own else status
+    check(lib.qlora_nf4_quantize(_ptr(W), dt, C.byref(st), _ptr(ws),
+                                 ws.numel() if ws is not None else 0, _ptr(status), _stream()),
+          "qlora_nf4_quantize")
+    _finish(status, own, "qlora_nf4_quantize")
+    return w
+
+
+def dequantize(w: NF4Weight, *, out: torch.Tensor | None = None,
+               status: torch.Tensor | None = None) -> torch.Tensor:
+    dev = w.packed.device
+    out = out if out is not None else torch.empty(w.shape, dtype=torch.bfloat16, device=dev)
+    st = w.cstruct()
+    own = status is None
+    status = new_status(dev) if own else status
+    check(lib.qlora_nf4_dequantize(C.byref(st), _ptr(out), _ptr(status), _stream()),
+          "qlora_nf4_dequantize")
+    _finish(status, own, "qlora_nf4_dequantize")
+    return out
+
+
+def _bf16(t, name):
+    if t.dtype != torch.bfloat16 or not t.is_contiguous() or not t.is_cuda:
+        raise TypeError(f"{name} must be a contiguous CUDA bfloat16 tensor")
+
+
+def linear_forward(X, w: NF4Weight, A, B, c: float, *, Y=None, Zc=None, status=None,
+                   workspace=None):
+    """Y = X·Ŵ + c·(X·A)·B with Ŵ decoded on the fly; returns (Y, Zc)."""
+    for t, n in ((X, "X"), (A, "A"), (B, "B")):
+        _bf16(t, n)
+    M, K = X.shape
+    Kw, N = w.shape
+    r = A.shape[1]
+    if Kw != K or A.shape[0] != K or tuple(B.shape) != (r, N):
+        raise ValueError("shape mismatch")
+    dev = X.device
+    Y = Y if Y is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    Zc = Zc if Zc is not None else torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+    need = int(lib.qlora_linear_fwd_workspace_size(M, K, N, r))
+    ws = workspace if workspace is not None else _ws.get(("f", dev), need, dev)
+    st = w.cstruct()
+    own = status is None
+    status = new_status(dev) if own else status
+    check(lib.qlora_linear_fwd(M, K, N, r, _ptr(X), C.byref(st), _ptr(A), _ptr(B), float(c),
+                               _ptr(Y), _ptr(Zc), _ptr(ws), ws.numel() if ws is not None else 0,
+                               _ptr(status), _stream()), "qlora_linear_fwd")
+    _finish(status, own, "qlora_linear_fwd")
+    return Y, Zc
+
+
+def linear_backward(dY, X, Zc, w: NF4Weight, A, B, c: float, *, dX=None, dA=None, dB=None,
+                    status=None, workspace=None):
+    """dX = dY·Ŵᵀ + c·(dY·Bᵀ)·Aᵀ, dA = Xᵀ·(c·dY·Bᵀ), dB = Zcᵀ·dY; returns (dX, dA, dB)."""
+    for t, n in ((dY, "dY"), (X, "X"), (Zc, "Zc"), (A, "A"), (B, "B")):
+        _bf16(t, n)
+    M, K = X.shape
+    N = dY.shape[1]
+    r = A.shape[1]
+    dev = X.device
+    dX = dX if dX is not None else torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    dA = dA if dA is not None else torch.empty((K, r), dtype=torch.float32, device=dev)
+    dB = dB if dB is not None else torch.empty((r, N), dtype=torch.float32, device=dev)
+    need = int(lib.qlora_linear_bwd_workspace_size(M, K, N, r))
+    ws = workspace if workspace is not None else _ws.get(("b", dev), need, dev)
+    st = w.cstruct()
+    own = status is None
+    status = new_status(dev) if own else status
+    check(lib.qlora_linear_bwd(M, K, N, r, _ptr(dY), _ptr(X), _ptr(Zc), C.byref(st), _ptr(A),
+                               _ptr(B), float(c), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws),
+                               ws.numel() if ws is not None else 0, _ptr(status), _stream()),
+          "qlora_linear_bwd")
+    _finish(status, own, "qlora_linear_bwd")
+    return dX, dA, dB

@@ -1,0 +1,68 @@
+// Launchers of the library's kernels and device helpers shared between
+// translation units.  Internal to the library (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace qnf4 {
+
+// The signed dynamic 8-bit codebook T8 of the scale codes (this library's own
+// definition; the page only requires "a signed dynamic 8-bit codebook, not
+// FP8 E4M3"): byte u, sign u >> 7, t = u & 127; t = 0 is 0; otherwise
+// f = floor(log2 t), e = 6 - f, m = t - 2^f and |v| = (2^f + 9(m+1)) /
+// (10^(e+1) 2^f), a correctly rounded double division rounded to fp32.
+__device__ __forceinline__ float t8_magnitude(int t) {
+  if (t == 0) return 0.0f;
+  const int f = 31 - __clz(t);
+  const int e = 6 - f;
+  const int m = t - (1 << f);
+  double p10 = 10.0;
+  for (int i = 0; i < e; ++i) p10 *= 10.0;
+  const double num = static_cast<double>((1 << f) + 9 * (m + 1));
+  const double den = p10 * static_cast<double>(1 << f);
+  return __double2float_rn(__ddiv_rn(num, den));
+}
+
+__device__ __forceinline__ void build_t8(float* t8 /*256*/) {
+  for (int u = threadIdx.x; u < 256; u += blockDim.x) {
+    const float v = t8_magnitude(u & 127);
+    t8[u] = (u >> 7) ? -v : v;
+  }
+}
+
+// quantize.cu
+cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* packed,
+                            float* absmax_out, bool dq, uint8_t* code8, float* s2, float* offset,
+                            void* ws, int32_t* d_status, cudaStream_t st, int num_sms);
+size_t quantize_workspace_bytes(int64_t numel, bool dq);
+
+// dequantize.cu
+cudaError_t launch_dequantize(const uint8_t* packed, int64_t numel, const float* absmax,
+                              const uint8_t* code8, const float* s2, const float* offset,
+                              uint16_t* out, int32_t* d_status, cudaStream_t st, int num_sms);
+
+// Decode-scale view of a quantized weight, shared by the GEMM and GEMV paths.
+struct ScaleView {
+  const float* absmax;   // non-null when not double-quantized
+  const uint8_t* code8;  // non-null when double-quantized
+  const float* s2;
+  const float* offset;
+};
+
+// linear.cu — forward and backward of the layer
+size_t linear_fwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r);
+size_t linear_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r);
+cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint16_t* X,
+                              const uint8_t* packed, ScaleView sv, const uint16_t* A,
+                              const uint16_t* B, float c, uint16_t* Y, uint16_t* Zc, void* ws,
+                              size_t ws_bytes, int32_t* d_status, cudaStream_t st, int num_sms);
+cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint16_t* dY,
+                              const uint16_t* X, const uint16_t* Zc, const uint8_t* packed,
+                              ScaleView sv, const uint16_t* A, const uint16_t* B, float c,
+                              uint16_t* dX, float* dA, float* dB, void* ws, size_t ws_bytes,
+                              int32_t* d_status, cudaStream_t st, int num_sms);
+
+}  // namespace qnf4

@@ -1,0 +1,931 @@
+// Forward and backward of the NF4 frozen-base LoRA linear layer on sm_100a.
+//
+// Page "QLoRA：冻结的 4-bit 权重怎样参与一次微调":
+//   §量化基座与可训练支路怎样相加      Z = X·A,  Y = X·Ŵ + c·Z·B
+//   §冻结权重为什么仍然需要输入梯度    dZ = c·G·Bᵀ, dX = G·Ŵᵀ + dZ·Aᵀ,
+//                                     dA = Xᵀ·dZ,  dB = c·Zᵀ·G
+//
+// Kernels in this file:
+//   skinny_gemm_kernel   rank-r contractions (X·A, G·Bᵀ, Xᵀ·dZ, Gᵀ·Zc): TMA
+//                        for both operands, tcgen05 MMA with N = 64, split-K
+//                        into fp32 partials, then skinny_reduce_kernel.
+//   fused_nf4_gemm_kernel  Y = X·Ŵ + Zc·B (forward) and dX = G·Ŵᵀ + dZ·Aᵀ
+//                        (backward): persistent, warp-specialised; TMA brings
+//                        activation tiles and packed-nibble tiles, decoder
+//                        warps turn nibbles into bf16 operand tiles in shared
+//                        memory, one thread issues tcgen05.mma into TMEM, and
+//                        the rank-r LoRA term is one extra K-step of the same
+//                        accumulator.
+//   nf4_gemv_kernel      M <= 16: split-K CUDA-core GEMV streaming the packed
+//                        payload, then gemv_reduce_kernel adds Zc·B.
+#include <cfloat>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "profile.cuh"
+#include "tmap.cuh"
+
+namespace qnf4 {
+
+__constant__ float kNF4g[16] = {QNF4_TABLE_VALUES};
+
+// ===========================================================================
+// Skinny contraction:  D[m'][n'] = sum_k' A(m',k') * B(n',k'),  n' < 64.
+// A tiles are 128 x 64 and B tiles 64 x 64 (bf16), each either K-major
+// (rows of 64 contiguous k') or MN-major (rows of 64 contiguous m'/n'), all
+// with the 128-byte swizzle.  blockIdx.x = 128-row tile, blockIdx.y = split.
+// ===========================================================================
+constexpr int kSkStages = 6;
+constexpr int kSkA = 16384, kSkB = 8192;
+constexpr int kSkThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr size_t kSkSmem = 1024 + kSkStages * (kSkA + kSkB) + 256;
+
+struct SkinnyArgs {
+  int Mp;            // rows of D
+  int nk;            // number of 64-wide k' blocks
+  int kb_per_split;  // k' blocks per split
+  float* partial;    // [splits][Mp][64]
+  int32_t* d_status;
+};
+
+template <bool kAmn, bool kBmn>
+__global__ void __launch_bounds__(kSkThreads, 1)
+    skinny_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmB, SkinnyArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kSkStages * kSkA;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kSkStages * kSkB);
+  uint64_t* empty = full + kSkStages;
+  uint64_t* done = empty + kSkStages;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * 128;
+  const int kb0 = blockIdx.y * args.kb_per_split;
+  const int kb1 = min(args.nk, kb0 + args.kb_per_split);
+  const int nkb = kb1 - kb0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSkStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 64);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    for (int i = 0; i < nkb; ++i) {
+      const int s = i % kSkStages;
+      const uint32_t ph = (i / kSkStages) & 1;
+      if (!mbar_wait(&empty[s], ph ^ 1)) { *abort_flag = 1; break; }
+      const int kb = kb0 + i;
+      mbar_arrive_expect_tx(&full[s], kSkA + kSkB);
+      if (kAmn) {
+        tma_load_2d(sA + s * kSkA, &tmA, &full[s], m0, kb * 64);
+        tma_load_2d(sA + s * kSkA + 8192, &tmA, &full[s], m0 + 64, kb * 64);
+      } else {
+        tma_load_2d(sA + s * kSkA, &tmA, &full[s], kb * 64, m0);
+      }
+      if (kBmn)
+        tma_load_2d(sB + s * kSkB, &tmB, &full[s], 0, kb * 64);
+      else
+        tma_load_2d(sB + s * kSkB, &tmB, &full[s], kb * 64, 0);
+    }
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc = idesc_bf16_f32(128, 64, kAmn ? 1 : 0, kBmn ? 1 : 0);
+    bool ok = true;
+    for (int i = 0; i < nkb; ++i) {
+      const int s = i % kSkStages;
+      const uint32_t ph = (i / kSkStages) & 1;
+      if (!mbar_wait(&full[s], ph)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t a0 = smem_u32(sA + s * kSkA), b0 = smem_u32(sB + s * kSkB);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint64_t ad = kAmn ? smem_desc(a0 + j * 2048, 8192, 1024) : smem_desc(a0 + j * 32, 16, 1024);
+        const uint64_t bd = kBmn ? smem_desc(b0 + j * 2048, 8192, 1024) : smem_desc(b0 + j * 32, 16, 1024);
+        umma_bf16(tmem, ad, bd, idesc, (i > 0 || j > 0) ? 1u : 0u);
+      }
+      umma_commit(&empty[s]);
+    }
+    if (!ok) *abort_flag = 1;
+    umma_commit(done);  // also drains whatever was issued
+  } else if (warp >= 2) {
+    const int q = warp & 3;
+    const bool ok = mbar_wait(done, 0);
+    tc_fence_after();
+    const int row = m0 + q * 32 + lane;
+    if (!ok) *abort_flag = 1;
+    if (ok && !*abort_flag) {
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c * 32, v);
+        tmem_ld_wait();
+        if (row < args.Mp) {
+          float4* dst = reinterpret_cast<float4*>(
+              args.partial + (static_cast<int64_t>(blockIdx.y) * args.Mp + row) * 64 + c * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) raise_status(args.d_status, QLORA_ERR_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
+  }
+}
+
+// out = scale * sum_s partial[s]; modes: 0 bf16 [Mp][ld], 1 fp32 [Mp][ld],
+// 2 fp32 transposed [ncols][Mp].
+__global__ void skinny_reduce_kernel(const float* __restrict__ partial, int splits, int Mp,
+                                     int ncols, float scale, int mode, void* out, int ld) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<int64_t>(Mp) * ncols) return;
+  const int row = static_cast<int>(idx / ncols), col = static_cast<int>(idx % ncols);
+  float acc = 0.0f;
+  for (int s = 0; s < splits; ++s) acc += partial[(static_cast<int64_t>(s) * Mp + row) * 64 + col];
+  acc *= scale;
+  if (mode == 0) {
+    static_cast<uint16_t*>(out)[static_cast<int64_t>(row) * ld + col] =
+        static_cast<uint16_t>(pack_bf16x2(acc, 0.0f) & 0xFFFFu);
+  } else if (mode == 1) {
+    static_cast<float*>(out)[static_cast<int64_t>(row) * ld + col] = acc;
+  } else {
+    static_cast<float*>(out)[static_cast<int64_t>(col) * Mp + row] = acc;
+  }
+}
+
+// ===========================================================================
+// Fused NF4-decode GEMM (forward: kBwd = false, input gradient: kBwd = true)
+//
+// Output tile 128 (rows of X or G) x 256, K-step 64.  Per stage the shared
+// memory holds the activation tile (128 x 64 bf16, K-major, TMA) and the
+// decoded weight tile (256 x 64 bf16).  The weight tile is written by the
+// decoder warps as 256 rows of 128 bytes, each row one NF4 block of 64
+// consecutive weights (row R at R*128, 16-byte chunk c at (c ^ (R & 7))*16,
+// the 128-byte swizzle pattern):
+//   forward   row R = 64*nb + k: weights (k0+k, n0+64nb .. +63) — an MN-major
+//             operand (atoms of 8 k-rows x 64 n; 8 KB between n-atoms);
+//   backward  row R: weights (n0+R, k0 .. k0+63) of W, i.e. row R of Ŵᵀ's
+//             K-major operand.
+// After the last K-step, one more step accumulates the LoRA term: Zc (or dZ)
+// as the A tile and B (or A) as the weight tile, both by TMA (rank padded to
+// a multiple of 16 with zeros by TMA's out-of-bounds fill).
+// ===========================================================================
+constexpr int kFStages = 4;
+constexpr int kFPStages = 2;
+constexpr int kFA = 16384;           // 128 x 64 bf16
+constexpr int kFB = 32768;           // 256 x 64 bf16
+constexpr int kFP = 8192;            // packed tile
+constexpr int kFThreads = 448;       // warp 0 TMA, 1 MMA, 2..9 decode, 10..13 epilogue
+constexpr int kFDecWarps = 8;
+constexpr int kFEpiWarps = 4;
+constexpr size_t kFSmem = 1024 + kFStages * (kFA + kFB) + kFPStages * kFP + 1024 + 512;
+
+struct FusedArgs {
+  int M;          // rows of the activation / output
+  int Nout;       // output columns (forward: N, backward: K)
+  int Nw;         // row length of the weight (N); blocks per weight row = Nw/64
+  int nk;         // K-steps over the contraction (forward: K/64, backward: N/64)
+  int rsteps;     // MMAs of K=16 in the LoRA step (ceil(r/16))
+  int m_tiles, n_tiles;
+  ScaleView sv;
+  uint16_t* out;  // bf16 [M][Nout]
+  int32_t* d_status;
+};
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// 8 packed nibbles (4 bytes, first weight in the high nibble of byte 0) ->
+// 8 bf16 from the per-block table whose high and low bytes are split into
+// H[0..3] and L[0..3] (entry j's byte in byte j%4 of H[j/4] / L[j/4]).
+__device__ __forceinline__ uint4 decode8(uint32_t p, const uint32_t (&H)[4],
+                                         const uint32_t (&L)[4]) {
+  uint4 o;
+  {
+    const uint32_t s = p & 0x7777u;
+    const uint32_t b = ((p >> 1) & 0x4444u) | 0x3210u;
+    const uint32_t hF = prmt(prmt(H[0], H[1], s), prmt(H[2], H[3], s), b);
+    const uint32_t lF = prmt(prmt(L[0], L[1], s), prmt(L[2], L[3], s), b);
+    o.x = prmt(lF, hF, 0x4051u);
+    o.y = prmt(lF, hF, 0x6273u);
+  }
+  {
+    const uint32_t q = p >> 16;
+    const uint32_t s = q & 0x7777u;
+    const uint32_t b = ((q >> 1) & 0x4444u) | 0x3210u;
+    const uint32_t hF = prmt(prmt(H[0], H[1], s), prmt(H[2], H[3], s), b);
+    const uint32_t lF = prmt(prmt(L[0], L[1], s), prmt(L[2], L[3], s), b);
+    o.z = prmt(lF, hF, 0x4051u);
+    o.w = prmt(lF, hF, 0x6273u);
+  }
+  return o;
+}
+
+// Per-block table: entry j = bf16(C_j * a) (fp32 product, then bf16).
+__device__ __forceinline__ void build_lut(float a, uint32_t (&H)[4], uint32_t (&L)[4]) {
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(kNF4g[2 * i] * a, kNF4g[2 * i + 1] * a);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    H[q] = prmt(w[2 * q], w[2 * q + 1], 0x7531u);
+    L[q] = prmt(w[2 * q], w[2 * q + 1], 0x6420u);
+  }
+}
+
+struct ScaleFetch {
+  float absv;    // absmax (no double quant)
+  uint32_t q;    // code8
+  float s2v;
+};
+
+__device__ __forceinline__ ScaleFetch fetch_scale(const ScaleView& sv, int64_t blk, bool valid) {
+  ScaleFetch f{1.0f, 0u, 1.0f};
+  if (!valid) return f;
+  if (sv.code8 == nullptr) {
+    f.absv = __ldg(sv.absmax + blk);
+  } else {
+    f.q = __ldg(sv.code8 + blk);
+    f.s2v = __ldg(sv.s2 + (blk >> 8));
+  }
+  return f;
+}
+
+__device__ __forceinline__ float finish_scale(const ScaleView& sv, const ScaleFetch& f, float off,
+                                              const float* t8) {
+  if (sv.code8 == nullptr) return f.absv;
+  return __fadd_rn(__fmul_rn(t8[f.q], f.s2v), off);
+}
+
+template <bool kBwd>
+__global__ void __launch_bounds__(kFThreads, 1)
+    fused_nf4_gemm_kernel(const __grid_constant__ CUtensorMap tmAct,
+                          const __grid_constant__ CUtensorMap tmPk,
+                          const __grid_constant__ CUtensorMap tmLA,
+                          const __grid_constant__ CUtensorMap tmLB, FusedArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + kFStages * kFA;
+  uint8_t* sP = sB + kFStages * kFB;
+  float* t8 = reinterpret_cast<float*>(sP + kFPStages * kFP);
+  uint64_t* full_a = reinterpret_cast<uint64_t*>(t8 + 256);
+  uint64_t* full_b = full_a + kFStages;
+  uint64_t* empty = full_b + kFStages;
+  uint64_t* pfull = empty + kFStages;
+  uint64_t* pempty = pfull + kFPStages;
+  uint64_t* tfull = pempty + kFPStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (args.sv.code8 != nullptr) build_t8(t8);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kFStages; ++s) {
+      mbar_init(&full_a[s], 1);
+      mbar_init(&full_b[s], kFDecWarps);
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < kFPStages; ++s) {
+      mbar_init(&pfull[s], 1);
+      mbar_init(&pempty[s], kFDecWarps);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], kFEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int num_tiles = args.m_tiles * args.n_tiles;
+  const int nsteps = args.nk + 1;  // + the LoRA step
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer ---------------------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tmAct);
+      tma_prefetch_desc(&tmPk);
+      tma_prefetch_desc(&tmLA);
+      tma_prefetch_desc(&tmLB);
+      uint32_t it = 0, pit = 0;
+      uint32_t last_parity[kFStages] = {2, 2, 2, 2};
+      uint32_t last_pparity[kFPStages] = {2, 2};
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int m0 = (tile % args.m_tiles) * 128;
+        const int n0 = (tile / args.m_tiles) * 256;
+        for (int kk = 0; kk < nsteps; ++kk, ++it) {
+          const int s = it % kFStages;
+          const uint32_t ph = (it / kFStages) & 1;
+          if (*abort_flag || !mbar_wait(&empty[s], ph ^ 1)) { ok = false; break; }
+          if (kk < args.nk) {
+            mbar_arrive_expect_tx(&full_a[s], kFA);
+            tma_load_2d(sA + s * kFA, &tmAct, &full_a[s], kk * 64, m0);
+            const int ps = pit % kFPStages;
+            const uint32_t pph = (pit / kFPStages) & 1;
+            if (!mbar_wait(&pempty[ps], pph ^ 1)) { last_parity[s] = ph; ok = false; break; }
+            mbar_arrive_expect_tx(&pfull[ps], kFP);
+            if (!kBwd)
+              tma_load_2d(sP + ps * kFP, &tmPk, &pfull[ps], n0 / 2, kk * 64);
+            else
+              tma_load_2d(sP + ps * kFP, &tmPk, &pfull[ps], kk * 32, n0);
+            last_pparity[ps] = pph;
+            ++pit;
+          } else {
+            mbar_arrive_expect_tx(&full_a[s], kFA + kFB);
+            tma_load_2d(sA + s * kFA, &tmLA, &full_a[s], 0, m0);
+            if (!kBwd) {
+#pragma unroll
+              for (int nb = 0; nb < 4; ++nb)
+                tma_load_2d(sB + s * kFB + nb * 8192, &tmLB, &full_a[s], n0 + nb * 64, 0);
+            } else {
+              tma_load_2d(sB + s * kFB, &tmLB, &full_a[s], 0, n0);
+            }
+          }
+          last_parity[s] = ph;
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        // let copies already in flight land before the CTA can exit
+        for (int s = 0; s < kFStages; ++s)
+          if (last_parity[s] < 2) (void)mbar_wait(&full_a[s], last_parity[s]);
+        for (int s = 0; s < kFPStages; ++s)
+          if (last_pparity[s] < 2) (void)mbar_wait(&pfull[s], last_pparity[s]);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer -----------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 256, 0, kBwd ? 0 : 1);
+      uint32_t it = 0, tc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tc) {
+        const uint32_t ab = tc & 1, aph = (tc >> 1) & 1;
+        if (*abort_flag || !mbar_wait(&tempty[ab], aph ^ 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t dt = tmem + ab * 256;
+        for (int kk = 0; kk < nsteps; ++kk, ++it) {
+          const int s = it % kFStages;
+          const uint32_t ph = (it / kFStages) & 1;
+          if (*abort_flag || !mbar_wait(&full_a[s], ph) || !mbar_wait(&full_b[s], ph)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * kFA), b0 = smem_u32(sB + s * kFB);
+          const int nm = (kk < args.nk) ? 4 : args.rsteps;
+          for (int j = 0; j < nm; ++j) {
+            const uint64_t ad = smem_desc(a0 + j * 32, 16, 1024);
+            const uint64_t bd = kBwd ? smem_desc(b0 + j * 32, 16, 1024)
+                                     : smem_desc(b0 + j * 2048, 8192, 1024);
+            umma_bf16(dt, ad, bd, idesc, (kk > 0 || j > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        umma_commit(&tfull[ab]);
+      }
+      if (!ok) *abort_flag = 1;
+      umma_commit(drain);
+      (void)mbar_wait(drain, 0);
+    }
+  } else if (warp < 2 + kFDecWarps) {
+    // ------------------------------ decoders -------------------------------
+    const int R = threadIdx.x - 64;  // weight-tile row 0..255
+    const float off = args.sv.code8 != nullptr ? __ldg(args.sv.offset) : 0.0f;
+    const int bpr = args.Nw / 64;    // NF4 blocks per weight row
+    uint32_t it = 0, pit = 0;
+    bool ok = true;
+    // coordinates of this thread's row for (tile, kk)
+    auto row_block = [&](int tile, int kk, bool& valid) -> int64_t {
+      const int n0 = (tile / args.m_tiles) * 256;
+      if (!kBwd) {
+        const int nb = R >> 6, kr = R & 63;
+        valid = n0 + nb * 64 < args.Nout;
+        return static_cast<int64_t>(kk * 64 + kr) * bpr + (n0 / 64 + nb);
+      } else {
+        valid = n0 + R < args.Nout;
+        return static_cast<int64_t>(n0 + R) * bpr + kk;
+      }
+    };
+    // prefetch the scale of the first decoded step
+    int tile = blockIdx.x;
+    bool v0 = false;
+    ScaleFetch nextf{};
+    if (tile < num_tiles) nextf = fetch_scale(args.sv, row_block(tile, 0, v0), v0);
+    bool nextv = v0;
+    for (; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int kk = 0; kk < nsteps; ++kk, ++it) {
+        const int s = it % kFStages;
+        const uint32_t ph = (it / kFStages) & 1;
+        if (*abort_flag || !mbar_wait(&empty[s], ph ^ 1)) { ok = false; break; }
+        if (kk < args.nk) {
+          const ScaleFetch f = nextf;
+          const bool valid = nextv;
+          // prefetch the next decoded step's scale
+          {
+            int ntile = tile, nkk = kk + 1;
+            if (nkk >= args.nk) { ntile = tile + gridDim.x; nkk = 0; }
+            if (ntile < num_tiles) {
+              bool vv = false;
+              const int64_t nb = row_block(ntile, nkk, vv);
+              nextf = fetch_scale(args.sv, nb, vv);
+              nextv = vv;
+            }
+          }
+          const int ps = pit % kFPStages;
+          const uint32_t pph = (pit / kFPStages) & 1;
+          if (!mbar_wait(&pfull[ps], pph)) { ok = false; break; }
+          const uint8_t* prow;
+          uint32_t c0, c1;
+          if (!kBwd) {
+            const int nb = R >> 6, kr = R & 63;
+            prow = sP + ps * kFP + kr * 128;
+            c0 = static_cast<uint32_t>((2 * nb) ^ (kr & 7));
+            c1 = static_cast<uint32_t>((2 * nb + 1) ^ (kr & 7));
+          } else {
+            prow = sP + ps * kFP + R * 32;
+            c0 = static_cast<uint32_t>((R >> 2) & 1);
+            c1 = c0 ^ 1u;
+          }
+          const uint4 p0 = *reinterpret_cast<const uint4*>(prow + c0 * 16);
+          const uint4 p1 = *reinterpret_cast<const uint4*>(prow + c1 * 16);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&pempty[ps]);
+          ++pit;
+          uint8_t* brow = sB + s * kFB + R * 128;
+          const uint32_t sw = static_cast<uint32_t>(R & 7);
+          if (valid) {
+            const float a = finish_scale(args.sv, f, off, t8);
+            uint32_t H[4], L[4];
+            build_lut(a, H, L);
+            const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(brow + ((static_cast<uint32_t>(c) ^ sw) << 4)) =
+                  decode8(pw[c], H, L);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(brow + (c << 4)) = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full_b[s]);
+        } else {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full_b[s]);
+        }
+      }
+    }
+    if (!ok) *abort_flag = 1;
+  } else {
+    // ------------------------------ epilogue -------------------------------
+    const int q = warp & 3;
+    uint32_t tc = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tc) {
+      const int m0 = (tile % args.m_tiles) * 128;
+      const int n0 = (tile / args.m_tiles) * 256;
+      const uint32_t ab = tc & 1, aph = (tc >> 1) & 1;
+      if (*abort_flag || !mbar_wait(&tfull[ab], aph)) { ok = false; break; }
+      tc_fence_after();
+      const int row = m0 + q * 32 + lane;
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * 256 + c * 32, v);
+        tmem_ld_wait();
+        const int col = n0 + c * 32;
+        if (row < args.M && col < args.Nout) {
+          uint4* dst = reinterpret_cast<uint4*>(args.out + static_cast<int64_t>(row) * args.Nout + col);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1])),
+                                pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
+                                pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
+                                pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[ab]);
+    }
+    if (!ok) *abort_flag = 1;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) raise_status(args.d_status, QLORA_ERR_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ===========================================================================
+// GEMV for M <= 16 (CUDA cores).  CTA = 256 columns x a K-range; lane owns 8
+// consecutive columns (one 32-bit packed word per weight row), warps stride
+// over rows.  fp32 partials per split, reduced in gemv_reduce_kernel.
+// ===========================================================================
+constexpr int kGvRows = 64;  // rows of X staged in shared memory per pass
+
+template <int MT>
+__global__ void __launch_bounds__(256) nf4_gemv_kernel(const uint16_t* __restrict__ X, int M,
+                                                       int K, int N, const uint8_t* __restrict__ packed,
+                                                       ScaleView sv, int rows_per_split,
+                                                       float* __restrict__ partial) {
+  __shared__ float xs[kGvRows][MT];
+  __shared__ float t8[256];
+  __shared__ float red[8][256];
+  if (sv.code8 != nullptr) build_t8(t8);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = blockIdx.x * 256 + lane * 8;
+  const int k0 = blockIdx.y * rows_per_split;
+  const int k1 = min(K, k0 + rows_per_split);
+  const float off = sv.code8 != nullptr ? __ldg(sv.offset) : 0.0f;
+  const bool colok = n < N;
+  float acc[MT][8];
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[m][i] = 0.0f;
+  for (int kb = k0; kb < k1; kb += kGvRows) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < kGvRows * MT; i += blockDim.x) {
+      const int kr = i / MT, m = i % MT;
+      const int k = kb + kr;
+      xs[kr][m] = (m < M && k < k1) ? bf16_bits_to_f32(__ldg(X + static_cast<int64_t>(m) * K + k)) : 0.0f;
+    }
+    __syncthreads();
+    if (colok) {
+      for (int kr = warp; kr < kGvRows && kb + kr < k1; kr += 8) {
+        const int k = kb + kr;
+        const int64_t blk = static_cast<int64_t>(k) * (N / 64) + (n >> 6);
+        float a;
+        if (sv.code8 == nullptr)
+          a = __ldg(sv.absmax + blk);
+        else
+          a = __fadd_rn(__fmul_rn(t8[__ldg(sv.code8 + blk)], __ldg(sv.s2 + (blk >> 8))), off);
+        const uint32_t p = __ldg(reinterpret_cast<const uint32_t*>(packed + ((static_cast<int64_t>(k) * N + n) >> 1)));
+        float w[8];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const uint32_t byte = (p >> (8 * b)) & 0xFFu;
+          const uint32_t pr = pack_bf16x2(kNF4g[byte >> 4] * a, kNF4g[byte & 15u] * a);
+          w[2 * b] = __uint_as_float(pr << 16);
+          w[2 * b + 1] = __uint_as_float(pr & 0xFFFF0000u);
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          const float xv = xs[kr][m];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[m][i] = fmaf(xv, w[i], acc[m][i]);
+        }
+      }
+    }
+  }
+  // reduce the 8 warps' partial sums through shared memory, one row at a time
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    if (m < M) {
+      __syncthreads();
+#pragma unroll
+      for (int i = 0; i < 8; ++i) red[warp][lane * 8 + i] = acc[m][i];
+      __syncthreads();
+      const int col = threadIdx.x;
+      float s = 0.0f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) s += red[w][col];
+      if (blockIdx.x * 256 + col < N)
+        partial[(static_cast<int64_t>(blockIdx.y) * M + m) * N + blockIdx.x * 256 + col] = s;
+    }
+  }
+}
+
+// Y[m][n] = bf16( sum_s partial[s][m][n] + sum_j Zc[m][j] * B[j][n] )
+__global__ void gemv_reduce_kernel(const float* __restrict__ partial, int splits, int M, int N,
+                                   const uint16_t* __restrict__ Zc, const uint16_t* __restrict__ B,
+                                   int r, uint16_t* __restrict__ Y) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<int64_t>(M) * N) return;
+  const int m = static_cast<int>(idx / N), n = static_cast<int>(idx % N);
+  float acc = 0.0f;
+  for (int s = 0; s < splits; ++s) acc += partial[(static_cast<int64_t>(s) * M + m) * N + n];
+  float lora = 0.0f;
+  for (int j = 0; j < r; ++j)
+    lora = fmaf(bf16_bits_to_f32(Zc[static_cast<int64_t>(m) * r + j]),
+                bf16_bits_to_f32(B[static_cast<int64_t>(j) * N + n]), lora);
+  Y[idx] = static_cast<uint16_t>(pack_bf16x2(acc + lora, 0.0f) & 0xFFFFu);
+}
+
+// ===========================================================================
+// Host side
+// ===========================================================================
+namespace {
+
+int skinny_splits(int Mp, int nk, int num_sms) {
+  const int mt = (Mp + 127) / 128;
+  int want = (2 * num_sms + mt - 1) / mt;
+  if (want < 1) want = 1;
+  if (want > nk) want = nk;
+  const int per = (nk + want - 1) / want;
+  return (nk + per - 1) / per;
+}
+
+struct WsCursor {
+  char* p;
+  size_t left;
+  bool ok = true;
+  void* take(size_t bytes) {
+    bytes = (bytes + 255) & ~static_cast<size_t>(255);
+    if (bytes > left) { ok = false; return nullptr; }
+    void* r = p;
+    p += bytes;
+    left -= bytes;
+    return r;
+  }
+};
+
+size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+template <bool A, bool B>
+cudaError_t set_skinny_attr() {
+  static bool done = false;
+  if (done) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(skinny_gemm_kernel<A, B>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSkSmem));
+  if (e == cudaSuccess) done = true;
+  return e;
+}
+
+// D = scale * A(m',k') B(n',k') ; writes through skinny_reduce_kernel.
+template <bool kAmn, bool kBmn>
+cudaError_t run_skinny(const CUtensorMap& ta, const CUtensorMap& tb, int Mp, int Kp, int ncols,
+                       float scale, int mode, void* out, int ld, float* partial, int splits,
+                       int32_t* d_status, cudaStream_t st) {
+  cudaError_t e = set_skinny_attr<kAmn, kBmn>();
+  if (e != cudaSuccess) return e;
+  const int nk = (Kp + 63) / 64;
+  SkinnyArgs a;
+  a.Mp = Mp;
+  a.nk = nk;
+  a.kb_per_split = (nk + splits - 1) / splits;
+  a.partial = partial;
+  a.d_status = d_status;
+  dim3 grid((Mp + 127) / 128, splits);
+  {
+    ProfScope prof(kProfSkinny, st);
+    skinny_gemm_kernel<kAmn, kBmn><<<grid, kSkThreads, kSkSmem, st>>>(ta, tb, a);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t total = static_cast<int64_t>(Mp) * ncols;
+  {
+    ProfScope prof(kProfOther, st);
+    skinny_reduce_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(
+        partial, splits, Mp, ncols, scale, mode, out, ld);
+  }
+  return cudaGetLastError();
+}
+
+template <bool kBwd>
+cudaError_t set_fused_attr() {
+  static bool done = false;
+  if (done) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(fused_nf4_gemm_kernel<kBwd>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kFSmem));
+  if (e == cudaSuccess) done = true;
+  return e;
+}
+
+constexpr CUtensorMapDataType kBF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+constexpr CUtensorMapDataType kU8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+constexpr CUtensorMapSwizzle kSW128 = CU_TENSOR_MAP_SWIZZLE_128B;
+constexpr CUtensorMapSwizzle kSW32 = CU_TENSOR_MAP_SWIZZLE_32B;
+
+int rsteps_of(int r) { return (r + 15) / 16; }
+
+size_t gemv_splits_and_bytes(int64_t M, int64_t K, int64_t N, int num_sms, int* splits_out) {
+  const int ntiles = static_cast<int>((N + 255) / 256);
+  int s = (2 * num_sms + ntiles - 1) / ntiles;
+  const int maxs = static_cast<int>((K + kGvRows - 1) / kGvRows);
+  if (s > maxs) s = maxs;
+  if (s < 1) s = 1;
+  if (splits_out) *splits_out = s;
+  return align256(static_cast<size_t>(s) * M * N * 4);
+}
+
+}  // namespace
+
+static int g_ws_sms = 148;  // sizing assumption for workspace queries (B200)
+
+size_t linear_fwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) {
+  (void)r;
+  const int S = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
+  size_t b = align256(static_cast<size_t>(S) * M * 64 * 4);
+  if (M <= 16) b += gemv_splits_and_bytes(M, K, N, g_ws_sms, nullptr);
+  return b;
+}
+
+size_t linear_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) {
+  (void)r;
+  const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(N / 64), g_ws_sms);
+  const int nkm = static_cast<int>((M + 63) / 64);
+  const int Sa = skinny_splits(static_cast<int>(K), nkm, g_ws_sms);
+  const int Sb = skinny_splits(static_cast<int>(N), nkm, g_ws_sms);
+  size_t b = align256(static_cast<size_t>(M) * 64 * 2);                 // dZ (bf16, padded to 64)
+  b += align256(static_cast<size_t>(Sz) * M * 64 * 4);                  // dZ partials
+  b += align256(static_cast<size_t>(Sa) * K * 64 * 4);                  // dA partials
+  b += align256(static_cast<size_t>(Sb) * N * 64 * 4);                  // dB partials
+  return b;
+}
+
+cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint16_t* X,
+                              const uint8_t* packed, ScaleView sv, const uint16_t* A,
+                              const uint16_t* B, float c, uint16_t* Y, uint16_t* Zc, void* ws,
+                              size_t ws_bytes, int32_t* d_status, cudaStream_t st, int num_sms) {
+  (void)num_sms;
+  WsCursor cur{static_cast<char*>(ws), ws_bytes};
+  // Zc = bf16(c * X A): A operand X (K-major), B operand A (MN-major over r)
+  CUtensorMap tX, tAl, tZc, tBl, tPk;
+  if (!make_tmap_2d(&tX, X, kBF16, 2, M, K, K, 64, 128, kSW128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tAl, A, kBF16, 2, K, r, r, 64, 64, kSW128)) return cudaErrorInvalidValue;
+  const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
+  float* pz = static_cast<float*>(cur.take(static_cast<size_t>(Sz) * M * 64 * 4));
+  if (!cur.ok) return cudaErrorInvalidValue;
+  cudaError_t e = run_skinny<false, true>(tX, tAl, static_cast<int>(M), static_cast<int>(K), r,
+                                          c, 0, Zc, r, pz, Sz, d_status, st);
+  if (e != cudaSuccess) return e;
+
+  if (M <= 16) {
+    int S = 1;
+    gemv_splits_and_bytes(M, K, N, g_ws_sms, &S);
+    float* pg = static_cast<float*>(cur.take(static_cast<size_t>(S) * M * N * 4));
+    if (!cur.ok) return cudaErrorInvalidValue;
+    const int rows = static_cast<int>(((K + S - 1) / S + kGvRows - 1) / kGvRows * kGvRows);
+    const int splits = static_cast<int>((K + rows - 1) / rows);
+    dim3 grid(static_cast<unsigned>((N + 255) / 256), splits);
+    const int Mi = static_cast<int>(M), Ki = static_cast<int>(K), Ni = static_cast<int>(N);
+    {
+    ProfScope prof(kProfGemv, st);
+    if (M <= 1)
+      nf4_gemv_kernel<1><<<grid, 256, 0, st>>>(X, Mi, Ki, Ni, packed, sv, rows, pg);
+    else if (M <= 4)
+      nf4_gemv_kernel<4><<<grid, 256, 0, st>>>(X, Mi, Ki, Ni, packed, sv, rows, pg);
+    else if (M <= 8)
+      nf4_gemv_kernel<8><<<grid, 256, 0, st>>>(X, Mi, Ki, Ni, packed, sv, rows, pg);
+    else
+      nf4_gemv_kernel<16><<<grid, 256, 0, st>>>(X, Mi, Ki, Ni, packed, sv, rows, pg);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t total = M * N;
+    {
+      ProfScope prof(kProfOther, st);
+      gemv_reduce_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(
+          pg, splits, Mi, Ni, Zc, B, r, Y);
+    }
+    return cudaGetLastError();
+  }
+
+  e = set_fused_attr<false>();
+  if (e != cudaSuccess) return e;
+  if (!make_tmap_2d(&tPk, packed, kU8, 1, K, N / 2, N / 2, 128, 64, kSW128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tZc, Zc, kBF16, 2, M, r, r, 64, 128, kSW128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tBl, B, kBF16, 2, r, N, N, 64, 64, kSW128)) return cudaErrorInvalidValue;
+  FusedArgs fa;
+  fa.M = static_cast<int>(M);
+  fa.Nout = static_cast<int>(N);
+  fa.Nw = static_cast<int>(N);
+  fa.nk = static_cast<int>(K / 64);
+  fa.rsteps = rsteps_of(r);
+  fa.m_tiles = static_cast<int>((M + 127) / 128);
+  fa.n_tiles = static_cast<int>((N + 255) / 256);
+  fa.sv = sv;
+  fa.out = Y;
+  fa.d_status = d_status;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int tiles = fa.m_tiles * fa.n_tiles;
+  const int grid = tiles < sms ? tiles : sms;
+  {
+    ProfScope prof(kProfFusedFwd, st);
+    fused_nf4_gemm_kernel<false><<<grid, kFThreads, kFSmem, st>>>(tX, tPk, tZc, tBl, fa);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint16_t* dY,
+                              const uint16_t* X, const uint16_t* Zc, const uint8_t* packed,
+                              ScaleView sv, const uint16_t* A, const uint16_t* B, float c,
+                              uint16_t* dX, float* dA, float* dB, void* ws, size_t ws_bytes,
+                              int32_t* d_status, cudaStream_t st, int num_sms) {
+  (void)num_sms;
+  WsCursor cur{static_cast<char*>(ws), ws_bytes};
+  uint16_t* dZ = static_cast<uint16_t*>(cur.take(static_cast<size_t>(M) * 64 * 2));
+  const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(N / 64), g_ws_sms);
+  const int nkm = static_cast<int>((M + 63) / 64);
+  const int Sa = skinny_splits(static_cast<int>(K), nkm, g_ws_sms);
+  const int Sb = skinny_splits(static_cast<int>(N), nkm, g_ws_sms);
+  float* pz = static_cast<float*>(cur.take(static_cast<size_t>(Sz) * M * 64 * 4));
+  float* pa = static_cast<float*>(cur.take(static_cast<size_t>(Sa) * K * 64 * 4));
+  float* pb = static_cast<float*>(cur.take(static_cast<size_t>(Sb) * N * 64 * 4));
+  if (!cur.ok) return cudaErrorInvalidValue;
+  cudaError_t e = cudaMemsetAsync(dZ, 0, static_cast<size_t>(M) * 64 * 2, st);
+  if (e != cudaSuccess) return e;
+
+  CUtensorMap tG, tBk, tXmn, tdZ, tGmn, tZcmn, tPk, tAl;
+  // dZ = c * G B^T : A operand G (K-major over N), B operand B (K-major: rows r, cols N)
+  if (!make_tmap_2d(&tG, dY, kBF16, 2, M, N, N, 64, 128, kSW128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tBk, B, kBF16, 2, r, N, N, 64, 64, kSW128)) return cudaErrorInvalidValue;
+  e = run_skinny<false, false>(tG, tBk, static_cast<int>(M), static_cast<int>(N), r, c, 0, dZ, 64,
+                               pz, Sz, d_status, st);
+  if (e != cudaSuccess) return e;
+  // dA = X^T dZ : A operand X^T (MN-major over K), B operand dZ (MN-major over r)
+  if (!make_tmap_2d(&tXmn, X, kBF16, 2, M, K, K, 64, 64, kSW128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tdZ, dZ, kBF16, 2, M, 64, 64, 64, 64, kSW128)) return cudaErrorInvalidValue;
+  e = run_skinny<true, true>(tXmn, tdZ, static_cast<int>(K), static_cast<int>(M), r, 1.0f, 1, dA,
+                             r, pa, Sa, d_status, st);
+  if (e != cudaSuccess) return e;
+  // dB^T = G^T Zc : A operand G^T (MN-major over N), B operand Zc (MN-major over r)
+  if (!make_tmap_2d(&tGmn, dY, kBF16, 2, M, N, N, 64, 64, kSW128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tZcmn, Zc, kBF16, 2, M, r, r, 64, 64, kSW128)) return cudaErrorInvalidValue;
+  e = run_skinny<true, true>(tGmn, tZcmn, static_cast<int>(N), static_cast<int>(M), r, 1.0f, 2,
+                             dB, r, pb, Sb, d_status, st);
+  if (e != cudaSuccess) return e;
+  // dX = G W^T + dZ A^T
+  e = set_fused_attr<true>();
+  if (e != cudaSuccess) return e;
+  if (!make_tmap_2d(&tPk, packed, kU8, 1, K, N / 2, N / 2, 32, 256, kSW32)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tAl, A, kBF16, 2, K, r, r, 64, 256, kSW128)) return cudaErrorInvalidValue;
+  CUtensorMap tdZa;
+  if (!make_tmap_2d(&tdZa, dZ, kBF16, 2, M, 64, 64, 64, 128, kSW128)) return cudaErrorInvalidValue;
+  FusedArgs fa;
+  fa.M = static_cast<int>(M);
+  fa.Nout = static_cast<int>(K);
+  fa.Nw = static_cast<int>(N);
+  fa.nk = static_cast<int>(N / 64);
+  fa.rsteps = rsteps_of(r);
+  fa.m_tiles = static_cast<int>((M + 127) / 128);
+  fa.n_tiles = static_cast<int>((K + 255) / 256);
+  fa.sv = sv;
+  fa.out = dX;
+  fa.d_status = d_status;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int tiles = fa.m_tiles * fa.n_tiles;
+  const int grid = tiles < sms ? tiles : sms;
+  {
+    ProfScope prof(kProfFusedBwd, st);
+    fused_nf4_gemm_kernel<true><<<grid, kFThreads, kFSmem, st>>>(tG, tPk, tdZa, tAl, fa);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace qnf4

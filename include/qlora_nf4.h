@@ -1,0 +1,220 @@
+/*
+ * qlora_nf4.h — C ABI of the NF4 frozen-base LoRA linear layer for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The layer (page "QLoRA：冻结的 4-bit 权重怎样参与一次微调", §量化基座与可训练支路
+ * 怎样相加 and §冻结权重为什么仍然需要输入梯度):
+ *
+ *     Z = X·A,   Y = X·Ŵ + c·Z·B               X: M×K, Ŵ: K×N, A: K×r, B: r×N
+ *     dZ = c·G·Bᵀ,  dX = G·Ŵᵀ + dZ·Aᵀ,  dA = Xᵀ·dZ,  dB = c·Zᵀ·G
+ *
+ * where Ŵ is decoded on the fly from blockwise NF4 codes and G = ∂L/∂Y.
+ * No gradient is produced for Ŵ or its packed codes and scales.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers named d_* or documented as "device" are CUDA device pointers;
+ *   everything else (the state struct itself, scalars, the status output of
+ *   qlora_status_sync) is host memory.
+ * - All matrices are dense, row-major and contiguous.  bf16 tensors are passed
+ *   as uint16_t bit patterns.  Device pointers must be 16-byte aligned.
+ * - Ownership: the caller allocates and frees every buffer, including the
+ *   workspace whose size the *_workspace_size functions report.  The library
+ *   never allocates device memory and never synchronizes the stream, except
+ *   in qlora_status_sync.
+ * - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default).
+ * - Errors: a host-side validation failure returns its qlora_status at once and
+ *   enqueues nothing.  Errors that only the device can see (non-finite input,
+ *   bad padding, an internal wait that ran out) are OR-ed as bit (1 << code)
+ *   into the caller's device word `d_status` (may be NULL to ignore them) and
+ *   the kernel finishes normally; outputs are then unspecified.  Read the word
+ *   with qlora_status_sync and clear it with qlora_status_clear.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* qlora_stream_t;   /* same type as cudaStream_t */
+
+typedef int32_t qlora_status;
+#define QLORA_OK               0
+#define QLORA_ERR_INVALID_ARG  1   /* null pointer, bad size, misaligned buffer, small workspace */
+#define QLORA_ERR_UNSUPPORTED  2   /* shape outside the supported set (see each call) */
+#define QLORA_ERR_NONFINITE    3   /* NaN/Inf weight or non-finite reconstruction */
+#define QLORA_ERR_BAD_PADDING  4   /* odd-length payload whose last low nibble is not code 7 */
+#define QLORA_ERR_CUDA         5   /* a CUDA runtime call failed (no device, launch error) */
+#define QLORA_ERR_TIMEOUT      6   /* a bounded device-side wait ran out */
+
+typedef int32_t qlora_dtype;
+#define QLORA_DTYPE_BF16 0
+#define QLORA_DTYPE_F32  1
+
+/*
+ * Quantized state of one K×N weight (page "QLoRA：冻结的 4-bit 权重怎样参与一次
+ * 微调", §从 NF4 索引打包成字节 and §Double Quantization 压缩的是 Scale).
+ *
+ * The weight is flattened row-major (index i = k·N + n) and cut into blocks
+ * of 64 consecutive elements; block b holds elements [64b, 64b+64), the last
+ * one possibly shorter.  n1 = ceil(numel/64), n2 = ceil(n1/256).
+ *   packed : ceil(numel/2) bytes; byte i = (code[2i] << 4) | code[2i+1]; an odd
+ *            tail is padded with code 7 in the low nibble.           (device)
+ *   absmax : n1 fp32 first-level scales, used when double_quant == 0. (device)
+ *   code8  : n1 8-bit codes of the centred scales (double_quant == 1). (device)
+ *   s2     : n2 fp32 second-level scales (double_quant == 1).          (device)
+ *   offset : 1 fp32, the mean of the first-level scales (double_quant == 1).
+ *            Decode scale a' = (T8[code8[b]] · s2[b/256]) + offset, each
+ *            operation rounded to fp32.                                (device)
+ * Unused pointers may be NULL.  The struct itself lives in host memory.
+ */
+typedef struct qlora_nf4_state {
+  int64_t  numel;         /* logical element count (K·N for a weight), >= 1 */
+  int32_t  blocksize;     /* must be 64 */
+  int32_t  double_quant;  /* 0 or 1 */
+  int32_t  dq_blocksize;  /* must be 256 */
+  int32_t  reserved;      /* must be 0 */
+  uint8_t* packed;
+  float*   absmax;
+  uint8_t* code8;
+  float*   s2;
+  float*   offset;
+} qlora_nf4_state;
+
+/* ABI version of this header (bumped on any incompatible change). */
+#define QLORA_NF4_ABI_VERSION 1
+int32_t qlora_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* qlora_status_str(qlora_status s);
+
+/* Element counts: n1 = ceil(numel/64), n2 = ceil(n1/256); 0 for numel < 1. */
+int64_t qlora_nf4_n1(int64_t numel);
+int64_t qlora_nf4_n2(int64_t numel);
+
+/*
+ * Read the device status word on `stream` (this call synchronizes the stream)
+ * into *h_mask (host) and return the lowest-numbered error whose bit is set,
+ * or QLORA_OK.  Returns QLORA_ERR_CUDA if the copy fails.
+ */
+qlora_status qlora_status_sync(const int32_t* d_status, qlora_stream_t stream, int32_t* h_mask);
+
+/* Enqueue a reset of the device status word to 0. */
+qlora_status qlora_status_clear(int32_t* d_status, qlora_stream_t stream);
+
+/*
+ * NF4 quantization — page "QLoRA：冻结的 4-bit 权重怎样参与一次微调",
+ * §NF4 保存的是索引而不是均匀整数值, §从 NF4 索引打包成字节 and
+ * §Double Quantization 压缩的是 Scale.
+ *
+ * Per 64-block: a = max|w| (exact), scale s = a, or 1 for an all-zero block;
+ * code = the index of the nearest of the 16 NF4 values to w/s, ties to the
+ * smaller index (decided exactly, as real numbers); codes packed high nibble
+ * first.  Without double quantization s goes to st->absmax.  With it, the
+ * n1 scales are centred on their exactly computed, once-rounded fp32 mean
+ * (st->offset), cut into groups of 256 with an fp32 absmax each (st->s2; 1
+ * for an all-zero group), and each centred scale gets the 8-bit code of the
+ * nearest value of the signed dynamic codebook T8 (ties to the smaller value)
+ * in st->code8.  The codes always come from the exact first-level scale.
+ *
+ *   W        : device, numel elements of `dtype` (QLORA_DTYPE_BF16 or _F32).
+ *   st       : host struct; numel >= 1; its device buffers receive the result.
+ *   ws       : device workspace of at least
+ *              qlora_nf4_quantize_workspace_size(numel, double_quant) bytes
+ *              (may be NULL when that size is 0).
+ * Device errors: QLORA_ERR_NONFINITE if any weight is NaN or ±Inf.
+ * Host errors: INVALID_ARG (null/misaligned pointers, numel < 1, bad
+ * blocksize, small workspace), UNSUPPORTED (numel > 2^40), CUDA.
+ */
+size_t qlora_nf4_quantize_workspace_size(int64_t numel, int32_t double_quant);
+qlora_status qlora_nf4_quantize(const void* W, qlora_dtype dtype, const qlora_nf4_state* st,
+                                void* ws, size_t ws_bytes, int32_t* d_status,
+                                qlora_stream_t stream);
+
+/*
+ * NF4 dequantization — page "QLoRA：冻结的 4-bit 权重怎样参与一次微调",
+ * §NF4 保存的是索引而不是均匀整数值 (reconstruction a·C_j) and §量化基座与可训练
+ * 支路怎样相加 (BF16 compute type).
+ *
+ * W_hat[i] = bf16(C[code_i] · a'_b), the exact product rounded once to bf16
+ * (nearest, ties to even), a'_b the decode scale of block b = i/64.
+ *   W_hat : device, numel bf16 outputs.
+ * Device errors: BAD_PADDING (odd numel whose last low nibble is not 7),
+ * NONFINITE (a decode scale that is not finite).
+ */
+qlora_status qlora_nf4_dequantize(const qlora_nf4_state* st, uint16_t* W_hat,
+                                  int32_t* d_status, qlora_stream_t stream);
+
+/*
+ * Forward — Z = X·A, Y = X·Ŵ + c·Z·B (page "QLoRA：冻结的 4-bit 权重怎样参与一次
+ * 微调", §量化基座与可训练支路怎样相加; c = α/r).
+ *
+ *   X  : device bf16 M×K      A : device bf16 K×r      B : device bf16 r×N
+ *   W  : NF4 state of the K×N weight (numel must equal K·N)
+ *   Y  : device bf16 M×N output
+ *   Zc : device bf16 M×r output, bf16(c·X·A); pass it to qlora_linear_bwd.
+ * The product is computed in fp32 on bf16 operands: Ŵ is decoded in tiles
+ * to bf16 (each weight within one bf16 ulp of qlora_nf4_dequantize's output)
+ * and never written to memory.  M <= 16 runs the HBM-bound GEMV path, larger
+ * M the fused tensor-core path.
+ * Shapes: M >= 1, K % 64 == 0, N % 64 == 0, 1 <= r <= 64, else UNSUPPORTED.
+ * ws: at least qlora_linear_fwd_workspace_size(M, K, N, r) bytes.
+ */
+size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t K, int64_t N, int32_t r);
+qlora_status qlora_linear_fwd(int64_t M, int64_t K, int64_t N, int32_t r,
+                              const uint16_t* X, const qlora_nf4_state* W,
+                              const uint16_t* A, const uint16_t* B, float c,
+                              uint16_t* Y, uint16_t* Zc,
+                              void* ws, size_t ws_bytes, int32_t* d_status,
+                              qlora_stream_t stream);
+
+/*
+ * Backward — page "QLoRA：冻结的 4-bit 权重怎样参与一次微调",
+ * §冻结权重为什么仍然需要输入梯度:
+ *   dZ = c·dY·Bᵀ,   dX = dY·Ŵᵀ + dZ·Aᵀ,   dA = Xᵀ·dZ,   dB = Zcᵀ·dY  (= c·Zᵀ·dY)
+ *
+ *   dY : device bf16 M×N       X : device bf16 M×K      Zc : the forward's Zc
+ *   dX : device bf16 M×K output
+ *   dA : device fp32 K×r output     dB : device fp32 r×N output
+ * No gradient is produced for W (the frozen base).  Same shape rules and
+ * workspace convention as the forward.
+ */
+size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t K, int64_t N, int32_t r);
+qlora_status qlora_linear_bwd(int64_t M, int64_t K, int64_t N, int32_t r,
+                              const uint16_t* dY, const uint16_t* X, const uint16_t* Zc,
+                              const qlora_nf4_state* W, const uint16_t* A, const uint16_t* B,
+                              float c, uint16_t* dX, float* dA, float* dB,
+                              void* ws, size_t ws_bytes, int32_t* d_status,
+                              qlora_stream_t stream);
+
+/*
+ * Launch timing, for measurement tools (no counterpart on the pages).  While
+ * enabled, each kernel launch of the library is bracketed by two CUDA events
+ * recorded on the stream the kernel runs on.  qlora_profile_read waits for
+ * the recorded events, adds their elapsed times to per-class totals and
+ * returns the total milliseconds and the launch count of class `kind`
+ * (QLORA_PROF_*), or of all classes for kind = -1.  Launch counts are kept
+ * whether or not timing is enabled.  qlora_profile_reset zeroes the totals.
+ * Not thread-safe across devices; meant for one measuring process.
+ */
+#define QLORA_PROF_FUSED_FWD  0   /* fused NF4 GEMM, forward (Y)        */
+#define QLORA_PROF_FUSED_BWD  1   /* fused NF4 GEMM, input gradient (dX) */
+#define QLORA_PROF_SKINNY     2   /* rank-r contractions (Zc, dZ, dA, dB) */
+#define QLORA_PROF_QUANTIZE   3   /* NF4 encoder and double quantization */
+#define QLORA_PROF_DEQUANTIZE 4   /* standalone dequantization           */
+#define QLORA_PROF_GEMV       5   /* M <= 16 GEMV                        */
+#define QLORA_PROF_OTHER      6   /* split-K reductions                  */
+qlora_status qlora_profile_enable(int32_t on);
+qlora_status qlora_profile_read(int32_t kind, double* total_ms, int64_t* launches);
+qlora_status qlora_profile_reset(void);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* QLORA_NF4_H */

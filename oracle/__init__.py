@@ -18,7 +18,7 @@ Parity status of each function is stated in its module header.
 """
 from .nf4 import (  # noqa: F401
     NF4, BLOCKSIZE, DQ_BLOCKSIZE, NonFiniteError, PaddingError,
-    encode_block, quantize_nf4, pack_codes, unpack_codes,
+    encode_block, block_scales, quantize_nf4, pack_codes, unpack_codes,
     dq_codebook, exact_mean_f32, double_quantize, decode_scales,
     round_to_bf16, dequantize, bit_budget,
 )

@@ -94,6 +94,25 @@ def encode_block(values):
     return codes, restored, scale
 
 
+def block_scales(w, blocksize: int = BLOCKSIZE):
+    """The scale step alone: max|w| per block of the row-major flattening, or
+    1.0 for an all-zero block, as fp32 (exact: it is an input magnitude)."""
+    w = np.asarray(w, dtype=np.float32).ravel()
+    P = w.size
+    if P == 0:
+        raise ValueError("empty tensor")
+    n1 = -(-P // blocksize)
+    full = (P // blocksize) * blocksize
+    amax = np.empty(n1, dtype=np.float32)
+    if full:
+        amax[:P // blocksize] = np.max(np.abs(w[:full].reshape(-1, blocksize)), axis=1)
+    if full < P:
+        amax[-1] = np.max(np.abs(w[full:]))
+    if not np.all(np.isfinite(amax)):
+        raise NonFiniteError("nonempty finite block required")
+    return np.where(amax > 0, amax, np.float32(1.0)).astype(np.float32)
+
+
 def quantize_nf4(w, blocksize: int = BLOCKSIZE, chunk_blocks: int = 1 << 15):
     """Blockwise NF4 codes and fp32 scales for a flat array of weights.
 

@@ -1,0 +1,67 @@
+"""Helpers shared by the GPU parity tests (oracle side and device side kept
+apart: the oracle only ever sees NumPy inputs from the seeded generators)."""
+import numpy as np
+import torch
+
+from oracle import nf4
+
+
+def dev():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return torch.device("cuda:0")
+
+
+def to_dev(x, dtype=torch.bfloat16):
+    """NumPy fp32 array (bf16-valued for bf16 tensors) -> contiguous CUDA tensor."""
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(dev()).to(dtype).contiguous()
+
+
+def to_np(t):
+    return t.detach().to(torch.float32).cpu().numpy().astype(np.float64)
+
+
+def bf16_bits(t):
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().astype(np.uint16)
+
+
+def rel_fro(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    den = np.linalg.norm(ref)
+    return float(np.linalg.norm(got - ref) / (den if den > 0 else 1.0))
+
+
+class OracleWeight:
+    """The oracle's own quantization of a weight, from the same NumPy input."""
+
+    def __init__(self, W, double_quant):
+        w = np.asarray(W, dtype=np.float32).ravel()
+        self.shape = np.asarray(W).shape
+        self.codes, self.absmax = nf4.quantize_nf4(w)
+        self.packed, self.length = nf4.pack_codes(self.codes)
+        self.dq = double_quant
+        if double_quant:
+            self.code8, self.s2, self.offset = nf4.double_quantize(self.absmax)
+            self.scales = nf4.decode_scales(self.absmax.size, code8=self.code8, s2=self.s2,
+                                            offset=self.offset)
+        else:
+            self.scales = self.absmax
+        self._what = None
+
+    @property
+    def w_hat(self):
+        if self._what is None:
+            self._what = nf4.dequantize(self.packed, self.length, self.scales).reshape(self.shape)
+        return self._what
+
+
+def assert_state_equal(w_gpu, ow: OracleWeight):
+    assert np.array_equal(w_gpu.packed.cpu().numpy(), ow.packed), "packed bytes differ"
+    if ow.dq:
+        assert np.array_equal(w_gpu.code8.cpu().numpy(), ow.code8), "scale codes differ"
+        assert np.array_equal(w_gpu.s2.cpu().numpy().view(np.uint32), ow.s2.view(np.uint32)), "s2 differs"
+        assert w_gpu.offset.cpu().numpy().view(np.uint32)[0] == np.float32(ow.offset).view(np.uint32), \
+            "offset differs"
+    else:
+        assert np.array_equal(w_gpu.absmax.cpu().numpy().view(np.uint32), ow.absmax.view(np.uint32)), \
+            "absmax differs"

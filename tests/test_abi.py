@@ -1,0 +1,124 @@
+"""The C-ABI library loads without a GPU, exports every symbol the header
+declares, and its host-side validation rejects bad arguments before any
+device work.  No compute call is made here."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "qlora_nf4.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from tests.conftest import ensure_built
+    ensure_built()
+    from bit_nf4_quantized_pack_b200 import _lib
+    return _lib
+
+
+def header_functions():
+    text = open(HEADER, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(qlora_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(L):
+    declared = header_functions()
+    assert len(declared) >= 13
+    assert sorted(L.SIGNATURES) == declared
+    out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (qlora_\w+)", out))
+    assert set(declared) <= exported
+    for name in declared:
+        assert getattr(L.lib, name) is not None
+
+
+def test_library_needs_no_libcuda_to_load(L):
+    out = subprocess.run(["ldd", L.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out
+
+
+def test_status_strings_and_counts(L):
+    lib = L.lib
+    assert lib.qlora_abi_version() == L.ABI_VERSION
+    for code in range(7):
+        assert lib.qlora_status_str(code)
+    assert lib.qlora_status_str(99) == b"unknown status"
+    assert lib.qlora_nf4_n1(1) == 1 and lib.qlora_nf4_n1(64) == 1 and lib.qlora_nf4_n1(65) == 2
+    assert lib.qlora_nf4_n2(64 * 256) == 1 and lib.qlora_nf4_n2(64 * 256 + 1) == 2
+    assert lib.qlora_nf4_n1(0) == 0 and lib.qlora_nf4_n2(0) == 0
+
+
+def test_workspace_sizes(L):
+    lib = L.lib
+    assert lib.qlora_nf4_quantize_workspace_size(1000, 0) == 0
+    assert lib.qlora_nf4_quantize_workspace_size(64 * 100, 1) >= 2048 + 4 * 100
+    assert lib.qlora_linear_fwd_workspace_size(4096, 4096, 4096, 16) > 0
+    assert lib.qlora_linear_bwd_workspace_size(4096, 4096, 4096, 16) > 0
+    # unsupported shapes report 0
+    assert lib.qlora_linear_fwd_workspace_size(16, 100, 64, 16) == 0
+    assert lib.qlora_linear_fwd_workspace_size(16, 64, 64, 12) == 0
+
+
+def _state(L, numel=128, dq=0, packed=4096):
+    st = L.NF4StateC()
+    st.numel, st.blocksize, st.double_quant, st.dq_blocksize, st.reserved = numel, 64, dq, 256, 0
+    st.packed = packed
+    st.absmax = 4096
+    st.code8, st.s2, st.offset = 4096, 4096, 4096
+    return st
+
+
+def test_host_validation_rejects_before_device_work(L):
+    lib, E = L.lib, L
+    st = _state(L)
+    fake = C.c_void_p(4096)
+    # null W, misaligned W, bad dtype, empty tensor, bad blocksize
+    assert lib.qlora_nf4_quantize(None, 0, C.byref(st), None, 0, None, None) == E.QLORA_ERR_INVALID_ARG
+    assert lib.qlora_nf4_quantize(C.c_void_p(4097), 0, C.byref(st), None, 0, None, None) == E.QLORA_ERR_INVALID_ARG
+    assert lib.qlora_nf4_quantize(fake, 7, C.byref(st), None, 0, None, None) == E.QLORA_ERR_INVALID_ARG
+    bad = _state(L, numel=0)
+    assert lib.qlora_nf4_quantize(fake, 0, C.byref(bad), None, 0, None, None) == E.QLORA_ERR_INVALID_ARG
+    bad = _state(L)
+    bad.blocksize = 128
+    assert lib.qlora_nf4_quantize(fake, 0, C.byref(bad), None, 0, None, None) == E.QLORA_ERR_INVALID_ARG
+    bad = _state(L, numel=1 << 39)
+    assert lib.qlora_nf4_quantize(fake, 0, C.byref(bad), None, 0, None, None) == E.QLORA_ERR_UNSUPPORTED
+    # double quant without workspace
+    dq = _state(L, dq=1)
+    assert lib.qlora_nf4_quantize(fake, 0, C.byref(dq), None, 0, None, None) == E.QLORA_ERR_INVALID_ARG
+    assert lib.qlora_nf4_quantize(None, 0, None, None, 0, None, None) == E.QLORA_ERR_INVALID_ARG
+    assert lib.qlora_nf4_dequantize(C.byref(st), None, None, None) == E.QLORA_ERR_INVALID_ARG
+    # linear: unsupported shapes and rank
+    w = _state(L, numel=64 * 64)
+    args = [fake, C.byref(w), fake, fake, 1.0, fake, fake, fake, 1 << 20, None, None]
+    assert lib.qlora_linear_fwd(8, 100, 64, 16, *args) == E.QLORA_ERR_UNSUPPORTED
+    assert lib.qlora_linear_fwd(8, 64, 64, 4, *args) == E.QLORA_ERR_UNSUPPORTED
+    assert lib.qlora_linear_fwd(8, 64, 64, 72, *args) == E.QLORA_ERR_UNSUPPORTED
+    assert lib.qlora_linear_fwd(0, 64, 64, 16, *args) == E.QLORA_ERR_INVALID_ARG
+    assert lib.qlora_linear_fwd(8, 128, 64, 16, *args) == E.QLORA_ERR_INVALID_ARG   # numel != K*N
+    args_nan = [fake, C.byref(w), fake, fake, float("nan"), fake, fake, fake, 1 << 20, None, None]
+    assert lib.qlora_linear_fwd(8, 64, 64, 16, *args_nan) == E.QLORA_ERR_INVALID_ARG
+    args_small_ws = [fake, C.byref(w), fake, fake, 1.0, fake, fake, fake, 16, None, None]
+    assert lib.qlora_linear_fwd(8, 64, 64, 16, *args_small_ws) == E.QLORA_ERR_INVALID_ARG
+    bargs = [fake, fake, fake, C.byref(w), fake, fake, 1.0, fake, fake, None, None, 0, None, None]
+    assert lib.qlora_linear_bwd(8, 64, 64, 16, *bargs) == E.QLORA_ERR_INVALID_ARG  # null dB
+    assert lib.qlora_status_sync(None, None, None) == E.QLORA_ERR_INVALID_ARG
+    assert lib.qlora_status_clear(None, None) == E.QLORA_ERR_INVALID_ARG
+
+
+def test_product_path_has_no_fallback():
+    """The binding loads the CUDA library or fails; it never imports the oracle."""
+    pkg = os.path.join(ROOT, "bit_nf4_quantized_pack_b200")
+    for f in os.listdir(pkg):
+        if f.endswith(".py"):
+            src = open(os.path.join(pkg, f), encoding="utf-8").read()
+            assert not re.search(r"^\s*(from|import)\s+oracle\b", src, flags=re.M), f
+            assert "import_module(\"oracle" not in src and "__import__(\"oracle" not in src, f

@@ -1,0 +1,139 @@
+"""GPU parity of qlora_linear_fwd / qlora_linear_bwd against the fp64 oracle.
+
+Bar: relative Frobenius error <= 5e-3 for Y, dX, dA, dB (each against the
+oracle's fp64 result on the oracle's own dequantized weight), with exact
+special cases where the arithmetic makes them exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+from bit_nf4_quantized_pack_b200 import synthetic as S
+from oracle.linear import lora_backward, lora_forward
+from tests._gpu_util import OracleWeight, rel_fro, to_dev, to_np
+
+pytestmark = pytest.mark.gpu
+TOL = 5e-3
+
+
+def _q():
+    import bit_nf4_quantized_pack_b200 as q
+    return q
+
+
+def run_case(lin, r, c, dq, *, backward=True, w_dtype=torch.bfloat16):
+    q = _q()
+    X, W, A, B = lin.X, lin.W, lin.A, lin.B
+    wq = q.quantize(to_dev(W, w_dtype), double_quant=dq)
+    Xt, At, Bt = to_dev(X), to_dev(A), to_dev(B)
+    Y, Zc = q.linear_forward(Xt, wq, At, Bt, c)
+    ow = OracleWeight(W, dq)
+    Yr, Zr = lora_forward(X, ow.w_hat, A, B, c)
+    out = {"Y": rel_fro(to_np(Y), Yr), "Zc": rel_fro(to_np(Zc), c * Zr)}
+    if backward:
+        G = lin.dY
+        dX, dA, dB = q.linear_backward(to_dev(G), Xt, Zc, wq, At, Bt, c)
+        dXr, dAr, dBr = lora_backward(G, X, ow.w_hat, A, B, c)
+        out.update(dX=rel_fro(to_np(dX), dXr), dA=rel_fro(to_np(dA), dAr),
+                   dB=rel_fro(to_np(dB), dBr))
+    return out
+
+
+CASES = [
+    # (M, K, N, r, dq)  — several tiles in every dimension plus ragged edges
+    (200, 320, 384, 16, True),
+    (129, 256, 512, 8, False),
+    (300, 512, 192, 64, True),
+    (257, 1024, 768, 32, True),
+    (17, 128, 256, 16, False),
+    (128, 64, 64, 8, True),
+]
+
+
+@pytest.mark.parametrize("M,K,N,r,dq", CASES)
+def test_fwd_bwd_parity(M, K, N, r, dq):
+    lin = S.random_case(M + K + N + r, M, K, N, r)
+    lin.dY = S.normal(7, M, 4, (M, N), 1.0)
+    errs = run_case(lin, r, 32.0 / r, dq)
+    for k, v in errs.items():
+        assert v <= TOL, (k, v, errs)
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 5, 8, 16])
+def test_gemv_parity(M):
+    lin = S.random_case(100 + M, M, 640, 576, 16)
+    errs = run_case(lin, 16, 2.0, True, backward=False)
+    for k, v in errs.items():
+        assert v <= TOL, (k, v, errs)
+
+
+def test_config1_tiny():
+    wl = S.config1()
+    lin = wl.linears[0]
+    errs = run_case(lin, wl.r, wl.c, wl.double_quant, w_dtype=torch.float32)
+    for k, v in errs.items():
+        assert v <= TOL, (k, v, errs)
+
+
+def test_special_cases():
+    q = _q()
+    M, K, N, r = 160, 256, 320, 16
+    lin = S.random_case(5, M, K, N, r)
+    X, W = lin.X, lin.W
+    Xt = to_dev(X)
+    wq = q.quantize(to_dev(W), double_quant=True)
+    ow = OracleWeight(W, True)
+    zA, zB = torch.zeros((K, r), dtype=torch.bfloat16, device="cuda"), \
+        torch.zeros((r, N), dtype=torch.bfloat16, device="cuda")
+    # A = B = 0: a plain product with the decoded weight
+    Y, Zc = q.linear_forward(Xt, wq, zA, zB, 2.0)
+    assert rel_fro(to_np(Y), X.astype(np.float64) @ ow.w_hat) <= TOL
+    assert torch.count_nonzero(Zc) == 0
+    # W = 0: only the LoRA branch remains (every code 7, every weight exactly 0)
+    w0 = q.quantize(torch.zeros((K, N), dtype=torch.bfloat16, device="cuda"), double_quant=True)
+    At, Bt = to_dev(lin.A), to_dev(lin.B)
+    Y, _ = q.linear_forward(Xt, w0, At, Bt, 2.0)
+    assert rel_fro(to_np(Y), 2.0 * (X.astype(np.float64) @ lin.A) @ lin.B) <= TOL
+    # B = 0: dA is exactly zero while dB is not
+    G = S.normal(9, 9, 9, (M, N), 1.0)
+    Y, Zc = q.linear_forward(Xt, wq, At, zB, 2.0)
+    dX, dA, dB = q.linear_backward(to_dev(G), Xt, Zc, wq, At, zB, 2.0)
+    assert torch.count_nonzero(dA) == 0 and torch.count_nonzero(dB) > 0
+
+
+def test_no_gradient_for_the_frozen_base():
+    """Backward leaves every buffer of the quantized state untouched."""
+    q = _q()
+    lin = S.random_case(11, 256, 256, 256, 16)
+    wq = q.quantize(to_dev(lin.W), double_quant=True)
+    before = [t.clone() for t in (wq.packed, wq.code8, wq.s2, wq.offset)]
+    Xt = to_dev(lin.X)
+    Y, Zc = q.linear_forward(Xt, wq, to_dev(lin.A), to_dev(lin.B), 2.0)
+    q.linear_backward(to_dev(lin.dY), Xt, Zc, wq, to_dev(lin.A), to_dev(lin.B), 2.0)
+    torch.cuda.synchronize()
+    for a, b in zip(before, (wq.packed, wq.code8, wq.s2, wq.offset)):
+        assert torch.equal(a, b)
+
+
+def test_full_size_projection_sampled_rows():
+    """4096 x 4096, M = 4096 (the benchmark shape): sampled rows of Y and dX,
+    full dA and dB."""
+    q = _q()
+    wl = S.config2()
+    lin = wl.linears[0]
+    X, W, A, B, G, c = lin.X, lin.W, lin.A, lin.B, lin.dY, wl.c
+    wq = q.quantize(to_dev(W), double_quant=True)
+    Xt = to_dev(X)
+    Y, Zc = q.linear_forward(Xt, wq, to_dev(A), to_dev(B), c)
+    dX, dA, dB = q.linear_backward(to_dev(G), Xt, Zc, wq, to_dev(A), to_dev(B), c)
+    ow = OracleWeight(W, True)
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([[0, 4095], rng.integers(0, 4096, 96)]))
+    Yr, _ = lora_forward(X[rows], ow.w_hat, A, B, c)
+    assert rel_fro(to_np(Y)[rows], Yr) <= TOL
+    dXr, _, _ = lora_backward(G[rows], X[rows], ow.w_hat, A, B, c)
+    assert rel_fro(to_np(dX)[rows], dXr) <= TOL
+    X64, G64 = X.astype(np.float64), G.astype(np.float64)
+    dZ = c * (G64 @ B.T)
+    assert rel_fro(to_np(dA), X64.T @ dZ) <= TOL
+    assert rel_fro(to_np(dB), c * ((X64 @ A).T @ G64)) <= TOL

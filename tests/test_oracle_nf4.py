@@ -238,3 +238,15 @@ def test_dequantize_worked_examples(golden):
     for got, r in zip(w, e["restored"]):
         lo, hi = sorted(_bf16_neighbours(abs(r))) if r else (0.0, 0.0)
         assert abs(got) in (lo, hi) and abs(abs(got) - abs(r)) <= abs(r) * 2 ** -8
+
+
+def test_block_scales_is_the_scale_step_of_quantize():
+    rng = np.random.default_rng(13)
+    for P in (1, 64, 65, 1000):
+        w = (rng.standard_normal(P) * 0.02).astype(np.float32)
+        if P > 64:
+            w[:64] = 0
+        _, s = nf4.quantize_nf4(w)
+        assert np.array_equal(nf4.block_scales(w), s)
+    with pytest.raises(nf4.NonFiniteError):
+        nf4.block_scales(np.array([1.0, np.nan], np.float32))
