@@ -196,7 +196,7 @@ __global__ void skinny_reduce_kernel(const float* __restrict__ partial, int spli
 // a multiple of 16 with zeros by TMA's out-of-bounds fill).
 // ===========================================================================
 constexpr int kFStages = 4;
-constexpr int kFPStages = 2;
+constexpr int kFPStages = 3;
 constexpr int kFA = 16384;           // 128 x 64 bf16
 constexpr int kFB = 32768;           // 256 x 64 bf16
 constexpr int kFP = 8192;            // packed tile
@@ -349,7 +349,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
       tma_prefetch_desc(&tmLB);
       uint32_t it = 0, pit = 0;
       uint32_t last_parity[kFStages] = {2, 2, 2, 2};
-      uint32_t last_pparity[kFPStages] = {2, 2};
+      uint32_t last_pparity[kFPStages] = {2, 2, 2};
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int m0 = (tile % args.m_tiles) * 128;
@@ -491,9 +491,6 @@ __global__ void __launch_bounds__(kFThreads, 1)
           }
           const uint4 p0 = *reinterpret_cast<const uint4*>(prow + c0 * 16);
           const uint4 p1 = *reinterpret_cast<const uint4*>(prow + c1 * 16);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&pempty[ps]);
-          ++pit;
           uint8_t* brow = sB + s * kFB + R * 128;
           const uint32_t sw = static_cast<uint32_t>(R & 7);
           if (valid) {
@@ -512,7 +509,15 @@ __global__ void __launch_bounds__(kFThreads, 1)
           }
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&full_b[s]);
+          // The packed stage is released only now, after every lane has used
+          // the bytes it loaded: a release right after issuing the shared
+          // loads let the next TMA overwrite the stage before slow warps'
+          // loads had returned.
+          if (lane == 0) {
+            mbar_arrive(&pempty[ps]);
+            mbar_arrive(&full_b[s]);
+          }
+          ++pit;
         } else {
           __syncwarp();
           if (lane == 0) mbar_arrive(&full_b[s]);
