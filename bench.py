@@ -296,6 +296,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip the GEMV and quantize sweeps")
+    ap.add_argument("--kernels-only", action="store_true",
+                    help="only the timed steps (no e2e, sweeps or CPU baseline): for profilers")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -389,7 +391,7 @@ def main():
 
     # ---------------- end to end through the public API with host buffers ----------------
     e2e = None
-    if rank == 0 or world > 1:
+    if not args.kernels_only:
         h = sets[0]["host"]
         pin = lambda a: torch.from_numpy(a.astype("float32")).to(torch.bfloat16).pin_memory()
         hW, hX, hG = pin(h.W), pin(h.X), pin(h.dY)
@@ -435,12 +437,12 @@ def main():
                "ms_per_step": ems, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     extras = {}
-    if rank == 0 and not args.no_extras:
+    if rank == 0 and not args.no_extras and not args.kernels_only:
         extras["gemv"] = gemv_sweep(torch, q, dev, peaks)
         extras["quantize"] = quantize_bench(torch, q, dev, peaks)
 
     cpu = None
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and not args.kernels_only:
         inputs = oracle_sample_inputs()
         t0 = time.perf_counter()
         oracle_step(inputs)

@@ -181,29 +181,34 @@ __global__ void skinny_reduce_kernel(const float* __restrict__ partial, int spli
 // ===========================================================================
 // Fused NF4-decode GEMM (forward: kBwd = false, input gradient: kBwd = true)
 //
-// Output tile 128 (rows of X or G) x 256, K-step 64.  Per stage the shared
-// memory holds the activation tile (128 x 64 bf16, K-major, TMA) and the
-// decoded weight tile (256 x 64 bf16).  The weight tile is written by the
-// decoder warps as 256 rows of 128 bytes, each row one NF4 block of 64
-// consecutive weights (row R at R*128, 16-byte chunk c at (c ^ (R & 7))*16,
-// the 128-byte swizzle pattern):
+// Output tile 256 (rows of X or G) x 128, K-step 64.  One decoded weight tile
+// (128 x 64 bf16) feeds two tcgen05.mma of M = 128 (rows m0..m0+127 and
+// m0+128..m0+255), so each decoded weight is used by 256 rows.  Per stage the
+// shared memory holds the activation tile (256 x 64 bf16, K-major, two TMA
+// boxes) and the decoded weight tile, written by the decoder warps as 128 rows
+// of 128 bytes, each row one NF4 block of 64 consecutive weights (row R at
+// R*128, 16-byte chunk c at (c ^ (R & 7))*16, the 128-byte swizzle pattern):
 //   forward   row R = 64*nb + k: weights (k0+k, n0+64nb .. +63) — an MN-major
 //             operand (atoms of 8 k-rows x 64 n; 8 KB between n-atoms);
 //   backward  row R: weights (n0+R, k0 .. k0+63) of W, i.e. row R of Ŵᵀ's
 //             K-major operand.
-// After the last K-step, one more step accumulates the LoRA term: Zc (or dZ)
-// as the A tile and B (or A) as the weight tile, both by TMA (rank padded to
-// a multiple of 16 with zeros by TMA's out-of-bounds fill).
+// Decoder warps form two groups that take alternate K-steps; each thread owns
+// one row, and loads its 32 packed bytes and its block scale straight from
+// global memory two of its K-steps ahead.  After the last K-step, one more
+// step accumulates the LoRA term: Zc (or dZ) as the activation tile and B (or
+// A) as the weight tile, both by TMA (rank padded to a multiple of 16 with
+// zeros by TMA's out-of-bounds fill).  TMEM holds two tile buffers of two
+// 128 x 128 fp32 accumulators (512 columns), so the epilogue of one tile
+// overlaps the main loop of the next.
 // ===========================================================================
 constexpr int kFStages = 4;
-constexpr int kFPStages = 3;
-constexpr int kFA = 16384;           // 128 x 64 bf16
-constexpr int kFB = 32768;           // 256 x 64 bf16
-constexpr int kFP = 8192;            // packed tile
+constexpr int kFBM = 256, kFBN = 128;
+constexpr int kFA = 32768;           // 256 x 64 bf16
+constexpr int kFB = 16384;           // 128 x 64 bf16
 constexpr int kFThreads = 448;       // warp 0 TMA, 1 MMA, 2..9 decode, 10..13 epilogue
-constexpr int kFDecWarps = 8;
+constexpr int kFGroupWarps = 4;      // decoder warps per group (two groups)
 constexpr int kFEpiWarps = 4;
-constexpr size_t kFSmem = 1024 + kFStages * (kFA + kFB) + kFPStages * kFP + 1024 + 512;
+constexpr size_t kFSmem = 1024 + kFStages * (kFA + kFB) + 1024 + 512;
 
 struct FusedArgs {
   int M;          // rows of the activation / output
@@ -213,6 +218,7 @@ struct FusedArgs {
   int rsteps;     // MMAs of K=16 in the LoRA step (ceil(r/16))
   int m_tiles, n_tiles;
   ScaleView sv;
+  const uint8_t* packed;
   uint16_t* out;  // bf16 [M][Nout]
   int32_t* d_status;
 };
@@ -261,34 +267,67 @@ __device__ __forceinline__ void build_lut(float a, uint32_t (&H)[4], uint32_t (&
   }
 }
 
-struct ScaleFetch {
-  float absv;    // absmax (no double quant)
-  uint32_t q;    // code8
-  float s2v;
+// What one decoder thread needs for one K-step, loaded ahead of use.
+struct RowFetch {
+  uint4 p0, p1;   // 32 packed bytes of the row's NF4 block
+  float absv;     // absmax (no double quant)
+  uint32_t q;     // scale code (double quant)
+  float s2v;      // second-level scale (double quant)
+  bool valid;     // row inside the weight; false also for LoRA steps
 };
 
-__device__ __forceinline__ ScaleFetch fetch_scale(const ScaleView& sv, int64_t blk, bool valid) {
-  ScaleFetch f{1.0f, 0u, 1.0f};
-  if (!valid) return f;
-  if (sv.code8 == nullptr) {
-    f.absv = __ldg(sv.absmax + blk);
+template <bool kBwd>
+__device__ __forceinline__ RowFetch fetch_row(const FusedArgs& a, int tile, int kk, int R,
+                                              int num_tiles) {
+  RowFetch f;
+  f.p0 = make_uint4(0, 0, 0, 0);
+  f.p1 = f.p0;
+  f.absv = 1.0f;
+  f.q = 0;
+  f.s2v = 1.0f;
+  f.valid = false;
+  if (tile >= num_tiles || kk >= a.nk) return f;
+  const int n0 = (tile / a.m_tiles) * kFBN;
+  const int64_t rowbytes = a.Nw / 2;
+  const int64_t bpr = a.Nw / 64;
+  int64_t blk;
+  const uint8_t* src;
+  if (!kBwd) {
+    const int nb = R >> 6, kr = R & 63;
+    if (n0 + nb * 64 >= a.Nout) return f;
+    const int64_t k = static_cast<int64_t>(kk) * 64 + kr;
+    src = a.packed + k * rowbytes + n0 / 2 + nb * 32;
+    blk = k * bpr + n0 / 64 + nb;
   } else {
-    f.q = __ldg(sv.code8 + blk);
-    f.s2v = __ldg(sv.s2 + (blk >> 8));
+    if (n0 + R >= a.Nout) return f;
+    const int64_t kw = n0 + R;
+    src = a.packed + kw * rowbytes + kk * 32;
+    blk = kw * bpr + kk;
+  }
+  f.valid = true;
+  f.p0 = __ldg(reinterpret_cast<const uint4*>(src));
+  f.p1 = __ldg(reinterpret_cast<const uint4*>(src + 16));
+  if (a.sv.code8 == nullptr) {
+    f.absv = __ldg(a.sv.absmax + blk);
+  } else {
+    f.q = __ldg(a.sv.code8 + blk);
+    f.s2v = __ldg(a.sv.s2 + (blk >> 8));
   }
   return f;
 }
 
-__device__ __forceinline__ float finish_scale(const ScaleView& sv, const ScaleFetch& f, float off,
-                                              const float* t8) {
-  if (sv.code8 == nullptr) return f.absv;
-  return __fadd_rn(__fmul_rn(t8[f.q], f.s2v), off);
+// Advance an iteration cursor (tile, kk) by `n` steps of nsteps per tile.
+__device__ __forceinline__ void advance(int& tile, int& kk, int n, int nsteps) {
+  kk += n;
+  while (kk >= nsteps) {
+    kk -= nsteps;
+    tile += gridDim.x;
+  }
 }
 
 template <bool kBwd>
 __global__ void __launch_bounds__(kFThreads, 1)
     fused_nf4_gemm_kernel(const __grid_constant__ CUtensorMap tmAct,
-                          const __grid_constant__ CUtensorMap tmPk,
                           const __grid_constant__ CUtensorMap tmLA,
                           const __grid_constant__ CUtensorMap tmLB, FusedArgs args) {
   extern __shared__ uint8_t smem_raw[];
@@ -296,14 +335,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + kFStages * kFA;
-  uint8_t* sP = sB + kFStages * kFB;
-  float* t8 = reinterpret_cast<float*>(sP + kFPStages * kFP);
+  float* t8 = reinterpret_cast<float*>(sB + kFStages * kFB);
   uint64_t* full_a = reinterpret_cast<uint64_t*>(t8 + 256);
   uint64_t* full_b = full_a + kFStages;
   uint64_t* empty = full_b + kFStages;
-  uint64_t* pfull = empty + kFStages;
-  uint64_t* pempty = pfull + kFPStages;
-  uint64_t* tfull = pempty + kFPStages;
+  uint64_t* tfull = empty + kFStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
@@ -314,12 +350,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kFStages; ++s) {
       mbar_init(&full_a[s], 1);
-      mbar_init(&full_b[s], kFDecWarps);
+      mbar_init(&full_b[s], kFGroupWarps);
       mbar_init(&empty[s], 1);
-    }
-    for (int s = 0; s < kFPStages; ++s) {
-      mbar_init(&pfull[s], 1);
-      mbar_init(&pempty[s], kFDecWarps);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
@@ -344,42 +376,33 @@ __global__ void __launch_bounds__(kFThreads, 1)
     // ------------------------------ TMA producer ---------------------------
     if (lane == 0) {
       tma_prefetch_desc(&tmAct);
-      tma_prefetch_desc(&tmPk);
       tma_prefetch_desc(&tmLA);
       tma_prefetch_desc(&tmLB);
-      uint32_t it = 0, pit = 0;
+      uint32_t it = 0;
       uint32_t last_parity[kFStages] = {2, 2, 2, 2};
-      uint32_t last_pparity[kFPStages] = {2, 2, 2};
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m0 = (tile % args.m_tiles) * 128;
-        const int n0 = (tile / args.m_tiles) * 256;
+        const int m0 = (tile % args.m_tiles) * kFBM;
+        const int n0 = (tile / args.m_tiles) * kFBN;
         for (int kk = 0; kk < nsteps; ++kk, ++it) {
           const int s = it % kFStages;
           const uint32_t ph = (it / kFStages) & 1;
           if (*abort_flag || !mbar_wait(&empty[s], ph ^ 1)) { ok = false; break; }
+          uint8_t* a = sA + s * kFA;
           if (kk < args.nk) {
             mbar_arrive_expect_tx(&full_a[s], kFA);
-            tma_load_2d(sA + s * kFA, &tmAct, &full_a[s], kk * 64, m0);
-            const int ps = pit % kFPStages;
-            const uint32_t pph = (pit / kFPStages) & 1;
-            if (!mbar_wait(&pempty[ps], pph ^ 1)) { last_parity[s] = ph; ok = false; break; }
-            mbar_arrive_expect_tx(&pfull[ps], kFP);
-            if (!kBwd)
-              tma_load_2d(sP + ps * kFP, &tmPk, &pfull[ps], n0 / 2, kk * 64);
-            else
-              tma_load_2d(sP + ps * kFP, &tmPk, &pfull[ps], kk * 32, n0);
-            last_pparity[ps] = pph;
-            ++pit;
+            tma_load_2d(a, &tmAct, &full_a[s], kk * 64, m0);
+            tma_load_2d(a + 16384, &tmAct, &full_a[s], kk * 64, m0 + 128);
           } else {
             mbar_arrive_expect_tx(&full_a[s], kFA + kFB);
-            tma_load_2d(sA + s * kFA, &tmLA, &full_a[s], 0, m0);
+            tma_load_2d(a, &tmLA, &full_a[s], 0, m0);
+            tma_load_2d(a + 16384, &tmLA, &full_a[s], 0, m0 + 128);
+            uint8_t* b = sB + s * kFB;
             if (!kBwd) {
-#pragma unroll
-              for (int nb = 0; nb < 4; ++nb)
-                tma_load_2d(sB + s * kFB + nb * 8192, &tmLB, &full_a[s], n0 + nb * 64, 0);
+              tma_load_2d(b, &tmLB, &full_a[s], n0, 0);
+              tma_load_2d(b + 8192, &tmLB, &full_a[s], n0 + 64, 0);
             } else {
-              tma_load_2d(sB + s * kFB, &tmLB, &full_a[s], 0, n0);
+              tma_load_2d(b, &tmLB, &full_a[s], 0, n0);
             }
           }
           last_parity[s] = ph;
@@ -390,21 +413,19 @@ __global__ void __launch_bounds__(kFThreads, 1)
         // let copies already in flight land before the CTA can exit
         for (int s = 0; s < kFStages; ++s)
           if (last_parity[s] < 2) (void)mbar_wait(&full_a[s], last_parity[s]);
-        for (int s = 0; s < kFPStages; ++s)
-          if (last_pparity[s] < 2) (void)mbar_wait(&pfull[s], last_pparity[s]);
       }
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer -----------------------------
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, 256, 0, kBwd ? 0 : 1);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, kFBN, 0, kBwd ? 0 : 1);
       uint32_t it = 0, tc = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tc) {
         const uint32_t ab = tc & 1, aph = (tc >> 1) & 1;
         if (*abort_flag || !mbar_wait(&tempty[ab], aph ^ 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t dt = tmem + ab * 256;
+        const uint32_t d0 = tmem + ab * 256, d1 = d0 + 128;
         for (int kk = 0; kk < nsteps; ++kk, ++it) {
           const int s = it % kFStages;
           const uint32_t ph = (it / kFStages) & 1;
@@ -416,10 +437,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
           const uint32_t a0 = smem_u32(sA + s * kFA), b0 = smem_u32(sB + s * kFB);
           const int nm = (kk < args.nk) ? 4 : args.rsteps;
           for (int j = 0; j < nm; ++j) {
-            const uint64_t ad = smem_desc(a0 + j * 32, 16, 1024);
             const uint64_t bd = kBwd ? smem_desc(b0 + j * 32, 16, 1024)
                                      : smem_desc(b0 + j * 2048, 8192, 1024);
-            umma_bf16(dt, ad, bd, idesc, (kk > 0 || j > 0) ? 1u : 0u);
+            const uint32_t acc = (kk > 0 || j > 0) ? 1u : 0u;
+            umma_bf16(d0, smem_desc(a0 + j * 32, 16, 1024), bd, idesc, acc);
+            umma_bf16(d1, smem_desc(a0 + 16384 + j * 32, 16, 1024), bd, idesc, acc);
           }
           umma_commit(&empty[s]);
         }
@@ -430,99 +452,54 @@ __global__ void __launch_bounds__(kFThreads, 1)
       umma_commit(drain);
       (void)mbar_wait(drain, 0);
     }
-  } else if (warp < 2 + kFDecWarps) {
+  } else if (warp < 2 + 2 * kFGroupWarps) {
     // ------------------------------ decoders -------------------------------
-    const int R = threadIdx.x - 64;  // weight-tile row 0..255
+    const int d = threadIdx.x - 64;
+    const int grp = d / (kFGroupWarps * 32);   // group 0 takes even steps, 1 odd
+    const int R = d % (kFGroupWarps * 32);     // weight-tile row 0..127
     const float off = args.sv.code8 != nullptr ? __ldg(args.sv.offset) : 0.0f;
-    const int bpr = args.Nw / 64;    // NF4 blocks per weight row
-    uint32_t it = 0, pit = 0;
     bool ok = true;
-    // coordinates of this thread's row for (tile, kk)
-    auto row_block = [&](int tile, int kk, bool& valid) -> int64_t {
-      const int n0 = (tile / args.m_tiles) * 256;
-      if (!kBwd) {
-        const int nb = R >> 6, kr = R & 63;
-        valid = n0 + nb * 64 < args.Nout;
-        return static_cast<int64_t>(kk * 64 + kr) * bpr + (n0 / 64 + nb);
-      } else {
-        valid = n0 + R < args.Nout;
-        return static_cast<int64_t>(n0 + R) * bpr + kk;
-      }
-    };
-    // prefetch the scale of the first decoded step
-    int tile = blockIdx.x;
-    bool v0 = false;
-    ScaleFetch nextf{};
-    if (tile < num_tiles) nextf = fetch_scale(args.sv, row_block(tile, 0, v0), v0);
-    bool nextv = v0;
-    for (; tile < num_tiles && ok; tile += gridDim.x) {
-      for (int kk = 0; kk < nsteps; ++kk, ++it) {
-        const int s = it % kFStages;
-        const uint32_t ph = (it / kFStages) & 1;
-        if (*abort_flag || !mbar_wait(&empty[s], ph ^ 1)) { ok = false; break; }
-        if (kk < args.nk) {
-          const ScaleFetch f = nextf;
-          const bool valid = nextv;
-          // prefetch the next decoded step's scale
-          {
-            int ntile = tile, nkk = kk + 1;
-            if (nkk >= args.nk) { ntile = tile + gridDim.x; nkk = 0; }
-            if (ntile < num_tiles) {
-              bool vv = false;
-              const int64_t nb = row_block(ntile, nkk, vv);
-              nextf = fetch_scale(args.sv, nb, vv);
-              nextv = vv;
-            }
-          }
-          const int ps = pit % kFPStages;
-          const uint32_t pph = (pit / kFPStages) & 1;
-          if (!mbar_wait(&pfull[ps], pph)) { ok = false; break; }
-          const uint8_t* prow;
-          uint32_t c0, c1;
-          if (!kBwd) {
-            const int nb = R >> 6, kr = R & 63;
-            prow = sP + ps * kFP + kr * 128;
-            c0 = static_cast<uint32_t>((2 * nb) ^ (kr & 7));
-            c1 = static_cast<uint32_t>((2 * nb + 1) ^ (kr & 7));
-          } else {
-            prow = sP + ps * kFP + R * 32;
-            c0 = static_cast<uint32_t>((R >> 2) & 1);
-            c1 = c0 ^ 1u;
-          }
-          const uint4 p0 = *reinterpret_cast<const uint4*>(prow + c0 * 16);
-          const uint4 p1 = *reinterpret_cast<const uint4*>(prow + c1 * 16);
-          uint8_t* brow = sB + s * kFB + R * 128;
-          const uint32_t sw = static_cast<uint32_t>(R & 7);
-          if (valid) {
-            const float a = finish_scale(args.sv, f, off, t8);
-            uint32_t H[4], L[4];
-            build_lut(a, H, L);
-            const uint32_t pw[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    // cursors: the step being decoded, and the one being prefetched (2 ahead)
+    int tile = blockIdx.x, kk = 0;
+    advance(tile, kk, grp, nsteps);
+    int ptile = tile, pkk = kk;
+    RowFetch q0 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
+    advance(ptile, pkk, 2, nsteps);
+    RowFetch q1 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
+    advance(ptile, pkk, 2, nsteps);
+    for (uint32_t it = grp; tile < num_tiles && ok; it += 2) {
+      const int s = it % kFStages;
+      const uint32_t ph = (it / kFStages) & 1;
+      const RowFetch f = q0;
+      q0 = q1;
+      q1 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
+      advance(ptile, pkk, 2, nsteps);
+      if (*abort_flag || !mbar_wait(&empty[s], ph ^ 1)) { ok = false; break; }
+      if (kk < args.nk) {
+        uint8_t* brow = sB + s * kFB + R * 128;
+        const uint32_t sw = static_cast<uint32_t>(R & 7);
+        if (f.valid) {
+          const float a = args.sv.code8 == nullptr
+                              ? f.absv
+                              : __fadd_rn(__fmul_rn(t8[f.q], f.s2v), off);
+          uint32_t H[4], L[4];
+          build_lut(a, H, L);
+          const uint32_t pw[8] = {f.p0.x, f.p0.y, f.p0.z, f.p0.w,
+                                  f.p1.x, f.p1.y, f.p1.z, f.p1.w};
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              *reinterpret_cast<uint4*>(brow + ((static_cast<uint32_t>(c) ^ sw) << 4)) =
-                  decode8(pw[c], H, L);
-          } else {
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-              *reinterpret_cast<uint4*>(brow + (c << 4)) = make_uint4(0, 0, 0, 0);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          // The packed stage is released only now, after every lane has used
-          // the bytes it loaded: a release right after issuing the shared
-          // loads let the next TMA overwrite the stage before slow warps'
-          // loads had returned.
-          if (lane == 0) {
-            mbar_arrive(&pempty[ps]);
-            mbar_arrive(&full_b[s]);
-          }
-          ++pit;
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(brow + ((static_cast<uint32_t>(c) ^ sw) << 4)) =
+                decode8(pw[c], H, L);
         } else {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&full_b[s]);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(brow + (c << 4)) = make_uint4(0, 0, 0, 0);
         }
+        fence_proxy_async_smem();
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full_b[s]);
+      advance(tile, kk, 2, nsteps);
     }
     if (!ok) *abort_flag = 1;
   } else {
@@ -531,26 +508,32 @@ __global__ void __launch_bounds__(kFThreads, 1)
     uint32_t tc = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tc) {
-      const int m0 = (tile % args.m_tiles) * 128;
-      const int n0 = (tile / args.m_tiles) * 256;
+      const int m0 = (tile % args.m_tiles) * kFBM;
+      const int n0 = (tile / args.m_tiles) * kFBN;
       const uint32_t ab = tc & 1, aph = (tc >> 1) & 1;
       if (*abort_flag || !mbar_wait(&tfull[ab], aph)) { ok = false; break; }
       tc_fence_after();
-      const int row = m0 + q * 32 + lane;
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * 256 + c * 32, v);
-        tmem_ld_wait();
-        const int col = n0 + c * 32;
-        if (row < args.M && col < args.Nout) {
-          uint4* dst = reinterpret_cast<uint4*>(args.out + static_cast<int64_t>(row) * args.Nout + col);
+      for (int h = 0; h < 2; ++h) {
+        const int row = m0 + h * 128 + q * 32 + lane;
+#pragma unroll 1
+        for (int c = 0; c < kFBN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(
+              tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * 256 + h * 128 + c * 32, v);
+          tmem_ld_wait();
+          const int col = n0 + c * 32;
+          if (row < args.M && col < args.Nout) {
+            uint4* dst =
+                reinterpret_cast<uint4*>(args.out + static_cast<int64_t>(row) * args.Nout + col);
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1])),
-                                pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
-                                pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
-                                pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(
+                  pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1])),
+                  pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
+                  pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
+                  pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
+          }
         }
       }
       tc_fence_before();
@@ -748,9 +731,7 @@ cudaError_t set_fused_attr() {
 }
 
 constexpr CUtensorMapDataType kBF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-constexpr CUtensorMapDataType kU8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
 constexpr CUtensorMapSwizzle kSW128 = CU_TENSOR_MAP_SWIZZLE_128B;
-constexpr CUtensorMapSwizzle kSW32 = CU_TENSOR_MAP_SWIZZLE_32B;
 
 int rsteps_of(int r) { return (r + 15) / 16; }
 
@@ -796,7 +777,7 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
   (void)num_sms;
   WsCursor cur{static_cast<char*>(ws), ws_bytes};
   // Zc = bf16(c * X A): A operand X (K-major), B operand A (MN-major over r)
-  CUtensorMap tX, tAl, tZc, tBl, tPk;
+  CUtensorMap tX, tAl, tZc, tBl;
   if (!make_tmap_2d(&tX, X, kBF16, 2, M, K, K, 64, 128, kSW128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tAl, A, kBF16, 2, K, r, r, 64, 64, kSW128)) return cudaErrorInvalidValue;
   const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
@@ -839,7 +820,6 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
 
   e = set_fused_attr<false>();
   if (e != cudaSuccess) return e;
-  if (!make_tmap_2d(&tPk, packed, kU8, 1, K, N / 2, N / 2, 128, 64, kSW128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tZc, Zc, kBF16, 2, M, r, r, 64, 128, kSW128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tBl, B, kBF16, 2, r, N, N, 64, 64, kSW128)) return cudaErrorInvalidValue;
   FusedArgs fa;
@@ -848,9 +828,10 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
   fa.Nw = static_cast<int>(N);
   fa.nk = static_cast<int>(K / 64);
   fa.rsteps = rsteps_of(r);
-  fa.m_tiles = static_cast<int>((M + 127) / 128);
-  fa.n_tiles = static_cast<int>((N + 255) / 256);
+  fa.m_tiles = static_cast<int>((M + kFBM - 1) / kFBM);
+  fa.n_tiles = static_cast<int>((N + kFBN - 1) / kFBN);
   fa.sv = sv;
+  fa.packed = packed;
   fa.out = Y;
   fa.d_status = d_status;
   int dev = 0, sms = 148;
@@ -860,7 +841,7 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
   const int grid = tiles < sms ? tiles : sms;
   {
     ProfScope prof(kProfFusedFwd, st);
-    fused_nf4_gemm_kernel<false><<<grid, kFThreads, kFSmem, st>>>(tX, tPk, tZc, tBl, fa);
+    fused_nf4_gemm_kernel<false><<<grid, kFThreads, kFSmem, st>>>(tX, tZc, tBl, fa);
   }
   return cudaGetLastError();
 }
@@ -884,7 +865,7 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   cudaError_t e = cudaMemsetAsync(dZ, 0, static_cast<size_t>(M) * 64 * 2, st);
   if (e != cudaSuccess) return e;
 
-  CUtensorMap tG, tBk, tXmn, tdZ, tGmn, tZcmn, tPk, tAl;
+  CUtensorMap tG, tBk, tXmn, tdZ, tGmn, tZcmn, tAl;
   // dZ = c * G B^T : A operand G (K-major over N), B operand B (K-major: rows r, cols N)
   if (!make_tmap_2d(&tG, dY, kBF16, 2, M, N, N, 64, 128, kSW128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tBk, B, kBF16, 2, r, N, N, 64, 64, kSW128)) return cudaErrorInvalidValue;
@@ -906,8 +887,7 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   // dX = G W^T + dZ A^T
   e = set_fused_attr<true>();
   if (e != cudaSuccess) return e;
-  if (!make_tmap_2d(&tPk, packed, kU8, 1, K, N / 2, N / 2, 32, 256, kSW32)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&tAl, A, kBF16, 2, K, r, r, 64, 256, kSW128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tAl, A, kBF16, 2, K, r, r, 64, 128, kSW128)) return cudaErrorInvalidValue;
   CUtensorMap tdZa;
   if (!make_tmap_2d(&tdZa, dZ, kBF16, 2, M, 64, 64, 64, 128, kSW128)) return cudaErrorInvalidValue;
   FusedArgs fa;
@@ -916,9 +896,10 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   fa.Nw = static_cast<int>(N);
   fa.nk = static_cast<int>(N / 64);
   fa.rsteps = rsteps_of(r);
-  fa.m_tiles = static_cast<int>((M + 127) / 128);
-  fa.n_tiles = static_cast<int>((K + 255) / 256);
+  fa.m_tiles = static_cast<int>((M + kFBM - 1) / kFBM);
+  fa.n_tiles = static_cast<int>((K + kFBN - 1) / kFBN);
   fa.sv = sv;
+  fa.packed = packed;
   fa.out = dX;
   fa.d_status = d_status;
   int dev = 0, sms = 148;
@@ -928,7 +909,7 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   const int grid = tiles < sms ? tiles : sms;
   {
     ProfScope prof(kProfFusedBwd, st);
-    fused_nf4_gemm_kernel<true><<<grid, kFThreads, kFSmem, st>>>(tG, tPk, tdZa, tAl, fa);
+    fused_nf4_gemm_kernel<true><<<grid, kFThreads, kFSmem, st>>>(tG, tdZa, tAl, fa);
   }
   return cudaGetLastError();
 }
