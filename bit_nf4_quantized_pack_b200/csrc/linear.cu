@@ -181,32 +181,32 @@ __global__ void skinny_reduce_kernel(const float* __restrict__ partial, int spli
 // ===========================================================================
 // Fused NF4-decode GEMM (forward: kBwd = false, input gradient: kBwd = true)
 //
-// Output tile 256 (rows of X or G) x 128, K-step 64.  One decoded weight tile
-// (128 x 64 bf16) feeds two tcgen05.mma of M = 128 (rows m0..m0+127 and
-// m0+128..m0+255), so each decoded weight is used by 256 rows.  Per stage the
-// shared memory holds the activation tile (256 x 64 bf16, K-major, two TMA
-// boxes) and the decoded weight tile, written by the decoder warps as 128 rows
-// of 128 bytes, each row one NF4 block of 64 consecutive weights (row R at
+// Output tile 256 (rows of X or G) x 256, K-step 64.  One decoded weight tile
+// (256 x 64 bf16) feeds two tcgen05.mma of M = 128, N = 256 (rows m0..m0+127
+// and m0+128..m0+255), so each decoded weight is used by 256 rows.  Per stage
+// the shared memory holds the activation tile (256 x 64 bf16, K-major, two
+// TMA boxes) and the decoded weight tile, written by the decoder warps as 256
+// rows of 128 bytes, each row one NF4 block of 64 consecutive weights (row R at
 // R*128, 16-byte chunk c at (c ^ (R & 7))*16, the 128-byte swizzle pattern):
 //   forward   row R = 64*nb + k: weights (k0+k, n0+64nb .. +63) — an MN-major
 //             operand (atoms of 8 k-rows x 64 n; 8 KB between n-atoms);
 //   backward  row R: weights (n0+R, k0 .. k0+63) of W, i.e. row R of Ŵᵀ's
 //             K-major operand.
-// Decoder warps form two groups that take alternate K-steps; each thread owns
-// one row, and loads its 32 packed bytes and its block scale straight from
-// global memory two of its K-steps ahead.  After the last K-step, one more
+// Each decoder thread owns one row and loads its 32 packed bytes and its
+// block scale straight from global memory three K-steps ahead.  After the last K-step, one more
 // step accumulates the LoRA term: Zc (or dZ) as the activation tile and B (or
 // A) as the weight tile, both by TMA (rank padded to a multiple of 16 with
-// zeros by TMA's out-of-bounds fill).  TMEM holds two tile buffers of two
-// 128 x 128 fp32 accumulators (512 columns), so the epilogue of one tile
-// overlaps the main loop of the next.
+// zeros by TMA's out-of-bounds fill).  TMEM holds the two 128 x 256 fp32
+// accumulators (all 512 columns); the epilogue drains them before the next
+// tile's first MMA.
 // ===========================================================================
-constexpr int kFStages = 4;
-constexpr int kFBM = 256, kFBN = 128;
+constexpr int kFStages = 3;
+constexpr int kFBM = 256, kFBN = 256;
 constexpr int kFA = 32768;           // 256 x 64 bf16
-constexpr int kFB = 16384;           // 128 x 64 bf16
+constexpr int kFB = 32768;           // 256 x 64 bf16
 constexpr int kFThreads = 448;       // warp 0 TMA, 1 MMA, 2..9 decode, 10..13 epilogue
-constexpr int kFGroupWarps = 4;      // decoder warps per group (two groups)
+constexpr int kFDecWarps = 8;
+constexpr int kFPrefetch = 3;        // K-steps of packed bytes and scales in flight per thread
 constexpr int kFEpiWarps = 4;
 constexpr size_t kFSmem = 1024 + kFStages * (kFA + kFB) + 1024 + 512;
 
@@ -234,21 +234,21 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 // H[0..3] and L[0..3] (entry j's byte in byte j%4 of H[j/4] / L[j/4]).
 __device__ __forceinline__ uint4 decode8(uint32_t p, const uint32_t (&H)[4],
                                          const uint32_t (&L)[4]) {
+  // selector nibbles: low 3 bits pick a byte within a plane pair, bit 3
+  // (moved to the "+4" position) picks the pair
+  const uint32_t s = p & 0x77777777u;
+  const uint32_t b = ((p >> 1) & 0x44444444u) | 0x32103210u;
   uint4 o;
   {
-    const uint32_t s = p & 0x7777u;
-    const uint32_t b = ((p >> 1) & 0x4444u) | 0x3210u;
     const uint32_t hF = prmt(prmt(H[0], H[1], s), prmt(H[2], H[3], s), b);
     const uint32_t lF = prmt(prmt(L[0], L[1], s), prmt(L[2], L[3], s), b);
     o.x = prmt(lF, hF, 0x4051u);
     o.y = prmt(lF, hF, 0x6273u);
   }
   {
-    const uint32_t q = p >> 16;
-    const uint32_t s = q & 0x7777u;
-    const uint32_t b = ((q >> 1) & 0x4444u) | 0x3210u;
-    const uint32_t hF = prmt(prmt(H[0], H[1], s), prmt(H[2], H[3], s), b);
-    const uint32_t lF = prmt(prmt(L[0], L[1], s), prmt(L[2], L[3], s), b);
+    const uint32_t s2 = s >> 16, b2 = b >> 16;
+    const uint32_t hF = prmt(prmt(H[0], H[1], s2), prmt(H[2], H[3], s2), b2);
+    const uint32_t lF = prmt(prmt(L[0], L[1], s2), prmt(L[2], L[3], s2), b2);
     o.z = prmt(lF, hF, 0x4051u);
     o.w = prmt(lF, hF, 0x6273u);
   }
@@ -305,13 +305,19 @@ __device__ __forceinline__ RowFetch fetch_row(const FusedArgs& a, int tile, int 
     blk = kw * bpr + kk;
   }
   f.valid = true;
-  f.p0 = __ldg(reinterpret_cast<const uint4*>(src));
-  f.p1 = __ldg(reinterpret_cast<const uint4*>(src + 16));
+  // volatile asm: the loads issue here, K-steps before their use, instead of
+  // being moved down to it
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(f.p0.x), "=r"(f.p0.y), "=r"(f.p0.z), "=r"(f.p0.w) : "l"(src));
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(f.p1.x), "=r"(f.p1.y), "=r"(f.p1.z), "=r"(f.p1.w) : "l"(src + 16));
   if (a.sv.code8 == nullptr) {
-    f.absv = __ldg(a.sv.absmax + blk);
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(f.absv) : "l"(a.sv.absmax + blk));
   } else {
-    f.q = __ldg(a.sv.code8 + blk);
-    f.s2v = __ldg(a.sv.s2 + (blk >> 8));
+    uint16_t qv;
+    asm volatile("ld.global.nc.u8 %0, [%1];" : "=h"(qv) : "l"(a.sv.code8 + blk));
+    f.q = qv;
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(f.s2v) : "l"(a.sv.s2 + (blk >> 8)));
   }
   return f;
 }
@@ -340,8 +346,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
   uint64_t* full_b = full_a + kFStages;
   uint64_t* empty = full_b + kFStages;
   uint64_t* tfull = empty + kFStages;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
+  uint64_t* tempty = tfull + 1;
+  uint64_t* drain = tempty + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -350,13 +356,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kFStages; ++s) {
       mbar_init(&full_a[s], 1);
-      mbar_init(&full_b[s], kFGroupWarps);
+      mbar_init(&full_b[s], kFDecWarps);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], kFEpiWarps);
-    }
+    mbar_init(tfull, 1);
+    mbar_init(tempty, kFEpiWarps);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -379,7 +383,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
       tma_prefetch_desc(&tmLA);
       tma_prefetch_desc(&tmLB);
       uint32_t it = 0;
-      uint32_t last_parity[kFStages] = {2, 2, 2, 2};
+      uint32_t last_parity[kFStages] = {2, 2, 2};
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int m0 = (tile % args.m_tiles) * kFBM;
@@ -399,8 +403,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
             tma_load_2d(a + 16384, &tmLA, &full_a[s], 0, m0 + 128);
             uint8_t* b = sB + s * kFB;
             if (!kBwd) {
-              tma_load_2d(b, &tmLB, &full_a[s], n0, 0);
-              tma_load_2d(b + 8192, &tmLB, &full_a[s], n0 + 64, 0);
+#pragma unroll
+              for (int nb = 0; nb < 4; ++nb)
+                tma_load_2d(b + nb * 8192, &tmLB, &full_a[s], n0 + nb * 64, 0);
             } else {
               tma_load_2d(b, &tmLB, &full_a[s], 0, n0);
             }
@@ -422,10 +427,10 @@ __global__ void __launch_bounds__(kFThreads, 1)
       uint32_t it = 0, tc = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tc) {
-        const uint32_t ab = tc & 1, aph = (tc >> 1) & 1;
-        if (*abort_flag || !mbar_wait(&tempty[ab], aph ^ 1)) { ok = false; break; }
+        // the epilogue of the previous tile has drained both accumulators
+        if (*abort_flag || !mbar_wait(tempty, (tc & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d0 = tmem + ab * 256, d1 = d0 + 128;
+        const uint32_t d0 = tmem, d1 = tmem + 256;
         for (int kk = 0; kk < nsteps; ++kk, ++it) {
           const int s = it % kFStages;
           const uint32_t ph = (it / kFStages) & 1;
@@ -446,34 +451,33 @@ __global__ void __launch_bounds__(kFThreads, 1)
           umma_commit(&empty[s]);
         }
         if (!ok) break;
-        umma_commit(&tfull[ab]);
+        umma_commit(tfull);
       }
       if (!ok) *abort_flag = 1;
       umma_commit(drain);
       (void)mbar_wait(drain, 0);
     }
-  } else if (warp < 2 + 2 * kFGroupWarps) {
+  } else if (warp < 2 + kFDecWarps) {
     // ------------------------------ decoders -------------------------------
-    const int d = threadIdx.x - 64;
-    const int grp = d / (kFGroupWarps * 32);   // group 0 takes even steps, 1 odd
-    const int R = d % (kFGroupWarps * 32);     // weight-tile row 0..127
+    const int R = threadIdx.x - 64;            // weight-tile row 0..255
     const float off = args.sv.code8 != nullptr ? __ldg(args.sv.offset) : 0.0f;
     bool ok = true;
-    // cursors: the step being decoded, and the one being prefetched (2 ahead)
-    int tile = blockIdx.x, kk = 0;
-    advance(tile, kk, grp, nsteps);
-    int ptile = tile, pkk = kk;
-    RowFetch q0 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
-    advance(ptile, pkk, 2, nsteps);
-    RowFetch q1 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
-    advance(ptile, pkk, 2, nsteps);
-    for (uint32_t it = grp; tile < num_tiles && ok; it += 2) {
+    int tile = blockIdx.x, kk = 0;             // the step being decoded
+    int ptile = tile, pkk = kk;                // the step being prefetched
+    RowFetch q[kFPrefetch];
+#pragma unroll
+    for (int i = 0; i < kFPrefetch; ++i) {
+      q[i] = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
+      advance(ptile, pkk, 1, nsteps);
+    }
+    for (uint32_t it = 0; tile < num_tiles && ok; ++it) {
       const int s = it % kFStages;
       const uint32_t ph = (it / kFStages) & 1;
-      const RowFetch f = q0;
-      q0 = q1;
-      q1 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
-      advance(ptile, pkk, 2, nsteps);
+      const RowFetch f = q[0];
+#pragma unroll
+      for (int i = 0; i + 1 < kFPrefetch; ++i) q[i] = q[i + 1];
+      q[kFPrefetch - 1] = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
+      advance(ptile, pkk, 1, nsteps);
       if (*abort_flag || !mbar_wait(&empty[s], ph ^ 1)) { ok = false; break; }
       if (kk < args.nk) {
         uint8_t* brow = sB + s * kFB + R * 128;
@@ -499,7 +503,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&full_b[s]);
-      advance(tile, kk, 2, nsteps);
+      advance(tile, kk, 1, nsteps);
     }
     if (!ok) *abort_flag = 1;
   } else {
@@ -510,8 +514,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tc) {
       const int m0 = (tile % args.m_tiles) * kFBM;
       const int n0 = (tile / args.m_tiles) * kFBN;
-      const uint32_t ab = tc & 1, aph = (tc >> 1) & 1;
-      if (*abort_flag || !mbar_wait(&tfull[ab], aph)) { ok = false; break; }
+      if (*abort_flag || !mbar_wait(tfull, tc & 1)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
@@ -519,8 +522,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < kFBN / 32; ++c) {
           uint32_t v[32];
-          tmem_ld_32x32b_x32(
-              tmem + (static_cast<uint32_t>(q * 32) << 16) + ab * 256 + h * 128 + c * 32, v);
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 256 + c * 32, v);
           tmem_ld_wait();
           const int col = n0 + c * 32;
           if (row < args.M && col < args.Nout) {
@@ -538,7 +540,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[ab]);
+      if (lane == 0) mbar_arrive(tempty);
     }
     if (!ok) *abort_flag = 1;
   }
@@ -553,84 +555,172 @@ __global__ void __launch_bounds__(kFThreads, 1)
 }
 
 // ===========================================================================
-// GEMV for M <= 16 (CUDA cores).  CTA = 256 columns x a K-range; lane owns 8
-// consecutive columns (one 32-bit packed word per weight row), warps stride
-// over rows.  fp32 partials per split, reduced in gemv_reduce_kernel.
+// GEMV for M <= 16 (decode-style small batches), HBM-bound.
+//
+// y[m][n] = sum_k x[m][k] * Ŵ[k][n] is evaluated with mma.sync m16n8k16 on a
+// 16-token tile, with the block scale folded into the activation:
+//   y[m][n] = sum_k bf16(x[m][k] * a'[k][n/64]) * bf16(C_{code(k,n)}).
+// The weight operand then needs no per-block table: a fixed 256-entry table of
+// bf16 pairs (C[hi nibble], C[lo nibble]) turns one byte into one B-fragment
+// register.  That byte is built from two adjacent weight rows (k, k+1) at the
+// same column by interleaving nibbles of their packed words, so each lookup
+// yields the (k, k+1) pair a B-fragment register holds.  The table lives in
+// shared memory as 32 copies, one per bank ((byte << 8) | lane*4 addresses a
+// lane's own copy), so lookups never conflict.  Columns are permuted inside a
+// 64-column block so that thread g's fragments cover its own packed word:
+// n-tile j, fragment column g is weight column 8g + j.
+//
+// Compared with the dequantized weight, bf16(C) * bf16(x a') differs from
+// x * bf16(C a') by at most a bf16 rounding of each factor (relative 2^-8 per
+// product); over K terms the relative error of y stays near 3e-3.
+//
+// CTA = 256 weight columns (four 64-column blocks) x a K-range; warp w works
+// on block w & 3 and every other 16-row step (w >> 2) of the range; the two
+// warps of a block are added through shared memory and the CTA writes one fp32
+// partial per split; gemv_reduce_kernel adds the splits and Zc·B.
 // ===========================================================================
-constexpr int kGvRows = 64;  // rows of X staged in shared memory per pass
+constexpr int kGvTable = 65536;  // 256 entries x 64 words (32 used) x 4 B
 
-template <int MT>
-__global__ void __launch_bounds__(256) nf4_gemv_kernel(const uint16_t* __restrict__ X, int M,
-                                                       int K, int N, const uint8_t* __restrict__ packed,
-                                                       ScaleView sv, int rows_per_split,
-                                                       float* __restrict__ partial) {
-  __shared__ float xs[kGvRows][MT];
-  __shared__ float t8[256];
-  __shared__ float red[8][256];
-  if (sv.code8 != nullptr) build_t8(t8);
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t saddr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(saddr));
+  return v;
+}
+
+template <bool kM16>
+__global__ void __launch_bounds__(256, 2) nf4_gemv_kernel(const uint16_t* __restrict__ X, int M,
+                                                          int K, int N,
+                                                          const uint8_t* __restrict__ packed,
+                                                          ScaleView sv, int steps_per_split,
+                                                          float* __restrict__ partial) {
+  extern __shared__ uint8_t gsm_raw[];
+  uint8_t* gsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsm_raw) + 255) &
+                                            ~static_cast<uintptr_t>(255));
+  uint32_t* table = reinterpret_cast<uint32_t*>(gsm);
+  float* t8 = reinterpret_cast<float*>(gsm + kGvTable);
+  float* red = t8 + 256;                       // [4 blocks][16 m][64 cols]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n = blockIdx.x * 256 + lane * 8;
-  const int k0 = blockIdx.y * rows_per_split;
-  const int k1 = min(K, k0 + rows_per_split);
+  // fixed table: entry e -> (bf16(C[e >> 4]) | bf16(C[e & 15]) << 16), 32 copies
+  for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
+    const int e = i >> 5, c = i & 31;
+    table[e * 64 + c] = pack_bf16x2(kNF4g[e >> 4], kNF4g[e & 15]);
+  }
+  if (sv.code8 != nullptr) build_t8(t8);
+  __syncthreads();
   const float off = sv.code8 != nullptr ? __ldg(sv.offset) : 0.0f;
-  const bool colok = n < N;
-  float acc[MT][8];
+  const int g = lane >> 2, t = lane & 3;
+  const int blk = blockIdx.x * 4 + (warp & 3);          // 64-column block
+  const bool colok = blk * 64 < N;
+  const int bpr = N / 64;
+  const int step0 = blockIdx.y * steps_per_split;
+  const int step1 = min(K / 16, step0 + steps_per_split);
+  const uint32_t tbase = smem_u32(table);
+  const uint32_t laneword = lane * 4;                    // byte 0 of the address
+  float acc[8][4];
 #pragma unroll
-  for (int m = 0; m < MT; ++m)
+  for (int j = 0; j < 8; ++j)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[m][i] = 0.0f;
-  for (int kb = k0; kb < k1; kb += kGvRows) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < kGvRows * MT; i += blockDim.x) {
-      const int kr = i / MT, m = i % MT;
-      const int k = kb + kr;
-      xs[kr][m] = (m < M && k < k1) ? bf16_bits_to_f32(__ldg(X + static_cast<int64_t>(m) * K + k)) : 0.0f;
-    }
-    __syncthreads();
-    if (colok) {
-      for (int kr = warp; kr < kGvRows && kb + kr < k1; kr += 8) {
-        const int k = kb + kr;
-        const int64_t blk = static_cast<int64_t>(k) * (N / 64) + (n >> 6);
-        float a;
-        if (sv.code8 == nullptr)
-          a = __ldg(sv.absmax + blk);
-        else
-          a = __fadd_rn(__fmul_rn(t8[__ldg(sv.code8 + blk)], __ldg(sv.s2 + (blk >> 8))), off);
-        const uint32_t p = __ldg(reinterpret_cast<const uint32_t*>(packed + ((static_cast<int64_t>(k) * N + n) >> 1)));
-        float w[8];
+    for (int i = 0; i < 4; ++i) acc[j][i] = 0.0f;
+
+  if (colok) {
+    const uint8_t* pcol = packed + blk * 32 + g * 4;    // this thread's packed word in a row
+    for (int st = step0 + (warp >> 2); st < step1; st += 2) {
+      const int kb = st * 16;
+      // block scales of rows kb..kb+15: lane i < 16 decodes row kb+i
+      float sc = 0.0f;
+      if (lane < 16) {
+        const int64_t b = static_cast<int64_t>(kb + lane) * bpr + blk;
+        sc = sv.code8 == nullptr
+                 ? __ldg(sv.absmax + b)
+                 : __fadd_rn(__fmul_rn(t8[__ldg(sv.code8 + b)], __ldg(sv.s2 + (b >> 8))), off);
+      }
+      const float s0 = __shfl_sync(0xFFFFFFFFu, sc, 2 * t);
+      const float s1 = __shfl_sync(0xFFFFFFFFu, sc, 2 * t + 1);
+      const float s2 = __shfl_sync(0xFFFFFFFFu, sc, 2 * t + 8);
+      const float s3 = __shfl_sync(0xFFFFFFFFu, sc, 2 * t + 9);
+      // activation fragment, scaled per row
+      uint32_t a[4] = {0u, 0u, 0u, 0u};
+      if (g < M) {
+        const uint16_t* xr = X + static_cast<int64_t>(g) * K + kb + 2 * t;
+        const uint32_t x0 = __ldg(reinterpret_cast<const uint32_t*>(xr));
+        const uint32_t x1 = __ldg(reinterpret_cast<const uint32_t*>(xr + 8));
+        a[0] = pack_bf16x2(__uint_as_float(x0 << 16) * s0, __uint_as_float(x0 & 0xFFFF0000u) * s1);
+        a[2] = pack_bf16x2(__uint_as_float(x1 << 16) * s2, __uint_as_float(x1 & 0xFFFF0000u) * s3);
+      }
+      if (kM16 && g + 8 < M) {
+        const uint16_t* xr = X + static_cast<int64_t>(g + 8) * K + kb + 2 * t;
+        const uint32_t x0 = __ldg(reinterpret_cast<const uint32_t*>(xr));
+        const uint32_t x1 = __ldg(reinterpret_cast<const uint32_t*>(xr + 8));
+        a[1] = pack_bf16x2(__uint_as_float(x0 << 16) * s0, __uint_as_float(x0 & 0xFFFF0000u) * s1);
+        a[3] = pack_bf16x2(__uint_as_float(x1 << 16) * s2, __uint_as_float(x1 & 0xFFFF0000u) * s3);
+      }
+      // packed words of rows kb+2t, kb+2t+1, kb+2t+8, kb+2t+9 (columns 8g..8g+7)
+      const int64_t rb = static_cast<int64_t>(N) / 2;
+      const uint8_t* p = pcol + static_cast<int64_t>(kb + 2 * t) * rb;
+      const uint32_t w0 = __ldg(reinterpret_cast<const uint32_t*>(p));
+      const uint32_t w1 = __ldg(reinterpret_cast<const uint32_t*>(p + rb));
+      const uint32_t w8 = __ldg(reinterpret_cast<const uint32_t*>(p + 8 * rb));
+      const uint32_t w9 = __ldg(reinterpret_cast<const uint32_t*>(p + 9 * rb));
+      // bytes (row k nibble, row k+1 nibble) per column: even and odd columns
+      const uint32_t lo_e = (w0 & 0xF0F0F0F0u) | ((w1 >> 4) & 0x0F0F0F0Fu);
+      const uint32_t lo_o = ((w0 << 4) & 0xF0F0F0F0u) | (w1 & 0x0F0F0F0Fu);
+      const uint32_t hi_e = (w8 & 0xF0F0F0F0u) | ((w9 >> 4) & 0x0F0F0F0Fu);
+      const uint32_t hi_o = ((w8 << 4) & 0xF0F0F0F0u) | (w9 & 0x0F0F0F0Fu);
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const uint32_t byte = (p >> (8 * b)) & 0xFFu;
-          const uint32_t pr = pack_bf16x2(kNF4g[byte >> 4] * a, kNF4g[byte & 15u] * a);
-          w[2 * b] = __uint_as_float(pr << 16);
-          w[2 * b + 1] = __uint_as_float(pr & 0xFFFF0000u);
-        }
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-          const float xv = xs[kr][m];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc[m][i] = fmaf(xv, w[i], acc[m][i]);
-        }
+      for (int i = 0; i < 4; ++i) {
+        // offset (byte i << 8) | lane*4: output byte 0 <- lane*4 (source byte
+        // 4), byte 1 <- byte i of the word, bytes 2 and 3 <- zero (source byte 5)
+        const uint32_t sel = 0x5504u | (static_cast<uint32_t>(i) << 4);
+        const uint32_t b0e = lds32(tbase + prmt(lo_e, laneword, sel));
+        const uint32_t b1e = lds32(tbase + prmt(hi_e, laneword, sel));
+        const uint32_t b0o = lds32(tbase + prmt(lo_o, laneword, sel));
+        const uint32_t b1o = lds32(tbase + prmt(hi_o, laneword, sel));
+        mma_bf16_16816(acc[2 * i], a, b0e, b1e);
+        mma_bf16_16816(acc[2 * i + 1], a, b0o, b1o);
       }
     }
   }
-  // reduce the 8 warps' partial sums through shared memory, one row at a time
+  // add the two warps of each block, then write this split's partial
+  float* myred = red + (warp & 3) * (16 * 64);
+  if (warp >= 4) {
 #pragma unroll
-  for (int m = 0; m < MT; ++m) {
-    if (m < M) {
-      __syncthreads();
+    for (int j = 0; j < 8; ++j) {
+      // acc[j]: (row g, cols 2t, 2t+1), (row g+8, ...) of n-tile j; column
+      // index c of n-tile j is weight column 8c + j
+      myred[g * 64 + 8 * (2 * t) + j] = acc[j][0];
+      myred[g * 64 + 8 * (2 * t + 1) + j] = acc[j][1];
+      myred[(g + 8) * 64 + 8 * (2 * t) + j] = acc[j][2];
+      myred[(g + 8) * 64 + 8 * (2 * t + 1) + j] = acc[j][3];
+    }
+  }
+  __syncthreads();
+  if (warp < 4 && colok) {
+    float* out = partial + static_cast<int64_t>(blockIdx.y) * M * N + blk * 64;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) red[warp][lane * 8 + i] = acc[m][i];
-      __syncthreads();
-      const int col = threadIdx.x;
-      float s = 0.0f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) s += red[w][col];
-      if (blockIdx.x * 256 + col < N)
-        partial[(static_cast<int64_t>(blockIdx.y) * M + m) * N + blockIdx.x * 256 + col] = s;
+    for (int j = 0; j < 8; ++j) {
+      const int c0 = 8 * (2 * t) + j, c1 = 8 * (2 * t + 1) + j;
+      if (g < M) {
+        out[static_cast<int64_t>(g) * N + c0] = acc[j][0] + myred[g * 64 + c0];
+        out[static_cast<int64_t>(g) * N + c1] = acc[j][1] + myred[g * 64 + c1];
+      }
+      if (g + 8 < M) {
+        out[static_cast<int64_t>(g + 8) * N + c0] = acc[j][2] + myred[(g + 8) * 64 + c0];
+        out[static_cast<int64_t>(g + 8) * N + c1] = acc[j][3] + myred[(g + 8) * 64 + c1];
+      }
     }
   }
 }
+
+constexpr size_t kGvSmem = 256 + kGvTable + 1024 + 4 * 16 * 64 * 4;
 
 // Y[m][n] = bf16( sum_s partial[s][m][n] + sum_j Zc[m][j] * B[j][n] )
 __global__ void gemv_reduce_kernel(const float* __restrict__ partial, int splits, int M, int N,
@@ -735,13 +825,17 @@ constexpr CUtensorMapSwizzle kSW128 = CU_TENSOR_MAP_SWIZZLE_128B;
 
 int rsteps_of(int r) { return (r + 15) / 16; }
 
-size_t gemv_splits_and_bytes(int64_t M, int64_t K, int64_t N, int num_sms, int* splits_out) {
+size_t gemv_splits_and_bytes(int64_t M, int64_t K, int64_t N, int num_sms, int* splits_out,
+                             int* steps_out) {
   const int ntiles = static_cast<int>((N + 255) / 256);
+  const int ksteps = static_cast<int>(K / 16);
   int s = (2 * num_sms + ntiles - 1) / ntiles;
-  const int maxs = static_cast<int>((K + kGvRows - 1) / kGvRows);
-  if (s > maxs) s = maxs;
+  if (s > ksteps / 2) s = ksteps / 2;
   if (s < 1) s = 1;
+  const int per = (ksteps + s - 1) / s;
+  s = (ksteps + per - 1) / per;
   if (splits_out) *splits_out = s;
+  if (steps_out) *steps_out = per;
   return align256(static_cast<size_t>(s) * M * N * 4);
 }
 
@@ -753,7 +847,7 @@ size_t linear_fwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) {
   (void)r;
   const int S = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
   size_t b = align256(static_cast<size_t>(S) * M * 64 * 4);
-  if (M <= 16) b += gemv_splits_and_bytes(M, K, N, g_ws_sms, nullptr);
+  if (M <= 16) b += gemv_splits_and_bytes(M, K, N, g_ws_sms, nullptr, nullptr);
   return b;
 }
 
@@ -788,24 +882,28 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
   if (e != cudaSuccess) return e;
 
   if (M <= 16) {
-    int S = 1;
-    gemv_splits_and_bytes(M, K, N, g_ws_sms, &S);
+    int S = 1, per = 1;
+    gemv_splits_and_bytes(M, K, N, g_ws_sms, &S, &per);
     float* pg = static_cast<float*>(cur.take(static_cast<size_t>(S) * M * N * 4));
     if (!cur.ok) return cudaErrorInvalidValue;
-    const int rows = static_cast<int>(((K + S - 1) / S + kGvRows - 1) / kGvRows * kGvRows);
-    const int splits = static_cast<int>((K + rows - 1) / rows);
-    dim3 grid(static_cast<unsigned>((N + 255) / 256), splits);
+    static bool attr_done = false;
+    if (!attr_done) {
+      e = cudaFuncSetAttribute(nf4_gemv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kGvSmem));
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(nf4_gemv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kGvSmem));
+      if (e != cudaSuccess) return e;
+      attr_done = true;
+    }
+    dim3 grid(static_cast<unsigned>((N + 255) / 256), S);
     const int Mi = static_cast<int>(M), Ki = static_cast<int>(K), Ni = static_cast<int>(N);
     {
-    ProfScope prof(kProfGemv, st);
-    if (M <= 1)
-      nf4_gemv_kernel<1><<<grid, 256, 0, st>>>(X, Mi, Ki, Ni, packed, sv, rows, pg);
-    else if (M <= 4)
-      nf4_gemv_kernel<4><<<grid, 256, 0, st>>>(X, Mi, Ki, Ni, packed, sv, rows, pg);
-    else if (M <= 8)
-      nf4_gemv_kernel<8><<<grid, 256, 0, st>>>(X, Mi, Ki, Ni, packed, sv, rows, pg);
-    else
-      nf4_gemv_kernel<16><<<grid, 256, 0, st>>>(X, Mi, Ki, Ni, packed, sv, rows, pg);
+      ProfScope prof(kProfGemv, st);
+      if (M <= 8)
+        nf4_gemv_kernel<false><<<grid, 256, kGvSmem, st>>>(X, Mi, Ki, Ni, packed, sv, per, pg);
+      else
+        nf4_gemv_kernel<true><<<grid, 256, kGvSmem, st>>>(X, Mi, Ki, Ni, packed, sv, per, pg);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -813,7 +911,7 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
     {
       ProfScope prof(kProfOther, st);
       gemv_reduce_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(
-          pg, splits, Mi, Ni, Zc, B, r, Y);
+          pg, S, Mi, Ni, Zc, B, r, Y);
     }
     return cudaGetLastError();
   }
@@ -887,7 +985,7 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   // dX = G W^T + dZ A^T
   e = set_fused_attr<true>();
   if (e != cudaSuccess) return e;
-  if (!make_tmap_2d(&tAl, A, kBF16, 2, K, r, r, 64, 128, kSW128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tAl, A, kBF16, 2, K, r, r, 64, 256, kSW128)) return cudaErrorInvalidValue;
   CUtensorMap tdZa;
   if (!make_tmap_2d(&tdZa, dZ, kBF16, 2, M, 64, 64, 64, 128, kSW128)) return cudaErrorInvalidValue;
   FusedArgs fa;

@@ -142,12 +142,19 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const T* __restrict__ W
     const bool finite = am <= FLT_MAX;
     bad |= !finite;
     const float s = (finite && am > 0.0f) ? am : 1.0f;
-    const float inv_s = __frcp_rn(s);
+    // For a block scale below 2^-126, 1/s would overflow: scale the block and
+    // its scale by 2^64 (exact for these tiny values) so the fast path stays
+    // finite; codes depend only on the ratio w/s.
+    const bool tiny = s < 1.17549435e-38f;
+    const float sc = tiny ? 18446744073709551616.0f : 1.0f;
+    const float s_eff = s * sc;
+    const float inv_s = __frcp_rn(s_eff);
     uint32_t word = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const uint32_t code =
-          (finite && e0 + i < numel) ? nearest_code(x[i], s, inv_s, tab, mexact) : kPadCode;
+      const uint32_t code = (finite && e0 + i < numel)
+                                ? nearest_code(x[i] * sc, s_eff, inv_s, tab, mexact)
+                                : kPadCode;
       // element 2k -> high nibble of byte k, element 2k+1 -> low nibble
       word |= code << ((i >> 1) * 8 + ((i & 1) ? 0 : 4));
     }
@@ -196,55 +203,122 @@ __device__ __forceinline__ void add_u32_at(uint32_t* L, int nl, int i, uint32_t 
 
 __device__ __forceinline__ int bit_of(const uint32_t* Q, int b) { return (Q[b >> 5] >> (b & 31)) & 1; }
 
-__global__ void dq_mean_kernel(const unsigned long long* __restrict__ bins, int64_t n1,
-                               float* __restrict__ offset) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  constexpr int NL = 12;
-  uint32_t L[NL];
-  for (int i = 0; i < NL; ++i) L[i] = 0;
-  for (int key = 1; key < 255; ++key) {
-    const unsigned long long v = bins[key];
-    if (!v) continue;
-    const int sh = key - 1, li = sh >> 5, bi = sh & 31;
-    const uint64_t p0 = (v & 0xFFFFFFFFull) << bi;   // < 2^63
-    const uint64_t p1 = (v >> 32) << bi;             // < 2^63
-    add_u32_at(L, NL, li, static_cast<uint32_t>(p0));
-    add_u32_at(L, NL, li + 1, static_cast<uint32_t>(p0 >> 32));
-    add_u32_at(L, NL, li + 1, static_cast<uint32_t>(p1));
-    add_u32_at(L, NL, li + 2, static_cast<uint32_t>(p1 >> 32));
-  }
-  const uint64_t d = static_cast<uint64_t>(n1);
-  uint32_t Q[NL];
-  uint64_t rem = 0;
-  for (int i = NL - 1; i >= 0; --i) {
-    const uint64_t cur = (rem << 32) | L[i];
-    Q[i] = static_cast<uint32_t>(cur / d);
-    rem = cur % d;
-  }
-  int h = -1;
-  for (int i = NL - 1; i >= 0 && h < 0; --i)
-    if (Q[i]) h = i * 32 + 31 - __clz(Q[i]);
-  uint32_t bits;
-  if (h < 23) {
-    // below 2^-126: Q itself is the subnormal significand
-    uint32_t q = Q[0];
-    const bool up = (2 * rem > d) || (2 * rem == d && (q & 1u));
-    bits = q + (up ? 1u : 0u);
-  } else {
-    const int shift = h - 23;
-    uint32_t mant = 0;
-    for (int b = 0; b < 24; ++b) mant |= static_cast<uint32_t>(bit_of(Q, shift + b)) << b;
-    bool up;
-    if (shift == 0) {
-      up = (2 * rem > d) || (2 * rem == d && (mant & 1u));
-    } else {
-      const int rb = bit_of(Q, shift - 1);
-      bool sticky = rem != 0;
-      for (int b = 0; b < shift - 1 && !sticky; ++b) sticky = bit_of(Q, b);
-      up = rb && (sticky || (mant & 1u));
+// Round q * 2^e (q > 0 a 128-bit integer, plus an extra fraction rem/d of
+// one unit 2^e, 0 <= rem < d) to the nearest fp32, ties to even.
+__device__ uint32_t round_q128_to_f32(unsigned __int128 q, uint64_t rem, uint64_t d, int e) {
+  if (q == 0) {
+    // below one unit: only possible when 2^e is below the subnormal quantum
+    // or the mean is exactly 0; scale up until the quantum is reached
+    while (e > -149 && q == 0) {
+      const unsigned __int128 t = static_cast<unsigned __int128>(rem) << 1;
+      q = static_cast<unsigned __int128>(t / d);
+      rem = static_cast<uint64_t>(t % d);
+      --e;
     }
-    mant += up ? 1u : 0u;
-    bits = (static_cast<uint32_t>(shift + 1) << 23) + (mant - 0x800000u);
+    if (q == 0) return 0u;
+  }
+  const uint64_t hi = static_cast<uint64_t>(q >> 64), lo = static_cast<uint64_t>(q);
+  const int h = hi ? 127 - __clzll(static_cast<long long>(hi)) : 63 - __clzll(static_cast<long long>(lo));
+  int qe = h + e - 23;                 // exponent of the fp32 quantum
+  if (qe < -149) qe = -149;
+  int shift = qe - e;
+  if (shift < 0) {                     // make room below: bring fraction bits in
+    const int up = -shift;
+    const unsigned __int128 t = static_cast<unsigned __int128>(rem) << up;
+    q = (q << up) + static_cast<unsigned __int128>(t / d);
+    rem = static_cast<uint64_t>(t % d);
+    shift = 0;
+  }
+  uint64_t mant = static_cast<uint64_t>(q >> shift);
+  bool up;
+  if (shift == 0) {
+    up = (2 * rem > d) || (2 * rem == d && (mant & 1u));
+  } else {
+    const unsigned __int128 below = q & ((static_cast<unsigned __int128>(1) << shift) - 1);
+    const unsigned __int128 half = static_cast<unsigned __int128>(1) << (shift - 1);
+    up = below > half || (below == half && (rem != 0 || (mant & 1u)));
+  }
+  mant += up ? 1u : 0u;
+  // value = mant * 2^qe with mant <= 2^24
+  if (qe == -149 && mant < (1u << 23)) return static_cast<uint32_t>(mant);   // subnormal
+  return (static_cast<uint32_t>(qe + 150) << 23) + static_cast<uint32_t>(mant - (1u << 23));
+}
+
+// One CTA of 256 threads: the bins are read in parallel, a warp ballot finds
+// the occupied exponent range, and one thread adds the occupied bins exactly:
+// in 128 bits when they span at most 64 binades (always, for any realistic
+// weight), else in a 384-bit integer.
+__global__ void __launch_bounds__(256) dq_mean_kernel(const unsigned long long* __restrict__ bins,
+                                                      int64_t n1, float* __restrict__ offset) {
+  __shared__ unsigned long long sb[256];
+  __shared__ int range[2];
+  sb[threadIdx.x] = bins[threadIdx.x];
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    uint32_t m = 0;
+    for (int i = 0; i < 8; ++i) m |= (sb[threadIdx.x * 8 + i] != 0ull ? 1u : 0u) << i;
+    const unsigned any = __ballot_sync(0xFFFFFFFFu, m != 0);
+    const int lmin = __ffs(any) - 1, lmax = 31 - __clz(any);
+    if (threadIdx.x == lmin) range[0] = threadIdx.x * 8 + (__ffs(m) - 1);
+    if (threadIdx.x == lmax) range[1] = threadIdx.x * 8 + (31 - __clz(m));
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  const int kmin = range[0], kmax = range[1];
+  const uint64_t d = static_cast<uint64_t>(n1);
+  uint32_t bits;
+  if (kmax - kmin <= 64) {
+    unsigned __int128 S = 0;
+    for (int key = kmin; key <= kmax; ++key)
+      S += static_cast<unsigned __int128>(sb[key]) << (key - kmin);
+    const unsigned __int128 Q = S / d;
+    const uint64_t rem = static_cast<uint64_t>(S % d);
+    bits = round_q128_to_f32(Q, rem, d, kmin - 1 - 149);
+  } else {
+    constexpr int NL = 12;
+    uint32_t L[NL];
+    for (int i = 0; i < NL; ++i) L[i] = 0;
+    for (int key = kmin; key <= kmax; ++key) {
+      const unsigned long long v = sb[key];
+      if (!v) continue;
+      const int sh = key - 1, li = sh >> 5, bi = sh & 31;
+      const uint64_t p0 = (v & 0xFFFFFFFFull) << bi;
+      const uint64_t p1 = (v >> 32) << bi;
+      add_u32_at(L, NL, li, static_cast<uint32_t>(p0));
+      add_u32_at(L, NL, li + 1, static_cast<uint32_t>(p0 >> 32));
+      add_u32_at(L, NL, li + 1, static_cast<uint32_t>(p1));
+      add_u32_at(L, NL, li + 2, static_cast<uint32_t>(p1 >> 32));
+    }
+    uint32_t Q[NL];
+    uint64_t rem = 0;
+    for (int i = NL - 1; i >= 0; --i) {
+      const uint64_t cur = (rem << 32) | L[i];
+      Q[i] = static_cast<uint32_t>(cur / d);
+      rem = cur % d;
+    }
+    int h = -1;
+    for (int i = NL - 1; i >= 0 && h < 0; --i)
+      if (Q[i]) h = i * 32 + 31 - __clz(Q[i]);
+    if (h < 23) {
+      const uint32_t q = Q[0];
+      const bool up = (2 * rem > d) || (2 * rem == d && (q & 1u));
+      bits = q + (up ? 1u : 0u);
+    } else {
+      const int shift = h - 23;
+      uint32_t mant = 0;
+      for (int b = 0; b < 24; ++b) mant |= static_cast<uint32_t>(bit_of(Q, shift + b)) << b;
+      bool up;
+      if (shift == 0) {
+        up = (2 * rem > d) || (2 * rem == d && (mant & 1u));
+      } else {
+        const int rb = bit_of(Q, shift - 1);
+        bool sticky = rem != 0;
+        for (int b = 0; b < shift - 1 && !sticky; ++b) sticky = bit_of(Q, b);
+        up = rb && (sticky || (mant & 1u));
+      }
+      mant += up ? 1u : 0u;
+      bits = (static_cast<uint32_t>(shift + 1) << 23) + (mant - 0x800000u);
+    }
   }
   *offset = __uint_as_float(bits);
 }
@@ -340,7 +414,7 @@ cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* pa
   if (e != cudaSuccess || !dq) return e;
   {
     ProfScope prof(kProfQuantize, st);
-    dq_mean_kernel<<<1, 32, 0, st>>>(bins, n1, offset);
+    dq_mean_kernel<<<1, 256, 0, st>>>(bins, n1, offset);
   }
   const int64_t n2 = (n1 + kDQBlock - 1) / kDQBlock;
   {

@@ -144,3 +144,26 @@ def test_full_size_65b_mlp_sampled():
         codes, _ = nf4.quantize_nf4(flat[b * 64:(b + 1) * 64])
         payload, _ = nf4.pack_codes(codes)
         assert np.array_equal(packed[b * 32:(b + 1) * 32], payload), b
+
+
+@pytest.mark.parametrize("scales", [
+    [1.0, 1.0 + 2.0 ** -23],                        # exact tie -> even (1.0)
+    [1.0 + 2.0 ** -23, 1.0 + 2.0 ** -22],           # exact tie -> even (upper)
+    [2.0 ** -149, 2.0 ** -149, 2.0 ** -148],        # subnormal scales
+    [1e-30, 1.0, 3.0],                              # > 64 binades apart: wide path
+    [1e-38, 3e38],                                  # extreme spread
+    [0.037] * 1000,                                 # equal scales
+    [2.0 ** 24] + [1.0] * 4095,                     # naive fp32 running sum would lose these
+])
+def test_double_quant_offset_is_the_exact_mean(scales):
+    """Blocks whose absmax equals each listed scale; the DQ offset must equal
+    the oracle's exactly rounded mean bit for bit."""
+    q = _q()
+    sc = np.array(scales, np.float32)
+    w = np.zeros(64 * sc.size, np.float32)
+    w[::64] = sc                                    # one element per block carries the scale
+    w[1::64] = -sc * np.float32(0.5)
+    g = q.quantize(to_dev(w, torch.float32), double_quant=True)
+    ow = OracleWeight(w, True)
+    assert_state_equal(g, ow)
+    assert np.array_equal(nf4.block_scales(w), sc)
