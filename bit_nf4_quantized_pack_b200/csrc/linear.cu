@@ -183,32 +183,36 @@ __global__ void skinny_reduce_kernel(const float* __restrict__ partial, int spli
 //
 // Output tile 256 (rows of X or G) x 256, K-step 64.  One decoded weight tile
 // (256 x 64 bf16) feeds two tcgen05.mma of M = 128, N = 256 (rows m0..m0+127
-// and m0+128..m0+255), so each decoded weight is used by 256 rows.  Per stage
-// the shared memory holds the activation tile (256 x 64 bf16, K-major, two
-// TMA boxes) and the decoded weight tile, written by the decoder warps as 256
-// rows of 128 bytes, each row one NF4 block of 64 consecutive weights (row R at
+// and m0+128..m0+255), so each decoded weight is used by 256 rows.
+//
+// Shared memory holds two rings.  Activation tiles (256 x 64 bf16, K-major,
+// two TMA boxes) have 4 stages so that TMA runs well ahead of the MMAs.
+// Decoded weight tiles have 3 stages; decoder warps write them as 256 rows of
+// 128 bytes, each row one NF4 block of 64 consecutive weights (row R at
 // R*128, 16-byte chunk c at (c ^ (R & 7))*16, the 128-byte swizzle pattern):
 //   forward   row R = 64*nb + k: weights (k0+k, n0+64nb .. +63) — an MN-major
 //             operand (atoms of 8 k-rows x 64 n; 8 KB between n-atoms);
 //   backward  row R: weights (n0+R, k0 .. k0+63) of W, i.e. row R of Ŵᵀ's
 //             K-major operand.
 // Each decoder thread owns one row and loads its 32 packed bytes and its
-// block scale straight from global memory three K-steps ahead.  After the last K-step, one more
-// step accumulates the LoRA term: Zc (or dZ) as the activation tile and B (or
-// A) as the weight tile, both by TMA (rank padded to a multiple of 16 with
-// zeros by TMA's out-of-bounds fill).  TMEM holds the two 128 x 256 fp32
-// accumulators (all 512 columns); the epilogue drains them before the next
-// tile's first MMA.
+// block scale straight from global memory three K-steps ahead.
+//
+// After the last K-step of a tile, the LoRA step takes two activation stages:
+// Zc (or dZ) as the activation tile and B (or A) as the weight tile, both by
+// TMA with the rank padded to a multiple of 16 by TMA's zero fill; the decoder
+// warps skip it.  TMEM holds the two 128 x 256 fp32 accumulators (all 512
+// columns); the epilogue releases each as soon as it has read it, so the next
+// tile's first MMAs into the first accumulator overlap the drain of the second.
 // ===========================================================================
-constexpr int kFStages = 3;
+constexpr int kFAStages = 4;         // activation tiles (TMA)
+constexpr int kFBStages = 3;         // decoded weight tiles (decoder warps)
 constexpr int kFBM = 256, kFBN = 256;
 constexpr int kFA = 32768;           // 256 x 64 bf16
 constexpr int kFB = 32768;           // 256 x 64 bf16
 constexpr int kFThreads = 448;       // warp 0 TMA, 1 MMA, 2..9 decode, 10..13 epilogue
 constexpr int kFDecWarps = 8;
-constexpr int kFPrefetch = 3;        // K-steps of packed bytes and scales in flight per thread
 constexpr int kFEpiWarps = 4;
-constexpr size_t kFSmem = 1024 + kFStages * (kFA + kFB) + 1024 + 512;
+constexpr size_t kFSmem = 1024 + kFAStages * kFA + kFBStages * kFB + 1024 + 512;
 
 struct FusedArgs {
   int M;          // rows of the activation / output
@@ -340,27 +344,32 @@ __global__ void __launch_bounds__(kFThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = sA + kFStages * kFA;
-  float* t8 = reinterpret_cast<float*>(sB + kFStages * kFB);
+  uint8_t* sB = sA + kFAStages * kFA;
+  float* t8 = reinterpret_cast<float*>(sB + kFBStages * kFB);
   uint64_t* full_a = reinterpret_cast<uint64_t*>(t8 + 256);
-  uint64_t* full_b = full_a + kFStages;
-  uint64_t* empty = full_b + kFStages;
-  uint64_t* tfull = empty + kFStages;
-  uint64_t* tempty = tfull + 1;
-  uint64_t* drain = tempty + 1;
+  uint64_t* empty_a = full_a + kFAStages;
+  uint64_t* full_b = empty_a + kFAStages;
+  uint64_t* empty_b = full_b + kFBStages;
+  uint64_t* tfull = empty_b + kFBStages;
+  uint64_t* tempty = tfull + 1;   // [2]: one per accumulator
+  uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (args.sv.code8 != nullptr) build_t8(t8);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kFStages; ++s) {
+    for (int s = 0; s < kFAStages; ++s) {
       mbar_init(&full_a[s], 1);
+      mbar_init(&empty_a[s], 1);
+    }
+    for (int s = 0; s < kFBStages; ++s) {
       mbar_init(&full_b[s], kFDecWarps);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty_b[s], 1);
     }
     mbar_init(tfull, 1);
-    mbar_init(tempty, kFEpiWarps);
+    mbar_init(&tempty[0], kFEpiWarps);
+    mbar_init(&tempty[1], kFEpiWarps);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -374,7 +383,6 @@ __global__ void __launch_bounds__(kFThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const int num_tiles = args.m_tiles * args.n_tiles;
-  const int nsteps = args.nk + 1;  // + the LoRA step
 
   if (warp == 0) {
     // ------------------------------ TMA producer ---------------------------
@@ -382,41 +390,51 @@ __global__ void __launch_bounds__(kFThreads, 1)
       tma_prefetch_desc(&tmAct);
       tma_prefetch_desc(&tmLA);
       tma_prefetch_desc(&tmLB);
-      uint32_t it = 0;
-      uint32_t last_parity[kFStages] = {2, 2, 2};
+      uint32_t ia = 0;                          // activation-ring slot counter
+      uint32_t last_parity[kFAStages] = {2, 2, 2, 2};
       bool ok = true;
+      auto take = [&](uint32_t& s_out) -> bool {
+        const uint32_t s = ia % kFAStages, ph = (ia / kFAStages) & 1;
+        if (*abort_flag || !mbar_wait(&empty_a[s], ph ^ 1)) return false;
+        last_parity[s] = ph;
+        s_out = s;
+        ++ia;
+        return true;
+      };
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int m0 = (tile % args.m_tiles) * kFBM;
         const int n0 = (tile / args.m_tiles) * kFBN;
-        for (int kk = 0; kk < nsteps; ++kk, ++it) {
-          const int s = it % kFStages;
-          const uint32_t ph = (it / kFStages) & 1;
-          if (*abort_flag || !mbar_wait(&empty[s], ph ^ 1)) { ok = false; break; }
+        for (int kk = 0; kk < args.nk && ok; ++kk) {
+          uint32_t s;
+          if (!take(s)) { ok = false; break; }
           uint8_t* a = sA + s * kFA;
-          if (kk < args.nk) {
-            mbar_arrive_expect_tx(&full_a[s], kFA);
-            tma_load_2d(a, &tmAct, &full_a[s], kk * 64, m0);
-            tma_load_2d(a + 16384, &tmAct, &full_a[s], kk * 64, m0 + 128);
-          } else {
-            mbar_arrive_expect_tx(&full_a[s], kFA + kFB);
-            tma_load_2d(a, &tmLA, &full_a[s], 0, m0);
-            tma_load_2d(a + 16384, &tmLA, &full_a[s], 0, m0 + 128);
-            uint8_t* b = sB + s * kFB;
-            if (!kBwd) {
+          mbar_arrive_expect_tx(&full_a[s], kFA);
+          tma_load_2d(a, &tmAct, &full_a[s], kk * 64, m0);
+          tma_load_2d(a + 16384, &tmAct, &full_a[s], kk * 64, m0 + 128);
+        }
+        if (!ok) break;
+        // LoRA step: Zc / dZ into one stage, B / A into the next
+        uint32_t s1, s2;
+        if (!take(s1)) { ok = false; break; }
+        uint8_t* a = sA + s1 * kFA;
+        mbar_arrive_expect_tx(&full_a[s1], kFA);
+        tma_load_2d(a, &tmLA, &full_a[s1], 0, m0);
+        tma_load_2d(a + 16384, &tmLA, &full_a[s1], 0, m0 + 128);
+        if (!take(s2)) { ok = false; break; }
+        uint8_t* b = sA + s2 * kFA;
+        mbar_arrive_expect_tx(&full_a[s2], kFB);
+        if (!kBwd) {
 #pragma unroll
-              for (int nb = 0; nb < 4; ++nb)
-                tma_load_2d(b + nb * 8192, &tmLB, &full_a[s], n0 + nb * 64, 0);
-            } else {
-              tma_load_2d(b, &tmLB, &full_a[s], 0, n0);
-            }
-          }
-          last_parity[s] = ph;
+          for (int nb = 0; nb < 4; ++nb)
+            tma_load_2d(b + nb * 8192, &tmLB, &full_a[s2], n0 + nb * 64, 0);
+        } else {
+          tma_load_2d(b, &tmLB, &full_a[s2], 0, n0);
         }
       }
       if (!ok) {
         *abort_flag = 1;
         // let copies already in flight land before the CTA can exit
-        for (int s = 0; s < kFStages; ++s)
+        for (int s = 0; s < kFAStages; ++s)
           if (last_parity[s] < 2) (void)mbar_wait(&full_a[s], last_parity[s]);
       }
     }
@@ -424,33 +442,55 @@ __global__ void __launch_bounds__(kFThreads, 1)
     // ------------------------------ MMA issuer -----------------------------
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, kFBN, 0, kBwd ? 0 : 1);
-      uint32_t it = 0, tc = 0;
+      uint32_t ia = 0, ib = 0, tc = 0;
       bool ok = true;
+      auto wait_a = [&](uint32_t& s) -> bool {
+        s = ia % kFAStages;
+        const uint32_t ph = (ia / kFAStages) & 1;
+        ++ia;
+        return !*abort_flag && mbar_wait(&full_a[s], ph);
+      };
+      auto bdesc = [&](uint32_t b0, int j) -> uint64_t {
+        return kBwd ? smem_desc(b0 + j * 32, 16, 1024) : smem_desc(b0 + j * 2048, 8192, 1024);
+      };
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tc) {
-        // the epilogue of the previous tile has drained both accumulators
-        if (*abort_flag || !mbar_wait(tempty, (tc & 1) ^ 1)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t d0 = tmem, d1 = tmem + 256;
-        for (int kk = 0; kk < nsteps; ++kk, ++it) {
-          const int s = it % kFStages;
-          const uint32_t ph = (it / kFStages) & 1;
-          if (*abort_flag || !mbar_wait(&full_a[s], ph) || !mbar_wait(&full_b[s], ph)) {
-            ok = false;
-            break;
-          }
+        const uint32_t tph = (tc & 1) ^ 1;       // parity of the previous tile's release
+        for (int kk = 0; kk < args.nk; ++kk) {
+          uint32_t sa;
+          if (!wait_a(sa)) { ok = false; break; }
+          const uint32_t sb = ib % kFBStages, phb = (ib / kFBStages) & 1;
+          ++ib;
+          if (*abort_flag || !mbar_wait(&full_b[sb], phb)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + s * kFA), b0 = smem_u32(sB + s * kFB);
-          const int nm = (kk < args.nk) ? 4 : args.rsteps;
-          for (int j = 0; j < nm; ++j) {
-            const uint64_t bd = kBwd ? smem_desc(b0 + j * 32, 16, 1024)
-                                     : smem_desc(b0 + j * 2048, 8192, 1024);
-            const uint32_t acc = (kk > 0 || j > 0) ? 1u : 0u;
-            umma_bf16(d0, smem_desc(a0 + j * 32, 16, 1024), bd, idesc, acc);
-            umma_bf16(d1, smem_desc(a0 + 16384 + j * 32, 16, 1024), bd, idesc, acc);
+          const uint32_t a0 = smem_u32(sA + sa * kFA), b0 = smem_u32(sB + sb * kFB);
+          const uint32_t acc = kk > 0 ? 1u : 0u;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (kk == 0) {   // first K-step of a tile: wait until this accumulator is drained
+              if (*abort_flag || !mbar_wait(&tempty[h], tph)) { ok = false; break; }
+              tc_fence_after();
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              umma_bf16(tmem + h * 256, smem_desc(a0 + h * 16384 + j * 32, 16, 1024),
+                        bdesc(b0, j), idesc, (acc || j > 0) ? 1u : 0u);
           }
-          umma_commit(&empty[s]);
+          if (!ok) break;
+          umma_commit(&empty_a[sa]);
+          umma_commit(&empty_b[sb]);
         }
         if (!ok) break;
+        // LoRA step
+        uint32_t s1, s2;
+        if (!wait_a(s1) || !wait_a(s2)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sA + s1 * kFA), b0 = smem_u32(sA + s2 * kFA);
+        for (int j = 0; j < args.rsteps; ++j) {
+          umma_bf16(tmem, smem_desc(a0 + j * 32, 16, 1024), bdesc(b0, j), idesc, 1u);
+          umma_bf16(tmem + 256, smem_desc(a0 + 16384 + j * 32, 16, 1024), bdesc(b0, j), idesc, 1u);
+        }
+        umma_commit(&empty_a[s1]);
+        umma_commit(&empty_a[s2]);
         umma_commit(tfull);
       }
       if (!ok) *abort_flag = 1;
@@ -461,49 +501,63 @@ __global__ void __launch_bounds__(kFThreads, 1)
     // ------------------------------ decoders -------------------------------
     const int R = threadIdx.x - 64;            // weight-tile row 0..255
     const float off = args.sv.code8 != nullptr ? __ldg(args.sv.offset) : 0.0f;
+    const int nsteps = args.nk;                // decoded steps per tile
     bool ok = true;
     int tile = blockIdx.x, kk = 0;             // the step being decoded
     int ptile = tile, pkk = kk;                // the step being prefetched
-    RowFetch q[kFPrefetch];
-#pragma unroll
-    for (int i = 0; i < kFPrefetch; ++i) {
-      q[i] = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
-      advance(ptile, pkk, 1, nsteps);
-    }
-    for (uint32_t it = 0; tile < num_tiles && ok; ++it) {
-      const int s = it % kFStages;
-      const uint32_t ph = (it / kFStages) & 1;
-      const RowFetch f = q[0];
-#pragma unroll
-      for (int i = 0; i + 1 < kFPrefetch; ++i) q[i] = q[i + 1];
-      q[kFPrefetch - 1] = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
-      advance(ptile, pkk, 1, nsteps);
-      if (*abort_flag || !mbar_wait(&empty[s], ph ^ 1)) { ok = false; break; }
-      if (kk < args.nk) {
-        uint8_t* brow = sB + s * kFB + R * 128;
-        const uint32_t sw = static_cast<uint32_t>(R & 7);
-        if (f.valid) {
-          const float a = args.sv.code8 == nullptr
-                              ? f.absv
-                              : __fadd_rn(__fmul_rn(t8[f.q], f.s2v), off);
-          uint32_t H[4], L[4];
-          build_lut(a, H, L);
-          const uint32_t pw[8] = {f.p0.x, f.p0.y, f.p0.z, f.p0.w,
-                                  f.p1.x, f.p1.y, f.p1.z, f.p1.w};
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(brow + ((static_cast<uint32_t>(c) ^ sw) << 4)) =
-                decode8(pw[c], H, L);
-        } else {
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(brow + (c << 4)) = make_uint4(0, 0, 0, 0);
-        }
-        fence_proxy_async_smem();
+    uint32_t ib = 0;
+    // One K-step: wait for a free weight stage, decode this thread's row.
+    auto step = [&](const RowFetch& f) {
+      const uint32_t s = ib % kFBStages, ph = (ib / kFBStages) & 1;
+      if (*abort_flag || !mbar_wait(&empty_b[s], ph ^ 1)) {
+        ok = false;
+        return;
       }
+      uint8_t* brow = sB + s * kFB + R * 128;
+      const uint32_t sw = static_cast<uint32_t>(R & 7);
+      if (f.valid) {
+        const float a = args.sv.code8 == nullptr
+                            ? f.absv
+                            : __fadd_rn(__fmul_rn(t8[f.q], f.s2v), off);
+        uint32_t H[4], L[4];
+        build_lut(a, H, L);
+        const uint32_t pw[8] = {f.p0.x, f.p0.y, f.p0.z, f.p0.w, f.p1.x, f.p1.y, f.p1.z, f.p1.w};
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(brow + ((static_cast<uint32_t>(c) ^ sw) << 4)) =
+              decode8(pw[c], H, L);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(brow + ((static_cast<uint32_t>(c) ^ sw) << 4)) =
+              make_uint4(0, 0, 0, 0);
+      }
+      fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&full_b[s]);
       advance(tile, kk, 1, nsteps);
+      ++ib;
+    };
+    // Three prefetch slots consumed and refilled in place (no register moves
+    // that would wait on loads still in flight).
+    RowFetch q0 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
+    advance(ptile, pkk, 1, nsteps);
+    RowFetch q1 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
+    advance(ptile, pkk, 1, nsteps);
+    RowFetch q2 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
+    advance(ptile, pkk, 1, nsteps);
+    while (ok && tile < num_tiles) {
+      step(q0);
+      q0 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
+      advance(ptile, pkk, 1, nsteps);
+      if (!ok || tile >= num_tiles) break;
+      step(q1);
+      q1 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
+      advance(ptile, pkk, 1, nsteps);
+      if (!ok || tile >= num_tiles) break;
+      step(q2);
+      q2 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
+      advance(ptile, pkk, 1, nsteps);
     }
     if (!ok) *abort_flag = 1;
   } else {
@@ -519,10 +573,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
         const int row = m0 + h * 128 + q * 32 + lane;
+        const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 256;
 #pragma unroll 1
         for (int c = 0; c < kFBN / 32; ++c) {
           uint32_t v[32];
-          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 256 + c * 32, v);
+          tmem_ld_32x32b_x32(tbase + c * 32, v);
           tmem_ld_wait();
           const int col = n0 + c * 32;
           if (row < args.M && col < args.Nout) {
@@ -537,10 +592,10 @@ __global__ void __launch_bounds__(kFThreads, 1)
                   pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[h]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tempty);
     }
     if (!ok) *abort_flag = 1;
   }
