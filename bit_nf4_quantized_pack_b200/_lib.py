@@ -21,6 +21,7 @@ QLORA_ERR_TIMEOUT = 6
 QLORA_DTYPE_BF16 = 0
 QLORA_DTYPE_F32 = 1
 ABI_VERSION = 1
+NOALLOC_MAX_NUMEL = 1 << 26
 
 
 class NF4StateC(C.Structure):
@@ -51,6 +52,7 @@ SIGNATURES = {
     "qlora_status_clear": (_I32, [_VP, _VP]),
     "qlora_nf4_quantize_workspace_size": (_SZ, [_I64, _I32]),
     "qlora_nf4_quantize": (_I32, [_VP, _I32, _PS, _VP, _SZ, _VP, _VP]),
+    "qlora_nf4_quantize_noalloc": (_I32, [_VP, _I32, _PS, _VP, _VP]),
     "qlora_nf4_dequantize": (_I32, [_PS, _VP, _VP, _VP]),
     "qlora_linear_fwd_workspace_size": (_SZ, [_I64, _I64, _I64, _I32]),
     "qlora_linear_fwd": (_I32, [_I64, _I64, _I64, _I32, _VP, _PS, _VP, _VP, _F, _VP, _VP,

@@ -137,6 +137,29 @@ qlora_status qlora_nf4_quantize(const void* W, qlora_dtype dtype, const qlora_nf
                                 qlora_stream_t stream);
 
 /*
+ * Allocation-free NF4 quantization (no counterpart on the pages: it is a
+ * property of this library, not of the method).  Same computation, arguments
+ * and errors as qlora_nf4_quantize, without the workspace: some callers cannot
+ * allocate device memory when they quantize (runtimes that plan every device
+ * buffer at start-up and forbid allocation in their steady state; plugins that
+ * only receive tensor pointers from a host framework).  The scratch it needs
+ * (2 KB of exponent bins plus one fp32 per 64-block, 4 MB at the limit) is a
+ * fixed array inside the library, allocated on each GPU that loads this part
+ * of the library and held until the process exits.
+ *   - numel must not exceed QLORA_NOALLOC_MAX_NUMEL, else QLORA_ERR_UNSUPPORTED.
+ *   - The first call on a device, made with that device current, looks up the
+ *     scratch's device address; make that first call before any stream
+ *     capture.
+ *   - All calls share the one scratch array (cleared where it must start at
+ *     zero by each call): calls that overlap on the GPU, from any stream or
+ *     thread, race with each other.  Serialize them.
+ */
+#define QLORA_NOALLOC_MAX_NUMEL (1ll << 26)
+qlora_status qlora_nf4_quantize_noalloc(const void* W, qlora_dtype dtype,
+                                        const qlora_nf4_state* st, int32_t* d_status,
+                                        qlora_stream_t stream);
+
+/*
  * NF4 dequantization — page "QLoRA：冻结的 4-bit 权重怎样参与一次微调",
  * §NF4 保存的是索引而不是均匀整数值 (reconstruction a·C_j) and §量化基座与可训练
  * 支路怎样相加 (BF16 compute type).
