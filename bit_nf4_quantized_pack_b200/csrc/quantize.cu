@@ -18,7 +18,7 @@ __constant__ float kNF4c[16] = {QNF4_TABLE_VALUES};
 // The rule is: code = argmin_j |w/s - C_j| with ties to the smaller index.
 // Since the table is sorted, that equals the number of midpoints
 // m_j = (C_j + C_{j+1})/2 strictly below w/s, i.e. #{j : w > s*m_j} (s > 0).
-// The fast path computes t = w * (1/s) in fp32 (absolute error < 2^-22) and
+// The fast path computes t = w * (1/s) in fp32 (absolute error < 2^-21) and
 // looks t up in 33 uniform buckets of width 1/16 that are offset by half a
 // bucket; every bucket holds at most one midpoint and no midpoint lies within
 // 0.004 of a bucket edge, so a bucket gives (number of midpoints below it,
@@ -54,130 +54,292 @@ __device__ __forceinline__ void build_buckets(Bucket* tab, double* mexact) {
     mexact[j] = 0.5 * (static_cast<double>(kNF4c[j]) + static_cast<double>(kNF4c[j + 1]));
 }
 
-__device__ __forceinline__ uint32_t nearest_code(float x, float s, float inv_s, const Bucket* tab,
-                                                 const double* mexact) {
-  const float t = x * inv_s;
-  int b = __float2int_rd(fmaf(t, 16.0f, 16.5f));
-  b = min(max(b, 0), kBuckets - 1);
-  const Bucket e = tab[b];
-  const float d = t - e.mid;
-  uint32_t code = static_cast<uint32_t>(e.jlo) + (d > 0.0f ? 1u : 0u);
-  if (fabsf(d) < kNearEps) {
-    const double thr = static_cast<double>(s) * mexact[e.jlo];
-    code = static_cast<uint32_t>(e.jlo) + (static_cast<double>(x) > thr ? 1u : 0u);
-  }
-  return code;
+// Exact decision for one element: code = jlo + (x > s*m_jlo) with the product
+// exact in fp64 (x, s already scaled alike).
+__device__ __forceinline__ uint32_t exact_code(float x, float s, int jlo, const double* mexact) {
+  return static_cast<uint32_t>(jlo) +
+         (static_cast<double>(x) > static_cast<double>(s) * mexact[jlo] ? 1u : 0u);
 }
 
+constexpr int kLaneElems = 16;   // consecutive elements per lane; 4 lanes per 64-block
+
 template <typename T>
-__device__ __forceinline__ void load8(const T* __restrict__ W, int64_t e0, int64_t numel, bool vec,
-                                      float (&x)[8]);
+__device__ __forceinline__ void load16(const T* __restrict__ W, int64_t e0, int64_t numel,
+                                       bool fast, float (&x)[kLaneElems]);
 
 template <>
-__device__ __forceinline__ void load8<uint16_t>(const uint16_t* __restrict__ W, int64_t e0,
-                                                int64_t numel, bool vec, float (&x)[8]) {
-  if (vec && e0 + 8 <= numel) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(W + e0));
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+__device__ __forceinline__ void load16<uint16_t>(const uint16_t* __restrict__ W, int64_t e0,
+                                                 int64_t numel, bool fast,
+                                                 float (&x)[kLaneElems]) {
+  if (fast) {
+    const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(W + e0));
+    const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(W + e0 + 8));
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 8; ++i) {
       x[2 * i] = __uint_as_float(w[i] << 16);
       x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < kLaneElems; ++i)
       x[i] = (e0 + i < numel) ? bf16_bits_to_f32(__ldg(W + e0 + i)) : 0.0f;
   }
 }
 
 template <>
-__device__ __forceinline__ void load8<float>(const float* __restrict__ W, int64_t e0, int64_t numel,
-                                             bool vec, float (&x)[8]) {
-  if (vec && e0 + 8 <= numel) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(W + e0));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(W + e0 + 4));
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+__device__ __forceinline__ void load16<float>(const float* __restrict__ W, int64_t e0,
+                                              int64_t numel, bool fast, float (&x)[kLaneElems]) {
+  if (fast) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(W + e0 + 4 * i));
+      x[4 * i] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
+    }
   } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) x[i] = (e0 + i < numel) ? __ldg(W + e0 + i) : 0.0f;
+    for (int i = 0; i < kLaneElems; ++i) x[i] = (e0 + i < numel) ? __ldg(W + e0 + i) : 0.0f;
   }
 }
 
-// One group of 8 lanes per 64-block; each lane owns 8 consecutive elements.
+// Per block-leader lane: the scales' exact sum per exponent is kept in two
+// (exponent, sum) register slots and only flushed to the CTA's shared bins
+// when a third exponent shows up, so the bins see few atomics.
+struct BinCache {
+  uint32_t k0 = 0, k1 = 0;
+  unsigned long long s0 = 0, s1 = 0;
+  __device__ __forceinline__ void add(float scale, unsigned long long* sbins) {
+    const uint32_t u = __float_as_uint(scale);
+    const uint32_t E = (u >> 23) & 0xFFu;
+    const uint32_t mant = (u & 0x7FFFFFu) | (E ? 0x800000u : 0u);
+    const uint32_t key = E ? E : 1u;
+    if (key == k0) {
+      s0 += mant;
+    } else if (key == k1) {
+      s1 += mant;
+    } else {
+      if (s1) atomicAdd(&sbins[k1], s1);
+      k1 = k0;
+      s1 = s0;
+      k0 = key;
+      s0 = mant;
+    }
+  }
+  __device__ __forceinline__ void flush(unsigned long long* sbins) {
+    if (s0) atomicAdd(&sbins[k0], s0);
+    if (s1) atomicAdd(&sbins[k1], s1);
+  }
+};
+
+// Encode the 16 elements x[] of one lane (lane `sub` of its 4-lane group,
+// elements e0..e0+15 of 64-block blk): absmax over the group, nearest codes,
+// packed store; the group leader stores the scale.
+//
+// Per element the fast path is: t = x/s by one multiply with an approximate
+// reciprocal; bucket = round(16 t + 16) by adding 2^23 + 16 (exact integer in
+// the low mantissa bits, no conversion instruction); one shared load of
+// (midpoint, codes below it); code = codes below + (t > midpoint) from the
+// sign of t - midpoint.  Exact fp64 decisions redo the rare elements within
+// 2^-20 of their midpoint (which includes t equal to it).
+template <bool kDQ>
+__device__ __forceinline__ void encode16(float (&x)[kLaneElems], int64_t blk, int64_t e0, int sub,
+                                         unsigned gmask, int64_t numel, bool full,
+                                         const Bucket* tab, const double* mexact,
+                                         uint8_t* __restrict__ packed, float* __restrict__ scales,
+                                         BinCache& bc, unsigned long long* sbins, bool& bad) {
+  float am = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kLaneElems; ++i) am = fmax_nan(am, fabsf(x[i]));
+  am = fmax_nan(am, __shfl_xor_sync(gmask, am, 1));
+  am = fmax_nan(am, __shfl_xor_sync(gmask, am, 2));
+  const bool finite = am <= FLT_MAX;
+  bad |= !finite;
+  const float s = (finite && am > 0.0f) ? am : 1.0f;
+  uint32_t w0 = 0x77777777u, w1 = 0x77777777u;   // all code 7 (non-finite blocks, padding)
+  if (finite) {
+    // Keep s and 1/s normal: a block scale below 2^-126 (1/s would overflow)
+    // is scaled up by 2^64, one above 2^126 (1/s would be subnormal) down by
+    // 2^-64, together with its elements; codes depend only on w/s, and an
+    // element that loses bits this way is far below any midpoint.
+    float s_eff = s;
+    if (s < 1.17549435e-38f || s > 8.50705917e37f) {
+      const float sc = s < 1.17549435e-38f ? 18446744073709551616.0f : 5.42101086e-20f;
+#pragma unroll
+      for (int i = 0; i < kLaneElems; ++i) x[i] *= sc;
+      s_eff = s * sc;
+    }
+    // relative error of t below 2^-21: inside the 2^-20 window of the exact check
+    float inv_s;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv_s) : "f"(s_eff));
+    const uint32_t tb = smem_u32(tab) - 0x4B000000u * 8u;   // (bits of 2^23 + b) * 8 + tb = &tab[b]
+    float dmin = 1.0f;
+    w0 = 0;
+    w1 = 0;
+#pragma unroll
+    for (int i = 0; i < kLaneElems; ++i) {
+      const float t = x[i] * inv_s;
+      const float y = fmaf(t, 16.0f, 8388624.0f);             // 2^23 + 16 + 16 t, rounded to an integer
+      float mid;
+      int jlo;
+      asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(mid), "=r"(jlo) : "r"(tb + __float_as_uint(y) * 8u));
+      const float d = t - mid;
+      const uint32_t code = static_cast<uint32_t>(jlo + 1 + (__float_as_int(d) >> 31));
+      dmin = fminf(dmin, fabsf(d));
+      const int sh = (i & 7) >> 1;
+      if (i < 8)
+        w0 += code << (sh * 8 + ((i & 1) ? 0 : 4));
+      else
+        w1 += code << (sh * 8 + ((i & 1) ? 0 : 4));
+    }
+    if (dmin < kNearEps) {
+      w0 = 0;
+      w1 = 0;
+#pragma unroll
+      for (int i = 0; i < kLaneElems; ++i) {
+        const float t = x[i] * inv_s;
+        const int b = __float2int_rd(fmaf(t, 16.0f, 16.5f));
+        const Bucket e = tab[b < 0 ? 0 : (b > kBuckets - 1 ? kBuckets - 1 : b)];
+        const float d = t - e.mid;
+        uint32_t code = static_cast<uint32_t>(e.jlo) + (d > 0.0f ? 1u : 0u);
+        if (fabsf(d) < kNearEps) code = exact_code(x[i], s_eff, e.jlo, mexact);
+        const int sh = (i & 7) >> 1;
+        if (i < 8)
+          w0 += code << (sh * 8 + ((i & 1) ? 0 : 4));
+        else
+          w1 += code << (sh * 8 + ((i & 1) ? 0 : 4));
+      }
+    }
+    if (!full) {
+#pragma unroll
+      for (int i = 0; i < kLaneElems; ++i)
+        if (e0 + i >= numel) {
+          const int sh = ((i & 7) >> 1) * 8 + ((i & 1) ? 0 : 4);
+          uint32_t& w = i < 8 ? w0 : w1;
+          w = (w & ~(0xFu << sh)) | (static_cast<uint32_t>(kPadCode) << sh);
+        }
+    }
+  }
+  const int64_t b0 = e0 >> 1;
+  if (full) {
+    *reinterpret_cast<uint2*>(packed + b0) = make_uint2(w0, w1);
+  } else {
+    const int64_t nbytes = (numel + 1) >> 1;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (b0 + k < nbytes) packed[b0 + k] = static_cast<uint8_t>((k < 4 ? w0 : w1) >> (8 * (k & 3)));
+  }
+  if (sub == 0) {
+    scales[blk] = s;
+    if (kDQ) bc.add(s, sbins);
+  }
+}
+
+constexpr int kChunkBlocks = 64;                 // 64-blocks per streamed chunk
+constexpr int kChunkElems = kChunkBlocks * kBlock;
+constexpr int kEncStages = 4;
+
+template <typename T>
+constexpr size_t encode_smem_bytes() {
+  return static_cast<size_t>(kEncStages) * kChunkElems * sizeof(T) + 128;
+}
+
+// CTA = 256 threads = 64 groups of 4 lanes = one chunk of 64 blocks per
+// iteration.  Whole chunks stream into a 4-stage shared-memory ring by 1-D
+// bulk copies; the remaining blocks (a partial last chunk, or everything when
+// W is not 16-byte aligned) are read directly from global memory.
 template <typename T, bool kDQ>
 __global__ void __launch_bounds__(256) nf4_encode_kernel(const T* __restrict__ W, int64_t numel,
                                                          int64_t n1, uint8_t* __restrict__ packed,
                                                          float* __restrict__ scales,
                                                          unsigned long long* __restrict__ bins,
                                                          int32_t* d_status) {
+  extern __shared__ uint8_t esm_raw[];
+  T* ring = reinterpret_cast<T*>((reinterpret_cast<uintptr_t>(esm_raw) + 127) &
+                                 ~static_cast<uintptr_t>(127));
   __shared__ Bucket tab[kBuckets];
   __shared__ double mexact[15];
   __shared__ unsigned long long sbins[kDQ ? 256 : 1];
+  __shared__ uint64_t full_bar[kEncStages];
+  __shared__ int abort_flag;
   build_buckets(tab, mexact);
   if (kDQ)
     for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = 0ull;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kEncStages; ++i) mbar_init(&full_bar[i], 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
   __syncthreads();
 
   const int lane = threadIdx.x & 31;
-  const int sub = lane & 7;
-  const unsigned gmask = 0xFFu << (lane & 24);
-  const bool vec = (reinterpret_cast<uintptr_t>(W) & 15u) == 0;
-  const int64_t nbytes = (numel + 1) >> 1;
-  const int64_t ngroups = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 3;
+  const int sub = lane & 3;
+  const unsigned gmask = 0xFu << (lane & 28);
+  const bool aligned16 = (reinterpret_cast<uintptr_t>(W) & 15u) == 0;
+  const int64_t nchunks = aligned16 ? numel / kChunkElems : 0;
+  const int64_t my_n =
+      nchunks > blockIdx.x ? (nchunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  constexpr uint32_t kChunkBytes = kChunkElems * sizeof(T);
+  BinCache bc;
   bool bad = false;
 
-  for (int64_t blk = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 3; blk < n1;
-       blk += ngroups) {
-    const int64_t e0 = blk * kBlock + sub * 8;
-    float x[8];
-    load8<T>(W, e0, numel, vec, x);
-    float am = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) am = fmax_nan(am, fabsf(x[i]));
-    am = fmax_nan(am, __shfl_xor_sync(gmask, am, 1));
-    am = fmax_nan(am, __shfl_xor_sync(gmask, am, 2));
-    am = fmax_nan(am, __shfl_xor_sync(gmask, am, 4));
-    const bool finite = am <= FLT_MAX;
-    bad |= !finite;
-    const float s = (finite && am > 0.0f) ? am : 1.0f;
-    // For a block scale below 2^-126, 1/s would overflow: scale the block and
-    // its scale by 2^64 (exact for these tiny values) so the fast path stays
-    // finite; codes depend only on the ratio w/s.
-    const bool tiny = s < 1.17549435e-38f;
-    const float sc = tiny ? 18446744073709551616.0f : 1.0f;
-    const float s_eff = s * sc;
-    const float inv_s = __frcp_rn(s_eff);
-    uint32_t word = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t code = (finite && e0 + i < numel)
-                                ? nearest_code(x[i] * sc, s_eff, inv_s, tab, mexact)
-                                : kPadCode;
-      // element 2k -> high nibble of byte k, element 2k+1 -> low nibble
-      word |= code << ((i >> 1) * 8 + ((i & 1) ? 0 : 4));
+  if (threadIdx.x == 0) {
+    for (int64_t j = 0; j < my_n && j < kEncStages; ++j) {
+      const int64_t c = blockIdx.x + j * gridDim.x;
+      mbar_arrive_expect_tx(&full_bar[j], kChunkBytes);
+      bulk_load_1d(ring + j * kChunkElems, W + c * kChunkElems, kChunkBytes, &full_bar[j]);
     }
-    const int64_t b0 = e0 >> 1;
-    if (e0 + 8 <= numel) {
-      *reinterpret_cast<uint32_t*>(packed + b0) = word;
+  }
+  for (int64_t j = 0; j < my_n; ++j) {
+    const int s = static_cast<int>(j % kEncStages);
+    const uint32_t ph = static_cast<uint32_t>((j / kEncStages) & 1);
+    if (!mbar_wait(&full_bar[s], ph)) abort_flag = 1;
+    __syncthreads();
+    if (abort_flag) break;
+    const int64_t c = blockIdx.x + j * gridDim.x;
+    const int local = threadIdx.x >> 2;
+    const int64_t blk = c * kChunkBlocks + local;
+    const int64_t e0 = blk * kBlock + sub * kLaneElems;
+    const T* src = ring + s * kChunkElems + local * kBlock + sub * kLaneElems;
+    float x[kLaneElems];
+    if (sizeof(T) == 2) {
+      const uint4 v0 = *reinterpret_cast<const uint4*>(src);
+      const uint4 v1 = *reinterpret_cast<const uint4*>(src + 8);
+      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
     } else {
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if (b0 + k < nbytes) packed[b0 + k] = static_cast<uint8_t>(word >> (8 * k));
-    }
-    if (sub == 0) {
-      scales[blk] = s;
-      if (kDQ) {
-        const uint32_t u = __float_as_uint(s);
-        const uint32_t E = (u >> 23) & 0xFFu;
-        const uint32_t mant = (u & 0x7FFFFFu) | (E ? 0x800000u : 0u);
-        atomicAdd(&sbins[E ? E : 1u], static_cast<unsigned long long>(mant));
+      for (int i = 0; i < 4; ++i) {
+        const float4 v = *reinterpret_cast<const float4*>(src + 4 * i);
+        x[4 * i] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
       }
     }
+    __syncthreads();   // every thread has its values: the stage may be refilled
+    if (threadIdx.x == 0 && j + kEncStages < my_n) {
+      const int64_t c2 = blockIdx.x + (j + kEncStages) * gridDim.x;
+      mbar_arrive_expect_tx(&full_bar[s], kChunkBytes);
+      bulk_load_1d(ring + s * kChunkElems, W + c2 * kChunkElems, kChunkBytes, &full_bar[s]);
+    }
+    encode16<kDQ>(x, blk, e0, sub, gmask, numel, true, tab, mexact, packed, scales, bc, sbins, bad);
+  }
+  if (abort_flag && threadIdx.x == 0) raise_status(d_status, QLORA_ERR_TIMEOUT);
+  // blocks not covered by whole streamed chunks
+  const int64_t first = nchunks * kChunkBlocks;
+  const int64_t ngroups = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 2;
+  for (int64_t blk = first + ((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 2);
+       blk < n1; blk += ngroups) {
+    const int64_t e0 = blk * kBlock + sub * kLaneElems;
+    const bool full = e0 + kLaneElems <= numel;
+    float x[kLaneElems];
+    load16<T>(W, e0, numel, full && aligned16, x);
+    encode16<kDQ>(x, blk, e0, sub, gmask, numel, full, tab, mexact, packed, scales, bc, sbins, bad);
   }
   if (bad) raise_status(d_status, QLORA_ERR_NONFINITE);
   if (kDQ) {
+    if (sub == 0) bc.flush(sbins);
     __syncthreads();
     for (int i = threadIdx.x; i < 256; i += blockDim.x)
       if (sbins[i]) atomicAdd(&bins[i], sbins[i]);
@@ -323,19 +485,21 @@ __global__ void __launch_bounds__(256) dq_mean_kernel(const unsigned long long* 
   *offset = __uint_as_float(bits);
 }
 
-// One CTA of 256 threads per group of 256 centred scales.  The 255 distinct
-// codebook values V_0 < ... < V_254 are: -|T|(127..1), 0, |T|(1..127); the
-// code of the nearest value to c/s2 (ties to the smaller value) is the number
-// k of midpoints (V_k + V_{k+1})/2 with s2 * mid < c, decided in fp64 where
-// s2 * mid is exact; k < 127 -> byte 0x80 | (127 - k), k = 127 -> 0x00,
-// k > 127 -> byte k - 127.
+// One warp per group of 256 centred scales (8 per lane, 8 groups per CTA).
+// The 255 distinct codebook values V_0 < ... < V_254 are: -|T|(127..1), 0,
+// |T|(1..127); the code of the nearest value to c/s2 (ties to the smaller
+// value) is the number k of midpoints m_k = (V_k + V_{k+1})/2 with
+// s2 * m_k < c.  s2 * m_k is exact in fp64, and for an fp32 c,
+// c > s2 * m_k  <=>  c > RD_fp32(s2 * m_k); so each warp turns its group's
+// 254 midpoints into fp32 thresholds once and counts them by binary search.
+// k < 127 -> byte 0x80 | (127 - k), k = 127 -> 0x00, k > 127 -> byte k - 127.
 __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict__ a, int64_t n1,
                                                         const float* __restrict__ offset_p,
                                                         uint8_t* __restrict__ code8,
                                                         float* __restrict__ s2) {
   __shared__ float mag[128];
   __shared__ double mid[254];
-  __shared__ float wmax[8];
+  __shared__ float thr[8][256];
   for (int t = threadIdx.x; t < 128; t += blockDim.x) mag[t] = t8_magnitude(t);
   __syncthreads();
   for (int k = threadIdx.x; k < 254; k += blockDim.x) {
@@ -345,33 +509,50 @@ __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict_
     };
     mid[k] = 0.5 * (V(k) + V(k + 1));
   }
-  const int64_t g = blockIdx.x;
-  const int64_t i = g * kDQBlock + threadIdx.x;
-  const float off = *offset_p;
-  const bool valid = i < n1;
-  const float c = valid ? __fsub_rn(a[i], off) : 0.0f;
-  float m = fabsf(c);
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
   __syncthreads();
-  float sg = wmax[0];
-  for (int w = 1; w < 8; ++w) sg = fmaxf(sg, wmax[w]);
-  if (!(sg > 0.0f)) sg = 1.0f;
-  if (threadIdx.x == 0) s2[g] = sg;
-  if (!valid) return;
-  const double cd = static_cast<double>(c), sd = static_cast<double>(sg);
-  int lo = 0, hi = 254;  // find the first k with sd*mid[k] >= cd
-  while (lo < hi) {
-    const int md = (lo + hi) >> 1;
-    if (sd * mid[md] < cd)
-      lo = md + 1;
-    else
-      hi = md;
+  const float off = *offset_p;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float* T = thr[warp];
+  const int64_t n2 = (n1 + kDQBlock - 1) / kDQBlock;
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * 8 + warp; g < n2;
+       g += static_cast<int64_t>(gridDim.x) * 8) {
+    float c[8];
+    float m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t i = g * kDQBlock + j * 32 + lane;
+      c[j] = i < n1 ? __fsub_rn(__ldg(a + i), off) : 0.0f;
+      m = fmaxf(m, fabsf(c[j]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    const float sg = m > 0.0f ? m : 1.0f;
+    if (lane == 0) s2[g] = sg;
+    const double sd = static_cast<double>(sg);
+    __syncwarp();                     // previous group's searches are done with T
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int k = j * 32 + lane;
+      if (k < 254) T[k] = __double2float_rd(sd * mid[k]);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t i = g * kDQBlock + j * 32 + lane;
+      int lo = 0, hi = 254;           // the first k with T[k] >= c
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        const int md = min((lo + hi) >> 1, 253);   // < 254 whenever lo < hi
+        const bool less = T[md] < c[j];
+        lo = (lo < hi && less) ? md + 1 : lo;
+        hi = (lo < hi && !less) ? md : hi;
+      }
+      const int k = lo;
+      if (i < n1)
+        code8[i] = static_cast<uint8_t>(k < 127 ? (0x80u | static_cast<uint32_t>(127 - k))
+                                                : (k == 127 ? 0u : static_cast<uint32_t>(k - 127)));
+    }
   }
-  const int k = lo;
-  const uint32_t byte = k < 127 ? (0x80u | static_cast<uint32_t>(127 - k))
-                                : (k == 127 ? 0u : static_cast<uint32_t>(k - 127));
-  code8[i] = static_cast<uint8_t>(byte);
 }
 
 // ---------------------------------------------------------------------------
@@ -382,8 +563,7 @@ cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* pa
                             void* ws, int32_t* d_status, cudaStream_t st, int num_sms) {
   const int64_t n1 = (numel + kBlock - 1) / kBlock;
   const int threads = 256;
-  const int64_t want = (n1 * 8 + threads - 1) / threads;
-  const int blocks = static_cast<int>(want < num_sms * 8LL ? want : num_sms * 8LL);
+  const int64_t want = (n1 * 4 + threads - 1) / threads;
   unsigned long long* bins = nullptr;
   float* scales = absmax_out;
   if (dq) {
@@ -394,19 +574,47 @@ cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* pa
   }
   {
   ProfScope prof(kProfQuantize, st);
+  // one wave of resident CTAs (each loops over chunks)
+  static int per_sm[4] = {0, 0, 0, 0};
+  {
+    static bool attr_done = false;
+    if (!attr_done) {
+      const int b16 = static_cast<int>(encode_smem_bytes<uint16_t>());
+      const int b32 = static_cast<int>(encode_smem_bytes<float>());
+      const void* fns[4] = {reinterpret_cast<const void*>(nf4_encode_kernel<uint16_t, false>),
+                            reinterpret_cast<const void*>(nf4_encode_kernel<uint16_t, true>),
+                            reinterpret_cast<const void*>(nf4_encode_kernel<float, false>),
+                            reinterpret_cast<const void*>(nf4_encode_kernel<float, true>)};
+      for (int i = 0; i < 4; ++i) {
+        const int bytes = i < 2 ? b16 : b32;
+        cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        cudaFuncSetAttribute(fns[i], cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        int nb = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fns[i], threads, bytes) != cudaSuccess || nb < 1)
+          nb = 1;
+        per_sm[i] = nb;
+      }
+      attr_done = true;
+    }
+  }
+  const int kind = (dtype == QLORA_DTYPE_BF16 ? 0 : 2) + (dq ? 1 : 0);
+  const int64_t cap = static_cast<int64_t>(num_sms) * per_sm[kind];
+  const int blocks = static_cast<int>(want < cap ? want : cap);
   if (dtype == QLORA_DTYPE_BF16) {
+    const size_t sm = encode_smem_bytes<uint16_t>();
     if (dq)
-      nf4_encode_kernel<uint16_t, true><<<blocks, threads, 0, st>>>(
+      nf4_encode_kernel<uint16_t, true><<<blocks, threads, sm, st>>>(
           static_cast<const uint16_t*>(W), numel, n1, packed, scales, bins, d_status);
     else
-      nf4_encode_kernel<uint16_t, false><<<blocks, threads, 0, st>>>(
+      nf4_encode_kernel<uint16_t, false><<<blocks, threads, sm, st>>>(
           static_cast<const uint16_t*>(W), numel, n1, packed, scales, bins, d_status);
   } else {
+    const size_t sm = encode_smem_bytes<float>();
     if (dq)
-      nf4_encode_kernel<float, true><<<blocks, threads, 0, st>>>(
+      nf4_encode_kernel<float, true><<<blocks, threads, sm, st>>>(
           static_cast<const float*>(W), numel, n1, packed, scales, bins, d_status);
     else
-      nf4_encode_kernel<float, false><<<blocks, threads, 0, st>>>(
+      nf4_encode_kernel<float, false><<<blocks, threads, sm, st>>>(
           static_cast<const float*>(W), numel, n1, packed, scales, bins, d_status);
   }
   }
@@ -419,7 +627,9 @@ cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* pa
   const int64_t n2 = (n1 + kDQBlock - 1) / kDQBlock;
   {
     ProfScope prof(kProfQuantize, st);
-    dq_encode_kernel<<<static_cast<unsigned>(n2), 256, 0, st>>>(scales, n1, offset, code8, s2);
+    const int64_t want_g = (n2 + 7) / 8;
+    const int64_t grid = want_g < num_sms * 8LL ? want_g : num_sms * 8LL;
+    dq_encode_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(scales, n1, offset, code8, s2);
   }
   return cudaGetLastError();
 }
