@@ -292,6 +292,41 @@ def quantize_bench(torch, q, dev, peaks):
     return {"shape": [Kq, Nq], "us": per * 1e6, "GB/s": gbs, "frac": gbs / peaks["hbm"]}
 
 
+def run_case(args):
+    """One kernel workload, --reps launches, no timing: the command ncu captures.
+    gemv: forward with M <= 16 tokens (DQ weight, r = 16, c = 2);
+    quantize: NF4 + DQ quantization of a K x N bf16 weight."""
+    import torch
+    import bit_nf4_quantized_pack_b200 as q
+    dev = torch.device("cuda", 0)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(11)
+    st = q.new_status(dev)
+    if args.case == "gemv":
+        Mg, Kg, Ng = (int(v) for v in (args.shape or "1,4096,11008").split(","))
+        # two weights, alternated, so no launch reads the previous one from L2
+        ws = []
+        for _ in range(2):
+            W = (torch.randn((Kg, Ng), generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+            ws.append(q.quantize(W, double_quant=True, status=st))
+            del W
+        A = (torch.randn((Kg, 16), generator=gen, device=dev) * 0.01).to(torch.bfloat16)
+        B = (torch.randn((16, Ng), generator=gen, device=dev) * 0.01).to(torch.bfloat16)
+        X = torch.randn((Mg, Kg), generator=gen, device=dev).to(torch.bfloat16)
+        for i in range(args.reps):
+            q.linear_forward(X, ws[i % 2], A, B, 2.0, status=st)
+    else:
+        Kq, Nq = (int(v) for v in (args.shape or "8192,22016").split(","))
+        W = (torch.randn((Kq, Nq), generator=gen, device=dev) * 0.015).to(torch.bfloat16)
+        w = q.quantize(W, double_quant=True, status=st)
+        for _ in range(args.reps):
+            q.quantize(W, double_quant=True, out=w, status=st)
+    torch.cuda.synchronize()
+    code = q.status_sync(st)
+    print(json.dumps({"case": args.case, "shape": args.shape, "reps": args.reps, "status": list(code)}))
+    return 0 if code[0] == 0 else 1
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -301,9 +336,16 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the GEMV and quantize sweeps")
     ap.add_argument("--kernels-only", action="store_true",
                     help="only the timed steps (no e2e, sweeps or CPU baseline): for profilers")
+    ap.add_argument("--case", choices=["gemv", "quantize"],
+                    help="run one kernel workload --reps times and exit (for profilers)")
+    ap.add_argument("--shape", default="",
+                    help="M,K,N for --case gemv (default 1,4096,11008); K,N for --case quantize")
+    ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.case:
+        return run_case(args)
 
     import torch
     import torch.distributed as dist

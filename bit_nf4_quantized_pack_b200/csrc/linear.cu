@@ -629,12 +629,42 @@ __global__ void __launch_bounds__(kFThreads, 1)
 // x * bf16(C a') by at most a bf16 rounding of each factor (relative 2^-8 per
 // product); over K terms the relative error of y stays near 3e-3.
 //
-// CTA = 256 weight columns (four 64-column blocks) x a K-range; warp w works
-// on block w & 3 and every other 16-row step (w >> 2) of the range; the two
-// warps of a block are added through shared memory and the CTA writes one fp32
-// partial per split; gemv_reduce_kernel adds the splits and Zc·B.
+// CTA = 256 weight columns x a K-range, one CTA per SM.  A producer warp
+// streams 128-row stages (packed 128 x 128 bytes and X 16 x 128 bf16, both by
+// TMA with the 128-byte swizzle) through a 6-stage ring; sixteen compute warps
+// cover a stage as 4 column blocks of 64 x 4 row slots, each slot two 16-row
+// steps 64 rows apart, and the four partial sums per block are added through
+// shared memory into one fp32 partial per split.  Each lane keeps the scale
+// loads of the next four stages in flight (lanes 0-15 the first step's rows,
+// lanes 16-31 the second's), so their latency never reaches the decode.
+// The stages also carry an 8-column slice of A: column group cg owns rank
+// columns [8cg, 8cg+8), and the warps of the first column block add that
+// slice of X·A with one more mma per step, using the raw activation fragment;
+// gemv_finish_kernel turns these partials into Zc = bf16(c·X·A) and adds the
+// splits and Zc·B.  The decode table sits at the start of the dynamic shared
+// window, so its base is a constant of the load instruction.
 // ===========================================================================
-constexpr int kGvTable = 65536;  // 256 entries x 64 words (32 used) x 4 B
+constexpr int kGvTable = 65536;        // 256 entries x 64 words (32 used) x 4 B
+constexpr int kGvRows = 128;           // k rows per stage
+constexpr int kGvStages = 6;
+constexpr int kGvPk = kGvRows * 128;   // packed weights of a stage
+constexpr int kGvXb = 2 * 2048;        // 16 tokens x 128 k bf16, two swizzled 64-k halves
+constexpr int kGvAb = kGvRows * 16;    // 128 k x 8 rank columns of A (bf16)
+constexpr int kGvCompute = 16;         // compute warps
+constexpr int kGvThreads = (kGvCompute + 1) * 32;
+constexpr int kGvAhead = 4;            // stages of scale loads in flight per lane
+constexpr size_t kGvSmem =
+    kGvTable + 1024 + kGvStages * (kGvPk + kGvXb + kGvAb) + 3 * 16 * 8 * 4 + 1024 + 256;
+static_assert(4 * 3 * 16 * 64 * 4 <= kGvStages * kGvPk, "block sums reuse the packed ring");
+
+struct GemvArgs {
+  int M, K, N, r;
+  int stages_per_split;   // 64-row stages per split
+  ScaleView sv;
+  float* partial;         // [splits][M][N]
+  float* zpart;           // [splits][M][r], or null when Zc is computed elsewhere
+  int32_t* d_status;
+};
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
                                                uint32_t b0, uint32_t b1) {
@@ -651,146 +681,346 @@ __device__ __forceinline__ uint32_t lds32(uint32_t saddr) {
   return v;
 }
 
-template <bool kM16>
-__global__ void __launch_bounds__(256, 2) nf4_gemv_kernel(const uint16_t* __restrict__ X, int M,
-                                                          int K, int N,
-                                                          const uint8_t* __restrict__ packed,
-                                                          ScaleView sv, int steps_per_split,
-                                                          float* __restrict__ partial) {
-  extern __shared__ uint8_t gsm_raw[];
-  uint8_t* gsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsm_raw) + 255) &
-                                            ~static_cast<uintptr_t>(255));
-  uint32_t* table = reinterpret_cast<uint32_t*>(gsm);
-  float* t8 = reinterpret_cast<float*>(gsm + kGvTable);
-  float* red = t8 + 256;                       // [4 blocks][16 m][64 cols]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // fixed table: entry e -> (bf16(C[e >> 4]) | bf16(C[e & 15]) << 16), 32 copies
-  for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) {
-    const int e = i >> 5, c = i & 31;
-    table[e * 64 + c] = pack_bf16x2(kNF4g[e >> 4], kNF4g[e & 15]);
-  }
-  if (sv.code8 != nullptr) build_t8(t8);
-  __syncthreads();
-  const float off = sv.code8 != nullptr ? __ldg(sv.offset) : 0.0f;
-  const int g = lane >> 2, t = lane & 3;
-  const int blk = blockIdx.x * 4 + (warp & 3);          // 64-column block
-  const bool colok = blk * 64 < N;
-  const int bpr = N / 64;
-  const int step0 = blockIdx.y * steps_per_split;
-  const int step1 = min(K / 16, step0 + steps_per_split);
-  const uint32_t tbase = smem_u32(table);
-  const uint32_t laneword = lane * 4;                    // byte 0 of the address
-  float acc[8][4];
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[j][i] = 0.0f;
+__device__ __forceinline__ uint32_t lds16(uint32_t saddr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(saddr));
+  return v;
+}
 
-  if (colok) {
-    const uint8_t* pcol = packed + blk * 32 + g * 4;    // this thread's packed word in a row
-    for (int st = step0 + (warp >> 2); st < step1; st += 2) {
-      const int kb = st * 16;
-      // block scales of rows kb..kb+15: lane i < 16 decodes row kb+i
-      float sc = 0.0f;
-      if (lane < 16) {
-        const int64_t b = static_cast<int64_t>(kb + lane) * bpr + blk;
-        sc = sv.code8 == nullptr
-                 ? __ldg(sv.absmax + b)
-                 : __fadd_rn(__fmul_rn(t8[__ldg(sv.code8 + b)], __ldg(sv.s2 + (b >> 8))), off);
+// Scale a'[row][blk] for the GEMV in two halves: the raw loads (issued where
+// called, several stages ahead) and the decode once they are needed.
+struct GvScale {
+  uint32_t q;   // code8 (double quantization)
+  float v;      // s2 of the block's 256-group, or the fp32 absmax
+};
+
+__device__ __forceinline__ GvScale gemv_scale_load(const ScaleView& sv, int64_t b) {
+  GvScale r;
+  r.q = 0u;
+  if (sv.code8 == nullptr) {
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(r.v) : "l"(sv.absmax + b));
+  } else {
+    uint16_t q;
+    asm volatile("ld.global.nc.u8 %0, [%1];" : "=h"(q) : "l"(sv.code8 + b));
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(r.v) : "l"(sv.s2 + (b >> 8)));
+    r.q = q;
+  }
+  return r;
+}
+
+__device__ __forceinline__ float gemv_scale_value(const ScaleView& sv, const GvScale& r, float off,
+                                                  const float* t8) {
+  if (sv.code8 == nullptr) return r.v;
+  return __fadd_rn(__fmul_rn(t8[r.q], r.v), off);
+}
+
+template <int kOff>
+__device__ __forceinline__ uint32_t lds32_at(uint32_t saddr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1+%2];" : "=r"(v) : "r"(saddr), "n"(kOff));
+  return v;
+}
+
+template <bool kM16>
+__global__ void __launch_bounds__(kGvThreads, 1)
+    nf4_gemv_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmX,
+                    const __grid_constant__ CUtensorMap tmA, GemvArgs args) {
+  extern __shared__ uint8_t gsm_raw[];
+  uint32_t* table = reinterpret_cast<uint32_t*>(gsm_raw);
+  uint8_t* gsm = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(gsm_raw + kGvTable) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sP = gsm;
+  uint8_t* sX = sP + kGvStages * kGvPk;
+  uint8_t* sAl = sX + kGvStages * kGvXb;
+  float* zred = reinterpret_cast<float*>(sAl + kGvStages * kGvAb);   // [3][16][8]
+  float* t8 = zred + 3 * 16 * 8;
+  uint64_t* full = reinterpret_cast<uint64_t*>(t8 + 256);
+  uint64_t* empty = full + kGvStages;
+  float* red = reinterpret_cast<float*>(sP);   // [4][3][16][64], after the last stage
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == kGvCompute * 32) {
+    for (int s = 0; s < kGvStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kGvCompute);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int M = args.M, N = args.N, K = args.K;
+  const int cg = blockIdx.x;                            // 256-column group
+  const int st0 = blockIdx.y * args.stages_per_split;
+  const int nst = min((K + kGvRows - 1) / kGvRows, st0 + args.stages_per_split) - st0;
+  bool ok = true;
+
+  if (warp == kGvCompute) {
+    // --------------------------------- producer ---------------------------------
+    // starts streaming while the compute warps build their tables; rows past K
+    // (a last stage of 64 rows) arrive as zeros
+    if (lane == 0) {
+      tma_prefetch_desc(&tmP);
+      tma_prefetch_desc(&tmX);
+      tma_prefetch_desc(&tmA);
+      auto issue = [&](int j, int s) {
+        const int k0 = (st0 + j) * kGvRows;
+        mbar_arrive_expect_tx(&full[s], kGvPk + kGvXb + kGvAb);
+        tma_load_2d(sP + s * kGvPk, &tmP, &full[s], cg * 128, k0);
+        tma_load_2d(sX + s * kGvXb, &tmX, &full[s], k0, 0);
+        tma_load_2d(sX + s * kGvXb + 2048, &tmX, &full[s], k0 + 64, 0);
+        tma_load_2d(sAl + s * kGvAb, &tmA, &full[s], cg * 8, k0);
+      };
+      for (int j = 0; j < nst && j < kGvStages; ++j) issue(j, j);
+      for (int j = 0; j + kGvStages < nst && ok; ++j) {
+        const int s = j % kGvStages;
+        const uint32_t ph = (j / kGvStages) & 1;
+        if (!mbar_wait(&empty[s], ph)) { ok = false; break; }
+        issue(j + kGvStages, s);
       }
-      const float s0 = __shfl_sync(0xFFFFFFFFu, sc, 2 * t);
-      const float s1 = __shfl_sync(0xFFFFFFFFu, sc, 2 * t + 1);
-      const float s2 = __shfl_sync(0xFFFFFFFFu, sc, 2 * t + 8);
-      const float s3 = __shfl_sync(0xFFFFFFFFu, sc, 2 * t + 9);
-      // activation fragment, scaled per row
-      uint32_t a[4] = {0u, 0u, 0u, 0u};
-      if (g < M) {
-        const uint16_t* xr = X + static_cast<int64_t>(g) * K + kb + 2 * t;
-        const uint32_t x0 = __ldg(reinterpret_cast<const uint32_t*>(xr));
-        const uint32_t x1 = __ldg(reinterpret_cast<const uint32_t*>(xr + 8));
-        a[0] = pack_bf16x2(__uint_as_float(x0 << 16) * s0, __uint_as_float(x0 & 0xFFFF0000u) * s1);
-        a[2] = pack_bf16x2(__uint_as_float(x1 << 16) * s2, __uint_as_float(x1 & 0xFFFF0000u) * s3);
+    }
+  } else {
+    // ------------------------------ compute warps ------------------------------
+    // fixed table: entry e -> (bf16(C[e >> 4]) | bf16(C[e & 15]) << 16), one
+    // copy per bank so that 32 lanes reading any entries never conflict
+    {
+      const float cv = kNF4g[lane & 15];
+      for (int e = warp; e < 256; e += kGvCompute)   // entry e is written by one warp
+        table[e * 64 + lane] =
+            pack_bf16x2(__shfl_sync(0xFFFFFFFFu, cv, e >> 4), __shfl_sync(0xFFFFFFFFu, cv, e & 15));
+    }
+    if (args.sv.code8 != nullptr) {
+      for (int u = threadIdx.x; u < 256; u += kGvCompute * 32) {
+        const float v = t8_magnitude(u & 127);
+        t8[u] = (u >> 7) ? -v : v;
       }
-      if (kM16 && g + 8 < M) {
-        const uint16_t* xr = X + static_cast<int64_t>(g + 8) * K + kb + 2 * t;
-        const uint32_t x0 = __ldg(reinterpret_cast<const uint32_t*>(xr));
-        const uint32_t x1 = __ldg(reinterpret_cast<const uint32_t*>(xr + 8));
-        a[1] = pack_bf16x2(__uint_as_float(x0 << 16) * s0, __uint_as_float(x0 & 0xFFFF0000u) * s1);
-        a[3] = pack_bf16x2(__uint_as_float(x1 << 16) * s2, __uint_as_float(x1 & 0xFFFF0000u) * s3);
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kGvCompute * 32) : "memory");   // compute warps only
+
+    const int b = warp & 3, p = warp >> 2;             // column block, row slot
+    const int blk = cg * 4 + b;                        // 64-column block
+    const bool colok = blk * 64 < N;
+    const int g = lane >> 2, t = lane & 3;
+    const int bpr = N / 64;
+    const int kb = 16 * p;                             // rows kb.. and kb+64.. of a stage
+    const float off = args.sv.code8 != nullptr ? __ldg(args.sv.offset) : 0.0f;
+    const uint32_t tbase = smem_u32(gsm_raw);
+    const uint32_t laneword = lane * 4;
+    // Per-lane shared offsets, fixed for the whole loop.  Packed stage (128-byte
+    // swizzle, row R at R*128, 16-byte chunk c at (c ^ (R & 7))*16): this lane
+    // reads the 4 bytes of columns 8g..8g+7 of block b in rows kb+2t, kb+2t+1
+    // and the same rows +8, +64 and +72 (all with the same swizzle phase).
+    const uint32_t cw = static_cast<uint32_t>(2 * b + (g >> 2));
+    const uint32_t wo = static_cast<uint32_t>((g & 3) * 4);
+    const uint32_t r0 = static_cast<uint32_t>(kb + 2 * t);
+    const uint32_t poff0 = r0 * 128 + ((cw ^ (r0 & 7)) << 4) + wo;
+    const uint32_t poff1 = (r0 + 1) * 128 + ((cw ^ ((r0 + 1) & 7)) << 4) + wo;
+    // X stage (two halves of 16 tokens x 64 k, swizzled): token g,
+    // k = kb + 2t (+1) and kb + 8 + 2t (+1), the second step 2048 bytes on
+    const uint32_t c0 = static_cast<uint32_t>(kb >> 3);
+    const uint32_t xoff0 = g * 128 + ((c0 ^ static_cast<uint32_t>(g)) << 4) + t * 4;
+    const uint32_t xoff1 = g * 128 + (((c0 + 1) ^ static_cast<uint32_t>(g)) << 4) + t * 4;
+    const uint32_t aoff = static_cast<uint32_t>((kb + 2 * t) * 16 + g * 2);   // A slice
+    const uint32_t sP0 = smem_u32(sP), sX0 = smem_u32(sX), sA0 = smem_u32(sAl);
+
+    // acc[f]: mma f covers weight columns 8g+2f (rows g) and 8g+2f+1 (rows g+8)
+    // against tokens 2t, 2t+1 (acc2: tokens 8+2t, 9+2t)
+    float acc[4][4], acc2[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[j][i] = acc2[j][i] = 0.0f;
+    float xa[4] = {0.0f, 0.0f, 0.0f, 0.0f};            // X·A slice (warps of block 0)
+    const bool do_xa = b == 0 && args.zpart != nullptr && cg * 8 < args.r;
+    // this lane's scale row inside a stage: kb + (lane & 15), second step for lanes 16-31
+    const int srow = kb + 64 * (lane >> 4) + (lane & 15);
+    auto scale_at = [&](int j) -> GvScale {
+      GvScale z;
+      z.q = 0u;
+      z.v = 0.0f;
+      const int row = (st0 + j) * kGvRows + srow;
+      if (colok && row < K) z = gemv_scale_load(args.sv, static_cast<int64_t>(row) * bpr + blk);
+      return z;
+    };
+    GvScale ring[kGvAhead];
+#pragma unroll
+    for (int u = 0; u < kGvAhead; ++u) {
+      ring[u].q = 0u;
+      ring[u].v = 0.0f;
+      if (u < nst) ring[u] = scale_at(u);
+    }
+
+    // one 16-row step h (0: rows kb.., 1: rows kb+64..) of stage slot s
+    auto step = [&](uint32_t ps, uint32_t xs, uint32_t as, float sc, int h) {
+      const uint32_t w0 = lds32(ps + poff0), w8 = lds32(ps + poff0 + 1024);
+      const uint32_t w1 = lds32(ps + poff1), w9 = lds32(ps + poff1 + 1024);
+      const uint32_t x0 = lds32(xs + xoff0), x1 = lds32(xs + xoff1);
+      const float s0 = __shfl_sync(0xFFFFFFFFu, sc, 16 * h + 2 * t);
+      const float s1 = __shfl_sync(0xFFFFFFFFu, sc, 16 * h + 2 * t + 1);
+      const float s2 = __shfl_sync(0xFFFFFFFFu, sc, 16 * h + 2 * t + 8);
+      const float s3 = __shfl_sync(0xFFFFFFFFu, sc, 16 * h + 2 * t + 9);
+      // B fragments: scaled activations of token g (and g + 8)
+      const uint32_t bx0 = pack_bf16x2(__uint_as_float(x0 << 16) * s0, __uint_as_float(x0 & 0xFFFF0000u) * s1);
+      const uint32_t bx1 = pack_bf16x2(__uint_as_float(x1 << 16) * s2, __uint_as_float(x1 & 0xFFFF0000u) * s3);
+      uint32_t y0 = 0u, y1 = 0u, by0 = 0u, by1 = 0u;
+      if (kM16) {
+        y0 = lds32(xs + xoff0 + 1024);
+        y1 = lds32(xs + xoff1 + 1024);
+        by0 = pack_bf16x2(__uint_as_float(y0 << 16) * s0, __uint_as_float(y0 & 0xFFFF0000u) * s1);
+        by1 = pack_bf16x2(__uint_as_float(y1 << 16) * s2, __uint_as_float(y1 & 0xFFFF0000u) * s3);
       }
-      // packed words of rows kb+2t, kb+2t+1, kb+2t+8, kb+2t+9 (columns 8g..8g+7)
-      const int64_t rb = static_cast<int64_t>(N) / 2;
-      const uint8_t* p = pcol + static_cast<int64_t>(kb + 2 * t) * rb;
-      const uint32_t w0 = __ldg(reinterpret_cast<const uint32_t*>(p));
-      const uint32_t w1 = __ldg(reinterpret_cast<const uint32_t*>(p + rb));
-      const uint32_t w8 = __ldg(reinterpret_cast<const uint32_t*>(p + 8 * rb));
-      const uint32_t w9 = __ldg(reinterpret_cast<const uint32_t*>(p + 9 * rb));
+      if (do_xa) {
+        // raw activations (tokens as rows) against A[k][8cg + g]
+        const uint32_t ab0 = lds16(as) | (lds16(as + 16) << 16);
+        const uint32_t ab1 = lds16(as + 128) | (lds16(as + 144) << 16);
+        const uint32_t araw[4] = {x0, y0, x1, y1};
+        mma_bf16_16816(xa, araw, ab0, ab1);
+      }
       // bytes (row k nibble, row k+1 nibble) per column: even and odd columns
       const uint32_t lo_e = (w0 & 0xF0F0F0F0u) | ((w1 >> 4) & 0x0F0F0F0Fu);
       const uint32_t lo_o = ((w0 << 4) & 0xF0F0F0F0u) | (w1 & 0x0F0F0F0Fu);
       const uint32_t hi_e = (w8 & 0xF0F0F0F0u) | ((w9 >> 4) & 0x0F0F0F0Fu);
       const uint32_t hi_o = ((w8 << 4) & 0xF0F0F0F0u) | (w9 & 0x0F0F0F0Fu);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        // offset (byte i << 8) | lane*4: output byte 0 <- lane*4 (source byte
-        // 4), byte 1 <- byte i of the word, bytes 2 and 3 <- zero (source byte 5)
-        const uint32_t sel = 0x5504u | (static_cast<uint32_t>(i) << 4);
-        const uint32_t b0e = lds32(tbase + prmt(lo_e, laneword, sel));
-        const uint32_t b1e = lds32(tbase + prmt(hi_e, laneword, sel));
-        const uint32_t b0o = lds32(tbase + prmt(lo_o, laneword, sel));
-        const uint32_t b1o = lds32(tbase + prmt(hi_o, laneword, sel));
-        mma_bf16_16816(acc[2 * i], a, b0e, b1e);
-        mma_bf16_16816(acc[2 * i + 1], a, b0o, b1o);
+      for (int f = 0; f < 4; ++f) {
+        // offset (byte f << 8) | lane*4: output byte 0 <- lane*4 (source byte
+        // 4), byte 1 <- byte f of the word, bytes 2 and 3 <- zero (source byte 5)
+        const uint32_t sel = 0x5504u | (static_cast<uint32_t>(f) << 4);
+        uint32_t wa[4];
+        wa[0] = lds32(tbase + prmt(lo_e, laneword, sel));   // column 8g+2f, k 2t..
+        wa[1] = lds32(tbase + prmt(lo_o, laneword, sel));   // column 8g+2f+1
+        wa[2] = lds32(tbase + prmt(hi_e, laneword, sel));   // column 8g+2f, k 2t+8..
+        wa[3] = lds32(tbase + prmt(hi_o, laneword, sel));
+        mma_bf16_16816(acc[f], wa, bx0, bx1);
+        if (kM16) mma_bf16_16816(acc2[f], wa, by0, by1);
+      }
+    };
+
+    for (int j0 = 0; j0 < nst && ok; j0 += kGvAhead) {
+#pragma unroll
+      for (int u = 0; u < kGvAhead; ++u) {
+        const int j = j0 + u;
+        if (j >= nst || !ok) break;
+        const int s = j % kGvStages;
+        const uint32_t ph = (j / kGvStages) & 1;
+        const float sc = gemv_scale_value(args.sv, ring[u], off, t8);
+        if (j + kGvAhead < nst) ring[u] = scale_at(j + kGvAhead);
+        if (!mbar_wait(&full[s], ph)) { ok = false; break; }
+        if (colok) {
+          const uint32_t ps = sP0 + s * kGvPk, xs = sX0 + s * kGvXb, as = sA0 + s * kGvAb + aoff;
+          step(ps, xs, as, sc, 0);
+          step(ps + 64 * 128, xs + 2048, as + 64 * 16, sc, 1);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
       }
     }
-  }
-  // add the two warps of each block, then write this split's partial
-  float* myred = red + (warp & 3) * (16 * 64);
-  if (warp >= 4) {
+    // every compute warp is past its last stage (and so every stage has
+    // landed) before the block sums overwrite the packed ring
+    asm volatile("bar.sync 1, %0;" ::"n"(kGvCompute * 32) : "memory");
+    // add the four row-slot warps of each block, then write this split's partial
+    // red[b][p-1][token][64 columns]
+    auto put = [&](float* dst, const float (&v)[4][4], int tok0) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      // acc[j]: (row g, cols 2t, 2t+1), (row g+8, ...) of n-tile j; column
-      // index c of n-tile j is weight column 8c + j
-      myred[g * 64 + 8 * (2 * t) + j] = acc[j][0];
-      myred[g * 64 + 8 * (2 * t + 1) + j] = acc[j][1];
-      myred[(g + 8) * 64 + 8 * (2 * t) + j] = acc[j][2];
-      myred[(g + 8) * 64 + 8 * (2 * t + 1) + j] = acc[j][3];
+      for (int f = 0; f < 4; ++f) {
+        const int ce = 8 * g + 2 * f;
+        dst[(tok0 + 2 * t) * 64 + ce] = v[f][0];
+        dst[(tok0 + 2 * t + 1) * 64 + ce] = v[f][1];
+        dst[(tok0 + 2 * t) * 64 + ce + 1] = v[f][2];
+        dst[(tok0 + 2 * t + 1) * 64 + ce + 1] = v[f][3];
+      }
+    };
+    if (p > 0) {
+      float* myred = red + (b * 3 + p - 1) * (16 * 64);
+      put(myred, acc, 0);
+      if (kM16) put(myred, acc2, 8);
+      if (do_xa) {
+        float* zr = zred + (p - 1) * 128;
+        zr[g * 8 + 2 * t] = xa[0];
+        zr[g * 8 + 2 * t + 1] = xa[1];
+        zr[(g + 8) * 8 + 2 * t] = xa[2];
+        zr[(g + 8) * 8 + 2 * t + 1] = xa[3];
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kGvCompute * 32) : "memory");   // compute warps only
+    if (do_xa && p == 0) {
+      float* zo = args.zpart + static_cast<int64_t>(blockIdx.y) * M * args.r + cg * 8;
+      const int q0 = 2 * t, q1 = 2 * t + 1;
+      auto zsum = [&](float v, int row, int col) {
+        return v + zred[row * 8 + col] + zred[128 + row * 8 + col] + zred[256 + row * 8 + col];
+      };
+      if (g < M) {
+        if (cg * 8 + q0 < args.r) zo[g * args.r + q0] = zsum(xa[0], g, q0);
+        if (cg * 8 + q1 < args.r) zo[g * args.r + q1] = zsum(xa[1], g, q1);
+      }
+      if (g + 8 < M) {
+        if (cg * 8 + q0 < args.r) zo[(g + 8) * args.r + q0] = zsum(xa[2], g + 8, q0);
+        if (cg * 8 + q1 < args.r) zo[(g + 8) * args.r + q1] = zsum(xa[3], g + 8, q1);
+      }
+    }
+    if (p == 0 && colok) {
+      const float* r1 = red + (b * 3) * (16 * 64);
+      float* out = args.partial + static_cast<int64_t>(blockIdx.y) * M * N + blk * 64;
+      auto emit = [&](const float (&v)[4][4], int tok0) {
+#pragma unroll
+        for (int f = 0; f < 4; ++f) {
+          const int ce = 8 * g + 2 * f;
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int tok = tok0 + 2 * t + (h & 1), col = ce + (h >> 1);
+            const int idx = tok * 64 + col;
+            if (tok < M)
+              out[static_cast<int64_t>(tok) * N + col] = v[f][h] + r1[idx] + r1[1024 + idx] + r1[2048 + idx];
+          }
+        }
+      };
+      emit(acc, 0);
+      if (kM16) emit(acc2, 8);
+    }
+  }
+  if (!ok && lane == 0) raise_status(args.d_status, QLORA_ERR_TIMEOUT);
+}
+
+// Zc = bf16(c * sum_s zpart[s]) (M x r, written by CTA 0; or read when zpart
+// is null), then per column n:
+// Y[m][n] = bf16( sum_s partial[s][m][n] + sum_j Zc[m][j] * B[j][n] ).
+__global__ void __launch_bounds__(128) gemv_finish_kernel(const float* __restrict__ partial,
+                                                          int splits, int M, int N,
+                                                          const float* __restrict__ zpart, int r,
+                                                          float c, const uint16_t* __restrict__ B,
+                                                          uint16_t* __restrict__ Zc,
+                                                          uint16_t* __restrict__ Y) {
+  // blockIdx.y = token m; this CTA needs row m of Zc only
+  __shared__ float zs[64];
+  const int m = blockIdx.y;
+  for (int j = threadIdx.x; j < r; j += blockDim.x) {
+    const int i = m * r + j;
+    if (zpart != nullptr) {
+      float acc = 0.0f;
+#pragma unroll 4
+      for (int s = 0; s < splits; ++s) acc += zpart[static_cast<int64_t>(s) * M * r + i];
+      const uint32_t zb = pack_bf16x2(c * acc, 0.0f) & 0xFFFFu;
+      zs[j] = bf16_bits_to_f32(zb);
+      if (blockIdx.x == 0) Zc[i] = static_cast<uint16_t>(zb);
+    } else {
+      zs[j] = bf16_bits_to_f32(Zc[i]);   // computed by the rank-r kernel
     }
   }
   __syncthreads();
-  if (warp < 4 && colok) {
-    float* out = partial + static_cast<int64_t>(blockIdx.y) * M * N + blk * 64;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int c0 = 8 * (2 * t) + j, c1 = 8 * (2 * t + 1) + j;
-      if (g < M) {
-        out[static_cast<int64_t>(g) * N + c0] = acc[j][0] + myred[g * 64 + c0];
-        out[static_cast<int64_t>(g) * N + c1] = acc[j][1] + myred[g * 64 + c1];
-      }
-      if (g + 8 < M) {
-        out[static_cast<int64_t>(g + 8) * N + c0] = acc[j][2] + myred[(g + 8) * 64 + c0];
-        out[static_cast<int64_t>(g + 8) * N + c1] = acc[j][3] + myred[(g + 8) * 64 + c1];
-      }
-    }
-  }
-}
-
-constexpr size_t kGvSmem = 256 + kGvTable + 1024 + 4 * 16 * 64 * 4;
-
-// Y[m][n] = bf16( sum_s partial[s][m][n] + sum_j Zc[m][j] * B[j][n] )
-__global__ void gemv_reduce_kernel(const float* __restrict__ partial, int splits, int M, int N,
-                                   const uint16_t* __restrict__ Zc, const uint16_t* __restrict__ B,
-                                   int r, uint16_t* __restrict__ Y) {
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= static_cast<int64_t>(M) * N) return;
-  const int m = static_cast<int>(idx / N), n = static_cast<int>(idx % N);
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
   float acc = 0.0f;
+#pragma unroll 4
   for (int s = 0; s < splits; ++s) acc += partial[(static_cast<int64_t>(s) * M + m) * N + n];
+  // r is a multiple of 8: eight independent loads of B per round
   float lora = 0.0f;
-  for (int j = 0; j < r; ++j)
-    lora = fmaf(bf16_bits_to_f32(Zc[static_cast<int64_t>(m) * r + j]),
-                bf16_bits_to_f32(B[static_cast<int64_t>(j) * N + n]), lora);
-  Y[idx] = static_cast<uint16_t>(pack_bf16x2(acc + lora, 0.0f) & 0xFFFFu);
+  for (int j0 = 0; j0 < r; j0 += 8) {
+    float bv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) bv[u] = bf16_bits_to_f32(__ldg(B + static_cast<int64_t>(j0 + u) * N + n));
+#pragma unroll
+    for (int u = 0; u < 8; ++u) lora = fmaf(zs[j0 + u], bv[u], lora);
+  }
+  Y[static_cast<int64_t>(m) * N + n] = static_cast<uint16_t>(pack_bf16x2(acc + lora, 0.0f) & 0xFFFFu);
 }
 
 // ===========================================================================
@@ -880,30 +1110,33 @@ constexpr CUtensorMapSwizzle kSW128 = CU_TENSOR_MAP_SWIZZLE_128B;
 
 int rsteps_of(int r) { return (r + 15) / 16; }
 
-size_t gemv_splits_and_bytes(int64_t M, int64_t K, int64_t N, int num_sms, int* splits_out,
-                             int* steps_out) {
-  const int ntiles = static_cast<int>((N + 255) / 256);
-  const int ksteps = static_cast<int>(K / 16);
-  int s = (2 * num_sms + ntiles - 1) / ntiles;
-  if (s > ksteps / 2) s = ksteps / 2;
+// GEMV split: one CTA per SM over (256-column groups) x (K splits).
+void gemv_plan(int64_t K, int64_t N, int num_sms, int* splits, int* stages_per_split) {
+  const int ncg = static_cast<int>((N + 255) / 256);
+  const int nstages = static_cast<int>((K + kGvRows - 1) / kGvRows);
+  int s = num_sms / ncg;
   if (s < 1) s = 1;
-  const int per = (ksteps + s - 1) / s;
-  s = (ksteps + per - 1) / per;
-  if (splits_out) *splits_out = s;
-  if (steps_out) *steps_out = per;
-  return align256(static_cast<size_t>(s) * M * N * 4);
+  if (s > nstages) s = nstages;
+  const int per = (nstages + s - 1) / s;
+  *stages_per_split = per;
+  *splits = (nstages + per - 1) / per;
 }
+
 
 }  // namespace
 
 static int g_ws_sms = 148;  // sizing assumption for workspace queries (B200)
 
 size_t linear_fwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) {
-  (void)r;
-  const int S = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
-  size_t b = align256(static_cast<size_t>(S) * M * 64 * 4);
-  if (M <= 16) b += gemv_splits_and_bytes(M, K, N, g_ws_sms, nullptr, nullptr);
-  return b;
+  const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
+  size_t skinny = align256(static_cast<size_t>(Sz) * M * 64 * 4);
+  if (M > 16) return skinny;
+  // GEMV partials and X·A partials; the rank-r kernel's partials reuse the
+  // latter region's size when it is the larger (never both at once)
+  int S = 1, per = 1;
+  gemv_plan(K, N, g_ws_sms, &S, &per);
+  const size_t zp = align256(static_cast<size_t>(S) * M * r * 4);
+  return align256(static_cast<size_t>(S) * M * N * 4) + (zp > skinny ? zp : skinny);
 }
 
 size_t linear_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) {
@@ -929,18 +1162,23 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
   CUtensorMap tX, tAl, tZc, tBl;
   if (!make_tmap_2d(&tX, X, kBF16, 2, M, K, K, 64, 128, kSW128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tAl, A, kBF16, 2, K, r, r, 64, 64, kSW128)) return cudaErrorInvalidValue;
-  const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
-  float* pz = static_cast<float*>(cur.take(static_cast<size_t>(Sz) * M * 64 * 4));
-  if (!cur.ok) return cudaErrorInvalidValue;
-  cudaError_t e = run_skinny<false, true>(tX, tAl, static_cast<int>(M), static_cast<int>(K), r,
-                                          c, 0, Zc, r, pz, Sz, d_status, st);
-  if (e != cudaSuccess) return e;
-
+  cudaError_t e = cudaSuccess;
   if (M <= 16) {
     int S = 1, per = 1;
-    gemv_splits_and_bytes(M, K, N, g_ws_sms, &S, &per);
+    gemv_plan(K, N, g_ws_sms, &S, &per);
+    const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
+    const size_t zbytes = static_cast<size_t>(S) * M * r * 4;
+    const size_t sbytes = static_cast<size_t>(Sz) * M * 64 * 4;
     float* pg = static_cast<float*>(cur.take(static_cast<size_t>(S) * M * N * 4));
+    float* pz = static_cast<float*>(cur.take(zbytes > sbytes ? zbytes : sbytes));
     if (!cur.ok) return cudaErrorInvalidValue;
+    const int ncg = static_cast<int>((N + 255) / 256);
+    const bool xa_in_gemv = ncg * 8 >= r;   // every 8-column rank slice has a column group
+    if (!xa_in_gemv) {
+      e = run_skinny<false, true>(tX, tAl, static_cast<int>(M), static_cast<int>(K), r, c, 0, Zc, r,
+                                  pz, Sz, d_status, st);
+      if (e != cudaSuccess) return e;
+    }
     static bool attr_done = false;
     if (!attr_done) {
       e = cudaFuncSetAttribute(nf4_gemv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -951,26 +1189,50 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
       if (e != cudaSuccess) return e;
       attr_done = true;
     }
-    dim3 grid(static_cast<unsigned>((N + 255) / 256), S);
-    const int Mi = static_cast<int>(M), Ki = static_cast<int>(K), Ni = static_cast<int>(N);
+    CUtensorMap tP, tXg, tAg;
+    if (!make_tmap_2d(&tP, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N / 2, N / 2, 128, kGvRows, kSW128))
+      return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&tXg, X, kBF16, 2, M, K, K, 64, 16, kSW128)) return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&tAg, A, kBF16, 2, K, r, r, 8, kGvRows, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+    GemvArgs ga;
+    ga.M = static_cast<int>(M);
+    ga.K = static_cast<int>(K);
+    ga.N = static_cast<int>(N);
+    ga.r = r;
+    ga.stages_per_split = per;
+    ga.sv = sv;
+    ga.partial = pg;
+    ga.zpart = xa_in_gemv ? pz : nullptr;
+    ga.d_status = d_status;
+    dim3 grid(static_cast<unsigned>(ncg), static_cast<unsigned>(S));
     {
       ProfScope prof(kProfGemv, st);
       if (M <= 8)
-        nf4_gemv_kernel<false><<<grid, 256, kGvSmem, st>>>(X, Mi, Ki, Ni, packed, sv, per, pg);
+        nf4_gemv_kernel<false><<<grid, kGvThreads, kGvSmem, st>>>(tP, tXg, tAg, ga);
       else
-        nf4_gemv_kernel<true><<<grid, 256, kGvSmem, st>>>(X, Mi, Ki, Ni, packed, sv, per, pg);
+        nf4_gemv_kernel<true><<<grid, kGvThreads, kGvSmem, st>>>(tP, tXg, tAg, ga);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const int64_t total = M * N;
     {
       ProfScope prof(kProfOther, st);
-      gemv_reduce_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(
-          pg, S, Mi, Ni, Zc, B, r, Y);
+      dim3 fgrid(static_cast<unsigned>((N + 127) / 128), static_cast<unsigned>(M));
+      gemv_finish_kernel<<<fgrid, 128, 0, st>>>(
+          pg, S, static_cast<int>(M), static_cast<int>(N), xa_in_gemv ? pz : nullptr, r, c, B, Zc, Y);
     }
     return cudaGetLastError();
   }
 
+  // rank-r product for the tensor-core path: Zc = bf16(c * X A)
+  {
+    const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
+    float* pz = static_cast<float*>(cur.take(static_cast<size_t>(Sz) * M * 64 * 4));
+    if (!cur.ok) return cudaErrorInvalidValue;
+    e = run_skinny<false, true>(tX, tAl, static_cast<int>(M), static_cast<int>(K), r, c, 0, Zc, r,
+                                pz, Sz, d_status, st);
+    if (e != cudaSuccess) return e;
+  }
   e = set_fused_attr<false>();
   if (e != cudaSuccess) return e;
   if (!make_tmap_2d(&tZc, Zc, kBF16, 2, M, r, r, 64, 128, kSW128)) return cudaErrorInvalidValue;

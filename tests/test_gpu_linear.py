@@ -67,6 +67,27 @@ def test_gemv_parity(M):
         assert v <= TOL, (k, v, errs)
 
 
+GEMV_SHAPES = [
+    # (M, K, N, r, dq): K not a multiple of 128 (a half stage of zeros), a ragged
+    # last column group, one 64-row stage, no double quantization, a rank wider
+    # than the column groups' 8-column slices (X·A by the rank-r kernel), and a
+    # single column group with one split per 128 rows
+    (1, 576, 576, 16, True),
+    (3, 64, 320, 8, False),
+    (16, 1088, 1344, 64, True),
+    (7, 2112, 256, 8, True),
+    (12, 832, 704, 24, False),
+]
+
+
+@pytest.mark.parametrize("M,K,N,r,dq", GEMV_SHAPES)
+def test_gemv_shapes(M, K, N, r, dq):
+    lin = S.random_case(1000 + M + K + N, M, K, N, r)
+    errs = run_case(lin, r, 16.0 / r, dq, backward=False)
+    for k, v in errs.items():
+        assert v <= TOL, (k, v, errs)
+
+
 def test_config1_tiny():
     wl = S.config1()
     lin = wl.linears[0]
