@@ -379,8 +379,9 @@ def main():
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     Zc = torch.empty((M, R), dtype=torch.bfloat16, device=dev)
     dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
-    dA = torch.empty((K, R), dtype=torch.float32, device=dev)
-    dB = torch.empty((R, N), dtype=torch.float32, device=dev)
+    from bit_nf4_quantized_pack_b200.dp import GradBucket
+    grads = GradBucket(K, N, R, dev)      # dA, dB as views of one all-reduce bucket
+    dA, dB = grads.dA, grads.dB
     status = q.new_status(dev)
 
     def step(i):
@@ -390,8 +391,7 @@ def main():
         q.linear_backward(s["dY"], s["X"], Zc, wbuf, s["A"], s["B"], c, dX=dX, dA=dA, dB=dB,
                           status=status)
         if world > 1:
-            dist.all_reduce(dA)
-            dist.all_reduce(dB)
+            grads.all_reduce()
 
     for i in range(args.warmup):
         step(i)
@@ -467,8 +467,7 @@ def main():
             q.linear_forward(dXin, wbuf, A_, B_, c, Y=Y, Zc=Zc, status=status)
             q.linear_backward(dG, dXin, Zc, wbuf, A_, B_, c, dX=dX, dA=dA, dB=dB, status=status)
             if world > 1:
-                dist.all_reduce(dA)
-                dist.all_reduce(dB)
+                grads.all_reduce()
             hdA.copy_(dA, non_blocking=True)
             hdB.copy_(dB, non_blocking=True)
 
