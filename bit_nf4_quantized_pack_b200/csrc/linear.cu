@@ -16,8 +16,9 @@
 //                        memory, one thread issues tcgen05.mma into TMEM, and
 //                        the rank-r LoRA term is one extra K-step of the same
 //                        accumulator.
-//   nf4_gemv_kernel      M <= 16: split-K CUDA-core GEMV streaming the packed
-//                        payload, then gemv_reduce_kernel adds Zc·B.
+//   nf4_gemv_kernel      M <= 16: split-K GEMV fed by TMA; decoded weight pairs
+//                        go from a shared table straight into mma.sync
+//                        fragments; gemv_finish_kernel adds the splits and Zc·B.
 #include <cfloat>
 
 #include "common.cuh"
