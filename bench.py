@@ -408,6 +408,9 @@ def main():
     if sampler:
         sampler.start()
     q.lib.qlora_profile_reset()
+    # launch events only around the roofline kernel's launches: events between
+    # the other launches would keep them from overlapping their predecessors
+    q.lib.qlora_profile_select(0x3)
     q.lib.qlora_profile_enable(1)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
@@ -428,6 +431,18 @@ def main():
     fwd_ms, fwd_n = prof_read(q, 0)
     bwd_ms, bwd_n = prof_read(q, 1)
     _, launches = prof_read(q, -1)
+    # per-class launch time per step, from a separate pass with every launch
+    # bracketed by events (outside the timed region)
+    q.lib.qlora_profile_reset()
+    q.lib.qlora_profile_select(0xFFFFFFFF)
+    q.lib.qlora_profile_enable(1)
+    nb = 10
+    for i in range(nb):
+        step(i)
+    torch.cuda.synchronize()
+    q.lib.qlora_profile_enable(0)
+    breakdown = {nm: prof_read(q, kind)[0] / nb * 1e3
+                 for kind, nm in ((0, "fused_fwd"), (1, "fused_dX"), (2, "rank_r"), (3, "quantize"))}
     code, mask = q.status_sync(status)
     if code != 0:
         raise SystemExit(f"device status {code} (mask {mask}) in the timed region")
@@ -522,7 +537,8 @@ def main():
                            "step": "quantize(W) + fwd + bwd" + (" + allreduce(dA,dB)" if world > 1 else ""),
                            "l2": f"{ROTATE} rotated input sets (W, X, dY: 96 MB each) > L2"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": int(launches), "clocks": clocks}
+                "gpu_launches": int(launches), "clocks": clocks,
+                "breakdown_us_per_step": breakdown}
         line.update(extras)
         print(json.dumps(line), flush=True)
     if world > 1:

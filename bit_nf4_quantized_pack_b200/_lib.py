@@ -63,6 +63,7 @@ SIGNATURES = {
     "qlora_profile_enable": (_I32, [_I32]),
     "qlora_profile_read": (_I32, [_I32, C.POINTER(C.c_double), C.POINTER(C.c_int64)]),
     "qlora_profile_reset": (_I32, []),
+    "qlora_profile_select": (_I32, [C.c_uint32]),
 }
 
 PROF_FUSED_FWD, PROF_FUSED_BWD, PROF_SKINNY, PROF_QUANTIZE = 0, 1, 2, 3

@@ -134,6 +134,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  Every kernel of the library is launched
+// with programmatic stream serialization: it lets its successor launch at once
+// (pdl_launch_dependents at its start) and, before its first access to global
+// memory that an earlier launch may write or read, waits for its predecessor
+// to complete and flush (pdl_wait).  Only set-up that touches no such memory
+// (shared memory, barriers, TMEM, tables of constants) runs before the wait.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,

@@ -29,9 +29,11 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(
     const float* __restrict__ offset, uint16_t* __restrict__ out, int32_t* d_status) {
   __shared__ float C[16];
   __shared__ float t8[256];
+  pdl_launch_dependents();
   if (threadIdx.x < 16) C[threadIdx.x] = kNF4d[threadIdx.x];
   if (code8 != nullptr) build_t8(t8);
   __syncthreads();
+  pdl_wait();   // the tables above read no global memory
   const float off = code8 != nullptr ? __ldg(offset) : 0.0f;
   const int64_t nbytes = (numel + 1) >> 1;
   const int64_t ngroups = (numel + 7) >> 3;
@@ -87,8 +89,9 @@ cudaError_t launch_dequantize(const uint8_t* packed, int64_t numel, const float*
   const int blocks = static_cast<int>(want < num_sms * 8LL ? want : num_sms * 8LL);
   {
     ProfScope prof(kProfDequantize, st);
-    nf4_dequant_kernel<<<blocks, threads, 0, st>>>(packed, numel, absmax, code8, s2, offset, out,
-                                                   d_status);
+    const cudaError_t e = launch_pdl(nf4_dequant_kernel, dim3(blocks), dim3(threads), 0, st, 1, packed,
+                                     numel, absmax, code8, s2, offset, out, d_status);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

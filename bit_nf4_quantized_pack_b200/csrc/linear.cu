@@ -8,7 +8,8 @@
 // Kernels in this file:
 //   skinny_gemm_kernel   rank-r contractions (X·A, G·Bᵀ, Xᵀ·dZ, Gᵀ·Zc): TMA
 //                        for both operands, tcgen05 MMA with N = 64, split-K
-//                        into fp32 partials, then skinny_reduce_kernel.
+//                        into fp32 partials; the last split of each row
+//                        tile adds them and writes the result.
 //   fused_nf4_gemm_kernel  Y = X·Ŵ + Zc·B (forward) and dX = G·Ŵᵀ + dZ·Aᵀ
 //                        (backward): persistent, warp-specialised; TMA brings
 //                        activation tiles and packed-nibble tiles, decoder
@@ -19,6 +20,7 @@
 //   nf4_gemv_kernel      M <= 16: split-K GEMV fed by TMA; decoded weight pairs
 //                        go from a shared table straight into mma.sync
 //                        fragments; gemv_finish_kernel adds the splits and Zc·B.
+#include <atomic>
 #include <cfloat>
 
 #include "common.cuh"
@@ -36,18 +38,41 @@ __constant__ float kNF4g[16] = {QNF4_TABLE_VALUES};
 // (rows of 64 contiguous k') or MN-major (rows of 64 contiguous m'/n'), all
 // with the 128-byte swizzle.  blockIdx.x = 128-row tile, blockIdx.y = split.
 // ===========================================================================
-constexpr int kSkStages = 6;
+constexpr int kSkStages = 8;
 constexpr int kSkA = 16384, kSkB = 8192;
 constexpr int kSkThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr size_t kSkSmem = 1024 + kSkStages * (kSkA + kSkB) + 256;
+static_assert(kSkStages * 8 * 3 + 16 <= 256, "skinny barriers and flags fit the tail");
 
 struct SkinnyArgs {
   int Mp;            // rows of D
   int nk;            // number of 64-wide k' blocks
   int kb_per_split;  // k' blocks per split
-  float* partial;    // [splits][Mp][64]
+  int splits;        // = cluster size along y (<= 8)
+  int ncols;         // columns of D that are kept (the rank r)
+  float scale;
+  int mode;          // 0: bf16 out[Mp][ld]; 1: fp32 out[Mp][ld]; 2: fp32 out[ncols][Mp]
+  void* out;
+  int ld;
   int32_t* d_status;
 };
+
+constexpr int kSkRedLd = 65;   // fp32 words per row of the split-sum buffer (bank spread)
+constexpr int kSkMaxSplits = 8;  // portable cluster size
+
+// Every thread of every CTA in the cluster (lanes may arrive diverged: the
+// producer and MMA lanes come from their own loops).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_saddr, uint32_t cta_rank) {
+  uint32_t remote;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_saddr), "r"(cta_rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
 
 template <bool kAmn, bool kBmn>
 __global__ void __launch_bounds__(kSkThreads, 1)
@@ -63,6 +88,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   uint64_t* done = empty + kSkStages;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_holder + 1);
+  float* red = reinterpret_cast<float*>(sA);   // [128][kSkRedLd], after the last MMA
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * 128;
@@ -87,6 +113,8 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  pdl_launch_dependents();   // after this CTA holds its TMEM
+  pdl_wait();
 
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
@@ -128,28 +156,70 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     if (!ok) *abort_flag = 1;
     umma_commit(done);  // also drains whatever was issued
   } else if (warp >= 2) {
+    // Epilogue, part 1: this split's fp32 sums into shared memory (the A ring
+    // is free once the last MMA has completed).
     const int q = warp & 3;
-    const bool ok = mbar_wait(done, 0);
+    const bool okd = mbar_wait(done, 0);
     tc_fence_after();
-    const int row = m0 + q * 32 + lane;
-    if (!ok) *abort_flag = 1;
-    if (ok && !*abort_flag) {
+    if (!okd) *abort_flag = 1;
+    const int row = q * 32 + lane;
+    const int nc = args.ncols;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+    for (int c = 0; c < 2; ++c) {
+      if (c * 32 < nc) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c * 32, v);
-        tmem_ld_wait();
-        if (row < args.Mp) {
-          float4* dst = reinterpret_cast<float4*>(
-              args.partial + (static_cast<int64_t>(blockIdx.y) * args.Mp + row) * 64 + c * 32);
+        if (okd) {
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c * 32, v);
+          tmem_ld_wait();
+        }
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        for (int i = 0; i < 32; ++i)
+          if (c * 32 + i < nc) red[row * kSkRedLd + c * 32 + i] = okd ? __uint_as_float(v[i]) : 0.0f;
+      }
+    }
+  }
+  // Part 2: the splits of a row tile are one thread-block cluster along y.
+  // Each adds a share of the tile's rows over all splits, in split order,
+  // reading the others' sums from distributed shared memory, and writes out.
+  cluster_sync_all();
+  if (warp >= 2) {
+    const int S = args.splits;
+    const int rank = static_cast<int>(blockIdx.y);   // cluster spans all of y
+    const int rows_per = (128 + S - 1) / S;
+    const int r0 = rank * rows_per;
+    const int nrow = min(rows_per, 128 - r0);
+    const int nc = args.ncols;
+    const int total = nrow > 0 ? nrow * nc : 0;
+    const uint32_t red_s = smem_u32(red);
+    for (int e = threadIdx.x - 64; e < total; e += 128) {
+      // mode 2 writes columns of out: let consecutive threads take consecutive rows
+      const int rr = args.mode == 2 ? e % nrow : e / nc;
+      const int cc = args.mode == 2 ? e / nrow : e % nc;
+      const int lrow = r0 + rr, grow = m0 + lrow;
+      // all S loads in flight first, then the sum in split order
+      const uint32_t off = red_s + static_cast<uint32_t>((lrow * kSkRedLd + cc) * 4);
+      float part[kSkMaxSplits];
+#pragma unroll
+      for (int sp = 0; sp < kSkMaxSplits; ++sp)
+        part[sp] = sp < S ? ld_dsmem_f32(off, static_cast<uint32_t>(sp)) : 0.0f;
+      float acc = 0.0f;
+#pragma unroll
+      for (int sp = 0; sp < kSkMaxSplits; ++sp)
+        if (sp < S) acc += part[sp];
+      acc *= args.scale;
+      if (grow < args.Mp) {
+        if (args.mode == 0) {
+          static_cast<uint16_t*>(args.out)[static_cast<int64_t>(grow) * args.ld + cc] =
+              static_cast<uint16_t>(pack_bf16x2(acc, 0.0f) & 0xFFFFu);
+        } else if (args.mode == 1) {
+          static_cast<float*>(args.out)[static_cast<int64_t>(grow) * args.ld + cc] = acc;
+        } else {
+          static_cast<float*>(args.out)[static_cast<int64_t>(cc) * args.Mp + grow] = acc;
         }
       }
     }
   }
+  cluster_sync_all();   // no CTA leaves while another still reads its sums
   tc_fence_before();
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0) raise_status(args.d_status, QLORA_ERR_TIMEOUT);
@@ -159,25 +229,6 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   }
 }
 
-// out = scale * sum_s partial[s]; modes: 0 bf16 [Mp][ld], 1 fp32 [Mp][ld],
-// 2 fp32 transposed [ncols][Mp].
-__global__ void skinny_reduce_kernel(const float* __restrict__ partial, int splits, int Mp,
-                                     int ncols, float scale, int mode, void* out, int ld) {
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= static_cast<int64_t>(Mp) * ncols) return;
-  const int row = static_cast<int>(idx / ncols), col = static_cast<int>(idx % ncols);
-  float acc = 0.0f;
-  for (int s = 0; s < splits; ++s) acc += partial[(static_cast<int64_t>(s) * Mp + row) * 64 + col];
-  acc *= scale;
-  if (mode == 0) {
-    static_cast<uint16_t*>(out)[static_cast<int64_t>(row) * ld + col] =
-        static_cast<uint16_t>(pack_bf16x2(acc, 0.0f) & 0xFFFFu);
-  } else if (mode == 1) {
-    static_cast<float*>(out)[static_cast<int64_t>(row) * ld + col] = acc;
-  } else {
-    static_cast<float*>(out)[static_cast<int64_t>(col) * Mp + row] = acc;
-  }
-}
 
 // ===========================================================================
 // Fused NF4-decode GEMM (forward: kBwd = false, input gradient: kBwd = true)
@@ -384,6 +435,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const int num_tiles = args.m_tiles * args.n_tiles;
+  pdl_launch_dependents();   // after this CTA holds its TMEM
+  pdl_wait();
 
   if (warp == 0) {
     // ------------------------------ TMA producer ---------------------------
@@ -740,6 +793,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   float* red = reinterpret_cast<float*>(sP);   // [4][3][16][64], after the last stage
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  pdl_launch_dependents();
   if (threadIdx.x == kGvCompute * 32) {
     for (int s = 0; s < kGvStages; ++s) {
       mbar_init(&full[s], 1);
@@ -760,6 +814,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     // starts streaming while the compute warps build their tables; rows past K
     // (a last stage of 64 rows) arrive as zeros
     if (lane == 0) {
+      pdl_wait();
       tma_prefetch_desc(&tmP);
       tma_prefetch_desc(&tmX);
       tma_prefetch_desc(&tmA);
@@ -796,6 +851,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       }
     }
     asm volatile("bar.sync 1, %0;" ::"n"(kGvCompute * 32) : "memory");   // compute warps only
+    pdl_wait();
 
     const int b = warp & 3, p = warp >> 2;             // column block, row slot
     const int blk = cg * 4 + b;                        // 64-column block
@@ -992,6 +1048,8 @@ __global__ void __launch_bounds__(128) gemv_finish_kernel(const float* __restric
                                                           uint16_t* __restrict__ Y) {
   // blockIdx.y = token m; this CTA needs row m of Zc only
   __shared__ float zs[64];
+  pdl_launch_dependents();
+  pdl_wait();
   const int m = blockIdx.y;
   for (int j = threadIdx.x; j < r; j += blockDim.x) {
     const int i = m * r + j;
@@ -1029,9 +1087,12 @@ __global__ void __launch_bounds__(128) gemv_finish_kernel(const float* __restric
 // ===========================================================================
 namespace {
 
+// K splits of a rank-r contraction: one CTA per SM (the kernel's shared
+// memory allows no second), so the grid is kept to a single wave.
 int skinny_splits(int Mp, int nk, int num_sms) {
   const int mt = (Mp + 127) / 128;
-  int want = (2 * num_sms + mt - 1) / mt;
+  int want = num_sms / mt;
+  if (want > kSkMaxSplits) want = kSkMaxSplits;
   if (want < 1) want = 1;
   if (want > nk) want = nk;
   const int per = (nk + want - 1) / want;
@@ -1065,11 +1126,11 @@ cudaError_t set_skinny_attr() {
   return e;
 }
 
-// D = scale * A(m',k') B(n',k') ; writes through skinny_reduce_kernel.
+// D = scale * A(m',k') B(n',k'): one launch, split-K sums added in-kernel.
 template <bool kAmn, bool kBmn>
 cudaError_t run_skinny(const CUtensorMap& ta, const CUtensorMap& tb, int Mp, int Kp, int ncols,
-                       float scale, int mode, void* out, int ld, float* partial, int splits,
-                       int32_t* d_status, cudaStream_t st) {
+                       float scale, int mode, void* out, int ld, int splits, int32_t* d_status,
+                       cudaStream_t st) {
   cudaError_t e = set_skinny_attr<kAmn, kBmn>();
   if (e != cudaSuccess) return e;
   const int nk = (Kp + 63) / 64;
@@ -1077,21 +1138,19 @@ cudaError_t run_skinny(const CUtensorMap& ta, const CUtensorMap& tb, int Mp, int
   a.Mp = Mp;
   a.nk = nk;
   a.kb_per_split = (nk + splits - 1) / splits;
-  a.partial = partial;
+  a.splits = (nk + a.kb_per_split - 1) / a.kb_per_split;
+  a.ncols = ncols;
+  a.scale = scale;
+  a.mode = mode;
+  a.out = out;
+  a.ld = ld;
   a.d_status = d_status;
-  dim3 grid((Mp + 127) / 128, splits);
   {
     ProfScope prof(kProfSkinny, st);
-    skinny_gemm_kernel<kAmn, kBmn><<<grid, kSkThreads, kSkSmem, st>>>(ta, tb, a);
+    e = launch_pdl(skinny_gemm_kernel<kAmn, kBmn>, dim3((Mp + 127) / 128, a.splits, 1),
+                   dim3(kSkThreads, 1, 1), kSkSmem, st, a.splits, ta, tb, a);
   }
-  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int64_t total = static_cast<int64_t>(Mp) * ncols;
-  {
-    ProfScope prof(kProfOther, st);
-    skinny_reduce_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(
-        partial, splits, Mp, ncols, scale, mode, out, ld);
-  }
   return cudaGetLastError();
 }
 
@@ -1129,28 +1188,17 @@ void gemv_plan(int64_t K, int64_t N, int num_sms, int* splits, int* stages_per_s
 static int g_ws_sms = 148;  // sizing assumption for workspace queries (B200)
 
 size_t linear_fwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) {
-  const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
-  size_t skinny = align256(static_cast<size_t>(Sz) * M * 64 * 4);
-  if (M > 16) return skinny;
-  // GEMV partials and X·A partials; the rank-r kernel's partials reuse the
-  // latter region's size when it is the larger (never both at once)
+  if (M > 16) return 0;   // the rank-r kernel adds its splits in shared memory
+  // GEMV partials and its per-split X·A slices
   int S = 1, per = 1;
   gemv_plan(K, N, g_ws_sms, &S, &per);
-  const size_t zp = align256(static_cast<size_t>(S) * M * r * 4);
-  return align256(static_cast<size_t>(S) * M * N * 4) + (zp > skinny ? zp : skinny);
+  return align256(static_cast<size_t>(S) * M * N * 4) + align256(static_cast<size_t>(S) * M * r * 4);
 }
 
 size_t linear_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) {
-  (void)r;
-  const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(N / 64), g_ws_sms);
-  const int nkm = static_cast<int>((M + 63) / 64);
-  const int Sa = skinny_splits(static_cast<int>(K), nkm, g_ws_sms);
-  const int Sb = skinny_splits(static_cast<int>(N), nkm, g_ws_sms);
-  size_t b = align256(static_cast<size_t>(M) * 64 * 2);                 // dZ (bf16, padded to 64)
-  b += align256(static_cast<size_t>(Sz) * M * 64 * 4);                  // dZ partials
-  b += align256(static_cast<size_t>(Sa) * K * 64 * 4);                  // dA partials
-  b += align256(static_cast<size_t>(Sb) * N * 64 * 4);                  // dB partials
-  return b;
+  (void)K;
+  (void)N;
+  return align256(static_cast<size_t>(M) * r * 2);   // dZ (bf16, M x r)
 }
 
 cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint16_t* X,
@@ -1168,16 +1216,14 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
     int S = 1, per = 1;
     gemv_plan(K, N, g_ws_sms, &S, &per);
     const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
-    const size_t zbytes = static_cast<size_t>(S) * M * r * 4;
-    const size_t sbytes = static_cast<size_t>(Sz) * M * 64 * 4;
     float* pg = static_cast<float*>(cur.take(static_cast<size_t>(S) * M * N * 4));
-    float* pz = static_cast<float*>(cur.take(zbytes > sbytes ? zbytes : sbytes));
+    float* pz = static_cast<float*>(cur.take(static_cast<size_t>(S) * M * r * 4));
     if (!cur.ok) return cudaErrorInvalidValue;
     const int ncg = static_cast<int>((N + 255) / 256);
     const bool xa_in_gemv = ncg * 8 >= r;   // every 8-column rank slice has a column group
     if (!xa_in_gemv) {
       e = run_skinny<false, true>(tX, tAl, static_cast<int>(M), static_cast<int>(K), r, c, 0, Zc, r,
-                                  pz, Sz, d_status, st);
+                                  Sz, d_status, st);
       if (e != cudaSuccess) return e;
     }
     static bool attr_done = false;
@@ -1210,28 +1256,27 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
     {
       ProfScope prof(kProfGemv, st);
       if (M <= 8)
-        nf4_gemv_kernel<false><<<grid, kGvThreads, kGvSmem, st>>>(tP, tXg, tAg, ga);
+        e = launch_pdl(nf4_gemv_kernel<false>, grid, dim3(kGvThreads), kGvSmem, st, 1, tP, tXg, tAg, ga);
       else
-        nf4_gemv_kernel<true><<<grid, kGvThreads, kGvSmem, st>>>(tP, tXg, tAg, ga);
+        e = launch_pdl(nf4_gemv_kernel<true>, grid, dim3(kGvThreads), kGvSmem, st, 1, tP, tXg, tAg, ga);
     }
-    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     {
       ProfScope prof(kProfOther, st);
       dim3 fgrid(static_cast<unsigned>((N + 127) / 128), static_cast<unsigned>(M));
-      gemv_finish_kernel<<<fgrid, 128, 0, st>>>(
-          pg, S, static_cast<int>(M), static_cast<int>(N), xa_in_gemv ? pz : nullptr, r, c, B, Zc, Y);
+      e = launch_pdl(gemv_finish_kernel, fgrid, dim3(128), 0, st, 1, static_cast<const float*>(pg), S,
+                     static_cast<int>(M), static_cast<int>(N),
+                     static_cast<const float*>(xa_in_gemv ? pz : nullptr), r, c, B, Zc, Y);
     }
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
 
   // rank-r product for the tensor-core path: Zc = bf16(c * X A)
   {
     const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
-    float* pz = static_cast<float*>(cur.take(static_cast<size_t>(Sz) * M * 64 * 4));
-    if (!cur.ok) return cudaErrorInvalidValue;
     e = run_skinny<false, true>(tX, tAl, static_cast<int>(M), static_cast<int>(K), r, c, 0, Zc, r,
-                                pz, Sz, d_status, st);
+                                Sz, d_status, st);
     if (e != cudaSuccess) return e;
   }
   e = set_fused_attr<false>();
@@ -1257,8 +1302,10 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
   const int grid = tiles < sms ? tiles : sms;
   {
     ProfScope prof(kProfFusedFwd, st);
-    fused_nf4_gemm_kernel<false><<<grid, kFThreads, kFSmem, st>>>(tX, tZc, tBl, fa);
+    e = launch_pdl(fused_nf4_gemm_kernel<false>, dim3(grid), dim3(kFThreads), kFSmem, st, 1, tX, tZc,
+                   tBl, fa);
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -1269,43 +1316,40 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
                               int32_t* d_status, cudaStream_t st, int num_sms) {
   (void)num_sms;
   WsCursor cur{static_cast<char*>(ws), ws_bytes};
-  uint16_t* dZ = static_cast<uint16_t*>(cur.take(static_cast<size_t>(M) * 64 * 2));
+  uint16_t* dZ = static_cast<uint16_t*>(cur.take(static_cast<size_t>(M) * r * 2));
   const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(N / 64), g_ws_sms);
   const int nkm = static_cast<int>((M + 63) / 64);
   const int Sa = skinny_splits(static_cast<int>(K), nkm, g_ws_sms);
   const int Sb = skinny_splits(static_cast<int>(N), nkm, g_ws_sms);
-  float* pz = static_cast<float*>(cur.take(static_cast<size_t>(Sz) * M * 64 * 4));
-  float* pa = static_cast<float*>(cur.take(static_cast<size_t>(Sa) * K * 64 * 4));
-  float* pb = static_cast<float*>(cur.take(static_cast<size_t>(Sb) * N * 64 * 4));
   if (!cur.ok) return cudaErrorInvalidValue;
-  cudaError_t e = cudaMemsetAsync(dZ, 0, static_cast<size_t>(M) * 64 * 2, st);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
 
   CUtensorMap tG, tBk, tXmn, tdZ, tGmn, tZcmn, tAl;
   // dZ = c * G B^T : A operand G (K-major over N), B operand B (K-major: rows r, cols N)
   if (!make_tmap_2d(&tG, dY, kBF16, 2, M, N, N, 64, 128, kSW128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tBk, B, kBF16, 2, r, N, N, 64, 64, kSW128)) return cudaErrorInvalidValue;
-  e = run_skinny<false, false>(tG, tBk, static_cast<int>(M), static_cast<int>(N), r, c, 0, dZ, 64,
-                               pz, Sz, d_status, st);
+  e = run_skinny<false, false>(tG, tBk, static_cast<int>(M), static_cast<int>(N), r, c, 0, dZ, r,
+                               Sz, d_status, st);
   if (e != cudaSuccess) return e;
   // dA = X^T dZ : A operand X^T (MN-major over K), B operand dZ (MN-major over r)
   if (!make_tmap_2d(&tXmn, X, kBF16, 2, M, K, K, 64, 64, kSW128)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&tdZ, dZ, kBF16, 2, M, 64, 64, 64, 64, kSW128)) return cudaErrorInvalidValue;
+  // (columns of dZ past r arrive as TMA zero fill)
+  if (!make_tmap_2d(&tdZ, dZ, kBF16, 2, M, r, r, 64, 64, kSW128)) return cudaErrorInvalidValue;
   e = run_skinny<true, true>(tXmn, tdZ, static_cast<int>(K), static_cast<int>(M), r, 1.0f, 1, dA,
-                             r, pa, Sa, d_status, st);
+                             r, Sa, d_status, st);
   if (e != cudaSuccess) return e;
   // dB^T = G^T Zc : A operand G^T (MN-major over N), B operand Zc (MN-major over r)
   if (!make_tmap_2d(&tGmn, dY, kBF16, 2, M, N, N, 64, 64, kSW128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tZcmn, Zc, kBF16, 2, M, r, r, 64, 64, kSW128)) return cudaErrorInvalidValue;
   e = run_skinny<true, true>(tGmn, tZcmn, static_cast<int>(N), static_cast<int>(M), r, 1.0f, 2,
-                             dB, r, pb, Sb, d_status, st);
+                             dB, r, Sb, d_status, st);
   if (e != cudaSuccess) return e;
   // dX = G W^T + dZ A^T
   e = set_fused_attr<true>();
   if (e != cudaSuccess) return e;
   if (!make_tmap_2d(&tAl, A, kBF16, 2, K, r, r, 64, 256, kSW128)) return cudaErrorInvalidValue;
   CUtensorMap tdZa;
-  if (!make_tmap_2d(&tdZa, dZ, kBF16, 2, M, 64, 64, 64, 128, kSW128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tdZa, dZ, kBF16, 2, M, r, r, 64, 128, kSW128)) return cudaErrorInvalidValue;
   FusedArgs fa;
   fa.M = static_cast<int>(M);
   fa.Nout = static_cast<int>(K);
@@ -1325,8 +1369,10 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   const int grid = tiles < sms ? tiles : sms;
   {
     ProfScope prof(kProfFusedBwd, st);
-    fused_nf4_gemm_kernel<true><<<grid, kFThreads, kFSmem, st>>>(tG, tdZa, tAl, fa);
+    e = launch_pdl(fused_nf4_gemm_kernel<true>, dim3(grid), dim3(kFThreads), kFSmem, st, 1, tG, tdZa,
+                   tAl, fa);
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -19,6 +19,7 @@ struct Pair {
 
 std::mutex g_mu;
 bool g_on = false;
+unsigned int g_mask = 0xFFFFFFFFu;
 std::vector<Pair> g_pending;
 std::vector<cudaEvent_t> g_free;
 long long g_launches[kProfKinds] = {0};
@@ -42,7 +43,7 @@ ProfScope::ProfScope(int id, cudaStream_t s) : id_(id), s_(s), a_(nullptr) {
   std::lock_guard<std::mutex> g(g_mu);
   ++g_total_launches;
   if (id_ >= 0 && id_ < kProfKinds) ++g_launches[id_];
-  if (!g_on) return;
+  if (!g_on || id_ < 0 || id_ >= 32 || !((g_mask >> id_) & 1u)) return;
   a_ = take_event();
   if (a_) cudaEventRecord(static_cast<cudaEvent_t>(a_), s_);
 }
@@ -69,6 +70,12 @@ extern "C" {
 qlora_status qlora_profile_enable(int32_t on) {
   std::lock_guard<std::mutex> g(qnf4::g_mu);
   qnf4::g_on = on != 0;
+  return QLORA_OK;
+}
+
+qlora_status qlora_profile_select(uint32_t kinds_mask) {
+  std::lock_guard<std::mutex> g(qnf4::g_mu);
+  qnf4::g_mask = kinds_mask;
   return QLORA_OK;
 }
 

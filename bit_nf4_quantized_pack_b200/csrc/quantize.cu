@@ -260,6 +260,8 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const T* __restrict__ W
   __shared__ double mexact[15];
   __shared__ unsigned long long sbins[kDQ ? 256 : 1];
   __shared__ uint64_t full_bar[kEncStages];
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ int abort_flag;
   build_buckets(tab, mexact);
   if (kDQ)
@@ -414,6 +416,8 @@ __global__ void __launch_bounds__(256) dq_mean_kernel(const unsigned long long* 
                                                       int64_t n1, float* __restrict__ offset) {
   __shared__ unsigned long long sb[256];
   __shared__ int range[2];
+  pdl_launch_dependents();
+  pdl_wait();
   sb[threadIdx.x] = bins[threadIdx.x];
   __syncthreads();
   if (threadIdx.x < 32) {
@@ -500,6 +504,7 @@ __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict_
   __shared__ float mag[128];
   __shared__ double mid[254];
   __shared__ float thr[8][256];
+  pdl_launch_dependents();
   for (int t = threadIdx.x; t < 128; t += blockDim.x) mag[t] = t8_magnitude(t);
   __syncthreads();
   for (int k = threadIdx.x; k < 254; k += blockDim.x) {
@@ -510,6 +515,7 @@ __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict_
     mid[k] = 0.5 * (V(k) + V(k + 1));
   }
   __syncthreads();
+  pdl_wait();   // the tables above read no global memory
   const float off = *offset_p;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float* T = thr[warp];
@@ -566,10 +572,11 @@ cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* pa
   const int64_t want = (n1 * 4 + threads - 1) / threads;
   unsigned long long* bins = nullptr;
   float* scales = absmax_out;
+  cudaError_t e = cudaSuccess;
   if (dq) {
     bins = static_cast<unsigned long long*>(ws);
     scales = reinterpret_cast<float*>(static_cast<char*>(ws) + 2048);
-    cudaError_t e = cudaMemsetAsync(bins, 0, 2048, st);
+    e = cudaMemsetAsync(bins, 0, 2048, st);
     if (e != cudaSuccess) return e;
   }
   {
@@ -602,35 +609,37 @@ cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* pa
   const int blocks = static_cast<int>(want < cap ? want : cap);
   if (dtype == QLORA_DTYPE_BF16) {
     const size_t sm = encode_smem_bytes<uint16_t>();
-    if (dq)
-      nf4_encode_kernel<uint16_t, true><<<blocks, threads, sm, st>>>(
-          static_cast<const uint16_t*>(W), numel, n1, packed, scales, bins, d_status);
-    else
-      nf4_encode_kernel<uint16_t, false><<<blocks, threads, sm, st>>>(
-          static_cast<const uint16_t*>(W), numel, n1, packed, scales, bins, d_status);
+    const uint16_t* w16 = static_cast<const uint16_t*>(W);
+    e = dq ? launch_pdl(nf4_encode_kernel<uint16_t, true>, dim3(blocks), dim3(threads), sm, st, 1, w16,
+                        numel, n1, packed, scales, bins, d_status)
+           : launch_pdl(nf4_encode_kernel<uint16_t, false>, dim3(blocks), dim3(threads), sm, st, 1, w16,
+                        numel, n1, packed, scales, bins, d_status);
   } else {
     const size_t sm = encode_smem_bytes<float>();
-    if (dq)
-      nf4_encode_kernel<float, true><<<blocks, threads, sm, st>>>(
-          static_cast<const float*>(W), numel, n1, packed, scales, bins, d_status);
-    else
-      nf4_encode_kernel<float, false><<<blocks, threads, sm, st>>>(
-          static_cast<const float*>(W), numel, n1, packed, scales, bins, d_status);
+    const float* w32 = static_cast<const float*>(W);
+    e = dq ? launch_pdl(nf4_encode_kernel<float, true>, dim3(blocks), dim3(threads), sm, st, 1, w32,
+                        numel, n1, packed, scales, bins, d_status)
+           : launch_pdl(nf4_encode_kernel<float, false>, dim3(blocks), dim3(threads), sm, st, 1, w32,
+                        numel, n1, packed, scales, bins, d_status);
   }
   }
-  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || !dq) return e;
   {
     ProfScope prof(kProfQuantize, st);
-    dq_mean_kernel<<<1, 256, 0, st>>>(bins, n1, offset);
+    e = launch_pdl(dq_mean_kernel, dim3(1), dim3(256), 0, st, 1,
+                   static_cast<const unsigned long long*>(bins), n1, offset);
   }
+  if (e != cudaSuccess) return e;
   const int64_t n2 = (n1 + kDQBlock - 1) / kDQBlock;
   {
     ProfScope prof(kProfQuantize, st);
     const int64_t want_g = (n2 + 7) / 8;
     const int64_t grid = want_g < num_sms * 8LL ? want_g : num_sms * 8LL;
-    dq_encode_kernel<<<static_cast<unsigned>(grid), 256, 0, st>>>(scales, n1, offset, code8, s2);
+    e = launch_pdl(dq_encode_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, 1,
+                   static_cast<const float*>(scales), n1, static_cast<const float*>(offset), code8, s2);
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -185,8 +185,11 @@ qlora_status qlora_nf4_dequantize(const qlora_nf4_state* st, uint16_t* W_hat,
  * to bf16 (each weight within one bf16 ulp of qlora_nf4_dequantize's output)
  * and never written to memory.  M <= 16 runs the HBM-bound GEMV path, larger
  * M the fused tensor-core path.
- * Shapes: M >= 1, K % 64 == 0, N % 64 == 0, 1 <= r <= 64, else UNSUPPORTED.
- * ws: at least qlora_linear_fwd_workspace_size(M, K, N, r) bytes.
+ * Shapes: M >= 1, K % 64 == 0, N % 64 == 0, 8 <= r <= 64 with r % 8 == 0,
+ * else UNSUPPORTED.
+ * ws: at least qlora_linear_fwd_workspace_size(M, K, N, r) bytes; that size is
+ * 0 for M > 16 (the rank-r kernel adds its K splits inside a thread-block
+ * cluster), and ws may then be null.
  */
 size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t K, int64_t N, int32_t r);
 qlora_status qlora_linear_fwd(int64_t M, int64_t K, int64_t N, int32_t r,
@@ -223,6 +226,11 @@ qlora_status qlora_linear_bwd(int64_t M, int64_t K, int64_t N, int32_t r,
  * returns the total milliseconds and the launch count of class `kind`
  * (QLORA_PROF_*), or of all classes for kind = -1.  Launch counts are kept
  * whether or not timing is enabled.  qlora_profile_reset zeroes the totals.
+ * qlora_profile_select restricts timing to the classes whose bit is set in
+ * `kinds_mask` (bit k = class k; all classes by default).  The events sit
+ * between launches and so keep a timed launch from overlapping its
+ * predecessor's tail (programmatic dependent launch): a measuring tool that
+ * wants the untouched launch chain times only the classes it needs.
  * Not thread-safe across devices; meant for one measuring process.
  */
 #define QLORA_PROF_FUSED_FWD  0   /* fused NF4 GEMM, forward (Y)        */
@@ -231,10 +239,11 @@ qlora_status qlora_linear_bwd(int64_t M, int64_t K, int64_t N, int32_t r,
 #define QLORA_PROF_QUANTIZE   3   /* NF4 encoder and double quantization */
 #define QLORA_PROF_DEQUANTIZE 4   /* standalone dequantization           */
 #define QLORA_PROF_GEMV       5   /* M <= 16 GEMV                        */
-#define QLORA_PROF_OTHER      6   /* split-K reductions                  */
+#define QLORA_PROF_OTHER      6   /* GEMV split sums                     */
 qlora_status qlora_profile_enable(int32_t on);
 qlora_status qlora_profile_read(int32_t kind, double* total_ms, int64_t* launches);
 qlora_status qlora_profile_reset(void);
+qlora_status qlora_profile_select(uint32_t kinds_mask);
 
 #ifdef __cplusplus
 }  /* extern "C" */

@@ -60,8 +60,11 @@ def test_workspace_sizes(L):
     lib = L.lib
     assert lib.qlora_nf4_quantize_workspace_size(1000, 0) == 0
     assert lib.qlora_nf4_quantize_workspace_size(64 * 100, 1) >= 2048 + 4 * 100
-    assert lib.qlora_linear_fwd_workspace_size(4096, 4096, 4096, 16) > 0
-    assert lib.qlora_linear_bwd_workspace_size(4096, 4096, 4096, 16) > 0
+    # the tensor-core path needs no forward workspace; the GEMV keeps split sums
+    assert lib.qlora_linear_fwd_workspace_size(4096, 4096, 4096, 16) == 0
+    assert lib.qlora_linear_fwd_workspace_size(4, 4096, 4096, 16) > 0
+    # backward: dZ (M x r bf16)
+    assert lib.qlora_linear_bwd_workspace_size(4096, 4096, 4096, 16) >= 4096 * 16 * 2
     # unsupported shapes report 0
     assert lib.qlora_linear_fwd_workspace_size(16, 100, 64, 16) == 0
     assert lib.qlora_linear_fwd_workspace_size(16, 64, 64, 12) == 0
