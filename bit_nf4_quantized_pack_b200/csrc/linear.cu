@@ -233,15 +233,18 @@ __global__ void __launch_bounds__(kSkThreads, 1)
 // ===========================================================================
 // Fused NF4-decode GEMM (forward: kBwd = false, input gradient: kBwd = true)
 //
-// Output tile 256 (rows of X or G) x 256, K-step 64.  One decoded weight tile
-// (256 x 64 bf16) feeds two tcgen05.mma of M = 128, N = 256 (rows m0..m0+127
-// and m0+128..m0+255), so each decoded weight is used by 256 rows.
+// Output tile 512 (rows of X or G) x 128, K-step 64.  One decoded weight tile
+// (128 x 64 bf16) feeds four tcgen05.mma of M = 128, N = 128 (rows m0+128h ..
+// m0+128h+127, h = 0..3), so each decoded weight is used by 512 rows: making
+// the decoded tile (decode, shared-memory stores, packed loads) is the costly
+// part of this kernel, and this shape halves it per FLOP against a 256 x 256
+// tile at the price of twice the activation bytes per K-step.
 //
-// Shared memory holds two rings.  Activation tiles (256 x 64 bf16, K-major,
-// two TMA boxes) have 4 stages so that TMA runs well ahead of the MMAs.
-// Decoded weight tiles have 3 stages; decoder warps write them as 256 rows of
-// 128 bytes, each row one NF4 block of 64 consecutive weights (row R at
-// R*128, 16-byte chunk c at (c ^ (R & 7))*16, the 128-byte swizzle pattern):
+// Shared memory holds two rings.  Activation tiles (512 x 64 bf16, K-major,
+// four TMA boxes) have 2 stages.  Decoded weight tiles have 4 stages; decoder
+// warps write them as 128 rows of 128 bytes, each row one NF4 block of 64
+// consecutive weights (row R at R*128, 16-byte chunk c at (c ^ (R & 7))*16,
+// the 128-byte swizzle pattern):
 //   forward   row R = 64*nb + k: weights (k0+k, n0+64nb .. +63) — an MN-major
 //             operand (atoms of 8 k-rows x 64 n; 8 KB between n-atoms);
 //   backward  row R: weights (n0+R, k0 .. k0+63) of W, i.e. row R of Ŵᵀ's
@@ -252,19 +255,22 @@ __global__ void __launch_bounds__(kSkThreads, 1)
 // After the last K-step of a tile, the LoRA step takes two activation stages:
 // Zc (or dZ) as the activation tile and B (or A) as the weight tile, both by
 // TMA with the rank padded to a multiple of 16 by TMA's zero fill; the decoder
-// warps skip it.  TMEM holds the two 128 x 256 fp32 accumulators (all 512
+// warps skip it.  TMEM holds the four 128 x 128 fp32 accumulators (all 512
 // columns); the epilogue releases each as soon as it has read it, so the next
-// tile's first MMAs into the first accumulator overlap the drain of the second.
+// tile's first MMAs into the first accumulators overlap the drain of the last.
 // ===========================================================================
-constexpr int kFAStages = 4;         // activation tiles (TMA)
-constexpr int kFBStages = 3;         // decoded weight tiles (decoder warps)
-constexpr int kFBM = 256, kFBN = 256;
-constexpr int kFA = 32768;           // 256 x 64 bf16
-constexpr int kFB = 32768;           // 256 x 64 bf16
-constexpr int kFThreads = 448;       // warp 0 TMA, 1 MMA, 2..9 decode, 10..13 epilogue
-constexpr int kFDecWarps = 8;
+constexpr int kFAStages = 2;         // activation tiles (TMA)
+constexpr int kFBStages = 4;         // decoded weight tiles (decoder warps)
+constexpr int kFBM = 512, kFBN = 128;
+constexpr int kFAcc = kFBM / 128;    // accumulators of 128 x kFBN fp32 in TMEM
+constexpr int kFA = kFBM * 128;      // 512 x 64 bf16
+constexpr int kFB = kFBN * 128;      // 128 x 64 bf16
+constexpr int kFDecWarps = kFBN / 32;   // one weight-tile row per decoder thread
 constexpr int kFEpiWarps = 4;
+constexpr int kFThreads = (2 + kFDecWarps + kFEpiWarps) * 32;  // TMA, MMA, decoders, epilogue
 constexpr size_t kFSmem = 1024 + kFAStages * kFA + kFBStages * kFB + 1024 + 512;
+static_assert(kFAcc * kFBN <= 512, "accumulators fit TMEM");
+static_assert(kFSmem <= 232448, "fused kernel shared memory");
 
 struct FusedArgs {
   int M;          // rows of the activation / output
@@ -403,8 +409,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
   uint64_t* full_b = empty_a + kFAStages;
   uint64_t* empty_b = full_b + kFBStages;
   uint64_t* tfull = empty_b + kFBStages;
-  uint64_t* tempty = tfull + 1;   // [2]: one per accumulator
-  uint64_t* drain = tempty + 2;
+  uint64_t* tempty = tfull + 1;   // [kFAcc]: one per accumulator
+  uint64_t* drain = tempty + kFAcc;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -420,8 +426,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
       mbar_init(&empty_b[s], 1);
     }
     mbar_init(tfull, 1);
-    mbar_init(&tempty[0], kFEpiWarps);
-    mbar_init(&tempty[1], kFEpiWarps);
+    for (int h = 0; h < kFAcc; ++h) mbar_init(&tempty[h], kFEpiWarps);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -445,7 +450,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
       tma_prefetch_desc(&tmLA);
       tma_prefetch_desc(&tmLB);
       uint32_t ia = 0;                          // activation-ring slot counter
-      uint32_t last_parity[kFAStages] = {2, 2, 2, 2};
+      uint32_t last_parity[kFAStages];
+#pragma unroll
+      for (int s = 0; s < kFAStages; ++s) last_parity[s] = 2;
       bool ok = true;
       auto take = [&](uint32_t& s_out) -> bool {
         const uint32_t s = ia % kFAStages, ph = (ia / kFAStages) & 1;
@@ -463,8 +470,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
           if (!take(s)) { ok = false; break; }
           uint8_t* a = sA + s * kFA;
           mbar_arrive_expect_tx(&full_a[s], kFA);
-          tma_load_2d(a, &tmAct, &full_a[s], kk * 64, m0);
-          tma_load_2d(a + 16384, &tmAct, &full_a[s], kk * 64, m0 + 128);
+#pragma unroll
+          for (int h = 0; h < kFAcc; ++h)
+            tma_load_2d(a + h * 16384, &tmAct, &full_a[s], kk * 64, m0 + h * 128);
         }
         if (!ok) break;
         // LoRA step: Zc / dZ into one stage, B / A into the next
@@ -472,14 +480,15 @@ __global__ void __launch_bounds__(kFThreads, 1)
         if (!take(s1)) { ok = false; break; }
         uint8_t* a = sA + s1 * kFA;
         mbar_arrive_expect_tx(&full_a[s1], kFA);
-        tma_load_2d(a, &tmLA, &full_a[s1], 0, m0);
-        tma_load_2d(a + 16384, &tmLA, &full_a[s1], 0, m0 + 128);
+#pragma unroll
+        for (int h = 0; h < kFAcc; ++h)
+          tma_load_2d(a + h * 16384, &tmLA, &full_a[s1], 0, m0 + h * 128);
         if (!take(s2)) { ok = false; break; }
         uint8_t* b = sA + s2 * kFA;
         mbar_arrive_expect_tx(&full_a[s2], kFB);
         if (!kBwd) {
 #pragma unroll
-          for (int nb = 0; nb < 4; ++nb)
+          for (int nb = 0; nb < kFBN / 64; ++nb)
             tma_load_2d(b + nb * 8192, &tmLB, &full_a[s2], n0 + nb * 64, 0);
         } else {
           tma_load_2d(b, &tmLB, &full_a[s2], 0, n0);
@@ -519,14 +528,14 @@ __global__ void __launch_bounds__(kFThreads, 1)
           const uint32_t a0 = smem_u32(sA + sa * kFA), b0 = smem_u32(sB + sb * kFB);
           const uint32_t acc = kk > 0 ? 1u : 0u;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
+          for (int h = 0; h < kFAcc; ++h) {
             if (kk == 0) {   // first K-step of a tile: wait until this accumulator is drained
               if (*abort_flag || !mbar_wait(&tempty[h], tph)) { ok = false; break; }
               tc_fence_after();
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              umma_bf16(tmem + h * 256, smem_desc(a0 + h * 16384 + j * 32, 16, 1024),
+              umma_bf16(tmem + h * kFBN, smem_desc(a0 + h * 16384 + j * 32, 16, 1024),
                         bdesc(b0, j), idesc, (acc || j > 0) ? 1u : 0u);
           }
           if (!ok) break;
@@ -539,10 +548,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
         if (!wait_a(s1) || !wait_a(s2)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a0 = smem_u32(sA + s1 * kFA), b0 = smem_u32(sA + s2 * kFA);
-        for (int j = 0; j < args.rsteps; ++j) {
-          umma_bf16(tmem, smem_desc(a0 + j * 32, 16, 1024), bdesc(b0, j), idesc, 1u);
-          umma_bf16(tmem + 256, smem_desc(a0 + 16384 + j * 32, 16, 1024), bdesc(b0, j), idesc, 1u);
-        }
+        for (int j = 0; j < args.rsteps; ++j)
+#pragma unroll
+          for (int h = 0; h < kFAcc; ++h)
+            umma_bf16(tmem + h * kFBN, smem_desc(a0 + h * 16384 + j * 32, 16, 1024), bdesc(b0, j),
+                      idesc, 1u);
         umma_commit(&empty_a[s1]);
         umma_commit(&empty_a[s2]);
         umma_commit(tfull);
@@ -553,7 +563,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     }
   } else if (warp < 2 + kFDecWarps) {
     // ------------------------------ decoders -------------------------------
-    const int R = threadIdx.x - 64;            // weight-tile row 0..255
+    const int R = threadIdx.x - 64;            // weight-tile row 0..kFBN-1
     const float off = args.sv.code8 != nullptr ? __ldg(args.sv.offset) : 0.0f;
     const int nsteps = args.nk;                // decoded steps per tile
     bool ok = true;
@@ -625,9 +635,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
       if (*abort_flag || !mbar_wait(tfull, tc & 1)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
+      for (int h = 0; h < kFAcc; ++h) {
         const int row = m0 + h * 128 + q * 32 + lane;
-        const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 256;
+        const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * kFBN;
 #pragma unroll 1
         for (int c = 0; c < kFBN / 32; ++c) {
           uint32_t v[32];
@@ -1347,7 +1357,7 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   // dX = G W^T + dZ A^T
   e = set_fused_attr<true>();
   if (e != cudaSuccess) return e;
-  if (!make_tmap_2d(&tAl, A, kBF16, 2, K, r, r, 64, 256, kSW128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tAl, A, kBF16, 2, K, r, r, 64, kFBN, kSW128)) return cudaErrorInvalidValue;
   CUtensorMap tdZa;
   if (!make_tmap_2d(&tdZa, dZ, kBF16, 2, M, r, r, 64, 128, kSW128)) return cudaErrorInvalidValue;
   FusedArgs fa;
