@@ -307,7 +307,8 @@ def quantize_bench(torch, q, dev, peaks):
 def run_case(args):
     """One kernel workload, --reps launches, no timing: the command ncu captures.
     gemv: forward with M <= 16 tokens (DQ weight, r = 16, c = 2);
-    quantize: NF4 + DQ quantization of a K x N bf16 weight."""
+    quantize: NF4 + DQ quantization of a K x N bf16 weight;
+    merge: the merged bf16 weight of a K x N DQ weight with r = 64."""
     import torch
     import bit_nf4_quantized_pack_b200 as q
     dev = torch.device("cuda", 0)
@@ -327,16 +328,57 @@ def run_case(args):
         X = torch.randn((Mg, Kg), generator=gen, device=dev).to(torch.bfloat16)
         for i in range(args.reps):
             q.linear_forward(X, ws[i % 2], A, B, 2.0, status=st)
-    else:
+    elif args.case == "quantize":
         Kq, Nq = (int(v) for v in (args.shape or "8192,22016").split(","))
         W = (torch.randn((Kq, Nq), generator=gen, device=dev) * 0.015).to(torch.bfloat16)
         w = q.quantize(W, double_quant=True, status=st)
         for _ in range(args.reps):
             q.quantize(W, double_quant=True, out=w, status=st)
+    else:
+        Kq, Nq = (int(v) for v in (args.shape or "8192,22016").split(","))
+        W = (torch.randn((Kq, Nq), generator=gen, device=dev) * 0.015).to(torch.bfloat16)
+        w = q.quantize(W, double_quant=True, status=st)
+        A = (torch.randn((Kq, 64), generator=gen, device=dev) * 0.01).to(torch.bfloat16)
+        B = (torch.randn((64, Nq), generator=gen, device=dev) * 0.01).to(torch.bfloat16)
+        for _ in range(args.reps):
+            q.merge(w, A, B, 0.25, out=W, status=st)
     torch.cuda.synchronize()
     code = q.status_sync(st)
     print(json.dumps({"case": args.case, "shape": args.shape, "reps": args.reps, "status": list(code)}))
     return 0 if code[0] == 0 else 1
+
+
+def merge_bench(torch, q, dev, peaks):
+    """Merge/export of the 8192x22016 weight with r = 64 (DQ state): GB/s of
+    P/2 + n1 + 4n2 + 4 (state) + 2r(K+N) (adapter) + 2P (bf16 output)."""
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(6)
+    Kq, Nq, rq = 8192, 22016, 64
+    W = (torch.randn((Kq, Nq), generator=gen, device=dev) * 0.015).to(torch.bfloat16)
+    w = q.quantize(W, double_quant=True)
+    del W
+    A = (torch.randn((Kq, rq), generator=gen, device=dev) * 0.01).to(torch.bfloat16)
+    B = (torch.randn((rq, Nq), generator=gen, device=dev) * 0.01).to(torch.bfloat16)
+    out = torch.empty((Kq, Nq), dtype=torch.bfloat16, device=dev)
+    st = q.new_status(dev)
+    for _ in range(3):
+        q.merge(w, A, B, 0.25, out=out, status=st)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 10
+    e0.record()
+    for _ in range(reps):
+        q.merge(w, A, B, 0.25, out=out, status=st)
+    e1.record()
+    torch.cuda.synchronize()
+    per = e0.elapsed_time(e1) / reps * 1e-3
+    P = Kq * Nq
+    n1 = P // 64
+    n2 = (n1 + 255) // 256
+    nbytes = P // 2 + n1 + 4 * n2 + 4 + 2 * rq * (Kq + Nq) + 2 * P
+    gbs = nbytes / per / 1e9
+    del out, w
+    return {"shape": [Kq, Nq], "r": rq, "us": per * 1e6, "GB/s": gbs, "frac": gbs / peaks["hbm"]}
 
 
 def main():
@@ -348,7 +390,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the GEMV and quantize sweeps")
     ap.add_argument("--kernels-only", action="store_true",
                     help="only the timed steps (no e2e, sweeps or CPU baseline): for profilers")
-    ap.add_argument("--case", choices=["gemv", "quantize"],
+    ap.add_argument("--case", choices=["gemv", "quantize", "merge"],
                     help="run one kernel workload --reps times and exit (for profilers)")
     ap.add_argument("--shape", default="",
                     help="M,K,N for --case gemv (default 1,4096,11008); K,N for --case quantize")
@@ -512,6 +554,7 @@ def main():
     if rank == 0 and not args.no_extras and not args.kernels_only:
         extras["gemv"] = gemv_sweep(torch, q, dev, peaks)
         extras["quantize"] = quantize_bench(torch, q, dev, peaks)
+        extras["merge"] = merge_bench(torch, q, dev, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.kernels_only:

@@ -23,7 +23,8 @@ import torch
 from . import _lib
 from ._lib import NF4StateC, QLoRAError, check, lib
 
-__all__ = ["NF4Weight", "quantize", "dequantize", "linear_forward", "linear_backward",
+__all__ = ["NF4Weight", "quantize", "dequantize", "merge", "merge_requantize",
+           "linear_forward", "linear_backward",
            "status_sync", "status_clear", "new_status", "QLoRAError", "lib"]
 
 BLOCKSIZE = 64
@@ -173,6 +174,33 @@ def dequantize(w: NF4Weight, *, out: torch.Tensor | None = None,
           "qlora_nf4_dequantize")
     _finish(status, own, "qlora_nf4_dequantize")
     return out
+
+
+def merge(w: NF4Weight, A, B, c: float, *, out: torch.Tensor | None = None,
+          status: torch.Tensor | None = None) -> torch.Tensor:
+    """The merged dense weight RN_bf16(Ŵ + c·A·B) (K x N bf16)."""
+    for t, n in ((A, "A"), (B, "B")):
+        _bf16(t, n)
+    K, N = w.shape
+    r = A.shape[1]
+    if A.shape[0] != K or tuple(B.shape) != (r, N):
+        raise ValueError("shape mismatch")
+    dev = w.packed.device
+    out = out if out is not None else torch.empty((K, N), dtype=torch.bfloat16, device=dev)
+    _bf16(out, "out")
+    st = w.cstruct()
+    own = status is None
+    status = new_status(dev) if own else status
+    check(lib.qlora_nf4_merge(K, N, r, C.byref(st), _ptr(A), _ptr(B), float(c), _ptr(out),
+                              _ptr(status), _stream()), "qlora_nf4_merge")
+    _finish(status, own, "qlora_nf4_merge")
+    return out
+
+
+def merge_requantize(w: NF4Weight, A, B, c: float, double_quant: bool = True, *,
+                     status: torch.Tensor | None = None) -> NF4Weight:
+    """The merged weight quantized again to NF4 (a new quantization step)."""
+    return quantize(merge(w, A, B, c, status=status), double_quant=double_quant, status=status)
 
 
 def _bf16(t, name):

@@ -178,6 +178,22 @@ qlora_status qlora_linear_fwd(int64_t M, int64_t K, int64_t N, int32_t r, const 
   return cuda_status(e);
 }
 
+qlora_status qlora_nf4_merge(int64_t K, int64_t N, int32_t r, const qlora_nf4_state* W,
+                             const uint16_t* A, const uint16_t* B, float c, uint16_t* out,
+                             int32_t* d_status, qlora_stream_t stream) {
+  qlora_status v = check_linear_shape(1, K, N, r);
+  if (v != QLORA_OK) return v;
+  v = check_state(W, true);
+  if (v != QLORA_OK) return v;
+  if (W->numel != K * N) return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(c)) return QLORA_ERR_INVALID_ARG;
+  const void* ptrs[] = {A, B, out};
+  for (const void* p : ptrs)
+    if (!p || !aligned(p, 16)) return QLORA_ERR_INVALID_ARG;
+  return cuda_status(qnf4::launch_merge(K, N, r, c, view_of(W), W->packed, A, B, out, d_status,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
 qlora_status qlora_linear_bwd(int64_t M, int64_t K, int64_t N, int32_t r, const uint16_t* dY,
                               const uint16_t* X, const uint16_t* Zc, const qlora_nf4_state* W,
                               const uint16_t* A, const uint16_t* B, float c, uint16_t* dX,

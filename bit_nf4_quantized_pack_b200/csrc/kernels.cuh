@@ -81,6 +81,11 @@ struct ScaleView {
   const float* offset;
 };
 
+// merge.cu — the merged dense weight RN_bf16(ŵ + c·A·B)
+cudaError_t launch_merge(int64_t K, int64_t N, int r, float c, ScaleView sv, const uint8_t* packed,
+                         const uint16_t* A, const uint16_t* B, uint16_t* out, int32_t* d_status,
+                         cudaStream_t st);
+
 // linear.cu — forward and backward of the layer
 size_t linear_fwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r);
 size_t linear_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r);

@@ -219,6 +219,27 @@ qlora_status qlora_linear_bwd(int64_t M, int64_t K, int64_t N, int32_t r,
                               qlora_stream_t stream);
 
 /*
+ * Merge / export — page "QLoRA：冻结的 4-bit 权重怎样参与一次微调",
+ * §Merge 后还是不是训练时的函数: after training, the layer's function is Ŵ
+ * together with the adapter; one delivery is the dense merged weight
+ *   out = RN_bf16( Ŵ + c·A·B ),   Ŵ = RN_bf16(C_j·a') as qlora_nf4_dequantize.
+ * The rank-r product is formed in fp32 (bf16 operands, fp32 accumulation) and
+ * added to Ŵ in one fp32 fma before the single rounding to bf16, so each
+ * output is within one bf16 ulp of the correctly rounded exact merge.  For
+ * the re-quantized delivery, pass `out` to qlora_nf4_quantize (a new
+ * quantization step: not the trained function in general).
+ *   W   : NF4 state of the K×N weight (numel must equal K·N)
+ *   A   : device bf16 K×r      B : device bf16 r×N     (row-major)
+ *   out : device bf16 K×N output (may not alias A, B or the state)
+ * Shapes as qlora_linear_fwd (K % 64 == 0, N % 64 == 0, 8 <= r <= 64, r % 8
+ * == 0).  A non-finite decode scale raises QLORA_ERR_NONFINITE in d_status.
+ * No workspace; asynchronous on `stream`.
+ */
+qlora_status qlora_nf4_merge(int64_t K, int64_t N, int32_t r, const qlora_nf4_state* W,
+                             const uint16_t* A, const uint16_t* B, float c, uint16_t* out,
+                             int32_t* d_status, qlora_stream_t stream);
+
+/*
  * Launch timing, for measurement tools (no counterpart on the pages).  While
  * enabled, each kernel launch of the library is bracketed by two CUDA events
  * recorded on the stream the kernel runs on.  qlora_profile_read waits for

@@ -158,3 +158,50 @@ def test_full_size_projection_sampled_rows():
     dZ = c * (G64 @ B.T)
     assert rel_fro(to_np(dA), X64.T @ dZ) <= TOL
     assert rel_fro(to_np(dB), c * ((X64 @ A).T @ G64)) <= TOL
+
+
+MERGE_CASES = [(64, 128, 8, True), (320, 384, 16, False), (256, 576, 64, True), (128, 64, 24, True)]
+
+
+@pytest.mark.parametrize("K,N,r,dq", MERGE_CASES)
+def test_merge_parity(K, N, r, dq):
+    """qlora_nf4_merge against the oracle's RN_bf16(W_hat + cAB): every output
+    within one bf16 ulp (fp32 rank-r sum on the device), nearly all exact."""
+    from oracle.merge import merge_bf16, merge_exact
+    q = _q()
+    lin = S.random_case(77 + K + N + r, 4, K, N, r)
+    c = 16.0 / r
+    wq = q.quantize(to_dev(lin.W), double_quant=dq)
+    got = to_np(q.merge(wq, to_dev(lin.A), to_dev(lin.B), c))
+    ow = OracleWeight(lin.W, dq)
+    ref = merge_bf16(ow.w_hat, lin.A, lin.B, c)
+    ex = merge_exact(ow.w_hat, lin.A, lin.B, c)
+    _, e = np.frexp(np.maximum(np.abs(ex), 1e-30))
+    ulp = np.ldexp(1.0, e - 8)
+    assert np.all(np.abs(got - ref) <= ulp), float(np.max(np.abs(got - ref) / ulp))
+    assert np.mean(got != ref) < 0.01
+
+
+def test_merge_zero_adapter_is_dequantize():
+    q = _q()
+    lin = S.random_case(91, 4, 192, 256, 16)
+    wq = q.quantize(to_dev(lin.W), double_quant=True)
+    A = torch.zeros((192, 16), dtype=torch.bfloat16, device="cuda")
+    got = q.merge(wq, A, to_dev(lin.B), 2.0)
+    assert torch.equal(got, q.dequantize(wq))
+
+
+def test_merge_requantize_matches_oracle_quantize_of_merged():
+    """Re-quantized delivery: the GPU's quantization of its merged weight is the
+    oracle's quantization of the same bf16 values, bit for bit."""
+    from oracle import nf4
+    q = _q()
+    lin = S.random_case(93, 4, 128, 256, 16)
+    wq = q.quantize(to_dev(lin.W), double_quant=True)
+    merged = q.merge(wq, to_dev(lin.A), to_dev(lin.B), 2.0)
+    rq = q.merge_requantize(wq, to_dev(lin.A), to_dev(lin.B), 2.0, double_quant=True)
+    codes, absmax = nf4.quantize_nf4(to_np(merged).ravel())
+    payload, _ = nf4.pack_codes(codes)
+    code8, s2, off = nf4.double_quantize(absmax)
+    assert np.array_equal(rq.packed.cpu().numpy(), payload)
+    assert np.array_equal(rq.code8.cpu().numpy(), code8)
