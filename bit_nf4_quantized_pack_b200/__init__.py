@@ -235,9 +235,12 @@ def linear_forward(X, w: NF4Weight, A, B, c: float, *, Y=None, Zc=None, status=N
 
 def linear_backward(dY, X, Zc, w: NF4Weight, A, B, c: float, *, dX=None, dA=None, dB=None,
                     status=None, workspace=None):
-    """dX = dY·Ŵᵀ + c·(dY·Bᵀ)·Aᵀ, dA = Xᵀ·(c·dY·Bᵀ), dB = Zcᵀ·dY; returns (dX, dA, dB)."""
-    for t, n in ((dY, "dY"), (X, "X"), (Zc, "Zc"), (A, "A"), (B, "B")):
+    """dX = dY·Ŵᵀ + c·(dY·Bᵀ)·Aᵀ, dA = Xᵀ·(c·dY·Bᵀ), dB = Zcᵀ·dY; returns (dX, dA, dB).
+    Zc=None recomputes bf16(c·X·A) inside the call (bit-identical to the forward's)."""
+    for t, n in ((dY, "dY"), (X, "X"), (A, "A"), (B, "B")):
         _bf16(t, n)
+    if Zc is not None:
+        _bf16(Zc, "Zc")
     M, K = X.shape
     N = dY.shape[1]
     r = A.shape[1]
@@ -250,7 +253,8 @@ def linear_backward(dY, X, Zc, w: NF4Weight, A, B, c: float, *, dX=None, dA=None
     st = w.cstruct()
     own = status is None
     status = new_status(dev) if own else status
-    check(lib.qlora_linear_bwd(M, K, N, r, _ptr(dY), _ptr(X), _ptr(Zc), C.byref(st), _ptr(A),
+    check(lib.qlora_linear_bwd(M, K, N, r, _ptr(dY), _ptr(X), _ptr(Zc) if Zc is not None else None,
+                               C.byref(st), _ptr(A),
                                _ptr(B), float(c), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws),
                                ws.numel() if ws is not None else 0, _ptr(status), _stream()),
           "qlora_linear_bwd")

@@ -205,9 +205,10 @@ qlora_status qlora_linear_bwd(int64_t M, int64_t K, int64_t N, int32_t r, const 
   if (v != QLORA_OK) return v;
   if (W->numel != K * N) return QLORA_ERR_INVALID_ARG;
   if (!std::isfinite(c)) return QLORA_ERR_INVALID_ARG;
-  const void* ptrs[] = {dY, X, Zc, A, B, dX, dA, dB};
+  const void* ptrs[] = {dY, X, A, B, dX, dA, dB};
   for (const void* p : ptrs)
     if (!p || !aligned(p, 16)) return QLORA_ERR_INVALID_ARG;
+  if (Zc && !aligned(Zc, 16)) return QLORA_ERR_INVALID_ARG;   // null: recompute it
   const size_t need = qlora_linear_bwd_workspace_size(M, K, N, r);
   if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 16))) return QLORA_ERR_INVALID_ARG;
   const int sms = sm_count();

@@ -1208,7 +1208,8 @@ size_t linear_fwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) {
 size_t linear_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) {
   (void)K;
   (void)N;
-  return align256(static_cast<size_t>(M) * r * 2);   // dZ (bf16, M x r)
+  // dZ, and Zc when the caller recomputes it instead of saving it (both bf16, M x r)
+  return 2 * align256(static_cast<size_t>(M) * r * 2);
 }
 
 cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint16_t* X,
@@ -1327,12 +1328,25 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   (void)num_sms;
   WsCursor cur{static_cast<char*>(ws), ws_bytes};
   uint16_t* dZ = static_cast<uint16_t*>(cur.take(static_cast<size_t>(M) * r * 2));
+  uint16_t* Zc_ws = static_cast<uint16_t*>(cur.take(static_cast<size_t>(M) * r * 2));
   const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(N / 64), g_ws_sms);
   const int nkm = static_cast<int>((M + 63) / 64);
   const int Sa = skinny_splits(static_cast<int>(K), nkm, g_ws_sms);
   const int Sb = skinny_splits(static_cast<int>(N), nkm, g_ws_sms);
   if (!cur.ok) return cudaErrorInvalidValue;
   cudaError_t e = cudaSuccess;
+  if (Zc == nullptr) {
+    // saved-activation policy "recompute": Zc = bf16(c X A) exactly as the
+    // forward forms it (same kernel, same splits, so the same bits)
+    CUtensorMap tXf, tAf;
+    if (!make_tmap_2d(&tXf, X, kBF16, 2, M, K, K, 64, 128, kSW128)) return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&tAf, A, kBF16, 2, K, r, r, 64, 64, kSW128)) return cudaErrorInvalidValue;
+    const int Sf = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
+    e = run_skinny<false, true>(tXf, tAf, static_cast<int>(M), static_cast<int>(K), r, c, 0, Zc_ws,
+                                r, Sf, d_status, st);
+    if (e != cudaSuccess) return e;
+    Zc = Zc_ws;
+  }
 
   CUtensorMap tG, tBk, tXmn, tdZ, tGmn, tZcmn, tAl;
   // dZ = c * G B^T : A operand G (K-major over N), B operand B (K-major: rows r, cols N)

@@ -204,7 +204,14 @@ qlora_status qlora_linear_fwd(int64_t M, int64_t K, int64_t N, int32_t r,
  * §冻结权重为什么仍然需要输入梯度:
  *   dZ = c·dY·Bᵀ,   dX = dY·Ŵᵀ + dZ·Aᵀ,   dA = Xᵀ·dZ,   dB = Zcᵀ·dY  (= c·Zᵀ·dY)
  *
- *   dY : device bf16 M×N       X : device bf16 M×K      Zc : the forward's Zc
+ *   dY : device bf16 M×N       X : device bf16 M×K
+ *   Zc : the forward's Zc, or NULL: the call then recomputes bf16(c·X·A) with
+ *        the forward's own kernel and split (bit-identical), so a chain of
+ *        layers need not keep M×r per layer between its forward and backward
+ *        (recompute instead of save, as gradient checkpointing trades
+ *        recomputation for stored activations: page "SFT（四）：QLoRA的4-bit
+ *        量化与LoRA微调原理", §26.2 为什么开启 Gradient Checkpointing; page
+ *        "QLoRA：冻结的 4-bit 权重怎样参与一次微调", §Paged Optimizer 管理哪一部分内存)
  *   dX : device bf16 M×K output
  *   dA : device fp32 K×r output     dB : device fp32 r×N output
  * No gradient is produced for W (the frozen base).  Same shape rules and
