@@ -30,3 +30,45 @@ def int4_quantize_block(values):
 
 def int4_dequantize_block(q, s):
     return [s * v for v in q]
+
+
+# ----------------------------------------------------------------------------
+# Library storage format of the same quantizer (whole weights, vectorised)
+# ----------------------------------------------------------------------------
+# Readings of the page's formula for a stored format (the page shows the
+# arithmetic only): blocks of 64 consecutive row-major elements, as NF4; the
+# stored per-block scale is fp32, s = RN_fp32(amax / 7) with amax / 7 formed
+# in fp64; q is decided on w / s in fp64 with the rule above (half away from
+# zero, then clip to [-7, 7]); the code is q + 8 (1 .. 15), packed two per byte
+# like NF4, and an odd tail is padded with code 8 (q = 0); the decoded weight
+# is RN_bf16(q * s), the product exact.
+INT4_PAD_CODE = 8
+
+
+def int4_quantize(w, blocksize: int = 64):
+    """Returns (codes uint8[numel], scales float32[n1]) of a flat weight."""
+    import numpy as np
+    x = np.asarray(w, dtype=np.float32).ravel().astype(np.float64)
+    if not np.all(np.isfinite(x)):
+        raise ValueError("nonfinite input")
+    n = x.size
+    n1 = (n + blocksize - 1) // blocksize
+    pad = n1 * blocksize - n
+    xb = np.concatenate([x, np.zeros(pad)]).reshape(n1, blocksize)
+    amax = np.max(np.abs(xb), axis=1)
+    s = np.where(amax > 0, amax / 7.0, 1.0).astype(np.float32)
+    t = xb / s.astype(np.float64)[:, None]
+    r = np.floor(np.abs(t) + 0.5) * np.where(t >= 0, 1.0, -1.0)
+    q = np.clip(r, -7, 7).astype(np.int64)
+    codes = (q + 8).astype(np.uint8).ravel()[:n]
+    return codes, s
+
+
+def int4_dequantize(codes, scales, blocksize: int = 64):
+    """RN_bf16((code - 8) * s) per element (fp64 holding bf16 values)."""
+    import numpy as np
+    from .nf4 import round_to_bf16
+    c = np.asarray(codes, dtype=np.int64).ravel()
+    s = np.asarray(scales, dtype=np.float32).astype(np.float64)
+    per = s[np.arange(c.size) // blocksize]
+    return round_to_bf16((c - 8) * per)

@@ -120,3 +120,43 @@ def test_int4_uniform_worked_example(golden):
     tol = g["approx_abs_tol"]
     assert all(abs(a - b) < tol for a, b in zip(w_hat, g["w_hat_approx"]))
     assert all(abs((w - h) - e) < tol for w, h, e in zip(g["W"], w_hat, g["error_approx"]))
+
+
+def test_int4_library_format_worked_example(golden):
+    """The stored format reproduces the page's example: q = [-7, -2, 1, 5]
+    (codes q + 8), scale ~0.1714, reconstruction ~[-1.200, -0.343, 0.171, 0.857]."""
+    from oracle.int4 import int4_dequantize, int4_quantize
+    g = golden("int4_uniform_example.json")
+    codes, s = int4_quantize(np.array(g["W"], dtype=np.float32))
+    assert list(codes.astype(int) - 8) == g["q"]
+    assert abs(float(s[0]) - g["s_approx"]) < 1e-4
+    w_hat = int4_dequantize(codes, s)
+    # the reconstruction is rounded to bf16 (3 significant digits)
+    assert np.all(np.abs(w_hat - np.array(g["w_hat_approx"])) < 5e-3)
+
+
+def test_int4_library_format_against_block_rule():
+    """Same codes as the fp64 per-block rule except where w/s sits within the
+    fp32 rounding of s from a .5 tie; all-zero blocks get scale 1; padding 8."""
+    from oracle.int4 import int4_quantize
+    rng = np.random.default_rng(8)
+    w = rng.normal(0, 0.02, 64 * 500).astype(np.float32)
+    w[64 * 7:64 * 8] = 0.0
+    codes, s = int4_quantize(w)
+    assert s[7] == 1.0 and np.all(codes[64 * 7:64 * 8] == 8)
+    agree = 0
+    for b in range(500):
+        q_ref, s_ref = int4_quantize_block(w[64 * b:64 * b + 64])
+        q = list(codes[64 * b:64 * b + 64].astype(int) - 8)
+        agree += sum(int(a == c) for a, c in zip(q, q_ref))
+        assert abs(float(s[b]) - s_ref) <= 2 ** -23 * s_ref
+    assert agree >= 64 * 500 - 5
+    # brute force on a tiny block: every q is the nearest integer (ties away
+    # from zero) of w / s within [-7, 7]
+    w = np.array([0.7, -0.05, 0.35, 0.0, -0.7, 0.2499], dtype=np.float32)
+    codes, s = int4_quantize(w)
+    for v, c in zip(w.astype(np.float64), codes.astype(int)):
+        t = v / float(s[0])
+        cands = list(range(-7, 8))
+        best = min(cands, key=lambda q: (abs(t - q), -abs(q)))
+        assert c - 8 == best
