@@ -58,6 +58,7 @@ class NF4Weight:
     code8: torch.Tensor | None = None
     s2: torch.Tensor | None = None
     offset: torch.Tensor | None = None
+    codebook: int = 0      # 0: NF4, 1: uniform INT4 (absmax then holds s = amax / 7)
 
     @property
     def numel(self) -> int:
@@ -72,7 +73,7 @@ class NF4Weight:
         st.blocksize = BLOCKSIZE
         st.double_quant = 1 if self.double_quant else 0
         st.dq_blocksize = DQ_BLOCKSIZE
-        st.reserved = 0
+        st.codebook = int(self.codebook)
         st.packed = self.packed.data_ptr()
         st.absmax = self.absmax.data_ptr() if self.absmax is not None else None
         st.code8 = self.code8.data_ptr() if self.code8 is not None else None
@@ -81,14 +82,16 @@ class NF4Weight:
         return st
 
     @staticmethod
-    def empty(shape, double_quant: bool, device="cuda") -> "NF4Weight":
+    def empty(shape, double_quant: bool, device="cuda", codebook: int = 0) -> "NF4Weight":
         numel = 1
         for s in shape:
             numel *= int(s)
         n1, n2 = n1_of(numel), n2_of(numel)
         u8, f32 = torch.uint8, torch.float32
+        if codebook and double_quant:
+            raise ValueError("the INT4 codebook has no double quantization")
         w = NF4Weight(tuple(int(s) for s in shape), bool(double_quant),
-                      torch.empty((numel + 1) // 2, dtype=u8, device=device))
+                      torch.empty((numel + 1) // 2, dtype=u8, device=device), codebook=int(codebook))
         if double_quant:
             w.code8 = torch.empty(n1, dtype=u8, device=device)
             w.s2 = torch.empty(n2, dtype=f32, device=device)
@@ -140,8 +143,15 @@ def _finish(status, own_status, where):
 
 
 def quantize(W: torch.Tensor, double_quant: bool = True, *, out: NF4Weight | None = None,
-             status: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> NF4Weight:
-    """Blockwise NF4 quantization of a contiguous bf16 or fp32 CUDA tensor."""
+             status: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+             codebook: str = "nf4") -> NF4Weight:
+    """Blockwise 4-bit quantization of a contiguous bf16 or fp32 CUDA tensor:
+    codebook "nf4" (optionally double-quantized) or "int4" (uniform signed)."""
+    if codebook not in ("nf4", "int4"):
+        raise ValueError("codebook must be 'nf4' or 'int4'")
+    cb = 1 if codebook == "int4" else 0
+    if cb:
+        double_quant = False
     if W.dtype == torch.bfloat16:
         dt = _lib.QLORA_DTYPE_BF16
     elif W.dtype == torch.float32:
@@ -150,7 +160,9 @@ def quantize(W: torch.Tensor, double_quant: bool = True, *, out: NF4Weight | Non
         raise TypeError("W must be bfloat16 or float32")
     if not W.is_contiguous():
         raise ValueError("W must be contiguous")
-    w = out if out is not None else NF4Weight.empty(W.shape, double_quant, W.device)
+    w = out if out is not None else NF4Weight.empty(W.shape, double_quant, W.device, codebook=cb)
+    if w.codebook != cb:
+        raise ValueError("out has another codebook")
     st = w.cstruct()
     need = int(lib.qlora_nf4_quantize_workspace_size(w.numel, st.double_quant))
     ws = workspace if workspace is not None else _ws.get(("q", W.device), need, W.device)

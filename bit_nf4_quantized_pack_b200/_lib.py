@@ -20,7 +20,7 @@ QLORA_ERR_CUDA = 5
 QLORA_ERR_TIMEOUT = 6
 QLORA_DTYPE_BF16 = 0
 QLORA_DTYPE_F32 = 1
-ABI_VERSION = 1
+ABI_VERSION = 2
 NOALLOC_MAX_NUMEL = 1 << 26
 
 
@@ -31,7 +31,7 @@ class NF4StateC(C.Structure):
         ("blocksize", C.c_int32),
         ("double_quant", C.c_int32),
         ("dq_blocksize", C.c_int32),
-        ("reserved", C.c_int32),
+        ("codebook", C.c_int32),
         ("packed", C.c_void_p),
         ("absmax", C.c_void_p),
         ("code8", C.c_void_p),

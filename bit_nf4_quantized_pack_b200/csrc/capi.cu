@@ -32,8 +32,10 @@ qlora_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : Q
 // Common checks of a quantized-state struct.
 qlora_status check_state(const qlora_nf4_state* st, bool need_scales) {
   if (!st) return QLORA_ERR_INVALID_ARG;
-  if (st->numel < 1 || st->blocksize != qnf4::kBlock || st->reserved != 0) return QLORA_ERR_INVALID_ARG;
+  if (st->numel < 1 || st->blocksize != qnf4::kBlock) return QLORA_ERR_INVALID_ARG;
+  if (st->codebook != QLORA_CODEBOOK_NF4 && st->codebook != QLORA_CODEBOOK_INT4) return QLORA_ERR_INVALID_ARG;
   if (st->double_quant != 0 && st->double_quant != 1) return QLORA_ERR_INVALID_ARG;
+  if (st->codebook == QLORA_CODEBOOK_INT4 && st->double_quant) return QLORA_ERR_UNSUPPORTED;
   if (st->numel > kMaxNumel) return QLORA_ERR_UNSUPPORTED;
   if (!st->packed || !aligned(st->packed, 16)) return QLORA_ERR_INVALID_ARG;
   if (!need_scales) return QLORA_OK;
@@ -49,6 +51,7 @@ qlora_status check_state(const qlora_nf4_state* st, bool need_scales) {
 
 qnf4::ScaleView view_of(const qlora_nf4_state* st) {
   qnf4::ScaleView v{};
+  v.codebook = st->codebook;
   if (st->double_quant) {
     v.code8 = st->code8;
     v.s2 = st->s2;
@@ -127,7 +130,8 @@ qlora_status qlora_nf4_quantize(const void* W, qlora_dtype dtype, const qlora_nf
   if (sms <= 0) return QLORA_ERR_CUDA;
   cudaError_t e = qnf4::launch_quantize(W, dtype, st->numel, st->packed, st->absmax,
                                         st->double_quant != 0, st->code8, st->s2, st->offset, ws,
-                                        d_status, reinterpret_cast<cudaStream_t>(stream), sms);
+                                        d_status, reinterpret_cast<cudaStream_t>(stream), sms,
+                                        st->codebook);
   return cuda_status(e);
 }
 
@@ -141,7 +145,7 @@ qlora_status qlora_nf4_dequantize(const qlora_nf4_state* st, uint16_t* W_hat, in
   const qnf4::ScaleView sv = view_of(st);
   cudaError_t e = qnf4::launch_dequantize(st->packed, st->numel, sv.absmax, sv.code8, sv.s2,
                                           sv.offset, W_hat, d_status,
-                                          reinterpret_cast<cudaStream_t>(stream), sms);
+                                          reinterpret_cast<cudaStream_t>(stream), sms, sv.codebook);
   return cuda_status(e);
 }
 

@@ -13,6 +13,7 @@ namespace qnf4 {
 constexpr int kBlock = 64;     // first-level NF4 block
 constexpr int kDQBlock = 256;  // second-level block of the scale codes
 constexpr int kPadCode = 7;    // odd-tail padding code (exact zero)
+constexpr int kPadCodeInt4 = 8;   // the same for the uniform INT4 codebook (q = 0)
 
 // The 16 NF4 reconstruction values as printed on the page "QLoRA：冻结的
 // 4-bit 权重怎样参与一次微调" (§从 NF4 索引打包成字节).  Every value is an exact
@@ -23,6 +24,13 @@ constexpr int kPadCode = 7;    // odd-tail padding code (exact zero)
       0.07958029955625534f, 0.16093020141124725f, 0.24611230194568634f,         \
       0.33791524171829224f, 0.44070982933044434f, 0.5626170039176941f,          \
       0.7229568362236023f, 1.0f
+
+// The uniform signed INT4 codebook (page "SFT（四）：QLoRA的4-bit量化与LoRA微调原理",
+// §6 先理解最普通的分块量化: w_hat = s·q, q in [-7, 7]): code j holds q = j - 8;
+// the quantizer emits codes 1 .. 15 and pads an odd tail with code 8 (q = 0).
+#define QNF4_INT4_VALUES                                                         \
+  -8.0f, -7.0f, -6.0f, -5.0f, -4.0f, -3.0f, -2.0f, -1.0f, 0.0f, 1.0f, 2.0f, 3.0f, \
+      4.0f, 5.0f, 6.0f, 7.0f
 
 // Raise an error bit in the caller's device status word.
 __device__ __forceinline__ void raise_status(int32_t* d_status, int code) {

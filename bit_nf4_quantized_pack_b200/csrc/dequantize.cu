@@ -9,7 +9,7 @@
 
 namespace qnf4 {
 
-__constant__ float kNF4d[16] = {QNF4_TABLE_VALUES};
+__constant__ float kNF4d[32] = {QNF4_TABLE_VALUES, QNF4_INT4_VALUES};   // NF4, INT4
 
 // Per 64-block decode scale: absmax, or T8[q]*s2 + offset with each operation
 // rounded to fp32 (no fusion).
@@ -26,11 +26,11 @@ __device__ __forceinline__ float decode_scale(int64_t blk, const float* __restri
 __global__ void __launch_bounds__(256) nf4_dequant_kernel(
     const uint8_t* __restrict__ packed, int64_t numel, const float* __restrict__ absmax,
     const uint8_t* __restrict__ code8, const float* __restrict__ s2,
-    const float* __restrict__ offset, uint16_t* __restrict__ out, int32_t* d_status) {
+    const float* __restrict__ offset, uint16_t* __restrict__ out, int32_t* d_status, int codebook) {
   __shared__ float C[16];
   __shared__ float t8[256];
   pdl_launch_dependents();
-  if (threadIdx.x < 16) C[threadIdx.x] = kNF4d[threadIdx.x];
+  if (threadIdx.x < 16) C[threadIdx.x] = kNF4d[16 * codebook + threadIdx.x];
   if (code8 != nullptr) build_t8(t8);
   __syncthreads();
   pdl_wait();   // the tables above read no global memory
@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(
         }
       if ((numel & 1) && ((nbytes - 1) - b0) < 4) {
         const int k = static_cast<int>((nbytes - 1) - b0);
-        badpad |= ((word >> (8 * k)) & 0xFu) != static_cast<uint32_t>(kPadCode);
+        badpad |= ((word >> (8 * k)) & 0xFu) != static_cast<uint32_t>(codebook ? kPadCodeInt4 : kPadCode);
       }
     }
     uint32_t o[4];
@@ -82,7 +82,8 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(
 
 cudaError_t launch_dequantize(const uint8_t* packed, int64_t numel, const float* absmax,
                               const uint8_t* code8, const float* s2, const float* offset,
-                              uint16_t* out, int32_t* d_status, cudaStream_t st, int num_sms) {
+                              uint16_t* out, int32_t* d_status, cudaStream_t st, int num_sms,
+                              int codebook) {
   const int threads = 256;
   const int64_t ngroups = (numel + 7) >> 3;
   const int64_t want = (ngroups + threads - 1) / threads;
@@ -90,7 +91,7 @@ cudaError_t launch_dequantize(const uint8_t* packed, int64_t numel, const float*
   {
     ProfScope prof(kProfDequantize, st);
     const cudaError_t e = launch_pdl(nf4_dequant_kernel, dim3(blocks), dim3(threads), 0, st, 1, packed,
-                                     numel, absmax, code8, s2, offset, out, d_status);
+                                     numel, absmax, code8, s2, offset, out, d_status, codebook);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();

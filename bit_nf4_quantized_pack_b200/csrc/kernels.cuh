@@ -65,16 +65,19 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // quantize.cu
 cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* packed,
                             float* absmax_out, bool dq, uint8_t* code8, float* s2, float* offset,
-                            void* ws, int32_t* d_status, cudaStream_t st, int num_sms);
+                            void* ws, int32_t* d_status, cudaStream_t st, int num_sms,
+                            int codebook = 0);
 size_t quantize_workspace_bytes(int64_t numel, bool dq);
 
 // dequantize.cu
 cudaError_t launch_dequantize(const uint8_t* packed, int64_t numel, const float* absmax,
                               const uint8_t* code8, const float* s2, const float* offset,
-                              uint16_t* out, int32_t* d_status, cudaStream_t st, int num_sms);
+                              uint16_t* out, int32_t* d_status, cudaStream_t st, int num_sms,
+                              int codebook = 0);
 
 // Decode-scale view of a quantized weight, shared by the GEMM and GEMV paths.
 struct ScaleView {
+  int codebook;          // 0: NF4, 1: uniform INT4 (its stored scale is amax / 7)
   const float* absmax;   // non-null when not double-quantized
   const uint8_t* code8;  // non-null when double-quantized
   const float* s2;

@@ -30,7 +30,8 @@
 
 namespace qnf4 {
 
-__constant__ float kNF4g[16] = {QNF4_TABLE_VALUES};
+// code values of the two codebooks: [0, 16) NF4, [16, 32) uniform INT4
+__constant__ float kNF4g[32] = {QNF4_TABLE_VALUES, QNF4_INT4_VALUES};
 
 // ===========================================================================
 // Skinny contraction:  D[m'][n'] = sum_k' A(m',k') * B(n',k'),  n' < 64.
@@ -318,10 +319,10 @@ __device__ __forceinline__ uint4 decode8(uint32_t p, const uint32_t (&H)[4],
 }
 
 // Per-block table: entry j = bf16(C_j * a) (fp32 product, then bf16).
-__device__ __forceinline__ void build_lut(float a, uint32_t (&H)[4], uint32_t (&L)[4]) {
+__device__ __forceinline__ void build_lut(const float* C, float a, uint32_t (&H)[4], uint32_t (&L)[4]) {
   uint32_t w[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(kNF4g[2 * i] * a, kNF4g[2 * i + 1] * a);
+  for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(C[2 * i] * a, C[2 * i + 1] * a);
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     H[q] = prmt(w[2 * q], w[2 * q + 1], 0x7531u);
@@ -584,7 +585,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
                             ? f.absv
                             : __fadd_rn(__fmul_rn(t8[f.q], f.s2v), off);
         uint32_t H[4], L[4];
-        build_lut(a, H, L);
+        build_lut(kNF4g + 16 * args.sv.codebook, a, H, L);
         const uint32_t pw[8] = {f.p0.x, f.p0.y, f.p0.z, f.p0.w, f.p1.x, f.p1.y, f.p1.z, f.p1.w};
 #pragma unroll
         for (int c = 0; c < 8; ++c)
@@ -849,7 +850,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     // fixed table: entry e -> (bf16(C[e >> 4]) | bf16(C[e & 15]) << 16), one
     // copy per bank so that 32 lanes reading any entries never conflict
     {
-      const float cv = kNF4g[lane & 15];
+      const float cv = kNF4g[16 * args.sv.codebook + (lane & 15)];
       for (int e = warp; e < 256; e += kGvCompute)   // entry e is written by one warp
         table[e * 64 + lane] =
             pack_bf16x2(__shfl_sync(0xFFFFFFFFu, cv, e >> 4), __shfl_sync(0xFFFFFFFFu, cv, e & 15));

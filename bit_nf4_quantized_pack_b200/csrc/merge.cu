@@ -17,7 +17,7 @@
 
 namespace qnf4 {
 
-__constant__ float kNF4m[16] = {QNF4_TABLE_VALUES};
+__constant__ float kNF4m[32] = {QNF4_TABLE_VALUES, QNF4_INT4_VALUES};   // NF4, INT4
 
 struct MergeArgs {
   int K, N, r;
@@ -98,13 +98,14 @@ __global__ void __launch_bounds__(256) nf4_merge_kernel(MergeArgs a) {
     const uint4* src = reinterpret_cast<const uint4*>(a.packed + (static_cast<int64_t>(k) * a.N + n0) / 2);
     const uint4 q0 = __ldg(src), q1 = __ldg(src + 1);
     const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    const float* Ctab = kNF4m + 16 * a.sv.codebook;
     uint16_t* dst = a.out + static_cast<int64_t>(k) * a.N + n0 + 2 * t;
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
       // byte 4s + t holds columns 8s + 2t (high nibble) and 8s + 2t + 1
       const uint32_t byte = (w[s] >> (8 * t)) & 0xFFu;
-      const float w0 = bf16_bits_to_f32(bf16_of_exact_product(kNF4m[byte >> 4], sc));
-      const float w1 = bf16_bits_to_f32(bf16_of_exact_product(kNF4m[byte & 15u], sc));
+      const float w0 = bf16_bits_to_f32(bf16_of_exact_product(Ctab[byte >> 4], sc));
+      const float w1 = bf16_bits_to_f32(bf16_of_exact_product(Ctab[byte & 15u], sc));
       const float m0 = fmaf(a.c, acc[s][2 * half], w0);
       const float m1 = fmaf(a.c, acc[s][2 * half + 1], w1);
       *reinterpret_cast<uint32_t*>(dst + 8 * s) = pack_bf16x2(m0, m1);

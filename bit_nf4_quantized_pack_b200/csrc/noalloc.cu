@@ -57,8 +57,10 @@ extern "C" qlora_status qlora_nf4_quantize_noalloc(const void* W, qlora_dtype dt
                                                    const qlora_nf4_state* st, int32_t* d_status,
                                                    qlora_stream_t stream) {
   if (!st || !W || !aligned(W, 16)) return QLORA_ERR_INVALID_ARG;
-  if (st->numel < 1 || st->blocksize != qnf4::kBlock || st->reserved != 0) return QLORA_ERR_INVALID_ARG;
+  if (st->numel < 1 || st->blocksize != qnf4::kBlock) return QLORA_ERR_INVALID_ARG;
+  if (st->codebook != QLORA_CODEBOOK_NF4 && st->codebook != QLORA_CODEBOOK_INT4) return QLORA_ERR_INVALID_ARG;
   if (st->double_quant != 0 && st->double_quant != 1) return QLORA_ERR_INVALID_ARG;
+  if (st->codebook == QLORA_CODEBOOK_INT4 && st->double_quant) return QLORA_ERR_UNSUPPORTED;
   if (dtype != QLORA_DTYPE_BF16 && dtype != QLORA_DTYPE_F32) return QLORA_ERR_INVALID_ARG;
   if (!st->packed || !aligned(st->packed, 16)) return QLORA_ERR_INVALID_ARG;
   if (st->double_quant) {
@@ -79,6 +81,6 @@ extern "C" qlora_status qlora_nf4_quantize_noalloc(const void* W, qlora_dtype dt
   cudaError_t e = qnf4::launch_quantize(W, dtype, st->numel, st->packed, st->absmax,
                                         st->double_quant != 0, st->code8, st->s2, st->offset,
                                         scratch, d_status,
-                                        reinterpret_cast<cudaStream_t>(stream), sms);
+                                        reinterpret_cast<cudaStream_t>(stream), sms, st->codebook);
   return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
 }

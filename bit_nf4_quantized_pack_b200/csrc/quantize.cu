@@ -564,11 +564,94 @@ __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict_
 // ---------------------------------------------------------------------------
 // Host launchers
 // ---------------------------------------------------------------------------
+// ---------------------------------------------------------------------------
+// Uniform signed INT4 (the comparator codebook; page "SFT（四）：QLoRA的4-bit量化与
+// LoRA微调原理", §6 先理解最普通的分块量化): per 64-block s = amax / 7 (formed in
+// fp64, stored as fp32; 1 for an all-zero block), q = clip(round(w / s), -7, 7)
+// with w / s in fp64 and ties away from zero, code q + 8; an odd tail is padded
+// with code 8.  One thread per block: 64 fp64 divisions, a comparator path.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) int4_encode_kernel(const T* __restrict__ W, int64_t numel,
+                                                          uint8_t* __restrict__ packed,
+                                                          float* __restrict__ scales,
+                                                          int32_t* d_status) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int64_t n1 = (numel + kBlock - 1) / kBlock;
+  const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (b >= n1) return;
+  const int64_t e0 = b * kBlock;
+  const int cnt = static_cast<int>(numel - e0 < kBlock ? numel - e0 : kBlock);
+  float x[kBlock];
+#pragma unroll
+  for (int i = 0; i < kBlock; ++i) {
+    float v = 0.0f;
+    if (i < cnt) {
+      if constexpr (sizeof(T) == 2) v = bf16_bits_to_f32(W[e0 + i]);
+      else v = W[e0 + i];
+    }
+    x[i] = v;
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kBlock; ++i) amax = fmax_nan(amax, fabsf(x[i]));
+  if (!(amax <= FLT_MAX)) {
+    raise_status(d_status, QLORA_ERR_NONFINITE);
+    amax = 0.0f;
+  }
+  const float sc = amax > 0.0f ? __double2float_rn(__ddiv_rn(static_cast<double>(amax), 7.0)) : 1.0f;
+  scales[b] = sc;
+  const double sd = static_cast<double>(sc);
+  uint32_t words[kBlock / 8];
+#pragma unroll
+  for (int wi = 0; wi < kBlock / 8; ++wi) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i = wi * 8 + k;
+      uint32_t code = static_cast<uint32_t>(kPadCodeInt4);
+      if (i < cnt) {
+        const double t = __ddiv_rn(static_cast<double>(x[i]), sd);
+        const double r = floor(__dadd_rn(fabs(t), 0.5));
+        const int q = static_cast<int>(fmin(r, 7.0)) * (t >= 0.0 ? 1 : -1);
+        code = static_cast<uint32_t>(q + 8);
+      }
+      // byte k/2 of the word: element 2m in the high nibble, 2m+1 in the low
+      w |= code << (8 * (k >> 1) + ((k & 1) ? 0 : 4));
+    }
+    words[wi] = w;
+  }
+  const int64_t nbytes = (numel + 1) >> 1;
+  const int64_t b0 = e0 >> 1;
+  if (cnt == kBlock) {
+    uint4* dst = reinterpret_cast<uint4*>(packed + b0);
+    dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+    dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+  } else {
+    for (int k = 0; k < kBlock / 2; ++k)
+      if (b0 + k < nbytes) packed[b0 + k] = static_cast<uint8_t>(words[k >> 2] >> (8 * (k & 3)));
+  }
+}
+
 cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* packed,
                             float* absmax_out, bool dq, uint8_t* code8, float* s2, float* offset,
-                            void* ws, int32_t* d_status, cudaStream_t st, int num_sms) {
+                            void* ws, int32_t* d_status, cudaStream_t st, int num_sms,
+                            int codebook) {
   const int64_t n1 = (numel + kBlock - 1) / kBlock;
   const int threads = 256;
+  if (codebook == 1) {   // uniform INT4: no double quantization, no workspace
+    const dim3 grid(static_cast<unsigned>((n1 + 255) / 256));
+    ProfScope prof(kProfQuantize, st);
+    const cudaError_t e1 =
+        dtype == QLORA_DTYPE_BF16
+            ? launch_pdl(int4_encode_kernel<uint16_t>, grid, dim3(256), 0, st, 1,
+                         static_cast<const uint16_t*>(W), numel, packed, absmax_out, d_status)
+            : launch_pdl(int4_encode_kernel<float>, grid, dim3(256), 0, st, 1,
+                         static_cast<const float*>(W), numel, packed, absmax_out, d_status);
+    if (e1 != cudaSuccess) return e1;
+    return cudaGetLastError();
+  }
   const int64_t want = (n1 * 4 + threads - 1) / threads;
   unsigned long long* bins = nullptr;
   float* scales = absmax_out;

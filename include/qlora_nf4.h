@@ -72,13 +72,25 @@ typedef int32_t qlora_dtype;
  *            Decode scale a' = (T8[code8[b]] · s2[b/256]) + offset, each
  *            operation rounded to fp32.                                (device)
  * Unused pointers may be NULL.  The struct itself lives in host memory.
+ *
+ * codebook selects the 16 code values:
+ *   QLORA_CODEBOOK_NF4  : the NF4 table; odd-tail padding code 7.
+ *   QLORA_CODEBOOK_INT4 : uniform signed INT4, the comparator type of page
+ *     "SFT（四）：QLoRA的4-bit量化与LoRA微调原理", §6 先理解最普通的分块量化:
+ *     code j holds q = j - 8 (the quantizer emits 1 .. 15: q = clip(round(w/s),
+ *     -7, 7), w/s in fp64, ties away from zero); `absmax` then holds the stored
+ *     scale s = RN_fp32(amax/7) (1 for an all-zero block); padding code 8;
+ *     double_quant must be 0 (else QLORA_ERR_UNSUPPORTED).
+ * Every kernel of the library decodes both: w_hat = RN_bf16(value(code) · scale).
  */
+#define QLORA_CODEBOOK_NF4  0
+#define QLORA_CODEBOOK_INT4 1
 typedef struct qlora_nf4_state {
   int64_t  numel;         /* logical element count (K·N for a weight), >= 1 */
   int32_t  blocksize;     /* must be 64 */
   int32_t  double_quant;  /* 0 or 1 */
   int32_t  dq_blocksize;  /* must be 256 */
-  int32_t  reserved;      /* must be 0 */
+  int32_t  codebook;      /* QLORA_CODEBOOK_NF4 (0) or QLORA_CODEBOOK_INT4 (1) */
   uint8_t* packed;
   float*   absmax;
   uint8_t* code8;
@@ -87,7 +99,7 @@ typedef struct qlora_nf4_state {
 } qlora_nf4_state;
 
 /* ABI version of this header (bumped on any incompatible change). */
-#define QLORA_NF4_ABI_VERSION 1
+#define QLORA_NF4_ABI_VERSION 2
 int32_t qlora_abi_version(void);
 
 /* Human-readable name of a status code (static string, never NULL). */
