@@ -61,6 +61,7 @@ SIGNATURES = {
     "qlora_linear_bwd": (_I32, [_I64, _I64, _I64, _I32, _VP, _VP, _VP, _PS, _VP, _VP, _F,
                                 _VP, _VP, _VP, _VP, _SZ, _VP, _VP]),
     "qlora_nf4_merge": (_I32, [_I64, _I64, _I32, _PS, _VP, _VP, _F, _VP, _VP, _VP]),
+    "qlora_selftest_bounded_wait": (_I32, [_I64, _VP, _VP]),
     "qlora_profile_enable": (_I32, [_I32]),
     "qlora_profile_read": (_I32, [_I32, C.POINTER(C.c_double), C.POINTER(C.c_int64)]),
     "qlora_profile_reset": (_I32, []),

@@ -5,6 +5,8 @@
 
 #include <cmath>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "kernels.cuh"
 #include "qlora_nf4.h"
 
@@ -28,6 +30,13 @@ int sm_count() {
 }
 
 qlora_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
+
+// An NVTX range around each compute entry point, so that a timeline tool
+// shows the library's calls (header-only NVTX: no cost without a tool).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
 
 // Common checks of a quantized-state struct.
 qlora_status check_state(const qlora_nf4_state* st, bool need_scales) {
@@ -120,6 +129,7 @@ size_t qlora_nf4_quantize_workspace_size(int64_t numel, int32_t double_quant) {
 qlora_status qlora_nf4_quantize(const void* W, qlora_dtype dtype, const qlora_nf4_state* st,
                                 void* ws, size_t ws_bytes, int32_t* d_status,
                                 qlora_stream_t stream) {
+  NvtxRange nvtx_range("qlora_nf4_quantize");
   qlora_status v = check_state(st, true);
   if (v != QLORA_OK) return v;
   if (!W || !aligned(W, 16)) return QLORA_ERR_INVALID_ARG;
@@ -137,6 +147,7 @@ qlora_status qlora_nf4_quantize(const void* W, qlora_dtype dtype, const qlora_nf
 
 qlora_status qlora_nf4_dequantize(const qlora_nf4_state* st, uint16_t* W_hat, int32_t* d_status,
                                   qlora_stream_t stream) {
+  NvtxRange nvtx_range("qlora_nf4_dequantize");
   qlora_status v = check_state(st, true);
   if (v != QLORA_OK) return v;
   if (!W_hat || !aligned(W_hat, 16)) return QLORA_ERR_INVALID_ARG;
@@ -163,6 +174,7 @@ qlora_status qlora_linear_fwd(int64_t M, int64_t K, int64_t N, int32_t r, const 
                               const qlora_nf4_state* W, const uint16_t* A, const uint16_t* B,
                               float c, uint16_t* Y, uint16_t* Zc, void* ws, size_t ws_bytes,
                               int32_t* d_status, qlora_stream_t stream) {
+  NvtxRange nvtx_range("qlora_linear_fwd");
   qlora_status v = check_linear_shape(M, K, N, r);
   if (v != QLORA_OK) return v;
   v = check_state(W, true);
@@ -185,6 +197,7 @@ qlora_status qlora_linear_fwd(int64_t M, int64_t K, int64_t N, int32_t r, const 
 qlora_status qlora_nf4_merge(int64_t K, int64_t N, int32_t r, const qlora_nf4_state* W,
                              const uint16_t* A, const uint16_t* B, float c, uint16_t* out,
                              int32_t* d_status, qlora_stream_t stream) {
+  NvtxRange nvtx_range("qlora_nf4_merge");
   qlora_status v = check_linear_shape(1, K, N, r);
   if (v != QLORA_OK) return v;
   v = check_state(W, true);
@@ -198,11 +211,19 @@ qlora_status qlora_nf4_merge(int64_t K, int64_t N, int32_t r, const qlora_nf4_st
                                         reinterpret_cast<cudaStream_t>(stream)));
 }
 
+qlora_status qlora_selftest_bounded_wait(int64_t limit_ns, int32_t* d_status, qlora_stream_t stream) {
+  NvtxRange nvtx_range("qlora_selftest_bounded_wait");
+  if (limit_ns < 1 || limit_ns > 10000000000ll || !d_status) return QLORA_ERR_INVALID_ARG;
+  return cuda_status(qnf4::launch_bounded_wait_selftest(d_status, static_cast<uint64_t>(limit_ns),
+                                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
 qlora_status qlora_linear_bwd(int64_t M, int64_t K, int64_t N, int32_t r, const uint16_t* dY,
                               const uint16_t* X, const uint16_t* Zc, const qlora_nf4_state* W,
                               const uint16_t* A, const uint16_t* B, float c, uint16_t* dX,
                               float* dA, float* dB, void* ws, size_t ws_bytes, int32_t* d_status,
                               qlora_stream_t stream) {
+  NvtxRange nvtx_range("qlora_linear_bwd");
   qlora_status v = check_linear_shape(M, K, N, r);
   if (v != QLORA_OK) return v;
   v = check_state(W, true);

@@ -62,6 +62,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// selftest.cu — a wait that nothing completes, bounded by limit_ns
+cudaError_t launch_bounded_wait_selftest(int32_t* d_status, uint64_t limit_ns, cudaStream_t st);
+
 // quantize.cu
 cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* packed,
                             float* absmax_out, bool dq, uint8_t* code8, float* s2, float* offset,

@@ -259,6 +259,17 @@ qlora_status qlora_nf4_merge(int64_t K, int64_t N, int32_t r, const qlora_nf4_st
                              int32_t* d_status, qlora_stream_t stream);
 
 /*
+ * Self-test of failure detection (no counterpart on the pages).  Launches one
+ * kernel that waits, with the library's bounded wait, on an mbarrier that
+ * nothing completes; after `limit_ns` (1 ns .. 10 s) of wall time the wait
+ * gives up, QLORA_ERR_TIMEOUT is OR-ed into *d_status and the kernel returns.
+ * Every wait inside the library's kernels is bounded the same way (2 s), so a
+ * lost arrival surfaces as this status instead of a hang, and the context
+ * stays usable.  Errors: INVALID_ARG (limit out of range, null status), CUDA.
+ */
+qlora_status qlora_selftest_bounded_wait(int64_t limit_ns, int32_t* d_status, qlora_stream_t stream);
+
+/*
  * Launch timing, for measurement tools (no counterpart on the pages).  While
  * enabled, each kernel launch of the library is bracketed by two CUDA events
  * recorded on the stream the kernel runs on.  qlora_profile_read waits for

@@ -125,3 +125,13 @@ def test_product_path_has_no_fallback():
             src = open(os.path.join(pkg, f), encoding="utf-8").read()
             assert not re.search(r"^\s*(from|import)\s+oracle\b", src, flags=re.M), f
             assert "import_module(\"oracle" not in src and "__import__(\"oracle" not in src, f
+
+
+def test_selftest_validation(L):
+    """The bounded-wait self-test rejects bad limits and a null status word on
+    the host, before any launch."""
+    lib = L.lib
+    fake = C.c_void_p(256)   # never dereferenced: validation fails first
+    assert lib.qlora_selftest_bounded_wait(0, fake, None) == 1
+    assert lib.qlora_selftest_bounded_wait(20_000_000_000, fake, None) == 1
+    assert lib.qlora_selftest_bounded_wait(1000, None, None) == 1

@@ -67,6 +67,35 @@ def test_gemv_parity(M):
         assert v <= TOL, (k, v, errs)
 
 
+MULTI_WAVE_CASES = [
+    # more 512 x 128 tiles than SMs, the last wave partial: the persistent
+    # CTAs take a second tile (forward in the first case, dX in the second)
+    (2048, 1024, 8192, 16, True),
+    (2048, 8192, 1024, 16, False),
+]
+
+
+@pytest.mark.parametrize("M,K,N,r,dq", MULTI_WAVE_CASES)
+def test_multi_wave_parity(M, K, N, r, dq):
+    lin = S.random_case(M + 3 * K + N, M, K, N, r)
+    lin.dY = S.normal(11, M, 4, (M, N), 1.0)
+    errs = run_case(lin, r, 32.0 / r, dq)
+    for k, v in errs.items():
+        assert v <= TOL, (k, v, errs)
+
+
+def test_forward_deterministic():
+    """Every sum has a fixed order: repeated launches give the same bits."""
+    q = _q()
+    lin = S.random_case(42, 2048, 1024, 8192, 16)
+    wq = q.quantize(to_dev(lin.W), double_quant=True)
+    Xt, At, Bt = to_dev(lin.X), to_dev(lin.A), to_dev(lin.B)
+    Y1, _ = q.linear_forward(Xt, wq, At, Bt, 2.0)
+    for _ in range(3):
+        Y2, _ = q.linear_forward(Xt, wq, At, Bt, 2.0)
+        assert torch.equal(Y1, Y2)
+
+
 GEMV_SHAPES = [
     # (M, K, N, r, dq): K not a multiple of 128 (a half stage of zeros), a ragged
     # last column group, one 64-row stage, no double quantization, a rank wider
