@@ -348,6 +348,61 @@ def run_case(args):
     return 0 if code[0] == 0 else 1
 
 
+def layers_bench(torch, q, dev, peaks):
+    """Forward + backward of the larger workloads, weights quantized (DQ) ahead:
+    the 7B decoder-layer linear set (q, k, v, o 4096x4096; gate, up 4096x11008;
+    down 11008x4096) and the 65B MLP slice (8192x22016, 22016x8192), M = 4096,
+    r = 64, alpha = 16.  TFLOP/s of sum 4MKN + 6Mr(K+N); seeded normal inputs
+    drawn on the GPU."""
+    from bit_nf4_quantized_pack_b200 import synthetic as S
+    gen = torch.Generator(device=dev)
+    out = {}
+    for name, shapes, sigma in (("layer7b", [(k, n) for _, k, n in S.LAYER7B], 0.02),
+                                ("mlp65b", [(8192, 22016), (22016, 8192)], 0.015)):
+        Mb, rb, c = 4096, 64, 16.0 / 64
+        gen.manual_seed(9)
+        layers = []
+        for (Kb, Nb) in shapes:
+            W = (torch.randn((Kb, Nb), generator=gen, device=dev) * sigma).to(torch.bfloat16)
+            w = q.quantize(W, double_quant=True)
+            del W
+            mk = lambda *sh, sc: (torch.randn(sh, generator=gen, device=dev) * sc).to(torch.bfloat16)
+            layers.append(dict(w=w, A=mk(Kb, rb, sc=0.01), B=mk(rb, Nb, sc=0.01), X=mk(Mb, Kb, sc=1.0),
+                               G=mk(Mb, Nb, sc=1.0), Y=torch.empty((Mb, Nb), dtype=torch.bfloat16, device=dev),
+                               Zc=torch.empty((Mb, rb), dtype=torch.bfloat16, device=dev),
+                               dX=torch.empty((Mb, Kb), dtype=torch.bfloat16, device=dev),
+                               dA=torch.empty((Kb, rb), dtype=torch.float32, device=dev),
+                               dB=torch.empty((rb, Nb), dtype=torch.float32, device=dev)))
+        st = q.new_status(dev)
+
+        def run():
+            for L in layers:
+                q.linear_forward(L["X"], L["w"], L["A"], L["B"], c, Y=L["Y"], Zc=L["Zc"], status=st)
+            for L in reversed(layers):
+                q.linear_backward(L["G"], L["X"], L["Zc"], L["w"], L["A"], L["B"], c, dX=L["dX"],
+                                  dA=L["dA"], dB=L["dB"], status=st)
+        for _ in range(2):
+            run()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 5
+        e0.record()
+        for _ in range(reps):
+            run()
+        e1.record()
+        torch.cuda.synchronize()
+        code, mask = q.status_sync(st)
+        if code != 0:
+            raise SystemExit(f"device status {code} (mask {mask}) in {name}")
+        ms = e0.elapsed_time(e1) / reps
+        flops = sum(4.0 * Mb * Kb * Nb + 6.0 * Mb * rb * (Kb + Nb) for Kb, Nb in shapes)
+        out[name] = {"ms": ms, "TFLOP/s": flops / (ms * 1e-3) / 1e12,
+                     "frac": flops / (ms * 1e-3) / 1e12 / peaks["bf16"], "linears": len(shapes)}
+        del layers
+        torch.cuda.empty_cache()
+    return out
+
+
 def merge_bench(torch, q, dev, peaks):
     """Merge/export of the 8192x22016 weight with r = 64 (DQ state): GB/s of
     P/2 + n1 + 4n2 + 4 (state) + 2r(K+N) (adapter) + 2P (bf16 output)."""
@@ -555,6 +610,7 @@ def main():
         extras["gemv"] = gemv_sweep(torch, q, dev, peaks)
         extras["quantize"] = quantize_bench(torch, q, dev, peaks)
         extras["merge"] = merge_bench(torch, q, dev, peaks)
+        extras["layers"] = layers_bench(torch, q, dev, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.kernels_only:

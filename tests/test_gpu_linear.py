@@ -234,3 +234,48 @@ def test_merge_requantize_matches_oracle_quantize_of_merged():
     code8, s2, off = nf4.double_quantize(absmax)
     assert np.array_equal(rq.packed.cpu().numpy(), payload)
     assert np.array_equal(rq.code8.cpu().numpy(), code8)
+
+
+@pytest.mark.slow
+def test_full_size_65b_mlp_sampled():
+    """The 65B MLP shapes at full size (M = 4096, r = 64, both 8192 x 22016 and
+    22016 x 8192), without double quantization so that the oracle can quantize
+    just the blocks it needs: sampled columns of Y, sampled columns of dX, full
+    dA and dB.  The oracle quantizes those blocks from the same input."""
+    from oracle import nf4
+    q = _q()
+    wl = S.config5()
+    rng = np.random.default_rng(5)
+    for lin in wl.linears:
+        X, W, A, B, G, c = lin.X, lin.W, lin.A, lin.B, lin.dY, wl.c
+        K, N = W.shape
+        M = X.shape[0]
+        wq = q.quantize(to_dev(W), double_quant=False)
+        Xt, At, Bt = to_dev(X), to_dev(A), to_dev(B)
+        Y, Zc = q.linear_forward(Xt, wq, At, Bt, c)
+        dX, dA, dB = q.linear_backward(to_dev(G), Xt, Zc, wq, At, Bt, c)
+        Y, dX, dA, dB = to_np(Y), to_np(dX), to_np(dA), to_np(dB)
+        X64, G64, A64, B64 = (np.asarray(t, np.float64) for t in (X, G, A, B))
+        Z = X64 @ A64
+        dZ = c * (G64 @ B64.T)
+
+        def w_hat_of(block):          # oracle quantization of a (rows x 64k) sub-matrix
+            codes, absmax = nf4.quantize_nf4(np.ascontiguousarray(block, np.float32).ravel())
+            payload, n = nf4.pack_codes(codes)
+            return nf4.dequantize(payload, n, absmax).reshape(block.shape)
+
+        # Y columns: each sampled column's 64-block in every row k
+        cols = np.unique(np.concatenate([[0, N - 1], rng.integers(0, N, 10)]))
+        for j in cols:
+            b0 = (j // 64) * 64
+            wcol = w_hat_of(W[:, b0:b0 + 64])[:, j - b0]
+            ref = X64 @ wcol + c * (Z @ B64[:, j])
+            assert rel_fro(Y[:, j], ref) <= TOL, ("Y", K, N, j)
+        # dX columns k: row k of W in full
+        ks = np.unique(np.concatenate([[0, K - 1], rng.integers(0, K, 10)]))
+        for k in ks:
+            wrow = w_hat_of(W[k:k + 1, :]).ravel()
+            ref = G64 @ wrow + dZ @ A64[k]
+            assert rel_fro(dX[:, k], ref) <= TOL, ("dX", K, N, k)
+        assert rel_fro(dA, X64.T @ dZ) <= TOL
+        assert rel_fro(dB, c * (Z.T @ G64)) <= TOL
