@@ -412,14 +412,9 @@ __device__ uint32_t round_q128_to_f32(unsigned __int128 q, uint64_t rem, uint64_
 // the occupied exponent range, and one thread adds the occupied bins exactly:
 // in 128 bits when they span at most 64 binades (always, for any realistic
 // weight), else in a 384-bit integer.
-__global__ void __launch_bounds__(256) dq_mean_kernel(const unsigned long long* __restrict__ bins,
-                                                      int64_t n1, float* __restrict__ offset) {
-  __shared__ unsigned long long sb[256];
-  __shared__ int range[2];
-  pdl_launch_dependents();
-  pdl_wait();
-  sb[threadIdx.x] = bins[threadIdx.x];
-  __syncthreads();
+// Exact mean of the n1 first-level scales from their exponent bins: the
+// range of non-empty keys (warp 0, ballots) ...
+__device__ __forceinline__ void bins_key_range(const unsigned long long* sb, int* range) {
   if (threadIdx.x < 32) {
     uint32_t m = 0;
     for (int i = 0; i < 8; ++i) m |= (sb[threadIdx.x * 8 + i] != 0ull ? 1u : 0u) << i;
@@ -428,9 +423,10 @@ __global__ void __launch_bounds__(256) dq_mean_kernel(const unsigned long long* 
     if (threadIdx.x == lmin) range[0] = threadIdx.x * 8 + (__ffs(m) - 1);
     if (threadIdx.x == lmax) range[1] = threadIdx.x * 8 + (31 - __clz(m));
   }
-  __syncthreads();
-  if (threadIdx.x != 0) return;
-  const int kmin = range[0], kmax = range[1];
+}
+
+// ... and the sum divided by n1 with one rounding to fp32 (one thread).
+__device__ uint32_t exact_mean_bits(const unsigned long long* sb, int kmin, int kmax, int64_t n1) {
   const uint64_t d = static_cast<uint64_t>(n1);
   uint32_t bits;
   if (kmax - kmin <= 64) {
@@ -486,7 +482,7 @@ __global__ void __launch_bounds__(256) dq_mean_kernel(const unsigned long long* 
       bits = (static_cast<uint32_t>(shift + 1) << 23) + (mant - 0x800000u);
     }
   }
-  *offset = __uint_as_float(bits);
+  return bits;
 }
 
 // One warp per group of 256 centred scales (8 per lane, 8 groups per CTA).
@@ -498,9 +494,14 @@ __global__ void __launch_bounds__(256) dq_mean_kernel(const unsigned long long* 
 // 254 midpoints into fp32 thresholds once and counts them by binary search.
 // k < 127 -> byte 0x80 | (127 - k), k = 127 -> 0x00, k > 127 -> byte k - 127.
 __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict__ a, int64_t n1,
-                                                        const float* __restrict__ offset_p,
+                                                        const unsigned long long* __restrict__ bins,
+                                                        float* __restrict__ offset_p,
                                                         uint8_t* __restrict__ code8,
                                                         float* __restrict__ s2) {
+  // every CTA forms the same exact mean from the bins (CTA 0 stores it)
+  __shared__ unsigned long long sb[256];
+  __shared__ int range[2];
+  __shared__ float s_off;
   __shared__ float mag[128];
   __shared__ double mid[254];
   __shared__ float thr[8][256];
@@ -516,7 +517,16 @@ __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict_
   }
   __syncthreads();
   pdl_wait();   // the tables above read no global memory
-  const float off = *offset_p;
+  sb[threadIdx.x] = bins[threadIdx.x];
+  __syncthreads();
+  bins_key_range(sb, range);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    s_off = __uint_as_float(exact_mean_bits(sb, range[0], range[1], n1));
+    if (blockIdx.x == 0) *offset_p = s_off;
+  }
+  __syncthreads();
+  const float off = s_off;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float* T = thr[warp];
   const int64_t n2 = (n1 + kDQBlock - 1) / kDQBlock;
@@ -708,19 +718,15 @@ cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* pa
   }
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || !dq) return e;
-  {
-    ProfScope prof(kProfQuantize, st);
-    e = launch_pdl(dq_mean_kernel, dim3(1), dim3(256), 0, st, 1,
-                   static_cast<const unsigned long long*>(bins), n1, offset);
-  }
-  if (e != cudaSuccess) return e;
+
   const int64_t n2 = (n1 + kDQBlock - 1) / kDQBlock;
   {
     ProfScope prof(kProfQuantize, st);
     const int64_t want_g = (n2 + 7) / 8;
     const int64_t grid = want_g < num_sms * 8LL ? want_g : num_sms * 8LL;
     e = launch_pdl(dq_encode_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, 1,
-                   static_cast<const float*>(scales), n1, static_cast<const float*>(offset), code8, s2);
+                   static_cast<const float*>(scales), n1, static_cast<const unsigned long long*>(bins),
+                   offset, code8, s2);
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
