@@ -124,10 +124,12 @@ def model(n_items, nk, A, B, n_dec, n_epi, n_acc, seed, producer_parity_bug=Fals
         assert idle < 200 * len(agents), "deadlock"
 
 
+# n_acc: four accumulators of 128 x 128 (forward), two of 128 x 256 (dX)
+@pytest.mark.parametrize("n_acc", [4, 2])
 @pytest.mark.parametrize("A,B", [(2, 4), (2, 2), (3, 2), (4, 3)])
-def test_fused_protocol_random_interleavings(A, B):
+def test_fused_protocol_random_interleavings(A, B, n_acc):
     for seed in range(20):
-        model(n_items=3, nk=5, A=A, B=B, n_dec=4, n_epi=4, n_acc=4, seed=seed)
+        model(n_items=3, nk=5, A=A, B=B, n_dec=4, n_epi=4, n_acc=n_acc, seed=seed)
 
 
 def test_mbarrier_model():
