@@ -22,6 +22,7 @@
 //                        fragments; gemv_finish_kernel adds the splits and Zc·B.
 #include <atomic>
 #include <cfloat>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -1242,6 +1243,41 @@ void gemv_plan(int64_t K, int64_t N, int num_sms, int* splits, int* stages_per_s
 
 static int g_ws_sms = 148;  // sizing assumption for workspace queries (B200)
 
+// A library-owned stream per device for work that runs beside the caller's
+// stream, and the two events of one fork and join.  Created on first use
+// (retried after a failure, e.g. inside a stream capture that forbids it);
+// g_side_mu is held from a fork to its join, so concurrent callers never
+// interleave their records and waits on the shared events.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+static std::mutex g_side_mu;
+static SideStream g_side[64];
+
+static SideStream* side_stream(int dev) {
+  if (dev < 0 || dev >= 64) return nullptr;
+  SideStream& ss = g_side[dev];
+  if (ss.s == nullptr) {
+    int least = 0, greatest = 0;
+    cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    cudaStream_t s = nullptr;
+    cudaEvent_t f = nullptr, j = nullptr;
+    if (cudaStreamCreateWithPriority(&s, cudaStreamNonBlocking, least) != cudaSuccess ||
+        cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess) {
+      if (s != nullptr) cudaStreamDestroy(s);
+      if (f != nullptr) cudaEventDestroy(f);
+      (void)cudaGetLastError();
+      return nullptr;
+    }
+    ss.fork = f;
+    ss.join = j;
+    ss.s = s;
+  }
+  return &ss;
+}
+
 size_t linear_fwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) {
   if (M > 16) return 0;   // the rank-r kernel adds its splits in shared memory
   // GEMV partials and its per-split X·A slices
@@ -1404,15 +1440,9 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   if (!make_tmap_2d(&tXmn, X, kBF16, 2, M, K, K, 64, 64, kSW128)) return cudaErrorInvalidValue;
   // (columns of dZ past r arrive as TMA zero fill)
   if (!make_tmap_2d(&tdZ, dZ, kBF16, 2, M, r, r, 64, 64, kSW128)) return cudaErrorInvalidValue;
-  e = run_skinny<true, true>(tXmn, tdZ, static_cast<int>(K), static_cast<int>(M), r, 1.0f, 1, dA,
-                             r, Sa, d_status, st);
-  if (e != cudaSuccess) return e;
   // dB^T = G^T Zc : A operand G^T (MN-major over N), B operand Zc (MN-major over r)
   if (!make_tmap_2d(&tGmn, dY, kBF16, 2, M, N, N, 64, 64, kSW128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tZcmn, Zc, kBF16, 2, M, r, r, 64, 64, kSW128)) return cudaErrorInvalidValue;
-  e = run_skinny<true, true>(tGmn, tZcmn, static_cast<int>(N), static_cast<int>(M), r, 1.0f, 2,
-                             dB, r, Sb, d_status, st);
-  if (e != cudaSuccess) return e;
   // dX = G W^T + dZ A^T
   e = set_fused_attr<true>();
   if (e != cudaSuccess) return e;
@@ -1436,13 +1466,42 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int tiles = fa.m_tiles * fa.n_tiles;
   const int grid = tiles < sms ? tiles : sms;
+
+  // dX on the caller's stream first; dA and dB, which need only dZ, Zc, X and
+  // G, on the side stream after dZ, so their CTAs take the SMs that dX's
+  // partial last wave of tiles leaves idle.  The caller's stream then waits
+  // for them: to the caller the call is ordered as one operation on st.
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  SideStream* ss = prof_timing(kProfSkinny) ? nullptr : side_stream(dev);
+  cudaStream_t s2 = st;
+  if (ss != nullptr && cudaEventRecord(ss->fork, st) == cudaSuccess) s2 = ss->s;
   {
     ProfScope prof(kProfFusedBwd, st);
     e = launch_pdl(fused_nf4_gemm_kernel<true>, dim3(grid), dim3(kFThreads), kFSmem, st, 1, tG, tdZa,
                    tAl, fa);
   }
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (s2 != st) {
+    const cudaError_t ew = cudaStreamWaitEvent(s2, ss->fork, 0);
+    if (ew != cudaSuccess) {
+      // no fork: dA and dB after dX on the caller's stream
+      s2 = st;
+      if (e == cudaSuccess) e = ew;
+    }
+  }
+  if (e == cudaSuccess)
+    e = run_skinny<true, true>(tXmn, tdZ, static_cast<int>(K), static_cast<int>(M), r, 1.0f, 1, dA,
+                               r, Sa, d_status, s2);
+  if (e == cudaSuccess)
+    e = run_skinny<true, true>(tGmn, tZcmn, static_cast<int>(N), static_cast<int>(M), r, 1.0f, 2,
+                               dB, r, Sb, d_status, s2);
+  if (s2 != st) {
+    // always join, so that nothing on st can run ahead of work already queued
+    const cudaError_t ej = cudaEventRecord(ss->join, s2);
+    const cudaError_t ew = ej == cudaSuccess ? cudaStreamWaitEvent(st, ss->join, 0) : ej;
+    if (e == cudaSuccess) e = ew;
+  }
+  return e;
 }
 
 }  // namespace qnf4

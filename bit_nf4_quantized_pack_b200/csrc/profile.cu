@@ -57,6 +57,11 @@ ProfScope::~ProfScope() {
   g_pending.push_back(Pair{id_, static_cast<cudaEvent_t>(a_), b});
 }
 
+bool prof_timing(int id) {
+  std::lock_guard<std::mutex> g(g_mu);
+  return g_on && id >= 0 && id < 32 && ((g_mask >> id) & 1u);
+}
+
 void prof_count_only(int id) {
   std::lock_guard<std::mutex> g(g_mu);
   ++g_total_launches;

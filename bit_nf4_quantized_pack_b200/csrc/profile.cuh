@@ -36,4 +36,9 @@ class ProfScope {
 
 void prof_count_only(int id);
 
+// True while launches of kind `id` are being timed.  The backward then runs
+// its rank-r launches in order on the caller's stream instead of beside dX,
+// so that each class's events bracket that class's work alone.
+bool prof_timing(int id);
+
 }  // namespace qnf4

@@ -23,6 +23,8 @@
  *   never allocates device memory and never synchronizes the stream, except
  *   in qlora_status_sync.
  * - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default).
+ *   qlora_linear_bwd forks part of its work onto a library stream and joins
+ *   it back before returning (see there).
  * - Errors: a host-side validation failure returns its qlora_status at once and
  *   enqueues nothing.  Errors that only the device can see (non-finite input,
  *   bad padding, an internal wait that ran out) are OR-ed as bit (1 << code)
@@ -228,6 +230,15 @@ qlora_status qlora_linear_fwd(int64_t M, int64_t K, int64_t N, int32_t r,
  *   dA : device fp32 K×r output     dB : device fp32 r×N output
  * No gradient is produced for W (the frozen base).  Same shape rules and
  * workspace convention as the forward.
+ * Streams: dA and dB run on a stream the library owns (one per device,
+ * created on first use), forked from `stream` after dZ and joined back into
+ * it before the call returns, so that they use the SMs that dX's last
+ * partial wave of tiles leaves idle.  To the caller the call is still one
+ * operation ordered on `stream` (later work on `stream` sees dX, dA and dB;
+ * it can be captured in a CUDA graph), and the results are the same bits as
+ * a run in order.  If the library stream cannot be created, or while
+ * rank-r launches are being timed (qlora_profile_*), everything runs in
+ * order on `stream`.
  */
 size_t qlora_linear_bwd_workspace_size(int64_t M, int64_t K, int64_t N, int32_t r);
 qlora_status qlora_linear_bwd(int64_t M, int64_t K, int64_t N, int32_t r,
@@ -281,7 +292,9 @@ qlora_status qlora_selftest_bounded_wait(int64_t limit_ns, int32_t* d_status, ql
  * `kinds_mask` (bit k = class k; all classes by default).  The events sit
  * between launches and so keep a timed launch from overlapping its
  * predecessor's tail (programmatic dependent launch): a measuring tool that
- * wants the untouched launch chain times only the classes it needs.
+ * wants the untouched launch chain times only the classes it needs.  While
+ * QLORA_PROF_SKINNY is timed, the backward runs dA and dB in order on the
+ * caller's stream (not beside dX), so that the class times do not overlap.
  * Not thread-safe across devices; meant for one measuring process.
  */
 #define QLORA_PROF_FUSED_FWD  0   /* fused NF4 GEMM, forward (Y)        */

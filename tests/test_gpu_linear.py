@@ -96,6 +96,58 @@ def test_forward_deterministic():
         assert torch.equal(Y1, Y2)
 
 
+def test_backward_streams_and_graph_capture():
+    """The backward runs dA and dB on a library stream beside dX and joins it
+    back into the caller's stream.  Bits must not depend on that: the same
+    call on the default stream, on another torch stream, repeated, and
+    captured in a CUDA graph and replayed gives identical dX, dA and dB."""
+    q = _q()
+    M, K, N, r = 1536, 1024, 2048, 16   # dX: 3 x 8 = 24 tiles; dA/dB: several clusters
+    lin = S.random_case(55, M, K, N, r)
+    wq = q.quantize(to_dev(lin.W), double_quant=True)
+    Xt, At, Bt = to_dev(lin.X), to_dev(lin.A), to_dev(lin.B)
+    G = to_dev(S.normal(9, M, 4, (M, N), 1.0))
+    _, Zc = q.linear_forward(Xt, wq, At, Bt, 2.0)
+    ref = q.linear_backward(G, Xt, Zc, wq, At, Bt, 2.0)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        again = q.linear_backward(G, Xt, Zc, wq, At, Bt, 2.0)
+        for a_, b_ in zip(ref, again):
+            assert torch.equal(a_, b_)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        on_side = q.linear_backward(G, Xt, Zc, wq, At, Bt, 2.0)
+    torch.cuda.current_stream().wait_stream(side)
+    for a_, b_ in zip(ref, on_side):
+        assert torch.equal(a_, b_)
+    # graph capture: outputs, workspace and status allocated before capture
+    dX = torch.empty_like(ref[0])
+    dA = torch.empty_like(ref[1])
+    dB = torch.empty_like(ref[2])
+    st = q.new_status()
+    ws = torch.empty(int(q.lib.qlora_linear_bwd_workspace_size(M, K, N, r)), dtype=torch.uint8,
+                     device="cuda")
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        q.linear_backward(G, Xt, Zc, wq, At, Bt, 2.0, dX=dX, dA=dA, dB=dB, status=st, workspace=ws)
+        cap.synchronize()
+        with torch.cuda.graph(g, stream=cap):
+            q.linear_backward(G, Xt, Zc, wq, At, Bt, 2.0, dX=dX, dA=dA, dB=dB, status=st,
+                              workspace=ws)
+    torch.cuda.synchronize()
+    for t in (dX, dA, dB):
+        t.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert q.status_sync(st) == (0, 0)
+    for a_, b_ in zip(ref, (dX, dA, dB)):
+        assert torch.equal(a_, b_)
+    del g
+
+
 GEMV_SHAPES = [
     # (M, K, N, r, dq): K not a multiple of 128 (a half stage of zeros), a ragged
     # last column group, one 64-row stage, no double quantization, a rank wider
