@@ -247,8 +247,10 @@ __global__ void __launch_bounds__(kSkThreads, 1)
 //             then reads 96 KB of operands per K-step from shared memory
 //             instead of 128 KB (the weight tile is read twice, not four
 //             times); measured 9% faster for dX.  The same transposition of
-//             the forward, with its MN-major tile as the A operand, measured
-//             3% slower than the untransposed form, so the forward keeps it.
+//             the forward measured slower than the untransposed form: 3% with
+//             its MN-major tile as the A operand, 6% with a K-major tile
+//             written by stmatrix .trans (two block scales per thread and
+//             K-step), so the forward keeps it.
 //
 // Shared memory holds two rings.  Activation tiles (512 x 64 bf16, K-major,
 // four TMA boxes) have 2 stages.  Decoded weight tiles have 4 stages; decoder
