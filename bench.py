@@ -246,6 +246,11 @@ def gemv_sweep(torch, q, dev, peaks):
             torch.cuda.synchronize()
             st = q.new_status(dev)
             s = torch.cuda.Stream(device=dev)
+            s.wait_stream(torch.cuda.current_stream(dev))
+            with torch.cuda.stream(s):         # warm-up on the capture stream (its workspace)
+                for w in ws:
+                    q.linear_forward(X, w, A, B, 2.0, Y=Y, Zc=Zc, status=st)
+            s.synchronize()
             g = torch.cuda.CUDAGraph()
             reps = 4
             with torch.cuda.stream(s):

@@ -117,8 +117,10 @@ def status_clear(status: torch.Tensor) -> None:
 
 
 class _WorkspaceCache:
-    """Reuses one device buffer per (device, purpose) so repeated calls do not
-    allocate; grows when a larger workspace is needed."""
+    """Reuses one device buffer per (purpose, device, current stream) so
+    repeated calls do not allocate; grows when a larger workspace is needed.
+    Keyed by stream as well: calls in flight on two streams never share a
+    buffer, and each buffer is allocated and used in one stream's order."""
 
     def __init__(self):
         self._bufs = {}
@@ -126,6 +128,7 @@ class _WorkspaceCache:
     def get(self, key, nbytes, device):
         if nbytes == 0:
             return None
+        key = (*key, torch.cuda.current_stream(device).cuda_stream)
         buf = self._bufs.get(key)
         if buf is None or buf.numel() < nbytes or buf.device != torch.device(device):
             buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
