@@ -157,3 +157,27 @@ def test_codes_independent_of_double_quant_and_zero_block_stays_zero():
     C = np.array(nf4.NF4)[codes]
     delta = (a_dq.astype(np.float64) - absmax)[np.arange(w.size) // 64]
     assert np.all(np.abs((w_dq - w_plain) - C * delta) <= 2 * 2 ** -8 * np.abs(w_plain) + 1e-12)
+
+
+def test_group_scale_is_the_max_over_every_position():
+    """s2 is the absmax of the whole 256-group of centred scales (the page's
+    blockwise absmax applied to the scales): placing the group's largest
+    deviation at its first or at its last position must give that deviation
+    as s2, and that scale must decode back within the error bound."""
+    rng = np.random.default_rng(10)
+    n1 = 256 * 3 + 40                       # ragged last group
+    a = np.abs(rng.standard_normal(n1) * 0.002 + 0.05).astype(np.float32)
+    a[255] = np.float32(0.9)                # last position of group 0
+    a[256] = np.float32(0.8)                # first position of group 1
+    a[n1 - 1] = np.float32(0.7)             # last position of the ragged group
+    code8, s2, off = nf4.double_quantize(a)
+    c = (a - off).astype(np.float32).astype(np.float64)
+    for g in range(s2.size):
+        grp = np.abs(c[g * 256:(g + 1) * 256])
+        assert np.all(grp <= s2[g]) and np.any(grp == s2[g])
+    dec = nf4.decode_scales(n1, code8=code8, s2=s2, offset=off).astype(np.float64)
+    vals = np.array(sorted(set(nf4.dq_codebook().astype(np.float64).tolist())))
+    half_gap = np.max(np.diff(vals)) / 2
+    for i in (255, 256, n1 - 1):
+        bound = float(s2[i // 256]) * half_gap + 4 * float(np.spacing(np.float32(1.0))) * a[i]
+        assert abs(dec[i] - a[i]) <= bound

@@ -160,3 +160,37 @@ def test_int4_library_format_against_block_rule():
         cands = list(range(-7, 8))
         best = min(cands, key=lambda q: (abs(t - q), -abs(q)))
         assert c - 8 == best
+
+
+def test_int4_ties_round_half_away_from_zero():
+    """The page does not say how round() breaks a tie; the reading taken is
+    half away from zero (the school rule).  With amax = 7 the scale is 1 and
+    w / s are exact halves."""
+    from oracle.int4 import int4_quantize
+    vals = [7.0, 2.5, -2.5, 0.5, -0.5, 1.5, -6.5]
+    want = [7, 3, -3, 1, -1, 2, -7]
+    q, s = int4_quantize_block(vals)
+    assert s == 1.0 and q == want
+    codes, sc = int4_quantize(np.array(vals, dtype=np.float32))
+    assert float(sc[0]) == 1.0 and list(codes.astype(int) - 8) == want
+
+
+def test_int4_dequantize_is_one_bf16_rounding_of_q_times_s():
+    """Decoded weights are bf16 values within half a bf16 ulp of the exact
+    q * s (s = RN_fp32(amax / 7) is not a bf16 number in general)."""
+    from oracle.int4 import int4_dequantize, int4_quantize
+    rng = np.random.default_rng(12)
+    w = rng.normal(0, 0.02, 64 * 50).astype(np.float32)
+    codes, s = int4_quantize(w)
+    out = int4_dequantize(codes, s)
+    exact = (codes.astype(np.float64) - 8) * s.astype(np.float64)[np.arange(w.size) // 64]
+    f32 = out.astype(np.float32)
+    assert np.all(f32.astype(np.float64) == out)               # fp32-exact
+    assert np.all((f32.view(np.uint32) & 0xFFFF) == 0)          # and bf16-exact
+    nz = exact != 0
+    _, e = np.frexp(exact[nz])
+    half_ulp = np.ldexp(1.0, e - 9)                             # bf16: 8 significant bits
+    assert np.all(np.abs(out[nz] - exact[nz]) <= half_ulp)
+    assert np.any(out[nz] != exact[nz])                         # rounding does happen
+    assert np.all(out[~nz] == 0)
+
