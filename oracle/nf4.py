@@ -26,8 +26,11 @@ What each function follows, and what pins it (tests under ``tests/``):
 * ``double_quantize`` / ``decode_scales`` — [P1] §"Double Quantization 压缩的是
   Scale" and [P3] §3.2: subtract the mean, 256-blocks, fp32 second-level
   absmax, nearest 8-bit code; restore = decode + offset.  Pinned by
-  invariants (equal group decodes to the offset; error bound) and by brute
-  force.
+  invariants (equal group decodes to the offset; error bound; s2 the max
+  over every group position) and by exact-rational brute force near every
+  codebook midpoint.  The decode's two fp32 roundings (product, then sum)
+  are a reading of "decode + offset" with fp32 storage: parity unpinned as
+  to that rounding order.
 * ``dequantize`` — [P1] §"NF4 保存的是索引而不是均匀整数值" (reconstruction
   a·C_j) and §"量化基座与可训练支路怎样相加" (computation in BF16): one
   rounding of the exact product to bf16.  Pinned by the page's printed

@@ -181,3 +181,60 @@ def test_group_scale_is_the_max_over_every_position():
     for i in (255, 256, n1 - 1):
         bound = float(s2[i // 256]) * half_gap + 4 * float(np.spacing(np.float32(1.0))) * a[i]
         assert abs(dec[i] - a[i]) <= bound
+
+
+def test_exact_mean_subnormal_closed_forms():
+    """Round to nearest even at the fp32 subnormal quantum 2^-149."""
+    q = 2.0 ** -149
+    assert nf4.exact_mean_f32(np.array([q, 0.0], np.float32)) == 0.0          # q/2: tie -> 0
+    assert nf4.exact_mean_f32(np.array([3 * q, 0.0], np.float32)) == np.float32(2 * q)  # 1.5q -> 2q
+    assert nf4.exact_mean_f32(np.array([q, q, q, 0.0], np.float32)) == np.float32(q)    # 0.75q -> q
+    assert nf4.exact_mean_f32(np.array([5 * q, 0.0], np.float32)) == np.float32(2 * q)  # 2.5q -> 2q
+
+
+def test_codebook_values_are_nearest_fp32_of_the_exact_ratio():
+    """Each magnitude is the fp32 value nearest (num / den) as an exact
+    rational, by enumeration of its fp32 neighbours."""
+    table = nf4.dq_codebook()
+    for t in range(1, 128):
+        f = t.bit_length() - 1
+        e, m = 6 - f, t - (1 << f)
+        x = Fraction((1 << f) + 9 * (m + 1), (10 ** (e + 1)) * (1 << f))
+        v = table[t]
+        lo, hi = np.nextafter(v, np.float32(0)), np.nextafter(v, np.float32(2))
+        d = abs(Fraction(float(v)) - x)
+        assert d <= abs(Fraction(float(lo)) - x) and d <= abs(Fraction(float(hi)) - x), t
+
+
+def test_double_quantize_exact_near_code_midpoints():
+    """Centred scales placed on fp32 neighbours of s2 * (every midpoint of the
+    8-bit codebook) get the exact-rational nearest code.  The values come in
+    +-pairs so that the mean is exactly 0 and c = a."""
+    table = nf4.dq_codebook()
+    vals = sorted(set(float(v) for v in table if v > 0))
+    pos_mids = [(Fraction(0) + Fraction(vals[0])) / 2]
+    pos_mids += [(Fraction(vals[i]) + Fraction(vals[i + 1])) / 2 for i in range(len(vals) - 1)]
+    D = np.float32(0.3)
+    pts = []
+    for mid in pos_mids:
+        t = np.float32(float(Fraction(float(D)) * mid))
+        for k in (-2, -1, 0, 1, 2):
+            v = t
+            for _ in range(abs(k)):
+                v = np.nextafter(v, np.float32(np.inf if k > 0 else -np.inf))
+            if 0 < v < D:
+                pts.append(v)
+    per = 127                                   # pairs per group after (D, -D)
+    groups = []
+    for i in range(0, len(pts), per):
+        chunk = pts[i:i + per]
+        g = [D, -D]
+        for v in chunk:
+            g += [v, -v]
+        g += [np.float32(0.0)] * (256 - len(g))
+        groups.append(g)
+    a = np.array([v for g in groups for v in g], dtype=np.float32)
+    code8, s2, off = nf4.double_quantize(a)
+    assert off == 0.0 and np.all(s2 == D)
+    for i in range(a.size):
+        assert code8[i] == _brute_code8(a[i], D), i

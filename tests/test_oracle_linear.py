@@ -194,3 +194,19 @@ def test_int4_dequantize_is_one_bf16_rounding_of_q_times_s():
     assert np.any(out[nz] != exact[nz])                         # rounding does happen
     assert np.all(out[~nz] == 0)
 
+
+def test_int4_ragged_tail_block():
+    """The stored format's last block holds only the tail: its scale comes
+    from the tail alone, and an all-zero tail gets scale 1 and code 8 (q = 0)."""
+    from oracle.int4 import int4_quantize
+    w = np.full(64 + 3, 0.01, np.float32)
+    w[63] = 5.0
+    w[64:] = [0.7, -0.3, 0.12]                  # no w / s near a .5 tie
+    codes, s = int4_quantize(w)
+    q_ref, s_ref = int4_quantize_block(w[64:])
+    assert abs(float(s[1]) - s_ref) <= 2 ** -23 * s_ref
+    assert list(codes[64:].astype(int) - 8) == q_ref == [7, -3, 1]
+    w[64:] = 0.0
+    codes, s = int4_quantize(w)
+    assert float(s[1]) == 1.0 and np.all(codes[64:] == 8)
+

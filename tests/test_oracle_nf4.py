@@ -250,3 +250,69 @@ def test_block_scales_is_the_scale_step_of_quantize():
         assert np.array_equal(nf4.block_scales(w), s)
     with pytest.raises(nf4.NonFiniteError):
         nf4.block_scales(np.array([1.0, np.nan], np.float32))
+
+
+def test_round_to_bf16_subnormal_and_overflow():
+    """Round to nearest even at the ends of the bf16 range: subnormals are
+    multiples of 2^-133 (fp32-exact inputs checked against the enumerated
+    bf16 grid), and past the largest bf16 value (2 - 2^-7) * 2^127 a tie
+    rounds to even, which is the overflow to infinity."""
+    rng = np.random.default_rng(21)
+    k = rng.integers(1, 1 << 23, 3000)
+    xs = np.ldexp(k.astype(np.float64), -149)          # fp32 subnormals: exact
+    xs = np.concatenate([xs, np.ldexp(rng.uniform(1, 2, 500), rng.integers(-130, -120, 500))])
+    xs = xs.astype(np.float32).astype(np.float64)      # keep them fp32-exact
+    out = nf4.round_to_bf16(xs)
+    for x, r in zip(xs, out):
+        lo, hi = _bf16_neighbours(x)
+        dl, dh = Fraction(x) - Fraction(lo), Fraction(hi) - Fraction(x)
+        if dl < dh:
+            assert r == lo, x
+        elif dh < dl:
+            assert r == hi, x
+        else:   # tie: the even bf16 pattern
+            even = lo if (int(np.array(np.float32(lo)).view(np.uint32)) >> 16) % 2 == 0 else hi
+            assert r == even, x
+    top = (2.0 - 2.0 ** -7) * 2.0 ** 127                # largest bf16, odd mantissa
+    ulp = 2.0 ** 120
+    assert nf4.round_to_bf16(top + ulp / 4) == top
+    assert nf4.round_to_bf16(top + ulp / 2) == np.inf   # tie -> even -> 2^128 overflows
+    assert nf4.round_to_bf16(-(top + 0.75 * ulp)) == -np.inf
+    assert nf4.round_to_bf16(2.0 ** -134) == 0.0        # half the smallest subnormal: tie -> 0
+    assert nf4.round_to_bf16(3 * 2.0 ** -134) == 2 * 2.0 ** -133   # tie -> even
+
+
+def test_ragged_tail_block_is_its_own_block():
+    """The last block holds only the tail (the page's blocks of 64 of the
+    flattening, the last one shorter): a large element just before it does
+    not enter its scale, and an all-zero tail gets scale 1 and code 7."""
+    w = np.full(64 + 5, 0.01, np.float32)
+    w[63] = 10.0
+    w[64:] = [0.2, -0.4, 0.0, 0.1, 0.05]
+    codes, absmax = nf4.quantize_nf4(w)
+    assert absmax[1] == np.float32(0.4) and nf4.block_scales(w)[1] == np.float32(0.4)
+    tail_codes, _, tail_scale = nf4.encode_block(w[64:])
+    assert list(codes[64:]) == tail_codes and tail_scale == np.float32(0.4)
+    w[64:] = 0.0
+    codes, absmax = nf4.quantize_nf4(w)
+    assert absmax[1] == 1.0 and nf4.block_scales(w)[1] == 1.0
+    assert np.all(codes[64:] == 7)
+
+
+def test_encode_block_exact_near_midpoints():
+    """The per-block rule in Python doubles agrees with exact rational
+    arithmetic on fp32 neighbours of every NF4 midpoint."""
+    rng = np.random.default_rng(22)
+    for a in (1.0, 0.3, 2.0 ** -20, 0.0123456, 3.0e4):
+        blk = _adversarial_block(rng, np.float32(a))
+        codes, _, _ = nf4.encode_block(blk)
+        assert codes == _brute_exact(blk)
+
+
+def test_dequantize_rejects_nonfinite_scale():
+    """A non-finite reconstruction is an error (the page's decode check)."""
+    payload, n = nf4.pack_codes(np.array([7, 9, 3, 15], dtype=np.uint8))
+    with pytest.raises(nf4.NonFiniteError):
+        nf4.dequantize(payload, n, np.array([np.inf], dtype=np.float32))
+    with pytest.raises(nf4.NonFiniteError):
+        nf4.dequantize(payload, n, np.array([np.nan], dtype=np.float32))
