@@ -141,7 +141,7 @@ def _copy(work):
     shutil.copytree(os.path.join(ROOT, "oracle"), os.path.join(work, "oracle"))
     os.makedirs(os.path.join(work, "tests"))
     for f in os.listdir(os.path.join(ROOT, "tests")):
-        if f.startswith("test_oracle") or f == "conftest.py":
+        if (f.startswith("test_oracle") and "mutants" not in f) or f == "conftest.py":
             shutil.copy(os.path.join(ROOT, "tests", f), os.path.join(work, "tests", f))
     shutil.copytree(os.path.join(ROOT, "tests", "golden"), os.path.join(work, "tests", "golden"))
 
