@@ -120,19 +120,24 @@ class _WorkspaceCache:
     """Reuses one device buffer per (purpose, device, current stream) so
     repeated calls do not allocate; grows when a larger workspace is needed.
     Keyed by stream as well: calls in flight on two streams never share a
-    buffer, and each buffer is allocated and used in one stream's order."""
+    buffer, and each buffer is allocated and used in one stream's order.
+    At most ``limit`` buffers are kept (the least recently used is dropped;
+    the caching allocator reuses its memory in its own stream's order)."""
 
-    def __init__(self):
+    def __init__(self, limit: int = 16):
         self._bufs = {}
+        self._limit = limit
 
     def get(self, key, nbytes, device):
         if nbytes == 0:
             return None
         key = (*key, torch.cuda.current_stream(device).cuda_stream)
-        buf = self._bufs.get(key)
+        buf = self._bufs.pop(key, None)
         if buf is None or buf.numel() < nbytes or buf.device != torch.device(device):
             buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
-            self._bufs[key] = buf
+        self._bufs[key] = buf                    # most recently used last
+        while len(self._bufs) > self._limit:
+            self._bufs.pop(next(iter(self._bufs)))
         return buf
 
 

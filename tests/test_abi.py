@@ -135,3 +135,34 @@ def test_selftest_validation(L):
     assert lib.qlora_selftest_bounded_wait(0, fake, None) == 1
     assert lib.qlora_selftest_bounded_wait(20_000_000_000, fake, None) == 1
     assert lib.qlora_selftest_bounded_wait(1000, None, None) == 1
+
+
+def test_workspace_cache_is_per_stream_and_bounded(L, monkeypatch):
+    """Host logic of the binding's workspace cache, on CPU tensors with a
+    stand-in for the current stream: one buffer per (purpose, device, stream),
+    grown when too small, and at most `limit` buffers kept."""
+    import torch
+
+    import bit_nf4_quantized_pack_b200 as q
+
+    class FakeStream:
+        def __init__(self, h):
+            self.cuda_stream = h
+
+    cur = {"h": 1}
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda device=None: FakeStream(cur["h"]))
+    cache = q._WorkspaceCache(limit=3)
+    a = cache.get(("b", "cpu"), 1000, "cpu")
+    assert a is cache.get(("b", "cpu"), 900, "cpu")          # reused on the same stream
+    cur["h"] = 2
+    b = cache.get(("b", "cpu"), 1000, "cpu")
+    assert b is not a                                          # another stream, another buffer
+    c = cache.get(("b", "cpu"), 5000, "cpu")
+    assert c is not b and c.numel() >= 5000                     # grown
+    assert cache.get(("b", "cpu"), 0, "cpu") is None
+    for h in (3, 4, 5):
+        cur["h"] = h
+        cache.get(("f", "cpu"), 10, "cpu")
+    assert len(cache._bufs) == 3                               # bounded, oldest dropped
+    cur["h"] = 1
+    assert cache.get(("b", "cpu"), 1000, "cpu") is not a       # stream 1's buffer was evicted
