@@ -133,7 +133,7 @@ CPU_BASELINE_REPS = 3
 
 def oracle_sample_inputs(ks=None, ms=None):
     import numpy as np
-    from bit_nf4_quantized_pack_b200 import synthetic as S
+    from inputs import synthetic as S
     ks = ORACLE_KS if ks is None else ks
     ms = ORACLE_MS if ms is None else ms
     lin = S.config2(M=ms).linears[0]
@@ -204,7 +204,7 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 def make_sets(torch, dev, nsets):
     import numpy as np
-    from bit_nf4_quantized_pack_b200 import synthetic as S
+    from inputs import synthetic as S
     sets = []
     for s in range(nsets):
         lin = S.config2(seed=s).linears[0]
@@ -359,7 +359,7 @@ def layers_bench(torch, q, dev, peaks):
     down 11008x4096) and the 65B MLP slice (8192x22016, 22016x8192), M = 4096,
     r = 64, alpha = 16.  TFLOP/s of sum 4MKN + 6Mr(K+N); seeded normal inputs
     drawn on the GPU."""
-    from bit_nf4_quantized_pack_b200 import synthetic as S
+    from inputs import synthetic as S
     gen = torch.Generator(device=dev)
     out = {}
     for name, shapes, sigma in (("layer7b", [(k, n) for _, k, n in S.LAYER7B], 0.02),

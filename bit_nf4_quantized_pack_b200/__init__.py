@@ -122,17 +122,36 @@ class _WorkspaceCache:
     Keyed by stream as well: calls in flight on two streams never share a
     buffer, and each buffer is allocated and used in one stream's order.
     At most ``limit`` buffers are kept (the least recently used is dropped;
-    the caching allocator reuses its memory in its own stream's order)."""
+    the caching allocator reuses its memory in its own stream's order).
+
+    CUDA graphs: a captured launch keeps the raw pointer of its workspace.
+    While the current stream is capturing, ``get`` never allocates, grows or
+    drops a buffer (a call that needs more than the cached buffer raises: pass
+    ``workspace=`` explicitly, or make the same call once before capturing),
+    and every buffer handed out during a capture stays referenced for the life
+    of the process, so a later, larger call that replaces it cannot hand its
+    memory to another tensor while a graph still writes into it."""
 
     def __init__(self, limit: int = 16):
         self._bufs = {}
         self._limit = limit
+        self._captured = []
 
     def get(self, key, nbytes, device):
         if nbytes == 0:
             return None
-        key = (*key, torch.cuda.current_stream(device).cuda_stream)
-        buf = self._bufs.pop(key, None)
+        stream = torch.cuda.current_stream(device)
+        key = (*key, stream.cuda_stream)
+        buf = self._bufs.get(key)
+        if stream.is_capturing():
+            if buf is None or buf.numel() < nbytes or buf.device != torch.device(device):
+                raise RuntimeError(
+                    "no workspace of the needed size is cached for this stream while it is "
+                    "capturing a CUDA graph: pass workspace= or run the call once before capture")
+            if not any(b is buf for b in self._captured):
+                self._captured.append(buf)
+            return buf
+        self._bufs.pop(key, None)
         if buf is None or buf.numel() < nbytes or buf.device != torch.device(device):
             buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
         self._bufs[key] = buf                    # most recently used last

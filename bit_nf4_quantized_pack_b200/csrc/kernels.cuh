@@ -5,11 +5,39 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
 #include <utility>
 
 #include "common.cuh"
 
 namespace qnf4 {
+
+// One-time set-up per device (kernel attributes, occupancy queries).
+// cudaFuncSetAttribute acts on the current device only, so every device that
+// runs a kernel gets its own run of `f(dev)`; a failed run is retried on the
+// next call.  Safe when several host threads make their first calls at once.
+constexpr int kMaxDevices = 64;
+class DeviceOnce {
+ public:
+  template <typename F>
+  cudaError_t run(F&& f) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (done_[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(mu_);
+    if (done_[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+    e = f(dev);
+    if (e == cudaSuccess) done_[dev].store(true, std::memory_order_release);
+    return e;
+  }
+
+ private:
+  std::mutex mu_;
+  std::atomic<bool> done_[kMaxDevices] = {};
+};
 
 // The signed dynamic 8-bit codebook T8 of the scale codes (this library's own
 // definition; the page only requires "a signed dynamic 8-bit codebook, not

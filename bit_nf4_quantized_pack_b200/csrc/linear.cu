@@ -1175,13 +1175,11 @@ size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
 
 template <bool A, bool B>
 cudaError_t set_skinny_attr() {
-  static bool done = false;
-  if (done) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(skinny_gemm_kernel<A, B>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSkSmem));
-  if (e == cudaSuccess) done = true;
-  return e;
+  static DeviceOnce once;
+  return once.run([](int) {
+    return cudaFuncSetAttribute(skinny_gemm_kernel<A, B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(kSkSmem));
+  });
 }
 
 // D = scale * A(m',k') B(n',k'): one launch, split-K sums added in-kernel.
@@ -1214,13 +1212,11 @@ cudaError_t run_skinny(const CUtensorMap& ta, const CUtensorMap& tb, int Mp, int
 
 template <bool kBwd>
 cudaError_t set_fused_attr() {
-  static bool done = false;
-  if (done) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(fused_nf4_gemm_kernel<kBwd>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kFSmem));
-  if (e == cudaSuccess) done = true;
-  return e;
+  static DeviceOnce once;
+  return once.run([](int) {
+    return cudaFuncSetAttribute(fused_nf4_gemm_kernel<kBwd>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(kFSmem));
+  });
 }
 
 constexpr CUtensorMapDataType kBF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -1320,16 +1316,17 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
                                   Sz, d_status, st);
       if (e != cudaSuccess) return e;
     }
-    static bool attr_done = false;
-    if (!attr_done) {
-      e = cudaFuncSetAttribute(nf4_gemv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kGvSmem));
-      if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(nf4_gemv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    static DeviceOnce gemv_once;
+    e = gemv_once.run([](int) {
+      cudaError_t r = cudaFuncSetAttribute(nf4_gemv_kernel<false>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(kGvSmem));
+      if (r == cudaSuccess)
+        r = cudaFuncSetAttribute(nf4_gemv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kGvSmem));
-      if (e != cudaSuccess) return e;
-      attr_done = true;
-    }
+      return r;
+    });
+    if (e != cudaSuccess) return e;
     CUtensorMap tP, tXg, tAg;
     if (!make_tmap_2d(&tP, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N / 2, N / 2, 128, kGvRows, kSW128))
       return cudaErrorInvalidValue;

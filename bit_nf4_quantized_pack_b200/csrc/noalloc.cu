@@ -18,6 +18,8 @@
 
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "kernels.cuh"
 #include "qlora_nf4.h"
 
@@ -51,11 +53,18 @@ cudaError_t scratch_on_current_device(void** out) {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// The same NVTX range as the library's other compute entry points.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+
 }  // namespace
 
 extern "C" qlora_status qlora_nf4_quantize_noalloc(const void* W, qlora_dtype dtype,
                                                    const qlora_nf4_state* st, int32_t* d_status,
                                                    qlora_stream_t stream) {
+  NvtxRange nvtx_range("qlora_nf4_quantize_noalloc");
   if (!st || !W || !aligned(W, 16)) return QLORA_ERR_INVALID_ARG;
   if (st->numel < 1 || st->blocksize != qnf4::kBlock) return QLORA_ERR_INVALID_ARG;
   if (st->codebook != QLORA_CODEBOOK_NF4 && st->codebook != QLORA_CODEBOOK_INT4) return QLORA_ERR_INVALID_ARG;

@@ -674,31 +674,35 @@ cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* pa
   }
   {
   ProfScope prof(kProfQuantize, st);
-  // one wave of resident CTAs (each loops over chunks)
-  static int per_sm[4] = {0, 0, 0, 0};
-  {
-    static bool attr_done = false;
-    if (!attr_done) {
-      const int b16 = static_cast<int>(encode_smem_bytes<uint16_t>());
-      const int b32 = static_cast<int>(encode_smem_bytes<float>());
-      const void* fns[4] = {reinterpret_cast<const void*>(nf4_encode_kernel<uint16_t, false>),
-                            reinterpret_cast<const void*>(nf4_encode_kernel<uint16_t, true>),
-                            reinterpret_cast<const void*>(nf4_encode_kernel<float, false>),
-                            reinterpret_cast<const void*>(nf4_encode_kernel<float, true>)};
-      for (int i = 0; i < 4; ++i) {
-        const int bytes = i < 2 ? b16 : b32;
-        cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-        cudaFuncSetAttribute(fns[i], cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-        int nb = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fns[i], threads, bytes) != cudaSuccess || nb < 1)
-          nb = 1;
-        per_sm[i] = nb;
-      }
-      attr_done = true;
+  // one wave of resident CTAs (each loops over chunks); attributes and
+  // occupancy per device
+  static int per_sm[kMaxDevices][4];
+  static DeviceOnce once;
+  e = once.run([&](int dev) {
+    const int b16 = static_cast<int>(encode_smem_bytes<uint16_t>());
+    const int b32 = static_cast<int>(encode_smem_bytes<float>());
+    const void* fns[4] = {reinterpret_cast<const void*>(nf4_encode_kernel<uint16_t, false>),
+                          reinterpret_cast<const void*>(nf4_encode_kernel<uint16_t, true>),
+                          reinterpret_cast<const void*>(nf4_encode_kernel<float, false>),
+                          reinterpret_cast<const void*>(nf4_encode_kernel<float, true>)};
+    for (int i = 0; i < 4; ++i) {
+      const int bytes = i < 2 ? b16 : b32;
+      cudaError_t r = cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+      if (r != cudaSuccess) return r;
+      cudaFuncSetAttribute(fns[i], cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      int nb = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fns[i], threads, bytes) != cudaSuccess || nb < 1)
+        nb = 1;
+      per_sm[dev][i] = nb;
     }
-  }
+    (void)cudaGetLastError();   // a refused carveout hint is not an error
+    return cudaSuccess;
+  });
+  if (e != cudaSuccess) return e;
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   const int kind = (dtype == QLORA_DTYPE_BF16 ? 0 : 2) + (dq ? 1 : 0);
-  const int64_t cap = static_cast<int64_t>(num_sms) * per_sm[kind];
+  const int64_t cap = static_cast<int64_t>(num_sms) * per_sm[dev][kind];
   const int blocks = static_cast<int>(want < cap ? want : cap);
   if (dtype == QLORA_DTYPE_BF16) {
     const size_t sm = encode_smem_bytes<uint16_t>();

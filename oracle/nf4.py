@@ -29,8 +29,8 @@ What each function follows, and what pins it (tests under ``tests/``):
   invariants (equal group decodes to the offset; error bound; s2 the max
   over every group position) and by exact-rational brute force near every
   codebook midpoint.  The decode's two fp32 roundings (product, then sum)
-  are a reading of "decode + offset" with fp32 storage: parity unpinned as
-  to that rounding order.
+  are a reading of "decode + offset" with fp32 storage, pinned by a
+  hand-worked case whose one-rounding result differs.
 * ``dequantize`` — [P1] §"NF4 保存的是索引而不是均匀整数值" (reconstruction
   a·C_j) and §"量化基座与可训练支路怎样相加" (computation in BF16): one
   rounding of the exact product to bf16.  Pinned by the page's printed

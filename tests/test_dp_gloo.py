@@ -37,7 +37,7 @@ def _free_port():
 
 
 def _case():
-    from bit_nf4_quantized_pack_b200 import synthetic as S
+    from inputs import synthetic as S
     from tests._gpu_util import OracleWeight
     M, K, N, r = 37, 128, 192, 8
     lin = S.random_case(4242, M, K, N, r)

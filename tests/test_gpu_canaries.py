@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 import torch
 
-from bit_nf4_quantized_pack_b200 import synthetic as S
+from inputs import synthetic as S
 from tests._gpu_util import to_dev
 
 pytestmark = pytest.mark.gpu

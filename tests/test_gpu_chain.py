@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 import torch
 
-from bit_nf4_quantized_pack_b200 import synthetic as S
+from inputs import synthetic as S
 from oracle.linear import lora_backward, lora_forward
 from tests._gpu_util import OracleWeight, rel_fro, to_dev, to_np
 

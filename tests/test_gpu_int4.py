@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 import torch
 
-from bit_nf4_quantized_pack_b200 import synthetic as S
+from inputs import synthetic as S
 from oracle.int4 import int4_dequantize, int4_quantize
 from oracle.linear import lora_backward, lora_forward
 from oracle.merge import merge_bf16, merge_exact

@@ -7,7 +7,7 @@ import numpy as np
 import pytest
 import torch
 
-from bit_nf4_quantized_pack_b200 import synthetic as S
+from inputs import synthetic as S
 from oracle import nf4
 from tests._gpu_util import OracleWeight, assert_state_equal, bf16_bits, dev, to_dev
 

@@ -238,3 +238,34 @@ def test_double_quantize_exact_near_code_midpoints():
     assert off == 0.0 and np.all(s2 == D)
     for i in range(a.size):
         assert code8[i] == _brute_code8(a[i], D), i
+
+
+def test_decode_rounds_the_product_before_adding_the_offset():
+    """Rounding order of the scale decode ([P1] §"Double Quantization 压缩的是
+    Scale": restore = decode + offset, every stored value fp32).  The reading
+    taken is two fp32 roundings, a' = RN32(RN32(T8[q] * s2) + offset), with no
+    fused multiply-add.  The values below separate it from a single rounding of
+    the exact T8[q] * s2 + offset; the expected bits are worked out by hand:
+
+      q = 0x43: sign 0, t = 67, f = 6, e = 0, m = 3, so
+                |T8| = (2^6 + 9 * 4) / (10 * 2^6) = 100/640 = 5/32 exactly.
+      s2 = 1 + 2^-23 (bits 0x3F800001).
+      T8 * s2 = 5/32 + 5 * 2^-28 = 2^-3 * (1.25 + 2^-23 + 2^-25); the 2^-25
+                term is below half an fp32 ulp of the product (2^-24 relative),
+                so RN32(T8 * s2) = 5/32 + 2^-26.
+      offset = -5/32 (bits 0xBE200000).
+      two roundings: RN32(2^-26) = 2^-26               -> bits 0x32800000
+      one rounding:  RN32(2^-26 + 2^-28) = 1.25 * 2^-26 -> bits 0x32A00000
+    """
+    code8 = np.array([0x43], dtype=np.uint8)
+    s2 = np.array([0x3F800001], dtype=np.uint32).view(np.float32)
+    offset = np.array([0xBE200000], dtype=np.uint32).view(np.float32)[0]
+    got = nf4.decode_scales(1, code8=code8, s2=s2, offset=offset)
+    assert got.dtype == np.float32
+    assert int(got.view(np.uint32)[0]) == 0x32800000
+    assert int(got.view(np.uint32)[0]) != 0x32A00000
+    # the same decode further into a group: the group index picks s2[1]
+    code8 = np.full(300, 0x43, dtype=np.uint8)
+    s2 = np.array([0x3F800000, 0x3F800001], dtype=np.uint32).view(np.float32)
+    got = nf4.decode_scales(300, code8=code8, s2=s2, offset=offset).view(np.uint32)
+    assert np.all(got[:256] == 0) and np.all(got[256:] == 0x32800000)

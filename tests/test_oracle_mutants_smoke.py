@@ -6,7 +6,7 @@ import pytest
 from tests import oracle_mutants as om
 
 SMOKE = ("encode_block ties to larger", "pack low nibble first", "DQ fp32 ratio", "dX sign",
-         "bf16 subnormal threshold", "int4 ties to even")
+         "bf16 subnormal threshold", "int4 ties to even", "decode fused")
 
 
 def test_smoke_mutants_are_caught(tmp_path):

@@ -15,8 +15,8 @@ import torch
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("dq", [True, False])
-def test_noalloc_quantize_matches_workspace_entry_point(dq):
+@pytest.mark.parametrize("dq,codebook", [(True, "nf4"), (False, "nf4"), (False, "int4")])
+def test_noalloc_quantize_matches_workspace_entry_point(dq, codebook):
     import bit_nf4_quantized_pack_b200 as q
     from bit_nf4_quantized_pack_b200 import _lib
     dev = torch.device("cuda", 0)
@@ -26,8 +26,8 @@ def test_noalloc_quantize_matches_workspace_entry_point(dq):
         g.manual_seed(seed)
         W = (torch.randn((K, N), generator=g, device=dev) * 0.02).to(torch.bfloat16)
         W[3, :64] = 0.0                                  # an all-zero block
-        ref = q.quantize(W, double_quant=dq)             # workspace entry point
-        out = q.NF4Weight.empty((K, N), dq, dev)
+        ref = q.quantize(W, double_quant=dq, codebook=codebook)   # workspace entry point
+        out = q.NF4Weight.empty((K, N), dq, dev, codebook=1 if codebook == "int4" else 0)
         st = out.cstruct()
         status = q.new_status(dev)
         rc = _lib.lib.qlora_nf4_quantize_noalloc(C.c_void_p(W.data_ptr()), _lib.QLORA_DTYPE_BF16,
@@ -47,7 +47,7 @@ def test_noalloc_quantize_matches_workspace_entry_point(dq):
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     from bit_nf4_quantized_pack_b200 import _lib
     st = _lib.NF4StateC()
-    st.numel, st.blocksize, st.double_quant, st.dq_blocksize, st.reserved = \
+    st.numel, st.blocksize, st.double_quant, st.dq_blocksize, st.codebook = \
         _lib.NOALLOC_MAX_NUMEL + 2, 64, 1, 256, 0
     st.packed = st.code8 = st.s2 = st.offset = 4096
     rc = _lib.lib.qlora_nf4_quantize_noalloc(C.c_void_p(4096), 0, C.byref(st), None, None)
