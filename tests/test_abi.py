@@ -72,7 +72,7 @@ def test_workspace_sizes(L):
 
 def _state(L, numel=128, dq=0, packed=4096):
     st = L.NF4StateC()
-    st.numel, st.blocksize, st.double_quant, st.dq_blocksize, st.reserved = numel, 64, dq, 256, 0
+    st.numel, st.blocksize, st.double_quant, st.dq_blocksize, st.codebook = numel, 64, dq, 256, 0
     st.packed = packed
     st.absmax = 4096
     st.code8, st.s2, st.offset = 4096, 4096, 4096
@@ -146,11 +146,16 @@ def test_workspace_cache_is_per_stream_and_bounded(L, monkeypatch):
     import bit_nf4_quantized_pack_b200 as q
 
     class FakeStream:
-        def __init__(self, h):
+        def __init__(self, h, capturing=False):
             self.cuda_stream = h
+            self._capturing = capturing
 
-    cur = {"h": 1}
-    monkeypatch.setattr(torch.cuda, "current_stream", lambda device=None: FakeStream(cur["h"]))
+        def is_capturing(self):
+            return self._capturing
+
+    cur = {"h": 1, "cap": False}
+    monkeypatch.setattr(torch.cuda, "current_stream",
+                        lambda device=None: FakeStream(cur["h"], cur["cap"]))
     cache = q._WorkspaceCache(limit=3)
     a = cache.get(("b", "cpu"), 1000, "cpu")
     assert a is cache.get(("b", "cpu"), 900, "cpu")          # reused on the same stream
@@ -166,3 +171,16 @@ def test_workspace_cache_is_per_stream_and_bounded(L, monkeypatch):
     assert len(cache._bufs) == 3                               # bounded, oldest dropped
     cur["h"] = 1
     assert cache.get(("b", "cpu"), 1000, "cpu") is not a       # stream 1's buffer was evicted
+    # while the stream captures a CUDA graph: no allocation, no growth, and the
+    # buffer handed out stays referenced after a later call replaces it
+    cur["h"] = 7
+    d = cache.get(("b", "cpu"), 1000, "cpu")
+    cur["cap"] = True
+    assert cache.get(("b", "cpu"), 800, "cpu") is d
+    with pytest.raises(RuntimeError):
+        cache.get(("b", "cpu"), 4000, "cpu")
+    with pytest.raises(RuntimeError):
+        cache.get(("q", "cpu"), 10, "cpu")
+    cur["cap"] = False
+    e = cache.get(("b", "cpu"), 4000, "cpu")
+    assert e is not d and any(x is d for x in cache._captured)
