@@ -74,7 +74,7 @@ qnf4::ScaleView view_of(const qlora_nf4_state* st) {
 qlora_status check_linear_shape(int64_t M, int64_t K, int64_t N, int32_t r) {
   if (M < 1 || K < 1 || N < 1) return QLORA_ERR_INVALID_ARG;
   if (K % 64 != 0 || N % 64 != 0) return QLORA_ERR_UNSUPPORTED;
-  if (r < 8 || r > 64 || r % 8 != 0) return QLORA_ERR_UNSUPPORTED;
+  if (r < 1 || r > 64) return QLORA_ERR_UNSUPPORTED;
   if (M > (1ll << 30) || K > (1ll << 30) || N > (1ll << 30)) return QLORA_ERR_UNSUPPORTED;
   if (K * N > kMaxNumel) return QLORA_ERR_UNSUPPORTED;
   return QLORA_OK;

@@ -51,11 +51,14 @@ struct SkinnyArgs {
   int nk;            // number of 64-wide k' blocks
   int kb_per_split;  // k' blocks per split
   int splits;        // = cluster size along y (<= 8)
-  int ncols;         // columns of D that are kept (the rank r)
+  int ncols;         // columns of D that are summed (the rank, or the padded rank)
+  int nout;          // columns written to `out` (<= ncols)
   float scale;
-  int mode;          // 0: bf16 out[Mp][ld]; 1: fp32 out[Mp][ld]; 2: fp32 out[ncols][Mp]
+  int mode;          // 0: bf16 out[Mp][ld]; 1: fp32 out[Mp][ld]; 2: fp32 out[nout][Mp]
   void* out;
   int ld;
+  uint16_t* out2;    // mode 0 only, may be null: all ncols columns again, bf16 [Mp][ld2]
+  int ld2;
   int32_t* d_status;
 };
 
@@ -211,12 +214,14 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       acc *= args.scale;
       if (grow < args.Mp) {
         if (args.mode == 0) {
-          static_cast<uint16_t*>(args.out)[static_cast<int64_t>(grow) * args.ld + cc] =
-              static_cast<uint16_t>(pack_bf16x2(acc, 0.0f) & 0xFFFFu);
-        } else if (args.mode == 1) {
-          static_cast<float*>(args.out)[static_cast<int64_t>(grow) * args.ld + cc] = acc;
-        } else {
-          static_cast<float*>(args.out)[static_cast<int64_t>(cc) * args.Mp + grow] = acc;
+          const uint16_t v = static_cast<uint16_t>(pack_bf16x2(acc, 0.0f) & 0xFFFFu);
+          if (cc < args.nout) static_cast<uint16_t*>(args.out)[static_cast<int64_t>(grow) * args.ld + cc] = v;
+          if (args.out2 != nullptr) args.out2[static_cast<int64_t>(grow) * args.ld2 + cc] = v;
+        } else if (cc < args.nout) {
+          if (args.mode == 1)
+            static_cast<float*>(args.out)[static_cast<int64_t>(grow) * args.ld + cc] = acc;
+          else
+            static_cast<float*>(args.out)[static_cast<int64_t>(cc) * args.Mp + grow] = acc;
         }
       }
     }
@@ -1128,16 +1133,35 @@ __global__ void __launch_bounds__(128) gemv_finish_kernel(const float* __restric
   float acc = 0.0f;
 #pragma unroll 4
   for (int s = 0; s < splits; ++s) acc += partial[(static_cast<int64_t>(s) * M + m) * N + n];
-  // r is a multiple of 8: eight independent loads of B per round
+  // eight independent loads of B per round (rows past r read as zero)
   float lora = 0.0f;
   for (int j0 = 0; j0 < r; j0 += 8) {
     float bv[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) bv[u] = bf16_bits_to_f32(__ldg(B + static_cast<int64_t>(j0 + u) * N + n));
+    for (int u = 0; u < 8; ++u)
+      bv[u] = j0 + u < r ? bf16_bits_to_f32(__ldg(B + static_cast<int64_t>(j0 + u) * N + n)) : 0.0f;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) lora = fmaf(zs[j0 + u], bv[u], lora);
+    for (int u = 0; u < 8; ++u)
+      if (j0 + u < r) lora = fmaf(zs[j0 + u], bv[u], lora);
   }
   Y[static_cast<int64_t>(m) * N + n] = static_cast<uint16_t>(pack_bf16x2(acc + lora, 0.0f) & 0xFFFFu);
+}
+
+// Zero-padded copy of a rows x r bf16 matrix into rows x rp (rp = r rounded
+// up to a multiple of 8), so that every row starts on a 16-byte boundary as
+// the tensor maps need.  Only used when r is not a multiple of 8.
+__global__ void __launch_bounds__(256) pad_cols_kernel(const uint16_t* __restrict__ src,
+                                                       int64_t rows, int r,
+                                                       uint16_t* __restrict__ dst, int rp) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int64_t total = rows * rp;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = i / rp;
+    const int col = static_cast<int>(i - row * rp);
+    dst[i] = col < r ? src[row * r + col] : static_cast<uint16_t>(0);
+  }
 }
 
 // ===========================================================================
@@ -1183,10 +1207,12 @@ cudaError_t set_skinny_attr() {
 }
 
 // D = scale * A(m',k') B(n',k'): one launch, split-K sums added in-kernel.
+// ncols columns of D are summed; the first nout go to `out`, and in mode 0 all
+// ncols also go to out2 (a padded copy) when it is not null.
 template <bool kAmn, bool kBmn>
 cudaError_t run_skinny(const CUtensorMap& ta, const CUtensorMap& tb, int Mp, int Kp, int ncols,
                        float scale, int mode, void* out, int ld, int splits, int32_t* d_status,
-                       cudaStream_t st) {
+                       cudaStream_t st, int nout = -1, uint16_t* out2 = nullptr, int ld2 = 0) {
   cudaError_t e = set_skinny_attr<kAmn, kBmn>();
   if (e != cudaSuccess) return e;
   const int nk = (Kp + 63) / 64;
@@ -1196,10 +1222,13 @@ cudaError_t run_skinny(const CUtensorMap& ta, const CUtensorMap& tb, int Mp, int
   a.kb_per_split = (nk + splits - 1) / splits;
   a.splits = (nk + a.kb_per_split - 1) / a.kb_per_split;
   a.ncols = ncols;
+  a.nout = nout < 0 ? ncols : nout;
   a.scale = scale;
   a.mode = mode;
   a.out = out;
   a.ld = ld;
+  a.out2 = out2;
+  a.ld2 = ld2;
   a.d_status = d_status;
   {
     ProfScope prof(kProfSkinny, st);
@@ -1223,6 +1252,23 @@ constexpr CUtensorMapDataType kBF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
 constexpr CUtensorMapSwizzle kSW128 = CU_TENSOR_MAP_SWIZZLE_128B;
 
 int rsteps_of(int r) { return (r + 15) / 16; }
+
+// Rank rounded up to a multiple of 8: the row pitch (rp * 2 bytes) of every
+// rank-r operand read by TMA must be a multiple of 16 bytes.
+int padded_rank(int r) { return (r + 7) & ~7; }
+
+cudaError_t launch_pad(const uint16_t* src, int64_t rows, int r, uint16_t* dst, int rp,
+                       cudaStream_t st) {
+  const int64_t want = (rows * rp + 255) / 256;
+  const unsigned grid = static_cast<unsigned>(want < 592 ? want : 592);
+  cudaError_t e;
+  {
+    ProfScope prof(kProfOther, st);
+    e = launch_pdl(pad_cols_kernel, dim3(grid), dim3(256), 0, st, 1, src, rows, r, dst, rp);
+  }
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
 
 // GEMV split: one CTA per SM over (256-column groups) x (K splits).
 void gemv_plan(int64_t K, int64_t N, int num_sms, int* splits, int* stages_per_split) {
@@ -1277,18 +1323,28 @@ static SideStream* side_stream(int dev) {
 }
 
 size_t linear_fwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) {
-  if (M > 16) return 0;   // the rank-r kernel adds its splits in shared memory
+  const int rp = padded_rank(r);
+  // A zero-padded to rp columns when r is not a multiple of 8
+  const size_t apad = rp != r ? align256(static_cast<size_t>(K) * rp * 2) : 0;
+  if (M > 16) {
+    // the rank-r kernel adds its splits in shared memory; a padded copy of Zc
+    // for the fused kernel's TMA when r is not a multiple of 8
+    return rp != r ? apad + align256(static_cast<size_t>(M) * rp * 2) : 0;
+  }
   // GEMV partials and its per-split X·A slices
   int S = 1, per = 1;
   gemv_plan(K, N, g_ws_sms, &S, &per);
-  return align256(static_cast<size_t>(S) * M * N * 4) + align256(static_cast<size_t>(S) * M * r * 4);
+  return align256(static_cast<size_t>(S) * M * N * 4) + align256(static_cast<size_t>(S) * M * r * 4) +
+         apad;
 }
 
 size_t linear_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) {
-  (void)K;
   (void)N;
-  // dZ, and Zc when the caller recomputes it instead of saving it (both bf16, M x r)
-  return 2 * align256(static_cast<size_t>(M) * r * 2);
+  const int rp = padded_rank(r);
+  // dZ, and Zc when the caller recomputes it instead of saving it (or a padded
+  // copy of the caller's Zc), both bf16 M x rp; A padded to rp columns
+  return 2 * align256(static_cast<size_t>(M) * rp * 2) +
+         (rp != r ? align256(static_cast<size_t>(K) * rp * 2) : 0);
 }
 
 cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint16_t* X,
@@ -1297,20 +1353,37 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
                               size_t ws_bytes, int32_t* d_status, cudaStream_t st, int num_sms) {
   (void)num_sms;
   WsCursor cur{static_cast<char*>(ws), ws_bytes};
+  const int rp = padded_rank(r);
+  const bool pad = rp != r;
+  cudaError_t e = cudaSuccess;
+  float* pg = nullptr;
+  float* pz = nullptr;
+  int S = 1, per = 1;
+  if (M <= 16) {
+    gemv_plan(K, N, g_ws_sms, &S, &per);
+    pg = static_cast<float*>(cur.take(static_cast<size_t>(S) * M * N * 4));
+    pz = static_cast<float*>(cur.take(static_cast<size_t>(S) * M * r * 4));
+  }
+  // A zero-padded to rp columns (16-byte row pitch for TMA) when r % 8 != 0
+  const uint16_t* At = A;
+  if (pad) {
+    uint16_t* Ap = static_cast<uint16_t*>(cur.take(static_cast<size_t>(K) * rp * 2));
+    if (!cur.ok) return cudaErrorInvalidValue;
+    e = launch_pad(A, K, r, Ap, rp, st);
+    if (e != cudaSuccess) return e;
+    At = Ap;
+  }
+  if (!cur.ok) return cudaErrorInvalidValue;
   // Zc = bf16(c * X A): A operand X (K-major), B operand A (MN-major over r)
   CUtensorMap tX, tAl, tZc, tBl;
   if (!make_tmap_2d(&tX, X, kBF16, 2, M, K, K, 64, 128, kSW128)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&tAl, A, kBF16, 2, K, r, r, 64, 64, kSW128)) return cudaErrorInvalidValue;
-  cudaError_t e = cudaSuccess;
+  if (!make_tmap_2d(&tAl, At, kBF16, 2, K, rp, rp, 64, 64, kSW128)) return cudaErrorInvalidValue;
   if (M <= 16) {
-    int S = 1, per = 1;
-    gemv_plan(K, N, g_ws_sms, &S, &per);
     const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
-    float* pg = static_cast<float*>(cur.take(static_cast<size_t>(S) * M * N * 4));
-    float* pz = static_cast<float*>(cur.take(static_cast<size_t>(S) * M * r * 4));
-    if (!cur.ok) return cudaErrorInvalidValue;
     const int ncg = static_cast<int>((N + 255) / 256);
-    const bool xa_in_gemv = ncg * 8 >= r;   // every 8-column rank slice has a column group
+    // Zc by the rank-r kernel, exactly as the backward recomputes it when the
+    // caller keeps no Zc (same kernel, same splits: the same bits)
+    const bool xa_in_gemv = false;
     if (!xa_in_gemv) {
       e = run_skinny<false, true>(tX, tAl, static_cast<int>(M), static_cast<int>(K), r, c, 0, Zc, r,
                                   Sz, d_status, st);
@@ -1331,7 +1404,7 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
     if (!make_tmap_2d(&tP, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N / 2, N / 2, 128, kGvRows, kSW128))
       return cudaErrorInvalidValue;
     if (!make_tmap_2d(&tXg, X, kBF16, 2, M, K, K, 64, 16, kSW128)) return cudaErrorInvalidValue;
-    if (!make_tmap_2d(&tAg, A, kBF16, 2, K, r, r, 8, kGvRows, CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!make_tmap_2d(&tAg, At, kBF16, 2, K, rp, rp, 8, kGvRows, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
     GemvArgs ga;
     ga.M = static_cast<int>(M);
@@ -1363,16 +1436,22 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
     return cudaGetLastError();
   }
 
-  // rank-r product for the tensor-core path: Zc = bf16(c * X A)
+  // rank-r product for the tensor-core path: Zc = bf16(c * X A), and a copy
+  // padded to rp columns for the fused kernel's TMA when r % 8 != 0
+  uint16_t* Zp = nullptr;
+  if (pad) {
+    Zp = static_cast<uint16_t*>(cur.take(static_cast<size_t>(M) * rp * 2));
+    if (!cur.ok) return cudaErrorInvalidValue;
+  }
   {
     const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
-    e = run_skinny<false, true>(tX, tAl, static_cast<int>(M), static_cast<int>(K), r, c, 0, Zc, r,
-                                Sz, d_status, st);
+    e = run_skinny<false, true>(tX, tAl, static_cast<int>(M), static_cast<int>(K), rp, c, 0, Zc, r,
+                                Sz, d_status, st, r, Zp, rp);
     if (e != cudaSuccess) return e;
   }
   e = set_fused_attr<false>();
   if (e != cudaSuccess) return e;
-  if (!make_tmap_2d(&tZc, Zc, kBF16, 2, M, r, r, 64, 128, kSW128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tZc, pad ? Zp : Zc, kBF16, 2, M, rp, rp, 64, 128, kSW128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tBl, B, kBF16, 2, r, N, N, 64, 64, kSW128)) return cudaErrorInvalidValue;
   FusedArgs fa;
   fa.M = static_cast<int>(M);
@@ -1407,47 +1486,62 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
                               int32_t* d_status, cudaStream_t st, int num_sms) {
   (void)num_sms;
   WsCursor cur{static_cast<char*>(ws), ws_bytes};
-  uint16_t* dZ = static_cast<uint16_t*>(cur.take(static_cast<size_t>(M) * r * 2));
-  uint16_t* Zc_ws = static_cast<uint16_t*>(cur.take(static_cast<size_t>(M) * r * 2));
+  const int rp = padded_rank(r);
+  const bool pad = rp != r;
+  // dZ and the working copy of Zc are bf16 M x rp (row pitch 16-byte aligned)
+  uint16_t* dZ = static_cast<uint16_t*>(cur.take(static_cast<size_t>(M) * rp * 2));
+  uint16_t* Zc_ws = static_cast<uint16_t*>(cur.take(static_cast<size_t>(M) * rp * 2));
+  uint16_t* Ap = pad ? static_cast<uint16_t*>(cur.take(static_cast<size_t>(K) * rp * 2)) : nullptr;
   const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(N / 64), g_ws_sms);
   const int nkm = static_cast<int>((M + 63) / 64);
   const int Sa = skinny_splits(static_cast<int>(K), nkm, g_ws_sms);
   const int Sb = skinny_splits(static_cast<int>(N), nkm, g_ws_sms);
   if (!cur.ok) return cudaErrorInvalidValue;
   cudaError_t e = cudaSuccess;
+  const uint16_t* At = A;
+  if (pad) {
+    e = launch_pad(A, K, r, Ap, rp, st);
+    if (e != cudaSuccess) return e;
+    At = Ap;
+  }
   if (Zc == nullptr) {
     // saved-activation policy "recompute": Zc = bf16(c X A) exactly as the
     // forward forms it (same kernel, same splits, so the same bits)
     CUtensorMap tXf, tAf;
     if (!make_tmap_2d(&tXf, X, kBF16, 2, M, K, K, 64, 128, kSW128)) return cudaErrorInvalidValue;
-    if (!make_tmap_2d(&tAf, A, kBF16, 2, K, r, r, 64, 64, kSW128)) return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&tAf, At, kBF16, 2, K, rp, rp, 64, 64, kSW128)) return cudaErrorInvalidValue;
     const int Sf = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
-    e = run_skinny<false, true>(tXf, tAf, static_cast<int>(M), static_cast<int>(K), r, c, 0, Zc_ws,
-                                r, Sf, d_status, st);
+    e = run_skinny<false, true>(tXf, tAf, static_cast<int>(M), static_cast<int>(K), rp, c, 0, Zc_ws,
+                                rp, Sf, d_status, st);
+    if (e != cudaSuccess) return e;
+    Zc = Zc_ws;
+  } else if (pad) {
+    e = launch_pad(Zc, M, r, Zc_ws, rp, st);
     if (e != cudaSuccess) return e;
     Zc = Zc_ws;
   }
 
   CUtensorMap tG, tBk, tXmn, tdZ, tGmn, tZcmn, tAl;
-  // dZ = c * G B^T : A operand G (K-major over N), B operand B (K-major: rows r, cols N)
+  // dZ = c * G B^T : A operand G (K-major over N), B operand B (K-major: rows r, cols N);
+  // B's rows past r arrive as zero fill, so dZ's padding columns are zero
   if (!make_tmap_2d(&tG, dY, kBF16, 2, M, N, N, 64, 128, kSW128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tBk, B, kBF16, 2, r, N, N, 64, 64, kSW128)) return cudaErrorInvalidValue;
-  e = run_skinny<false, false>(tG, tBk, static_cast<int>(M), static_cast<int>(N), r, c, 0, dZ, r,
+  e = run_skinny<false, false>(tG, tBk, static_cast<int>(M), static_cast<int>(N), rp, c, 0, dZ, rp,
                                Sz, d_status, st);
   if (e != cudaSuccess) return e;
   // dA = X^T dZ : A operand X^T (MN-major over K), B operand dZ (MN-major over r)
   if (!make_tmap_2d(&tXmn, X, kBF16, 2, M, K, K, 64, 64, kSW128)) return cudaErrorInvalidValue;
-  // (columns of dZ past r arrive as TMA zero fill)
-  if (!make_tmap_2d(&tdZ, dZ, kBF16, 2, M, r, r, 64, 64, kSW128)) return cudaErrorInvalidValue;
+  // (columns of dZ past rp arrive as TMA zero fill)
+  if (!make_tmap_2d(&tdZ, dZ, kBF16, 2, M, rp, rp, 64, 64, kSW128)) return cudaErrorInvalidValue;
   // dB^T = G^T Zc : A operand G^T (MN-major over N), B operand Zc (MN-major over r)
   if (!make_tmap_2d(&tGmn, dY, kBF16, 2, M, N, N, 64, 64, kSW128)) return cudaErrorInvalidValue;
-  if (!make_tmap_2d(&tZcmn, Zc, kBF16, 2, M, r, r, 64, 64, kSW128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tZcmn, Zc, kBF16, 2, M, rp, rp, 64, 64, kSW128)) return cudaErrorInvalidValue;
   // dX = G W^T + dZ A^T
   e = set_fused_attr<true>();
   if (e != cudaSuccess) return e;
-  if (!make_tmap_2d(&tAl, A, kBF16, 2, K, r, r, 64, kFBN, kSW128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tAl, At, kBF16, 2, K, rp, rp, 64, kFBN, kSW128)) return cudaErrorInvalidValue;
   CUtensorMap tdZa;
-  if (!make_tmap_2d(&tdZa, dZ, kBF16, 2, M, r, r, 64, 128, kSW128)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&tdZa, dZ, kBF16, 2, M, rp, rp, 64, 128, kSW128)) return cudaErrorInvalidValue;
   FusedArgs fa;
   fa.M = static_cast<int>(M);
   fa.Nout = static_cast<int>(K);

@@ -53,11 +53,14 @@ __global__ void __launch_bounds__(256) nf4_merge_kernel(MergeArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int nb = blockIdx.x, n0 = nb * 64;
-  // B[j][n0 .. n0+63] -> bt, rank rows in pairs (r is a multiple of 8)
-  for (int i = threadIdx.x; i < (a.r / 2) * 64; i += blockDim.x) {
+  // B[j][n0 .. n0+63] -> bt, rank rows in pairs; rows from r up to the next
+  // multiple of 16 (the last mma step) are zero
+  const int r16 = (a.r + 15) & ~15;
+  for (int i = threadIdx.x; i < (r16 / 2) * 64; i += blockDim.x) {
     const int jp = i >> 6, n = i & 63;
-    const uint32_t lo = __ldg(a.B + static_cast<int64_t>(2 * jp) * a.N + n0 + n);
-    const uint32_t hi = __ldg(a.B + static_cast<int64_t>(2 * jp + 1) * a.N + n0 + n);
+    const uint32_t lo = 2 * jp < a.r ? __ldg(a.B + static_cast<int64_t>(2 * jp) * a.N + n0 + n) : 0u;
+    const uint32_t hi =
+        2 * jp + 1 < a.r ? __ldg(a.B + static_cast<int64_t>(2 * jp + 1) * a.N + n0 + n) : 0u;
     bt[n * kMgLd + jp] = lo | (hi << 16);
   }
   __syncthreads();
@@ -76,17 +79,23 @@ __global__ void __launch_bounds__(256) nf4_merge_kernel(MergeArgs a) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[s8][i] = 0.0f;
     const int64_t rowA = static_cast<int64_t>(kA) * a.r, rowB = static_cast<int64_t>(kB) * a.r;
+    // A[row][j], A[row][j + 1] as one bf16 pair; columns from r on are zero
+    // (r may be odd, so the pair is read as two 16-bit values)
+    auto a_pair = [&](int64_t row, int j) -> uint32_t {
+      const uint32_t lo = j < a.r ? __ldg(a.A + row + j) : 0u;
+      const uint32_t hi = j + 1 < a.r ? __ldg(a.A + row + j + 1) : 0u;
+      return lo | (hi << 16);
+    };
     for (int j0 = 0; j0 < a.r; j0 += 16) {
-      const bool hi = j0 + 8 < a.r;   // the upper 8 rank columns of a step may be absent
       uint32_t af[4];
-      af[0] = __ldg(reinterpret_cast<const uint32_t*>(a.A + rowA + j0 + 2 * t));
-      af[1] = __ldg(reinterpret_cast<const uint32_t*>(a.A + rowB + j0 + 2 * t));
-      af[2] = hi ? __ldg(reinterpret_cast<const uint32_t*>(a.A + rowA + j0 + 8 + 2 * t)) : 0u;
-      af[3] = hi ? __ldg(reinterpret_cast<const uint32_t*>(a.A + rowB + j0 + 8 + 2 * t)) : 0u;
+      af[0] = a_pair(rowA, j0 + 2 * t);
+      af[1] = a_pair(rowB, j0 + 2 * t);
+      af[2] = a_pair(rowA, j0 + 8 + 2 * t);
+      af[3] = a_pair(rowB, j0 + 8 + 2 * t);
 #pragma unroll
       for (int s8 = 0; s8 < 8; ++s8) {
         const uint32_t* col = bt + (8 * s8 + g) * kMgLd + j0 / 2 + t;
-        mma_m16n8k16_bf16(acc[s8], af, col[0], hi ? col[4] : 0u);
+        mma_m16n8k16_bf16(acc[s8], af, col[0], col[4]);
       }
     }
     // decoded weights and the merge, rows kA and kB

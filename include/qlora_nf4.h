@@ -199,11 +199,14 @@ qlora_status qlora_nf4_dequantize(const qlora_nf4_state* st, uint16_t* W_hat,
  * to bf16 (each weight within one bf16 ulp of qlora_nf4_dequantize's output)
  * and never written to memory.  M <= 16 runs the HBM-bound GEMV path, larger
  * M the fused tensor-core path.
- * Shapes: M >= 1, K % 64 == 0, N % 64 == 0, 8 <= r <= 64 with r % 8 == 0,
- * else UNSUPPORTED.
+ * Shapes: M >= 1, K % 64 == 0, N % 64 == 0, 1 <= r <= 64, else UNSUPPORTED.
+ * A rank that is not a multiple of 8 is zero-padded to the next multiple of 8
+ * inside the workspace (A, and the copy of Zc the tensor-core path reads), so
+ * that every row the tensor maps read starts on a 16-byte boundary; the padded
+ * rank columns are zero and change no result.
  * ws: at least qlora_linear_fwd_workspace_size(M, K, N, r) bytes; that size is
- * 0 for M > 16 (the rank-r kernel adds its K splits inside a thread-block
- * cluster), and ws may then be null.
+ * 0 for M > 16 when r % 8 == 0 (the rank-r kernel adds its K splits inside a
+ * thread-block cluster), and ws may then be null.
  */
 size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t K, int64_t N, int32_t r);
 qlora_status qlora_linear_fwd(int64_t M, int64_t K, int64_t N, int32_t r,
@@ -261,8 +264,8 @@ qlora_status qlora_linear_bwd(int64_t M, int64_t K, int64_t N, int32_t r,
  *   W   : NF4 state of the K×N weight (numel must equal K·N)
  *   A   : device bf16 K×r      B : device bf16 r×N     (row-major)
  *   out : device bf16 K×N output (may not alias A, B or the state)
- * Shapes as qlora_linear_fwd (K % 64 == 0, N % 64 == 0, 8 <= r <= 64, r % 8
- * == 0).  A non-finite decode scale raises QLORA_ERR_NONFINITE in d_status.
+ * Shapes as qlora_linear_fwd (K % 64 == 0, N % 64 == 0, 1 <= r <= 64).  A
+ * non-finite decode scale raises QLORA_ERR_NONFINITE in d_status.
  * No workspace; asynchronous on `stream`.
  */
 qlora_status qlora_nf4_merge(int64_t K, int64_t N, int32_t r, const qlora_nf4_state* W,

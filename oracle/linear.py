@@ -31,17 +31,27 @@ def lora_forward(X, W_hat, A, B, c):
     return Y, Z
 
 
-def lora_backward(G, X, W_hat, A, B, c):
-    """Returns (dX, dA, dB) for the output gradient G, all fp64."""
+def lora_adapter_grads(G, X, A, B, c):
+    """The trainable branch's part of the backward, which needs no W_hat:
+    returns (dZ, dA, dB) with Z = X A, dZ = c G B^T, dA = X^T dZ, dB = c Z^T G,
+    all fp64 ([P1] §"冻结权重为什么仍然需要输入梯度")."""
     G = np.asarray(G, dtype=np.float64)
     X = np.asarray(X, dtype=np.float64)
-    W_hat = np.asarray(W_hat, dtype=np.float64)
     A = np.asarray(A, dtype=np.float64)
     B = np.asarray(B, dtype=np.float64)
     c = float(c)
     Z = X @ A
     dZ = c * (G @ B.T)
-    dX = G @ W_hat.T + dZ @ A.T
     dA = X.T @ dZ
     dB = c * (Z.T @ G)
+    return dZ, dA, dB
+
+
+def lora_backward(G, X, W_hat, A, B, c):
+    """Returns (dX, dA, dB) for the output gradient G, all fp64."""
+    G = np.asarray(G, dtype=np.float64)
+    W_hat = np.asarray(W_hat, dtype=np.float64)
+    A = np.asarray(A, dtype=np.float64)
+    dZ, dA, dB = lora_adapter_grads(G, X, A, B, c)
+    dX = G @ W_hat.T + dZ @ A.T
     return dX, dA, dB

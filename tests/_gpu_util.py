@@ -65,3 +65,49 @@ def assert_state_equal(w_gpu, ow: OracleWeight):
     else:
         assert np.array_equal(w_gpu.absmax.cpu().numpy().view(np.uint32), ow.absmax.view(np.uint32)), \
             "absmax differs"
+
+
+# Element-wise bounds on top of the whole-matrix relative Frobenius error: a
+# handful of wrong outputs, or one wrong 64-column block in one row, moves the
+# whole-matrix norm of a large output by far less than 5e-3, but not the error
+# of its row or of its tile.
+FRO_TOL = 5e-3
+ROW_TOL = 1e-2
+TILE_TOL = 2e-2
+
+
+def close_report(got, ref, tile=128):
+    """Relative errors of `got` against `ref`: whole matrix (Frobenius), worst
+    row, worst tile x tile block.  A row or tile whose reference norm is tiny
+    is measured against a tenth of the typical row or tile norm instead."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    if ref.ndim == 1:
+        got, ref = got[None, :], ref[None, :]
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    diff = got - ref
+    total = np.linalg.norm(ref)
+    out = {"fro": float(np.linalg.norm(diff) / (total if total > 0 else 1.0))}
+    R, C = ref.shape
+    row_rms = total / np.sqrt(R)
+    rn = np.linalg.norm(ref, axis=1)
+    dn = np.linalg.norm(diff, axis=1)
+    out["row"] = float(np.max(dn / np.maximum(rn, max(0.1 * row_rms, 1e-300))))
+    tr, tc = min(tile, R), min(tile, C)
+    Rp, Cp = -(-R // tr) * tr, -(-C // tc) * tc
+
+    def blocks(a):
+        p = np.zeros((Rp, Cp))
+        p[:R, :C] = a
+        return np.sqrt((p.reshape(Rp // tr, tr, Cp // tc, tc) ** 2).sum(axis=(1, 3)))
+
+    tn, td = blocks(ref), blocks(diff)
+    tile_rms = total / np.sqrt(tn.size)
+    out["tile"] = float(np.max(td / np.maximum(tn, max(0.1 * tile_rms, 1e-300))))
+    return out
+
+
+def assert_close(name, got, ref, fro=FRO_TOL, row=ROW_TOL, tile_tol=TILE_TOL):
+    rep = close_report(got, ref)
+    assert rep["fro"] <= fro and rep["row"] <= row and rep["tile"] <= tile_tol, (name, rep)
+    return rep

@@ -67,7 +67,11 @@ def test_workspace_sizes(L):
     assert lib.qlora_linear_bwd_workspace_size(4096, 4096, 4096, 16) >= 4096 * 16 * 2
     # unsupported shapes report 0
     assert lib.qlora_linear_fwd_workspace_size(16, 100, 64, 16) == 0
-    assert lib.qlora_linear_fwd_workspace_size(16, 64, 64, 12) == 0
+    assert lib.qlora_linear_fwd_workspace_size(16, 64, 64, 0) == 0
+    assert lib.qlora_linear_fwd_workspace_size(16, 64, 64, 65) == 0
+    # a rank that is not a multiple of 8: A (K x 16) and Zc (M x 16) padded copies
+    assert lib.qlora_linear_fwd_workspace_size(4096, 4096, 4096, 12) >= (4096 + 4096) * 16 * 2
+    assert lib.qlora_linear_bwd_workspace_size(4096, 4096, 4096, 3) >= (2 * 4096 + 4096) * 8 * 2
 
 
 def _state(L, numel=128, dq=0, packed=4096):
@@ -103,7 +107,8 @@ def test_host_validation_rejects_before_device_work(L):
     w = _state(L, numel=64 * 64)
     args = [fake, C.byref(w), fake, fake, 1.0, fake, fake, fake, 1 << 20, None, None]
     assert lib.qlora_linear_fwd(8, 100, 64, 16, *args) == E.QLORA_ERR_UNSUPPORTED
-    assert lib.qlora_linear_fwd(8, 64, 64, 4, *args) == E.QLORA_ERR_UNSUPPORTED
+    assert lib.qlora_linear_fwd(8, 64, 64, 0, *args) == E.QLORA_ERR_UNSUPPORTED
+    assert lib.qlora_linear_fwd(8, 64, 64, 65, *args) == E.QLORA_ERR_UNSUPPORTED
     assert lib.qlora_linear_fwd(8, 64, 64, 72, *args) == E.QLORA_ERR_UNSUPPORTED
     assert lib.qlora_linear_fwd(0, 64, 64, 16, *args) == E.QLORA_ERR_INVALID_ARG
     assert lib.qlora_linear_fwd(8, 128, 64, 16, *args) == E.QLORA_ERR_INVALID_ARG   # numel != K*N

@@ -1,16 +1,18 @@
 """GPU parity of qlora_linear_fwd / qlora_linear_bwd against the fp64 oracle.
 
-Bar: relative Frobenius error <= 5e-3 for Y, dX, dA, dB (each against the
-oracle's fp64 result on the oracle's own dequantized weight), with exact
-special cases where the arithmetic makes them exact.
+Bar: for Y, Zc, dX, dA, dB (each against the oracle's fp64 result on the
+oracle's own dequantized weight) a whole-matrix relative Frobenius error <=
+5e-3, and the worst row's and worst 128 x 128 tile's relative error within the
+bounds of tests/_gpu_util.py; exact special cases where the arithmetic makes
+them exact.
 """
 import numpy as np
 import pytest
 import torch
 
 from inputs import synthetic as S
-from oracle.linear import lora_backward, lora_forward
-from tests._gpu_util import OracleWeight, rel_fro, to_dev, to_np
+from oracle.linear import lora_adapter_grads, lora_backward, lora_forward
+from tests._gpu_util import OracleWeight, assert_close, close_report, rel_fro, to_dev, to_np
 
 pytestmark = pytest.mark.gpu
 TOL = 5e-3
@@ -29,13 +31,19 @@ def run_case(lin, r, c, dq, *, backward=True, w_dtype=torch.bfloat16):
     Y, Zc = q.linear_forward(Xt, wq, At, Bt, c)
     ow = OracleWeight(W, dq)
     Yr, Zr = lora_forward(X, ow.w_hat, A, B, c)
-    out = {"Y": rel_fro(to_np(Y), Yr), "Zc": rel_fro(to_np(Zc), c * Zr)}
+    out = {"Y": assert_close("Y", to_np(Y), Yr)["fro"],
+           "Zc": assert_close("Zc", to_np(Zc), c * Zr)["fro"]}
     if backward:
         G = lin.dY
         dX, dA, dB = q.linear_backward(to_dev(G), Xt, Zc, wq, At, Bt, c)
         dXr, dAr, dBr = lora_backward(G, X, ow.w_hat, A, B, c)
-        out.update(dX=rel_fro(to_np(dX), dXr), dA=rel_fro(to_np(dA), dAr),
-                   dB=rel_fro(to_np(dB), dBr))
+        out.update(dX=assert_close("dX", to_np(dX), dXr)["fro"],
+                   dA=assert_close("dA", to_np(dA), dAr)["fro"],
+                   dB=assert_close("dB", to_np(dB), dBr)["fro"])
+        # the recompute policy (no saved Zc) gives the same bits
+        dX2, dA2, dB2 = q.linear_backward(to_dev(G), Xt, None, wq, At, Bt, c)
+        for a_, b_ in zip((dX, dA, dB), (dX2, dA2, dB2)):
+            assert torch.equal(a_, b_)
     return out
 
 
@@ -55,6 +63,29 @@ def test_fwd_bwd_parity(M, K, N, r, dq):
     lin = S.random_case(M + K + N + r, M, K, N, r)
     lin.dY = S.normal(7, M, 4, (M, N), 1.0)
     errs = run_case(lin, r, 32.0 / r, dq)
+    for k, v in errs.items():
+        assert v <= TOL, (k, v, errs)
+
+
+ODD_RANK_CASES = [
+    # (M, K, N, r): ranks that are not multiples of 8, zero-padded inside the
+    # workspace; tensor-core path (M > 16) and GEMV (M <= 16), fwd and bwd
+    (200, 256, 320, 1),
+    (129, 320, 256, 3),
+    (300, 512, 192, 12),
+    (160, 384, 512, 40),
+    (1, 256, 320, 1),
+    (4, 320, 448, 3),
+    (9, 512, 384, 12),
+    (16, 576, 256, 40),
+]
+
+
+@pytest.mark.parametrize("M,K,N,r", ODD_RANK_CASES)
+def test_ranks_not_multiple_of_8(M, K, N, r):
+    lin = S.random_case(3000 + M + K + N + r, M, K, N, r)
+    lin.dY = S.normal(13, M + r, 4, (M, N), 1.0)
+    errs = run_case(lin, r, 16.0 / r, True)
     for k, v in errs.items():
         assert v <= TOL, (k, v, errs)
 
@@ -232,13 +263,12 @@ def test_full_size_projection_sampled_rows():
     rng = np.random.default_rng(0)
     rows = np.unique(np.concatenate([[0, 4095], rng.integers(0, 4096, 96)]))
     Yr, _ = lora_forward(X[rows], ow.w_hat, A, B, c)
-    assert rel_fro(to_np(Y)[rows], Yr) <= TOL
+    assert_close("Y rows", to_np(Y)[rows], Yr)
     dXr, _, _ = lora_backward(G[rows], X[rows], ow.w_hat, A, B, c)
-    assert rel_fro(to_np(dX)[rows], dXr) <= TOL
-    X64, G64 = X.astype(np.float64), G.astype(np.float64)
-    dZ = c * (G64 @ B.T)
-    assert rel_fro(to_np(dA), X64.T @ dZ) <= TOL
-    assert rel_fro(to_np(dB), c * ((X64 @ A).T @ G64)) <= TOL
+    assert_close("dX rows", to_np(dX)[rows], dXr)
+    _, dAr, dBr = lora_adapter_grads(G, X, A, B, c)
+    assert_close("dA", to_np(dA), dAr)
+    assert_close("dB", to_np(dB), dBr)
 
 
 MERGE_CASES = [(64, 128, 8, True), (320, 384, 16, False), (256, 576, 64, True), (128, 64, 24, True)]
@@ -286,48 +316,3 @@ def test_merge_requantize_matches_oracle_quantize_of_merged():
     code8, s2, off = nf4.double_quantize(absmax)
     assert np.array_equal(rq.packed.cpu().numpy(), payload)
     assert np.array_equal(rq.code8.cpu().numpy(), code8)
-
-
-@pytest.mark.slow
-def test_full_size_65b_mlp_sampled():
-    """The 65B MLP shapes at full size (M = 4096, r = 64, both 8192 x 22016 and
-    22016 x 8192), without double quantization so that the oracle can quantize
-    just the blocks it needs: sampled columns of Y, sampled columns of dX, full
-    dA and dB.  The oracle quantizes those blocks from the same input."""
-    from oracle import nf4
-    q = _q()
-    wl = S.config5()
-    rng = np.random.default_rng(5)
-    for lin in wl.linears:
-        X, W, A, B, G, c = lin.X, lin.W, lin.A, lin.B, lin.dY, wl.c
-        K, N = W.shape
-        M = X.shape[0]
-        wq = q.quantize(to_dev(W), double_quant=False)
-        Xt, At, Bt = to_dev(X), to_dev(A), to_dev(B)
-        Y, Zc = q.linear_forward(Xt, wq, At, Bt, c)
-        dX, dA, dB = q.linear_backward(to_dev(G), Xt, Zc, wq, At, Bt, c)
-        Y, dX, dA, dB = to_np(Y), to_np(dX), to_np(dA), to_np(dB)
-        X64, G64, A64, B64 = (np.asarray(t, np.float64) for t in (X, G, A, B))
-        Z = X64 @ A64
-        dZ = c * (G64 @ B64.T)
-
-        def w_hat_of(block):          # oracle quantization of a (rows x 64k) sub-matrix
-            codes, absmax = nf4.quantize_nf4(np.ascontiguousarray(block, np.float32).ravel())
-            payload, n = nf4.pack_codes(codes)
-            return nf4.dequantize(payload, n, absmax).reshape(block.shape)
-
-        # Y columns: each sampled column's 64-block in every row k
-        cols = np.unique(np.concatenate([[0, N - 1], rng.integers(0, N, 10)]))
-        for j in cols:
-            b0 = (j // 64) * 64
-            wcol = w_hat_of(W[:, b0:b0 + 64])[:, j - b0]
-            ref = X64 @ wcol + c * (Z @ B64[:, j])
-            assert rel_fro(Y[:, j], ref) <= TOL, ("Y", K, N, j)
-        # dX columns k: row k of W in full
-        ks = np.unique(np.concatenate([[0, K - 1], rng.integers(0, K, 10)]))
-        for k in ks:
-            wrow = w_hat_of(W[k:k + 1, :]).ravel()
-            ref = G64 @ wrow + dZ @ A64[k]
-            assert rel_fro(dX[:, k], ref) <= TOL, ("dX", K, N, k)
-        assert rel_fro(dA, X64.T @ dZ) <= TOL
-        assert rel_fro(dB, c * (Z.T @ G64)) <= TOL
