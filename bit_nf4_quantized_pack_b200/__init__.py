@@ -143,7 +143,7 @@ class _WorkspaceCache:
         stream = torch.cuda.current_stream(device)
         key = (*key, stream.cuda_stream)
         buf = self._bufs.get(key)
-        if stream.is_capturing():
+        if torch.cuda.is_current_stream_capturing():
             if buf is None or buf.numel() < nbytes or buf.device != torch.device(device):
                 raise RuntimeError(
                     "no workspace of the needed size is cached for this stream while it is "

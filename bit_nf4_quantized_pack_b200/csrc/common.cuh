@@ -32,6 +32,43 @@ constexpr int kPadCodeInt4 = 8;   // the same for the uniform INT4 codebook (q =
   -8.0f, -7.0f, -6.0f, -5.0f, -4.0f, -3.0f, -2.0f, -1.0f, 0.0f, 1.0f, 2.0f, 3.0f, \
       4.0f, 5.0f, 6.0f, 7.0f
 
+// The signed dynamic 8-bit codebook T8 of the scale codes (this library's own
+// definition; the page only requires "a signed dynamic 8-bit codebook, not
+// FP8 E4M3"): byte u, sign u >> 7, t = u & 127; t = 0 is 0; otherwise
+// f = floor(log2 t), e = 6 - f, m = t - 2^f and |v| = (2^f + 9(m+1)) /
+// (10^(e+1) 2^f), a correctly rounded double division rounded to fp32.
+// Evaluated by the compiler (IEEE double division, then round to nearest
+// float) into a table that decoding kernels copy from constant memory.
+struct T8Table {
+  float v[256];
+};
+
+constexpr double t8_pow10(int e) {
+  double p = 10.0;
+  for (int i = 0; i < e; ++i) p *= 10.0;
+  return p;
+}
+
+constexpr float t8_value(int u) {
+  const int t = u & 127;
+  if (t == 0) return 0.0f;
+  int f = 0;
+  while ((2 << f) <= t) ++f;
+  const int e = 6 - f, m = t - (1 << f);
+  const float mag = static_cast<float>(static_cast<double>((1 << f) + 9 * (m + 1)) /
+                                       (t8_pow10(e) * static_cast<double>(1 << f)));
+  return (u >> 7) ? -mag : mag;
+}
+
+constexpr T8Table make_t8_table() {
+  T8Table t{};
+  for (int u = 0; u < 256; ++u) t.v[u] = t8_value(u);
+  return t;
+}
+static_assert(make_t8_table().v[0x43] == 0.15625f && make_t8_table().v[0x7F] == 1.0f &&
+                  make_t8_table().v[0xFF] == -1.0f && make_t8_table().v[0x80] == 0.0f,
+              "T8 spot values");
+
 // Raise an error bit in the caller's device status word.
 __device__ __forceinline__ void raise_status(int32_t* d_status, int code) {
   if (d_status) atomicOr(d_status, 1 << code);
@@ -183,6 +220,23 @@ __device__ __forceinline__ void bulk_load_1d(void* smem_dst, const void* gsrc, u
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Thread-block clusters: a barrier over every thread of every CTA (lanes may
+// arrive diverged), and a load from a peer CTA's shared memory at the same
+// offset as `local_saddr` in this CTA.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_saddr, uint32_t cta_rank) {
+  uint32_t remote;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_saddr), "r"(cta_rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
 }
 
 // ---------------------------------------------------------------------------

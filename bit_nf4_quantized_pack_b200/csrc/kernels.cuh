@@ -120,6 +120,20 @@ cudaError_t launch_merge(int64_t K, int64_t N, int r, float c, ScaleView sv, con
                          const uint16_t* A, const uint16_t* B, uint16_t* out, int32_t* d_status,
                          cudaStream_t st);
 
+// gemv.cu — the M <= 16 forward (and, with zc_only, the recompute of its Zc):
+// A_pad is A with its rows padded to rp (a multiple of 8) columns; Zc is
+// written with row pitch ldz (columns r .. ldz-1 as 0) by one CTA.
+struct GemvPlan {
+  int G;     // 256-column groups
+  int S;     // K splits = cluster size
+  int per;   // 128-row stages per split
+};
+GemvPlan gemv_plan(int64_t K, int64_t N, int num_sms);
+cudaError_t launch_gemv(int64_t M, int64_t K, int64_t N, int r, const uint16_t* X,
+                        const uint8_t* packed, ScaleView sv, const uint16_t* A_pad, int rp,
+                        const uint16_t* B, float c, uint16_t* Y, uint16_t* Zc, int ldz,
+                        bool zc_only, int32_t* d_status, cudaStream_t st, int num_sms);
+
 // linear.cu — forward and backward of the layer
 size_t linear_fwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r);
 size_t linear_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r);

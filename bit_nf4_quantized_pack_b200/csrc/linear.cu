@@ -17,9 +17,7 @@
 //                        memory, one thread issues tcgen05.mma into TMEM, and
 //                        the rank-r LoRA term is one extra K-step of the same
 //                        accumulator.
-//   nf4_gemv_kernel      M <= 16: split-K GEMV fed by TMA; decoded weight pairs
-//                        go from a shared table straight into mma.sync
-//                        fragments; gemv_finish_kernel adds the splits and Zc·B.
+// The M <= 16 forward (a GEMV) is in gemv.cu.
 #include <atomic>
 #include <cfloat>
 #include <mutex>
@@ -64,20 +62,6 @@ struct SkinnyArgs {
 
 constexpr int kSkRedLd = 65;   // fp32 words per row of the split-sum buffer (bank spread)
 constexpr int kSkMaxSplits = 8;  // portable cluster size
-
-// Every thread of every CTA in the cluster (lanes may arrive diverged: the
-// producer and MMA lanes come from their own loops).
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
-}
-
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_saddr, uint32_t cta_rank) {
-  uint32_t remote;
-  float v;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_saddr), "r"(cta_rank));
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-  return v;
-}
 
 template <bool kAmn, bool kBmn>
 __global__ void __launch_bounds__(kSkThreads, 1)
@@ -726,427 +710,6 @@ __global__ void __launch_bounds__(kFThreads, 1)
   }
 }
 
-// ===========================================================================
-// GEMV for M <= 16 (decode-style small batches), HBM-bound.
-//
-// y[m][n] = sum_k x[m][k] * Ŵ[k][n] is evaluated with mma.sync m16n8k16 on a
-// 16-token tile, with the block scale folded into the activation:
-//   y[m][n] = sum_k bf16(x[m][k] * a'[k][n/64]) * bf16(C_{code(k,n)}).
-// The weight operand then needs no per-block table: a fixed 256-entry table of
-// bf16 pairs (C[hi nibble], C[lo nibble]) turns one byte into one B-fragment
-// register.  That byte is built from two adjacent weight rows (k, k+1) at the
-// same column by interleaving nibbles of their packed words, so each lookup
-// yields the (k, k+1) pair a B-fragment register holds.  The table lives in
-// shared memory as 32 copies, one per bank ((byte << 8) | lane*4 addresses a
-// lane's own copy), so lookups never conflict.  Columns are permuted inside a
-// 64-column block so that thread g's fragments cover its own packed word:
-// n-tile j, fragment column g is weight column 8g + j.
-//
-// Compared with the dequantized weight, bf16(C) * bf16(x a') differs from
-// x * bf16(C a') by at most a bf16 rounding of each factor (relative 2^-8 per
-// product); over K terms the relative error of y stays near 3e-3.
-//
-// CTA = 256 weight columns x a K-range, one CTA per SM.  A producer warp
-// streams 128-row stages (packed 128 x 128 bytes and X 16 x 128 bf16, both by
-// TMA with the 128-byte swizzle) through a 6-stage ring; sixteen compute warps
-// cover a stage as 4 column blocks of 64 x 4 row slots, each slot two 16-row
-// steps 64 rows apart, and the four partial sums per block are added through
-// shared memory into one fp32 partial per split.  Each lane keeps the scale
-// loads of the next four stages in flight (lanes 0-15 the first step's rows,
-// lanes 16-31 the second's), so their latency never reaches the decode.
-// The stages also carry an 8-column slice of A: column group cg owns rank
-// columns [8cg, 8cg+8), and the warps of the first column block add that
-// slice of X·A with one more mma per step, using the raw activation fragment;
-// gemv_finish_kernel turns these partials into Zc = bf16(c·X·A) and adds the
-// splits and Zc·B.  The decode table sits at the start of the dynamic shared
-// window, so its base is a constant of the load instruction.
-// ===========================================================================
-constexpr int kGvTable = 65536;        // 256 entries x 64 words (32 used) x 4 B
-constexpr int kGvRows = 128;           // k rows per stage
-constexpr int kGvStages = 6;
-constexpr int kGvPk = kGvRows * 128;   // packed weights of a stage
-constexpr int kGvXb = 2 * 2048;        // 16 tokens x 128 k bf16, two swizzled 64-k halves
-constexpr int kGvAb = kGvRows * 16;    // 128 k x 8 rank columns of A (bf16)
-constexpr int kGvCompute = 16;         // compute warps
-constexpr int kGvThreads = (kGvCompute + 1) * 32;
-constexpr int kGvAhead = 4;            // stages of scale loads in flight per lane
-constexpr size_t kGvSmem =
-    kGvTable + 1024 + kGvStages * (kGvPk + kGvXb + kGvAb) + 3 * 16 * 8 * 4 + 1024 + 256;
-static_assert(4 * 3 * 16 * 64 * 4 <= kGvStages * kGvPk, "block sums reuse the packed ring");
-
-struct GemvArgs {
-  int M, K, N, r;
-  int stages_per_split;   // 64-row stages per split
-  ScaleView sv;
-  float* partial;         // [splits][M][N]
-  float* zpart;           // [splits][M][r], or null when Zc is computed elsewhere
-  int32_t* d_status;
-};
-
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
-                                               uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t lds32(uint32_t saddr) {
-  uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(saddr));
-  return v;
-}
-
-__device__ __forceinline__ uint32_t lds16(uint32_t saddr) {
-  uint16_t v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(saddr));
-  return v;
-}
-
-// Scale a'[row][blk] for the GEMV in two halves: the raw loads (issued where
-// called, several stages ahead) and the decode once they are needed.
-struct GvScale {
-  uint32_t q;   // code8 (double quantization)
-  float v;      // s2 of the block's 256-group, or the fp32 absmax
-};
-
-__device__ __forceinline__ GvScale gemv_scale_load(const ScaleView& sv, int64_t b) {
-  GvScale r;
-  r.q = 0u;
-  if (sv.code8 == nullptr) {
-    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(r.v) : "l"(sv.absmax + b));
-  } else {
-    uint16_t q;
-    asm volatile("ld.global.nc.u8 %0, [%1];" : "=h"(q) : "l"(sv.code8 + b));
-    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(r.v) : "l"(sv.s2 + (b >> 8)));
-    r.q = q;
-  }
-  return r;
-}
-
-__device__ __forceinline__ float gemv_scale_value(const ScaleView& sv, const GvScale& r, float off,
-                                                  const float* t8) {
-  if (sv.code8 == nullptr) return r.v;
-  return __fadd_rn(__fmul_rn(t8[r.q], r.v), off);
-}
-
-template <int kOff>
-__device__ __forceinline__ uint32_t lds32_at(uint32_t saddr) {
-  uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1+%2];" : "=r"(v) : "r"(saddr), "n"(kOff));
-  return v;
-}
-
-template <bool kM16>
-__global__ void __launch_bounds__(kGvThreads, 1)
-    nf4_gemv_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmX,
-                    const __grid_constant__ CUtensorMap tmA, GemvArgs args) {
-  extern __shared__ uint8_t gsm_raw[];
-  uint32_t* table = reinterpret_cast<uint32_t*>(gsm_raw);
-  uint8_t* gsm = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(gsm_raw + kGvTable) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* sP = gsm;
-  uint8_t* sX = sP + kGvStages * kGvPk;
-  uint8_t* sAl = sX + kGvStages * kGvXb;
-  float* zred = reinterpret_cast<float*>(sAl + kGvStages * kGvAb);   // [3][16][8]
-  float* t8 = zred + 3 * 16 * 8;
-  uint64_t* full = reinterpret_cast<uint64_t*>(t8 + 256);
-  uint64_t* empty = full + kGvStages;
-  float* red = reinterpret_cast<float*>(sP);   // [4][3][16][64], after the last stage
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  pdl_launch_dependents();
-  if (threadIdx.x == kGvCompute * 32) {
-    for (int s = 0; s < kGvStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kGvCompute);
-    }
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  const int M = args.M, N = args.N, K = args.K;
-  const int cg = blockIdx.x;                            // 256-column group
-  const int st0 = blockIdx.y * args.stages_per_split;
-  const int nst = min((K + kGvRows - 1) / kGvRows, st0 + args.stages_per_split) - st0;
-  bool ok = true;
-
-  if (warp == kGvCompute) {
-    // --------------------------------- producer ---------------------------------
-    // starts streaming while the compute warps build their tables; rows past K
-    // (a last stage of 64 rows) arrive as zeros
-    if (lane == 0) {
-      pdl_wait();
-      tma_prefetch_desc(&tmP);
-      tma_prefetch_desc(&tmX);
-      tma_prefetch_desc(&tmA);
-      auto issue = [&](int j, int s) {
-        const int k0 = (st0 + j) * kGvRows;
-        mbar_arrive_expect_tx(&full[s], kGvPk + kGvXb + kGvAb);
-        tma_load_2d(sP + s * kGvPk, &tmP, &full[s], cg * 128, k0);
-        tma_load_2d(sX + s * kGvXb, &tmX, &full[s], k0, 0);
-        tma_load_2d(sX + s * kGvXb + 2048, &tmX, &full[s], k0 + 64, 0);
-        tma_load_2d(sAl + s * kGvAb, &tmA, &full[s], cg * 8, k0);
-      };
-      for (int j = 0; j < nst && j < kGvStages; ++j) issue(j, j);
-      for (int j = 0; j + kGvStages < nst && ok; ++j) {
-        const int s = j % kGvStages;
-        const uint32_t ph = (j / kGvStages) & 1;
-        if (!mbar_wait(&empty[s], ph)) { ok = false; break; }
-        issue(j + kGvStages, s);
-      }
-    }
-  } else {
-    // ------------------------------ compute warps ------------------------------
-    // fixed table: entry e -> (bf16(C[e >> 4]) | bf16(C[e & 15]) << 16), one
-    // copy per bank so that 32 lanes reading any entries never conflict
-    {
-      const float cv = kNF4g[16 * args.sv.codebook + (lane & 15)];
-      for (int e = warp; e < 256; e += kGvCompute)   // entry e is written by one warp
-        table[e * 64 + lane] =
-            pack_bf16x2(__shfl_sync(0xFFFFFFFFu, cv, e >> 4), __shfl_sync(0xFFFFFFFFu, cv, e & 15));
-    }
-    if (args.sv.code8 != nullptr) {
-      for (int u = threadIdx.x; u < 256; u += kGvCompute * 32) {
-        const float v = t8_magnitude(u & 127);
-        t8[u] = (u >> 7) ? -v : v;
-      }
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(kGvCompute * 32) : "memory");   // compute warps only
-    pdl_wait();
-
-    const int b = warp & 3, p = warp >> 2;             // column block, row slot
-    const int blk = cg * 4 + b;                        // 64-column block
-    const bool colok = blk * 64 < N;
-    const int g = lane >> 2, t = lane & 3;
-    const int bpr = N / 64;
-    const int kb = 16 * p;                             // rows kb.. and kb+64.. of a stage
-    const float off = args.sv.code8 != nullptr ? __ldg(args.sv.offset) : 0.0f;
-    const uint32_t tbase = smem_u32(gsm_raw);
-    const uint32_t laneword = lane * 4;
-    // Per-lane shared offsets, fixed for the whole loop.  Packed stage (128-byte
-    // swizzle, row R at R*128, 16-byte chunk c at (c ^ (R & 7))*16): this lane
-    // reads the 4 bytes of columns 8g..8g+7 of block b in rows kb+2t, kb+2t+1
-    // and the same rows +8, +64 and +72 (all with the same swizzle phase).
-    const uint32_t cw = static_cast<uint32_t>(2 * b + (g >> 2));
-    const uint32_t wo = static_cast<uint32_t>((g & 3) * 4);
-    const uint32_t r0 = static_cast<uint32_t>(kb + 2 * t);
-    const uint32_t poff0 = r0 * 128 + ((cw ^ (r0 & 7)) << 4) + wo;
-    const uint32_t poff1 = (r0 + 1) * 128 + ((cw ^ ((r0 + 1) & 7)) << 4) + wo;
-    // X stage (two halves of 16 tokens x 64 k, swizzled): token g,
-    // k = kb + 2t (+1) and kb + 8 + 2t (+1), the second step 2048 bytes on
-    const uint32_t c0 = static_cast<uint32_t>(kb >> 3);
-    const uint32_t xoff0 = g * 128 + ((c0 ^ static_cast<uint32_t>(g)) << 4) + t * 4;
-    const uint32_t xoff1 = g * 128 + (((c0 + 1) ^ static_cast<uint32_t>(g)) << 4) + t * 4;
-    const uint32_t aoff = static_cast<uint32_t>((kb + 2 * t) * 16 + g * 2);   // A slice
-    const uint32_t sP0 = smem_u32(sP), sX0 = smem_u32(sX), sA0 = smem_u32(sAl);
-
-    // acc[f]: mma f covers weight columns 8g+2f (rows g) and 8g+2f+1 (rows g+8)
-    // against tokens 2t, 2t+1 (acc2: tokens 8+2t, 9+2t)
-    float acc[4][4], acc2[4][4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[j][i] = acc2[j][i] = 0.0f;
-    float xa[4] = {0.0f, 0.0f, 0.0f, 0.0f};            // X·A slice (warps of block 0)
-    const bool do_xa = b == 0 && args.zpart != nullptr && cg * 8 < args.r;
-    // this lane's scale row inside a stage: kb + (lane & 15), second step for lanes 16-31
-    const int srow = kb + 64 * (lane >> 4) + (lane & 15);
-    auto scale_at = [&](int j) -> GvScale {
-      GvScale z;
-      z.q = 0u;
-      z.v = 0.0f;
-      const int row = (st0 + j) * kGvRows + srow;
-      if (colok && row < K) z = gemv_scale_load(args.sv, static_cast<int64_t>(row) * bpr + blk);
-      return z;
-    };
-    GvScale ring[kGvAhead];
-#pragma unroll
-    for (int u = 0; u < kGvAhead; ++u) {
-      ring[u].q = 0u;
-      ring[u].v = 0.0f;
-      if (u < nst) ring[u] = scale_at(u);
-    }
-
-    // one 16-row step h (0: rows kb.., 1: rows kb+64..) of stage slot s
-    auto step = [&](uint32_t ps, uint32_t xs, uint32_t as, float sc, int h) {
-      const uint32_t w0 = lds32(ps + poff0), w8 = lds32(ps + poff0 + 1024);
-      const uint32_t w1 = lds32(ps + poff1), w9 = lds32(ps + poff1 + 1024);
-      const uint32_t x0 = lds32(xs + xoff0), x1 = lds32(xs + xoff1);
-      const float s0 = __shfl_sync(0xFFFFFFFFu, sc, 16 * h + 2 * t);
-      const float s1 = __shfl_sync(0xFFFFFFFFu, sc, 16 * h + 2 * t + 1);
-      const float s2 = __shfl_sync(0xFFFFFFFFu, sc, 16 * h + 2 * t + 8);
-      const float s3 = __shfl_sync(0xFFFFFFFFu, sc, 16 * h + 2 * t + 9);
-      // B fragments: scaled activations of token g (and g + 8)
-      const uint32_t bx0 = pack_bf16x2(__uint_as_float(x0 << 16) * s0, __uint_as_float(x0 & 0xFFFF0000u) * s1);
-      const uint32_t bx1 = pack_bf16x2(__uint_as_float(x1 << 16) * s2, __uint_as_float(x1 & 0xFFFF0000u) * s3);
-      uint32_t y0 = 0u, y1 = 0u, by0 = 0u, by1 = 0u;
-      if (kM16) {
-        y0 = lds32(xs + xoff0 + 1024);
-        y1 = lds32(xs + xoff1 + 1024);
-        by0 = pack_bf16x2(__uint_as_float(y0 << 16) * s0, __uint_as_float(y0 & 0xFFFF0000u) * s1);
-        by1 = pack_bf16x2(__uint_as_float(y1 << 16) * s2, __uint_as_float(y1 & 0xFFFF0000u) * s3);
-      }
-      if (do_xa) {
-        // raw activations (tokens as rows) against A[k][8cg + g]
-        const uint32_t ab0 = lds16(as) | (lds16(as + 16) << 16);
-        const uint32_t ab1 = lds16(as + 128) | (lds16(as + 144) << 16);
-        const uint32_t araw[4] = {x0, y0, x1, y1};
-        mma_bf16_16816(xa, araw, ab0, ab1);
-      }
-      // bytes (row k nibble, row k+1 nibble) per column: even and odd columns
-      const uint32_t lo_e = (w0 & 0xF0F0F0F0u) | ((w1 >> 4) & 0x0F0F0F0Fu);
-      const uint32_t lo_o = ((w0 << 4) & 0xF0F0F0F0u) | (w1 & 0x0F0F0F0Fu);
-      const uint32_t hi_e = (w8 & 0xF0F0F0F0u) | ((w9 >> 4) & 0x0F0F0F0Fu);
-      const uint32_t hi_o = ((w8 << 4) & 0xF0F0F0F0u) | (w9 & 0x0F0F0F0Fu);
-#pragma unroll
-      for (int f = 0; f < 4; ++f) {
-        // offset (byte f << 8) | lane*4: output byte 0 <- lane*4 (source byte
-        // 4), byte 1 <- byte f of the word, bytes 2 and 3 <- zero (source byte 5)
-        const uint32_t sel = 0x5504u | (static_cast<uint32_t>(f) << 4);
-        uint32_t wa[4];
-        wa[0] = lds32(tbase + prmt(lo_e, laneword, sel));   // column 8g+2f, k 2t..
-        wa[1] = lds32(tbase + prmt(lo_o, laneword, sel));   // column 8g+2f+1
-        wa[2] = lds32(tbase + prmt(hi_e, laneword, sel));   // column 8g+2f, k 2t+8..
-        wa[3] = lds32(tbase + prmt(hi_o, laneword, sel));
-        mma_bf16_16816(acc[f], wa, bx0, bx1);
-        if (kM16) mma_bf16_16816(acc2[f], wa, by0, by1);
-      }
-    };
-
-    for (int j0 = 0; j0 < nst && ok; j0 += kGvAhead) {
-#pragma unroll
-      for (int u = 0; u < kGvAhead; ++u) {
-        const int j = j0 + u;
-        if (j >= nst || !ok) break;
-        const int s = j % kGvStages;
-        const uint32_t ph = (j / kGvStages) & 1;
-        const float sc = gemv_scale_value(args.sv, ring[u], off, t8);
-        if (j + kGvAhead < nst) ring[u] = scale_at(j + kGvAhead);
-        if (!mbar_wait(&full[s], ph)) { ok = false; break; }
-        if (colok) {
-          const uint32_t ps = sP0 + s * kGvPk, xs = sX0 + s * kGvXb, as = sA0 + s * kGvAb + aoff;
-          step(ps, xs, as, sc, 0);
-          step(ps + 64 * 128, xs + 2048, as + 64 * 16, sc, 1);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-      }
-    }
-    // every compute warp is past its last stage (and so every stage has
-    // landed) before the block sums overwrite the packed ring
-    asm volatile("bar.sync 1, %0;" ::"n"(kGvCompute * 32) : "memory");
-    // add the four row-slot warps of each block, then write this split's partial
-    // red[b][p-1][token][64 columns]
-    auto put = [&](float* dst, const float (&v)[4][4], int tok0) {
-#pragma unroll
-      for (int f = 0; f < 4; ++f) {
-        const int ce = 8 * g + 2 * f;
-        dst[(tok0 + 2 * t) * 64 + ce] = v[f][0];
-        dst[(tok0 + 2 * t + 1) * 64 + ce] = v[f][1];
-        dst[(tok0 + 2 * t) * 64 + ce + 1] = v[f][2];
-        dst[(tok0 + 2 * t + 1) * 64 + ce + 1] = v[f][3];
-      }
-    };
-    if (p > 0) {
-      float* myred = red + (b * 3 + p - 1) * (16 * 64);
-      put(myred, acc, 0);
-      if (kM16) put(myred, acc2, 8);
-      if (do_xa) {
-        float* zr = zred + (p - 1) * 128;
-        zr[g * 8 + 2 * t] = xa[0];
-        zr[g * 8 + 2 * t + 1] = xa[1];
-        zr[(g + 8) * 8 + 2 * t] = xa[2];
-        zr[(g + 8) * 8 + 2 * t + 1] = xa[3];
-      }
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(kGvCompute * 32) : "memory");   // compute warps only
-    if (do_xa && p == 0) {
-      float* zo = args.zpart + static_cast<int64_t>(blockIdx.y) * M * args.r + cg * 8;
-      const int q0 = 2 * t, q1 = 2 * t + 1;
-      auto zsum = [&](float v, int row, int col) {
-        return v + zred[row * 8 + col] + zred[128 + row * 8 + col] + zred[256 + row * 8 + col];
-      };
-      if (g < M) {
-        if (cg * 8 + q0 < args.r) zo[g * args.r + q0] = zsum(xa[0], g, q0);
-        if (cg * 8 + q1 < args.r) zo[g * args.r + q1] = zsum(xa[1], g, q1);
-      }
-      if (g + 8 < M) {
-        if (cg * 8 + q0 < args.r) zo[(g + 8) * args.r + q0] = zsum(xa[2], g + 8, q0);
-        if (cg * 8 + q1 < args.r) zo[(g + 8) * args.r + q1] = zsum(xa[3], g + 8, q1);
-      }
-    }
-    if (p == 0 && colok) {
-      const float* r1 = red + (b * 3) * (16 * 64);
-      float* out = args.partial + static_cast<int64_t>(blockIdx.y) * M * N + blk * 64;
-      auto emit = [&](const float (&v)[4][4], int tok0) {
-#pragma unroll
-        for (int f = 0; f < 4; ++f) {
-          const int ce = 8 * g + 2 * f;
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const int tok = tok0 + 2 * t + (h & 1), col = ce + (h >> 1);
-            const int idx = tok * 64 + col;
-            if (tok < M)
-              out[static_cast<int64_t>(tok) * N + col] = v[f][h] + r1[idx] + r1[1024 + idx] + r1[2048 + idx];
-          }
-        }
-      };
-      emit(acc, 0);
-      if (kM16) emit(acc2, 8);
-    }
-  }
-  if (!ok && lane == 0) raise_status(args.d_status, QLORA_ERR_TIMEOUT);
-}
-
-// Zc = bf16(c * sum_s zpart[s]) (M x r, written by CTA 0; or read when zpart
-// is null), then per column n:
-// Y[m][n] = bf16( sum_s partial[s][m][n] + sum_j Zc[m][j] * B[j][n] ).
-__global__ void __launch_bounds__(128) gemv_finish_kernel(const float* __restrict__ partial,
-                                                          int splits, int M, int N,
-                                                          const float* __restrict__ zpart, int r,
-                                                          float c, const uint16_t* __restrict__ B,
-                                                          uint16_t* __restrict__ Zc,
-                                                          uint16_t* __restrict__ Y) {
-  // blockIdx.y = token m; this CTA needs row m of Zc only
-  __shared__ float zs[64];
-  pdl_launch_dependents();
-  pdl_wait();
-  const int m = blockIdx.y;
-  for (int j = threadIdx.x; j < r; j += blockDim.x) {
-    const int i = m * r + j;
-    if (zpart != nullptr) {
-      float acc = 0.0f;
-#pragma unroll 4
-      for (int s = 0; s < splits; ++s) acc += zpart[static_cast<int64_t>(s) * M * r + i];
-      const uint32_t zb = pack_bf16x2(c * acc, 0.0f) & 0xFFFFu;
-      zs[j] = bf16_bits_to_f32(zb);
-      if (blockIdx.x == 0) Zc[i] = static_cast<uint16_t>(zb);
-    } else {
-      zs[j] = bf16_bits_to_f32(Zc[i]);   // computed by the rank-r kernel
-    }
-  }
-  __syncthreads();
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= N) return;
-  float acc = 0.0f;
-#pragma unroll 4
-  for (int s = 0; s < splits; ++s) acc += partial[(static_cast<int64_t>(s) * M + m) * N + n];
-  // eight independent loads of B per round (rows past r read as zero)
-  float lora = 0.0f;
-  for (int j0 = 0; j0 < r; j0 += 8) {
-    float bv[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u)
-      bv[u] = j0 + u < r ? bf16_bits_to_f32(__ldg(B + static_cast<int64_t>(j0 + u) * N + n)) : 0.0f;
-#pragma unroll
-    for (int u = 0; u < 8; ++u)
-      if (j0 + u < r) lora = fmaf(zs[j0 + u], bv[u], lora);
-  }
-  Y[static_cast<int64_t>(m) * N + n] = static_cast<uint16_t>(pack_bf16x2(acc + lora, 0.0f) & 0xFFFFu);
-}
-
 // Zero-padded copy of a rows x r bf16 matrix into rows x rp (rp = r rounded
 // up to a multiple of 8), so that every row starts on a 16-byte boundary as
 // the tensor maps need.  Only used when r is not a multiple of 8.
@@ -1270,19 +833,6 @@ cudaError_t launch_pad(const uint16_t* src, int64_t rows, int r, uint16_t* dst, 
   return cudaGetLastError();
 }
 
-// GEMV split: one CTA per SM over (256-column groups) x (K splits).
-void gemv_plan(int64_t K, int64_t N, int num_sms, int* splits, int* stages_per_split) {
-  const int ncg = static_cast<int>((N + 255) / 256);
-  const int nstages = static_cast<int>((K + kGvRows - 1) / kGvRows);
-  int s = num_sms / ncg;
-  if (s < 1) s = 1;
-  if (s > nstages) s = nstages;
-  const int per = (nstages + s - 1) / s;
-  *stages_per_split = per;
-  *splits = (nstages + per - 1) / per;
-}
-
-
 }  // namespace
 
 static int g_ws_sms = 148;  // sizing assumption for workspace queries (B200)
@@ -1331,11 +881,7 @@ size_t linear_fwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) {
     // for the fused kernel's TMA when r is not a multiple of 8
     return rp != r ? apad + align256(static_cast<size_t>(M) * rp * 2) : 0;
   }
-  // GEMV partials and its per-split X·A slices
-  int S = 1, per = 1;
-  gemv_plan(K, N, g_ws_sms, &S, &per);
-  return align256(static_cast<size_t>(S) * M * N * 4) + align256(static_cast<size_t>(S) * M * r * 4) +
-         apad;
+  return apad;   // the GEMV adds its K splits inside a thread-block cluster
 }
 
 size_t linear_bwd_workspace_bytes(int64_t M, int64_t K, int64_t N, int r) {
@@ -1351,19 +897,10 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
                               const uint8_t* packed, ScaleView sv, const uint16_t* A,
                               const uint16_t* B, float c, uint16_t* Y, uint16_t* Zc, void* ws,
                               size_t ws_bytes, int32_t* d_status, cudaStream_t st, int num_sms) {
-  (void)num_sms;
   WsCursor cur{static_cast<char*>(ws), ws_bytes};
   const int rp = padded_rank(r);
   const bool pad = rp != r;
   cudaError_t e = cudaSuccess;
-  float* pg = nullptr;
-  float* pz = nullptr;
-  int S = 1, per = 1;
-  if (M <= 16) {
-    gemv_plan(K, N, g_ws_sms, &S, &per);
-    pg = static_cast<float*>(cur.take(static_cast<size_t>(S) * M * N * 4));
-    pz = static_cast<float*>(cur.take(static_cast<size_t>(S) * M * r * 4));
-  }
   // A zero-padded to rp columns (16-byte row pitch for TMA) when r % 8 != 0
   const uint16_t* At = A;
   if (pad) {
@@ -1379,61 +916,10 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
   if (!make_tmap_2d(&tX, X, kBF16, 2, M, K, K, 64, 128, kSW128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tAl, At, kBF16, 2, K, rp, rp, 64, 64, kSW128)) return cudaErrorInvalidValue;
   if (M <= 16) {
-    const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
-    const int ncg = static_cast<int>((N + 255) / 256);
-    // Zc by the rank-r kernel, exactly as the backward recomputes it when the
-    // caller keeps no Zc (same kernel, same splits: the same bits)
-    const bool xa_in_gemv = false;
-    if (!xa_in_gemv) {
-      e = run_skinny<false, true>(tX, tAl, static_cast<int>(M), static_cast<int>(K), r, c, 0, Zc, r,
-                                  Sz, d_status, st);
-      if (e != cudaSuccess) return e;
-    }
-    static DeviceOnce gemv_once;
-    e = gemv_once.run([](int) {
-      cudaError_t r = cudaFuncSetAttribute(nf4_gemv_kernel<false>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(kGvSmem));
-      if (r == cudaSuccess)
-        r = cudaFuncSetAttribute(nf4_gemv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kGvSmem));
-      return r;
-    });
-    if (e != cudaSuccess) return e;
-    CUtensorMap tP, tXg, tAg;
-    if (!make_tmap_2d(&tP, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N / 2, N / 2, 128, kGvRows, kSW128))
-      return cudaErrorInvalidValue;
-    if (!make_tmap_2d(&tXg, X, kBF16, 2, M, K, K, 64, 16, kSW128)) return cudaErrorInvalidValue;
-    if (!make_tmap_2d(&tAg, At, kBF16, 2, K, rp, rp, 8, kGvRows, CU_TENSOR_MAP_SWIZZLE_NONE))
-      return cudaErrorInvalidValue;
-    GemvArgs ga;
-    ga.M = static_cast<int>(M);
-    ga.K = static_cast<int>(K);
-    ga.N = static_cast<int>(N);
-    ga.r = r;
-    ga.stages_per_split = per;
-    ga.sv = sv;
-    ga.partial = pg;
-    ga.zpart = xa_in_gemv ? pz : nullptr;
-    ga.d_status = d_status;
-    dim3 grid(static_cast<unsigned>(ncg), static_cast<unsigned>(S));
-    {
-      ProfScope prof(kProfGemv, st);
-      if (M <= 8)
-        e = launch_pdl(nf4_gemv_kernel<false>, grid, dim3(kGvThreads), kGvSmem, st, 1, tP, tXg, tAg, ga);
-      else
-        e = launch_pdl(nf4_gemv_kernel<true>, grid, dim3(kGvThreads), kGvSmem, st, 1, tP, tXg, tAg, ga);
-    }
-    if (e != cudaSuccess) return e;
-    {
-      ProfScope prof(kProfOther, st);
-      dim3 fgrid(static_cast<unsigned>((N + 127) / 128), static_cast<unsigned>(M));
-      e = launch_pdl(gemv_finish_kernel, fgrid, dim3(128), 0, st, 1, static_cast<const float*>(pg), S,
-                     static_cast<int>(M), static_cast<int>(N),
-                     static_cast<const float*>(xa_in_gemv ? pz : nullptr), r, c, B, Zc, Y);
-    }
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
+    // one launch: weights streamed once, X·A and its split sums in the same
+    // cluster, Zc and Y written (the GEMV's own SM count fixes its splits)
+    return launch_gemv(M, K, N, r, X, packed, sv, At, rp, B, c, Y, Zc, r, false, d_status, st,
+                       num_sms);
   }
 
   // rank-r product for the tensor-core path: Zc = bf16(c * X A), and a copy
@@ -1484,7 +970,6 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
                               ScaleView sv, const uint16_t* A, const uint16_t* B, float c,
                               uint16_t* dX, float* dA, float* dB, void* ws, size_t ws_bytes,
                               int32_t* d_status, cudaStream_t st, int num_sms) {
-  (void)num_sms;
   WsCursor cur{static_cast<char*>(ws), ws_bytes};
   const int rp = padded_rank(r);
   const bool pad = rp != r;
@@ -1504,7 +989,14 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
     if (e != cudaSuccess) return e;
     At = Ap;
   }
-  if (Zc == nullptr) {
+  if (Zc == nullptr && M <= 16) {
+    // saved-activation policy "recompute": Zc = bf16(c X A) exactly as the
+    // forward forms it for M <= 16 (the GEMV kernel, its splits and sums)
+    e = launch_gemv(M, K, N, r, X, packed, sv, At, rp, B, c, nullptr, Zc_ws, rp, true, d_status, st,
+                    num_sms);
+    if (e != cudaSuccess) return e;
+    Zc = Zc_ws;
+  } else if (Zc == nullptr) {
     // saved-activation policy "recompute": Zc = bf16(c X A) exactly as the
     // forward forms it (same kernel, same splits, so the same bits)
     CUtensorMap tXf, tAf;

@@ -205,7 +205,7 @@ qlora_status qlora_nf4_dequantize(const qlora_nf4_state* st, uint16_t* W_hat,
  * that every row the tensor maps read starts on a 16-byte boundary; the padded
  * rank columns are zero and change no result.
  * ws: at least qlora_linear_fwd_workspace_size(M, K, N, r) bytes; that size is
- * 0 for M > 16 when r % 8 == 0 (the rank-r kernel adds its K splits inside a
+ * 0 when r % 8 == 0 (every kernel of the forward adds its K splits inside a
  * thread-block cluster), and ws may then be null.
  */
 size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t K, int64_t N, int32_t r);

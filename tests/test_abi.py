@@ -60,9 +60,11 @@ def test_workspace_sizes(L):
     lib = L.lib
     assert lib.qlora_nf4_quantize_workspace_size(1000, 0) == 0
     assert lib.qlora_nf4_quantize_workspace_size(64 * 100, 1) >= 2048 + 4 * 100
-    # the tensor-core path needs no forward workspace; the GEMV keeps split sums
+    # neither forward path needs a workspace when r % 8 == 0: both add their K
+    # splits inside a thread-block cluster
     assert lib.qlora_linear_fwd_workspace_size(4096, 4096, 4096, 16) == 0
-    assert lib.qlora_linear_fwd_workspace_size(4, 4096, 4096, 16) > 0
+    assert lib.qlora_linear_fwd_workspace_size(4, 4096, 4096, 16) == 0
+    assert lib.qlora_linear_fwd_workspace_size(4, 4096, 4096, 12) >= 4096 * 16 * 2
     # backward: dZ (M x r bf16)
     assert lib.qlora_linear_bwd_workspace_size(4096, 4096, 4096, 16) >= 4096 * 16 * 2
     # unsupported shapes report 0
@@ -115,7 +117,8 @@ def test_host_validation_rejects_before_device_work(L):
     args_nan = [fake, C.byref(w), fake, fake, float("nan"), fake, fake, fake, 1 << 20, None, None]
     assert lib.qlora_linear_fwd(8, 64, 64, 16, *args_nan) == E.QLORA_ERR_INVALID_ARG
     args_small_ws = [fake, C.byref(w), fake, fake, 1.0, fake, fake, fake, 16, None, None]
-    assert lib.qlora_linear_fwd(8, 64, 64, 16, *args_small_ws) == E.QLORA_ERR_INVALID_ARG
+    # a rank that needs a padded copy of A in the workspace
+    assert lib.qlora_linear_fwd(8, 64, 64, 12, *args_small_ws) == E.QLORA_ERR_INVALID_ARG
     bargs = [fake, fake, fake, C.byref(w), fake, fake, 1.0, fake, fake, None, None, 0, None, None]
     assert lib.qlora_linear_bwd(8, 64, 64, 16, *bargs) == E.QLORA_ERR_INVALID_ARG  # null dB
     assert lib.qlora_status_sync(None, None, None) == E.QLORA_ERR_INVALID_ARG
@@ -151,16 +154,12 @@ def test_workspace_cache_is_per_stream_and_bounded(L, monkeypatch):
     import bit_nf4_quantized_pack_b200 as q
 
     class FakeStream:
-        def __init__(self, h, capturing=False):
+        def __init__(self, h):
             self.cuda_stream = h
-            self._capturing = capturing
-
-        def is_capturing(self):
-            return self._capturing
 
     cur = {"h": 1, "cap": False}
-    monkeypatch.setattr(torch.cuda, "current_stream",
-                        lambda device=None: FakeStream(cur["h"], cur["cap"]))
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda device=None: FakeStream(cur["h"]))
+    monkeypatch.setattr(torch.cuda, "is_current_stream_capturing", lambda: cur["cap"])
     cache = q._WorkspaceCache(limit=3)
     a = cache.get(("b", "cpu"), 1000, "cpu")
     assert a is cache.get(("b", "cpu"), 900, "cpu")          # reused on the same stream

@@ -63,7 +63,8 @@ def test_config4_decoder_layer_linear(i):
     name, K, N = S.LAYER7B[i]
     lin = S.make_linear(4, i, name, 4096, K, N, 0.02, wl.r, outlier_frac=0.001,
                         outlier_value=0.2)
-    assert np.count_nonzero(np.abs(lin.W) == np.float32(0.2)) > 0.0005 * K * N
+    # the outliers (+-0.2 before the bf16 rounding, 10 sigma) are all there
+    assert 0.0009 * K * N < np.count_nonzero(np.abs(lin.W) > 0.15) < 0.0011 * K * N
     ow = OracleWeight(lin.W, True)
     wq = q.quantize(to_dev(lin.W), double_quant=True)
     assert_state_equal(wq, ow)
