@@ -48,7 +48,6 @@ namespace qnf4 {
 namespace {
 
 __constant__ float kCodeVals[32] = {QNF4_TABLE_VALUES, QNF4_INT4_VALUES};   // NF4, INT4
-__constant__ T8Table kT8 = make_t8_table();
 
 constexpr int kGvTable = 65536;          // 256 entries x 64 words (32 used) x 4 B
 constexpr int kGvRows = 128;             // k rows per stage
@@ -171,7 +170,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       table[e * 64 + lane] =
           pack_bf16x2(__shfl_sync(0xFFFFFFFFu, cv, e >> 4), __shfl_sync(0xFFFFFFFFu, cv, e & 15));
   }
-  for (int u = threadIdx.x; u < 256; u += blockDim.x) t8[u] = kT8.v[u];
+  for (int u = threadIdx.x; u < 256; u += blockDim.x) t8[u] = kT8Table.v[u];
   __syncthreads();
 
   const int M = args.M, N = args.N, K = args.K;

@@ -39,28 +39,13 @@ class DeviceOnce {
   std::atomic<bool> done_[kMaxDevices] = {};
 };
 
-// The signed dynamic 8-bit codebook T8 of the scale codes (this library's own
-// definition; the page only requires "a signed dynamic 8-bit codebook, not
-// FP8 E4M3"): byte u, sign u >> 7, t = u & 127; t = 0 is 0; otherwise
-// f = floor(log2 t), e = 6 - f, m = t - 2^f and |v| = (2^f + 9(m+1)) /
-// (10^(e+1) 2^f), a correctly rounded double division rounded to fp32.
-__device__ __forceinline__ float t8_magnitude(int t) {
-  if (t == 0) return 0.0f;
-  const int f = 31 - __clz(t);
-  const int e = 6 - f;
-  const int m = t - (1 << f);
-  double p10 = 10.0;
-  for (int i = 0; i < e; ++i) p10 *= 10.0;
-  const double num = static_cast<double>((1 << f) + 9 * (m + 1));
-  const double den = p10 * static_cast<double>(1 << f);
-  return __double2float_rn(__ddiv_rn(num, den));
-}
+// The scale codebook T8 (see make_t8_table in common.cuh), one copy per
+// translation unit in constant memory; build_t8 stages it in shared memory,
+// where a warp's lookups of different codes do not serialize.
+static __constant__ T8Table kT8Table = make_t8_table();
 
 __device__ __forceinline__ void build_t8(float* t8 /*256*/) {
-  for (int u = threadIdx.x; u < 256; u += blockDim.x) {
-    const float v = t8_magnitude(u & 127);
-    t8[u] = (u >> 7) ? -v : v;
-  }
+  for (int u = threadIdx.x; u < 256; u += blockDim.x) t8[u] = kT8Table.v[u];
 }
 
 // Launch with programmatic stream serialization (and, when cluster_y > 1, a
@@ -93,7 +78,11 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // selftest.cu — a wait that nothing completes, bounded by limit_ns
 cudaError_t launch_bounded_wait_selftest(int32_t* d_status, uint64_t limit_ns, cudaStream_t st);
 
-// quantize.cu
+// quantize.cu.  With double quantization the workspace holds, from its
+// start: 256 exponent bins of the scales (2 KB), the counter of finished
+// encoder CTAs, then (at kQuantizeWsHead) one fp32 scale per 64-block; the
+// first kQuantizeWsHead bytes are cleared by every call.
+constexpr size_t kQuantizeWsHead = 2304;
 cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* packed,
                             float* absmax_out, bool dq, uint8_t* code8, float* s2, float* offset,
                             void* ws, int32_t* d_status, cudaStream_t st, int num_sms,

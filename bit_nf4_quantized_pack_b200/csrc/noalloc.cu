@@ -9,8 +9,8 @@
 // host framework and have no allocator of their own.  This entry point needs
 // nothing from them but the inputs and outputs.
 //
-// The scratch (2 KB of exponent bins for the exact mean, plus one fp32 scale
-// per 64-block) lives in this file's module, so it is allocated only once that
+// The scratch (2 KB of exponent bins for the exact mean and a counter, 2304
+// bytes in all, plus one fp32 scale per 64-block) lives in this file's module, so it is allocated only once that
 // module is loaded, and every GPU that loads it keeps it until the process
 // exits.  Its device address is looked up once per device, on the first call
 // made with that device current.
@@ -26,7 +26,7 @@
 namespace {
 
 constexpr int64_t kNoAllocMaxBlocks = QLORA_NOALLOC_MAX_NUMEL / 64;
-constexpr size_t kNoAllocScratchBytes = 2048 + static_cast<size_t>(kNoAllocMaxBlocks) * 4;
+constexpr size_t kNoAllocScratchBytes = qnf4::kQuantizeWsHead + static_cast<size_t>(kNoAllocMaxBlocks) * 4;
 
 __device__ __align__(256) unsigned char g_quantize_scratch[kNoAllocScratchBytes];
 
@@ -86,7 +86,7 @@ extern "C" qlora_status qlora_nf4_quantize_noalloc(const void* W, qlora_dtype dt
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return QLORA_ERR_CUDA;
-  // the exponent bins at the start of the scratch are cleared by the launcher
+  // the bins and the counter at the start of the scratch are cleared by the launcher
   cudaError_t e = qnf4::launch_quantize(W, dtype, st->numel, st->packed, st->absmax,
                                         st->double_quant != 0, st->code8, st->s2, st->offset,
                                         scratch, d_status,

@@ -22,21 +22,25 @@ __constant__ float kNF4c[16] = {QNF4_TABLE_VALUES};
 // looks t up in 33 uniform buckets of width 1/16 that are offset by half a
 // bucket; every bucket holds at most one midpoint and no midpoint lies within
 // 0.004 of a bucket edge, so a bucket gives (number of midpoints below it,
-// the midpoint inside it).  Only when t is within 2^-20 of that midpoint is
-// the comparison redone exactly: w > s*m_j in fp64, where s*m_j is exact
-// (24-bit times at most 26-bit significand).  An exact tie (w == s*m_j) is
-// not "greater", so it keeps the smaller index.
+// the midpoint inside it).  A bucket's entry is one 32-bit word: the fp32
+// midpoint (4.0 when the bucket holds none) with its low five mantissa bits
+// replaced by (number of midpoints below the bucket) + 1.  That moves the
+// midpoint by under 32 ulp, i.e. under 2^-19 since |m| < 1; with the 2^-21
+// error of t the computed t - m is within E < 2^-18 of the exact one, so its
+// sign can be wrong only when |t - m| < 2E < 2^-17.  Every element within
+// 2^-17 of the stored midpoint (exact ties included) is therefore redone
+// exactly: w > s*m_j in fp64, where s*m_j is exact (24-bit times at most
+// 26-bit significand).  An exact tie (w == s*m_j) is not "greater", so it
+// keeps the smaller index.  Each lane reads its own copy of the 33 words
+// (bucket b of lane l at word 32b + l), so the lookups of a warp never
+// conflict.
 // ---------------------------------------------------------------------------
-struct Bucket {
-  float mid;  // the midpoint inside this bucket, or 4.0 (none)
-  int jlo;    // number of midpoints below the bucket = code left of `mid`
-};
-
 constexpr int kBuckets = 33;
-constexpr float kNearEps = 9.5367431640625e-07f;  // 2^-20
+constexpr float kNearEps = 7.62939453125e-06f;   // 2^-17
 
-__device__ __forceinline__ void build_buckets(Bucket* tab, double* mexact) {
-  for (int b = threadIdx.x; b < kBuckets; b += blockDim.x) {
+__device__ __forceinline__ void build_buckets(uint32_t* tab /*[33][32]*/, double* mexact) {
+  for (int i = threadIdx.x; i < kBuckets * 32; i += blockDim.x) {
+    const int b = i >> 5;
     const double lo = (b - 16.5) / 16.0, hi = (b - 15.5) / 16.0;
     int jlo = 0;
     float mid = 4.0f;
@@ -47,8 +51,7 @@ __device__ __forceinline__ void build_buckets(Bucket* tab, double* mexact) {
       else if (mj < hi)
         mid = static_cast<float>(mj);
     }
-    tab[b].mid = mid;
-    tab[b].jlo = jlo;
+    tab[i] = (__float_as_uint(mid) & ~31u) | static_cast<uint32_t>(jlo + 1);
   }
   for (int j = threadIdx.x; j < 15; j += blockDim.x)
     mexact[j] = 0.5 * (static_cast<double>(kNF4c[j]) + static_cast<double>(kNF4c[j + 1]));
@@ -144,7 +147,7 @@ struct BinCache {
 template <bool kDQ>
 __device__ __forceinline__ void encode16(float (&x)[kLaneElems], int64_t blk, int64_t e0, int sub,
                                          unsigned gmask, int64_t numel, bool full,
-                                         const Bucket* tab, const double* mexact,
+                                         const uint32_t* tab, const double* mexact,
                                          uint8_t* __restrict__ packed, float* __restrict__ scales,
                                          BinCache& bc, unsigned long long* sbins, bool& bad) {
   float am = 0.0f;
@@ -168,10 +171,11 @@ __device__ __forceinline__ void encode16(float (&x)[kLaneElems], int64_t blk, in
       for (int i = 0; i < kLaneElems; ++i) x[i] *= sc;
       s_eff = s * sc;
     }
-    // relative error of t below 2^-21: inside the 2^-20 window of the exact check
+    // relative error of t below 2^-21 (inside the exact check's window, above)
     float inv_s;
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv_s) : "f"(s_eff));
-    const uint32_t tb = smem_u32(tab) - 0x4B000000u * 8u;   // (bits of 2^23 + b) * 8 + tb = &tab[b]
+    // (bits of 2^23 + b) * 128 + tb = this lane's word of bucket b
+    const uint32_t tb = smem_u32(tab) + (threadIdx.x & 31u) * 4u - 0x4B000000u * 128u;
     float dmin = 1.0f;
     w0 = 0;
     w1 = 0;
@@ -179,11 +183,11 @@ __device__ __forceinline__ void encode16(float (&x)[kLaneElems], int64_t blk, in
     for (int i = 0; i < kLaneElems; ++i) {
       const float t = x[i] * inv_s;
       const float y = fmaf(t, 16.0f, 8388624.0f);             // 2^23 + 16 + 16 t, rounded to an integer
-      float mid;
-      int jlo;
-      asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=f"(mid), "=r"(jlo) : "r"(tb + __float_as_uint(y) * 8u));
-      const float d = t - mid;
-      const uint32_t code = static_cast<uint32_t>(jlo + 1 + (__float_as_int(d) >> 31));
+      uint32_t ent;
+      asm("ld.shared.b32 %0, [%1];" : "=r"(ent) : "r"(tb + __float_as_uint(y) * 128u));
+      const float d = t - __uint_as_float(ent);
+      // codes below the bucket + 1, minus one when t is below the midpoint
+      const uint32_t code = (ent & 31u) - (__float_as_uint(d) >> 31);
       dmin = fminf(dmin, fabsf(d));
       const int sh = (i & 7) >> 1;
       if (i < 8)
@@ -198,10 +202,11 @@ __device__ __forceinline__ void encode16(float (&x)[kLaneElems], int64_t blk, in
       for (int i = 0; i < kLaneElems; ++i) {
         const float t = x[i] * inv_s;
         const int b = __float2int_rd(fmaf(t, 16.0f, 16.5f));
-        const Bucket e = tab[b < 0 ? 0 : (b > kBuckets - 1 ? kBuckets - 1 : b)];
-        const float d = t - e.mid;
-        uint32_t code = static_cast<uint32_t>(e.jlo) + (d > 0.0f ? 1u : 0u);
-        if (fabsf(d) < kNearEps) code = exact_code(x[i], s_eff, e.jlo, mexact);
+        const uint32_t ent = tab[32 * (b < 0 ? 0 : (b > kBuckets - 1 ? kBuckets - 1 : b))];
+        const int jlo = static_cast<int>(ent & 31u) - 1;
+        const float d = t - __uint_as_float(ent);
+        uint32_t code = static_cast<uint32_t>(jlo) + (d > 0.0f ? 1u : 0u);
+        if (fabsf(d) < kNearEps) code = exact_code(x[i], s_eff, jlo, mexact);
         const int sh = (i & 7) >> 1;
         if (i < 8)
           w0 += code << (sh * 8 + ((i & 1) ? 0 : 4));
@@ -231,120 +236,6 @@ __device__ __forceinline__ void encode16(float (&x)[kLaneElems], int64_t blk, in
   if (sub == 0) {
     scales[blk] = s;
     if (kDQ) bc.add(s, sbins);
-  }
-}
-
-constexpr int kChunkBlocks = 64;                 // 64-blocks per streamed chunk
-constexpr int kChunkElems = kChunkBlocks * kBlock;
-constexpr int kEncStages = 4;
-
-template <typename T>
-constexpr size_t encode_smem_bytes() {
-  return static_cast<size_t>(kEncStages) * kChunkElems * sizeof(T) + 128;
-}
-
-// CTA = 256 threads = 64 groups of 4 lanes = one chunk of 64 blocks per
-// iteration.  Whole chunks stream into a 4-stage shared-memory ring by 1-D
-// bulk copies; the remaining blocks (a partial last chunk, or everything when
-// W is not 16-byte aligned) are read directly from global memory.
-template <typename T, bool kDQ>
-__global__ void __launch_bounds__(256) nf4_encode_kernel(const T* __restrict__ W, int64_t numel,
-                                                         int64_t n1, uint8_t* __restrict__ packed,
-                                                         float* __restrict__ scales,
-                                                         unsigned long long* __restrict__ bins,
-                                                         int32_t* d_status) {
-  extern __shared__ uint8_t esm_raw[];
-  T* ring = reinterpret_cast<T*>((reinterpret_cast<uintptr_t>(esm_raw) + 127) &
-                                 ~static_cast<uintptr_t>(127));
-  __shared__ Bucket tab[kBuckets];
-  __shared__ double mexact[15];
-  __shared__ unsigned long long sbins[kDQ ? 256 : 1];
-  __shared__ uint64_t full_bar[kEncStages];
-  pdl_launch_dependents();
-  pdl_wait();
-  __shared__ int abort_flag;
-  build_buckets(tab, mexact);
-  if (kDQ)
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = 0ull;
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kEncStages; ++i) mbar_init(&full_bar[i], 1);
-    abort_flag = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  const int lane = threadIdx.x & 31;
-  const int sub = lane & 3;
-  const unsigned gmask = 0xFu << (lane & 28);
-  const bool aligned16 = (reinterpret_cast<uintptr_t>(W) & 15u) == 0;
-  const int64_t nchunks = aligned16 ? numel / kChunkElems : 0;
-  const int64_t my_n =
-      nchunks > blockIdx.x ? (nchunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  constexpr uint32_t kChunkBytes = kChunkElems * sizeof(T);
-  BinCache bc;
-  bool bad = false;
-
-  if (threadIdx.x == 0) {
-    for (int64_t j = 0; j < my_n && j < kEncStages; ++j) {
-      const int64_t c = blockIdx.x + j * gridDim.x;
-      mbar_arrive_expect_tx(&full_bar[j], kChunkBytes);
-      bulk_load_1d(ring + j * kChunkElems, W + c * kChunkElems, kChunkBytes, &full_bar[j]);
-    }
-  }
-  for (int64_t j = 0; j < my_n; ++j) {
-    const int s = static_cast<int>(j % kEncStages);
-    const uint32_t ph = static_cast<uint32_t>((j / kEncStages) & 1);
-    if (!mbar_wait(&full_bar[s], ph)) abort_flag = 1;
-    __syncthreads();
-    if (abort_flag) break;
-    const int64_t c = blockIdx.x + j * gridDim.x;
-    const int local = threadIdx.x >> 2;
-    const int64_t blk = c * kChunkBlocks + local;
-    const int64_t e0 = blk * kBlock + sub * kLaneElems;
-    const T* src = ring + s * kChunkElems + local * kBlock + sub * kLaneElems;
-    float x[kLaneElems];
-    if (sizeof(T) == 2) {
-      const uint4 v0 = *reinterpret_cast<const uint4*>(src);
-      const uint4 v1 = *reinterpret_cast<const uint4*>(src + 8);
-      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        x[2 * i] = __uint_as_float(w[i] << 16);
-        x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 v = *reinterpret_cast<const float4*>(src + 4 * i);
-        x[4 * i] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
-      }
-    }
-    __syncthreads();   // every thread has its values: the stage may be refilled
-    if (threadIdx.x == 0 && j + kEncStages < my_n) {
-      const int64_t c2 = blockIdx.x + (j + kEncStages) * gridDim.x;
-      mbar_arrive_expect_tx(&full_bar[s], kChunkBytes);
-      bulk_load_1d(ring + s * kChunkElems, W + c2 * kChunkElems, kChunkBytes, &full_bar[s]);
-    }
-    encode16<kDQ>(x, blk, e0, sub, gmask, numel, true, tab, mexact, packed, scales, bc, sbins, bad);
-  }
-  if (abort_flag && threadIdx.x == 0) raise_status(d_status, QLORA_ERR_TIMEOUT);
-  // blocks not covered by whole streamed chunks
-  const int64_t first = nchunks * kChunkBlocks;
-  const int64_t ngroups = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 2;
-  for (int64_t blk = first + ((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 2);
-       blk < n1; blk += ngroups) {
-    const int64_t e0 = blk * kBlock + sub * kLaneElems;
-    const bool full = e0 + kLaneElems <= numel;
-    float x[kLaneElems];
-    load16<T>(W, e0, numel, full && aligned16, x);
-    encode16<kDQ>(x, blk, e0, sub, gmask, numel, full, tab, mexact, packed, scales, bc, sbins, bad);
-  }
-  if (bad) raise_status(d_status, QLORA_ERR_NONFINITE);
-  if (kDQ) {
-    if (sub == 0) bc.flush(sbins);
-    __syncthreads();
-    for (int i = threadIdx.x; i < 256; i += blockDim.x)
-      if (sbins[i]) atomicAdd(&bins[i], sbins[i]);
   }
 }
 
@@ -485,6 +376,141 @@ __device__ uint32_t exact_mean_bits(const unsigned long long* sb, int kmin, int 
   return bits;
 }
 
+constexpr int kChunkBlocks = 64;                 // 64-blocks per streamed chunk
+constexpr int kChunkElems = kChunkBlocks * kBlock;
+constexpr int kEncStages = 4;
+
+template <typename T>
+constexpr size_t encode_smem_bytes() {
+  return static_cast<size_t>(kEncStages) * kChunkElems * sizeof(T) + 128;
+}
+
+// CTA = 256 threads = 64 groups of 4 lanes = one chunk of 64 blocks per
+// iteration.  Whole chunks stream into a 4-stage shared-memory ring by 1-D
+// bulk copies; the remaining blocks (a partial last chunk, or everything when
+// W is not 16-byte aligned) are read directly from global memory.
+template <typename T, bool kDQ>
+__global__ void __launch_bounds__(256) nf4_encode_kernel(const T* __restrict__ W, int64_t numel,
+                                                         int64_t n1, uint8_t* __restrict__ packed,
+                                                         float* __restrict__ scales,
+                                                         unsigned long long* __restrict__ bins,
+                                                         unsigned int* __restrict__ done_ctas,
+                                                         float* __restrict__ offset_out,
+                                                         int32_t* d_status) {
+  extern __shared__ uint8_t esm_raw[];
+  T* ring = reinterpret_cast<T*>((reinterpret_cast<uintptr_t>(esm_raw) + 127) &
+                                 ~static_cast<uintptr_t>(127));
+  __shared__ uint32_t tab[kBuckets * 32];
+  __shared__ double mexact[15];
+  __shared__ unsigned long long sbins[kDQ ? 256 : 1];
+  __shared__ uint64_t full_bar[kEncStages];
+  pdl_launch_dependents();
+  pdl_wait();
+  __shared__ int abort_flag;
+  build_buckets(tab, mexact);
+  if (kDQ)
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = 0ull;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kEncStages; ++i) mbar_init(&full_bar[i], 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int lane = threadIdx.x & 31;
+  const int sub = lane & 3;
+  const unsigned gmask = 0xFu << (lane & 28);
+  const bool aligned16 = (reinterpret_cast<uintptr_t>(W) & 15u) == 0;
+  const int64_t nchunks = aligned16 ? numel / kChunkElems : 0;
+  const int64_t my_n =
+      nchunks > blockIdx.x ? (nchunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  constexpr uint32_t kChunkBytes = kChunkElems * sizeof(T);
+  BinCache bc;
+  bool bad = false;
+
+  if (threadIdx.x == 0) {
+    for (int64_t j = 0; j < my_n && j < kEncStages; ++j) {
+      const int64_t c = blockIdx.x + j * gridDim.x;
+      mbar_arrive_expect_tx(&full_bar[j], kChunkBytes);
+      bulk_load_1d(ring + j * kChunkElems, W + c * kChunkElems, kChunkBytes, &full_bar[j]);
+    }
+  }
+  for (int64_t j = 0; j < my_n; ++j) {
+    const int s = static_cast<int>(j % kEncStages);
+    const uint32_t ph = static_cast<uint32_t>((j / kEncStages) & 1);
+    if (!mbar_wait(&full_bar[s], ph)) abort_flag = 1;
+    __syncthreads();
+    if (abort_flag) break;
+    const int64_t c = blockIdx.x + j * gridDim.x;
+    const int local = threadIdx.x >> 2;
+    const int64_t blk = c * kChunkBlocks + local;
+    const int64_t e0 = blk * kBlock + sub * kLaneElems;
+    const T* src = ring + s * kChunkElems + local * kBlock + sub * kLaneElems;
+    float x[kLaneElems];
+    if (sizeof(T) == 2) {
+      const uint4 v0 = *reinterpret_cast<const uint4*>(src);
+      const uint4 v1 = *reinterpret_cast<const uint4*>(src + 8);
+      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 v = *reinterpret_cast<const float4*>(src + 4 * i);
+        x[4 * i] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
+      }
+    }
+    __syncthreads();   // every thread has its values: the stage may be refilled
+    if (threadIdx.x == 0 && j + kEncStages < my_n) {
+      const int64_t c2 = blockIdx.x + (j + kEncStages) * gridDim.x;
+      mbar_arrive_expect_tx(&full_bar[s], kChunkBytes);
+      bulk_load_1d(ring + s * kChunkElems, W + c2 * kChunkElems, kChunkBytes, &full_bar[s]);
+    }
+    encode16<kDQ>(x, blk, e0, sub, gmask, numel, true, tab, mexact, packed, scales, bc, sbins, bad);
+  }
+  if (abort_flag && threadIdx.x == 0) raise_status(d_status, QLORA_ERR_TIMEOUT);
+  // blocks not covered by whole streamed chunks
+  const int64_t first = nchunks * kChunkBlocks;
+  const int64_t ngroups = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 2;
+  for (int64_t blk = first + ((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 2);
+       blk < n1; blk += ngroups) {
+    const int64_t e0 = blk * kBlock + sub * kLaneElems;
+    const bool full = e0 + kLaneElems <= numel;
+    float x[kLaneElems];
+    load16<T>(W, e0, numel, full && aligned16, x);
+    encode16<kDQ>(x, blk, e0, sub, gmask, numel, full, tab, mexact, packed, scales, bc, sbins, bad);
+  }
+  if (bad) raise_status(d_status, QLORA_ERR_NONFINITE);
+  if (kDQ) {
+    if (sub == 0) bc.flush(sbins);
+    __syncthreads();
+    for (int i = threadIdx.x; i < 256; i += blockDim.x)
+      if (sbins[i]) atomicAdd(&bins[i], sbins[i]);
+    // The last CTA to finish forms the exact mean of all first-level scales
+    // from the global bins (every other CTA's additions are visible to it:
+    // each made them before its fenced increment of the counter).
+    __shared__ int last_cta;
+    __shared__ int krange[2];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      last_cta = atomicAdd(done_ctas, 1u) == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (last_cta) {
+      __threadfence();
+      for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = __ldcg(bins + i);
+      __syncthreads();
+      bins_key_range(sbins, krange);
+      __syncthreads();
+      if (threadIdx.x == 0) *offset_out = __uint_as_float(exact_mean_bits(sbins, krange[0], krange[1], n1));
+    }
+  }
+}
+
 // One warp per group of 256 centred scales (8 per lane, 8 groups per CTA).
 // The 255 distinct codebook values V_0 < ... < V_254 are: -|T|(127..1), 0,
 // |T|(1..127); the code of the nearest value to c/s2 (ties to the smaller
@@ -494,19 +520,16 @@ __device__ uint32_t exact_mean_bits(const unsigned long long* sb, int kmin, int 
 // 254 midpoints into fp32 thresholds once and counts them by binary search.
 // k < 127 -> byte 0x80 | (127 - k), k = 127 -> 0x00, k > 127 -> byte k - 127.
 __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict__ a, int64_t n1,
-                                                        const unsigned long long* __restrict__ bins,
-                                                        float* __restrict__ offset_p,
+                                                        const float* __restrict__ offset_p,
                                                         uint8_t* __restrict__ code8,
                                                         float* __restrict__ s2) {
-  // every CTA forms the same exact mean from the bins (CTA 0 stores it)
-  __shared__ unsigned long long sb[256];
-  __shared__ int range[2];
+  // the exact mean (offset) was formed by the encoder's last CTA
   __shared__ float s_off;
   __shared__ float mag[128];
   __shared__ double mid[254];
   __shared__ float thr[8][256];
   pdl_launch_dependents();
-  for (int t = threadIdx.x; t < 128; t += blockDim.x) mag[t] = t8_magnitude(t);
+  for (int t = threadIdx.x; t < 128; t += blockDim.x) mag[t] = kT8Table.v[t];
   __syncthreads();
   for (int k = threadIdx.x; k < 254; k += blockDim.x) {
     auto V = [&](int i) -> double {
@@ -517,14 +540,7 @@ __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict_
   }
   __syncthreads();
   pdl_wait();   // the tables above read no global memory
-  sb[threadIdx.x] = bins[threadIdx.x];
-  __syncthreads();
-  bins_key_range(sb, range);
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    s_off = __uint_as_float(exact_mean_bits(sb, range[0], range[1], n1));
-    if (blockIdx.x == 0) *offset_p = s_off;
-  }
+  if (threadIdx.x == 0) s_off = *offset_p;
   __syncthreads();
   const float off = s_off;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -666,10 +682,13 @@ cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* pa
   unsigned long long* bins = nullptr;
   float* scales = absmax_out;
   cudaError_t e = cudaSuccess;
+  unsigned int* done_ctas = nullptr;
   if (dq) {
+    // workspace: 256 exponent bins, the finished-CTA counter, then the scales
     bins = static_cast<unsigned long long*>(ws);
-    scales = reinterpret_cast<float*>(static_cast<char*>(ws) + 2048);
-    e = cudaMemsetAsync(bins, 0, 2048, st);
+    done_ctas = reinterpret_cast<unsigned int*>(static_cast<char*>(ws) + 2048);
+    scales = reinterpret_cast<float*>(static_cast<char*>(ws) + kQuantizeWsHead);
+    e = cudaMemsetAsync(ws, 0, kQuantizeWsHead, st);
     if (e != cudaSuccess) return e;
   }
   {
@@ -708,16 +727,16 @@ cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* pa
     const size_t sm = encode_smem_bytes<uint16_t>();
     const uint16_t* w16 = static_cast<const uint16_t*>(W);
     e = dq ? launch_pdl(nf4_encode_kernel<uint16_t, true>, dim3(blocks), dim3(threads), sm, st, 1, w16,
-                        numel, n1, packed, scales, bins, d_status)
+                        numel, n1, packed, scales, bins, done_ctas, offset, d_status)
            : launch_pdl(nf4_encode_kernel<uint16_t, false>, dim3(blocks), dim3(threads), sm, st, 1, w16,
-                        numel, n1, packed, scales, bins, d_status);
+                        numel, n1, packed, scales, bins, done_ctas, offset, d_status);
   } else {
     const size_t sm = encode_smem_bytes<float>();
     const float* w32 = static_cast<const float*>(W);
     e = dq ? launch_pdl(nf4_encode_kernel<float, true>, dim3(blocks), dim3(threads), sm, st, 1, w32,
-                        numel, n1, packed, scales, bins, d_status)
+                        numel, n1, packed, scales, bins, done_ctas, offset, d_status)
            : launch_pdl(nf4_encode_kernel<float, false>, dim3(blocks), dim3(threads), sm, st, 1, w32,
-                        numel, n1, packed, scales, bins, d_status);
+                        numel, n1, packed, scales, bins, done_ctas, offset, d_status);
   }
   }
   if (e == cudaSuccess) e = cudaGetLastError();
@@ -729,8 +748,7 @@ cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* pa
     const int64_t want_g = (n2 + 7) / 8;
     const int64_t grid = want_g < num_sms * 8LL ? want_g : num_sms * 8LL;
     e = launch_pdl(dq_encode_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, 1,
-                   static_cast<const float*>(scales), n1, static_cast<const unsigned long long*>(bins),
-                   offset, code8, s2);
+                   static_cast<const float*>(scales), n1, static_cast<const float*>(offset), code8, s2);
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -739,7 +757,7 @@ cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* pa
 size_t quantize_workspace_bytes(int64_t numel, bool dq) {
   if (!dq) return 0;
   const int64_t n1 = (numel + kBlock - 1) / kBlock;
-  return 2048 + static_cast<size_t>(n1) * 4;
+  return kQuantizeWsHead + static_cast<size_t>(n1) * 4;
 }
 
 }  // namespace qnf4

@@ -157,7 +157,8 @@ qlora_status qlora_nf4_quantize(const void* W, qlora_dtype dtype, const qlora_nf
  * allocate device memory when they quantize (runtimes that plan every device
  * buffer at start-up and forbid allocation in their steady state; plugins that
  * only receive tensor pointers from a host framework).  The scratch it needs
- * (2 KB of exponent bins plus one fp32 per 64-block, 4 MB at the limit) is a
+ * (2304 bytes of exponent bins and a counter, plus one fp32 per 64-block;
+ * about 4 MB at the limit) is a
  * fixed array inside the library, allocated on each GPU that loads this part
  * of the library and held until the process exits.
  *   - numel must not exceed QLORA_NOALLOC_MAX_NUMEL, else QLORA_ERR_UNSUPPORTED.

@@ -76,10 +76,13 @@ ROW_TOL = 1e-2
 TILE_TOL = 2e-2
 
 
-def close_report(got, ref, tile=128):
+def close_report(got, ref, tile=128, row_elems=256):
     """Relative errors of `got` against `ref`: whole matrix (Frobenius), worst
-    row, worst tile x tile block.  A row or tile whose reference norm is tiny
-    is measured against a tenth of the typical row or tile norm instead."""
+    row, worst tile x tile block.  A "row" is a group of consecutive rows with
+    at least `row_elems` elements (one row of a wide matrix; several rows of a
+    narrow one such as dA, K x r, where a single element's relative error says
+    nothing).  A row or tile whose reference norm is tiny is measured against a
+    tenth of the typical row or tile norm instead."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     if ref.ndim == 1:
@@ -89,9 +92,16 @@ def close_report(got, ref, tile=128):
     total = np.linalg.norm(ref)
     out = {"fro": float(np.linalg.norm(diff) / (total if total > 0 else 1.0))}
     R, C = ref.shape
-    row_rms = total / np.sqrt(R)
-    rn = np.linalg.norm(ref, axis=1)
-    dn = np.linalg.norm(diff, axis=1)
+    rb = max(1, -(-row_elems // C))             # rows per group
+    Rg = -(-R // rb)
+
+    def row_norms(a):
+        p = np.zeros((Rg * rb, C))
+        p[:R] = a
+        return np.sqrt((p.reshape(Rg, rb * C) ** 2).sum(axis=1))
+
+    row_rms = total / np.sqrt(Rg)
+    rn, dn = row_norms(ref), row_norms(diff)
     out["row"] = float(np.max(dn / np.maximum(rn, max(0.1 * row_rms, 1e-300))))
     tr, tc = min(tile, R), min(tile, C)
     Rp, Cp = -(-R // tr) * tr, -(-C // tc) * tc
