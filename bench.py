@@ -64,61 +64,102 @@ def load_peaks():
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock and clock-event (throttle) reasons of this process's GPU,
+    sampled every 0.5 ms through NVML while the timed region runs (the GPU is
+    found by its UUID, so CUDA_VISIBLE_DEVICES does not matter); falls back to
+    `nvidia-smi -lms 20` when NVML is not available."""
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
+    def __init__(self, torch_device):
+        self.dev = torch_device
+        self.samples = []
+        self.stop_flag = False
+        self.thread = None
         self.proc = None
-        self.lines = []
-        self.t = None
+        self.smax = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+        if not uuid.startswith("GPU-"):
+            uuid = "GPU-" + uuid
+        return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid)
 
     def start(self):
         try:
+            nv, h = self._nvml_handle()
+            self.smax = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+
+            def loop():
+                while not self.stop_flag:
+                    try:
+                        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                        rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((float(sm), int(rs)))
+                    except Exception:
+                        pass
+                    time.sleep(0.0005)
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.thread = None
+        try:
+            idx = int(os.environ.get("LOCAL_RANK", "0"))
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", f"--id={idx}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.lines = []
+            self.thread = threading.Thread(target=lambda: [self.lines.append(ln.strip())
+                                                           for ln in self.proc.stdout], daemon=True)
+            self.thread.start()
+            time.sleep(0.2)
         except Exception:
             self.proc = None
-            return
-        self.t = threading.Thread(target=self._read, daemon=True)
-        self.t.start()
-        t0 = time.time()
-        while not self.lines and time.time() - t0 < 5.0:   # sampler is up
-            time.sleep(0.01)
-        self.n0 = len(self.lines)
-
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.03)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines[getattr(self, "n0", 0):]:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
+        self.stop_flag = True
+        sm, reasons = [], set()
+        if self.proc is not None:
+            time.sleep(0.05)
+            self.proc.terminate()
             try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            names = [n for n, _ in self.REASONS]
+            for ln in self.lines:
+                parts = [q.strip() for q in ln.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    self.smax = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+            src = "nvidia-smi"
+        elif self.thread is not None:
+            self.thread.join(timeout=1.0)
+            for f, rs in self.samples:
+                sm.append(f)
+                for nm, bit in self.REASONS:
+                    if rs & bit:
+                        reasons.add(nm)
+            src = "nvml"
+        else:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source"]}
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.smax,
+                "reasons": sorted(reasons), "samples": len(sm), "source": src}
 
 
 # ---------------------------------------------------------------------------
@@ -286,19 +327,23 @@ def quantize_bench(torch, q, dev, peaks):
     W = (torch.randn((Kq, Nq), generator=gen, device=dev) * 0.015).to(torch.bfloat16)
     w = q.quantize(W, double_quant=True)
     st = q.new_status(dev)
+    ws = torch.empty(int(q.lib.qlora_nf4_quantize_workspace_size(Kq * Nq, 1)), dtype=torch.uint8,
+                     device=dev)
     for _ in range(3):
-        q.quantize(W, double_quant=True, out=w, status=st)
-    q.lib.qlora_profile_reset()
-    q.lib.qlora_profile_enable(1)
+        q.quantize(W, double_quant=True, out=w, status=st, workspace=ws)
     torch.cuda.synchronize()
+    # launches back to back, no per-launch events (they would keep each launch
+    # from overlapping its predecessor's tail)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     reps = 10
     e0.record()
     for _ in range(reps):
-        q.quantize(W, double_quant=True, out=w, status=st)
+        q.quantize(W, double_quant=True, out=w, status=st, workspace=ws)
     e1.record()
     torch.cuda.synchronize()
-    q.lib.qlora_profile_enable(0)
+    code, _ = q.status_sync(st)
+    if code != 0:
+        raise SystemExit(f"device status {code} in the quantize sweep")
     per = e0.elapsed_time(e1) / reps * 1e-3
     P = Kq * Nq
     n1 = P // 64
@@ -503,7 +548,7 @@ def main():
         raise SystemExit(f"device status {code} (mask {mask}) during warm-up")
 
     # ---------------- timed region (device time, max over ranks) ----------------
-    sampler = ClockSampler(local) if rank == 0 else None
+    sampler = ClockSampler(dev) if rank == 0 else None
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -576,29 +621,51 @@ def main():
             torch.empty_like(sets[0]["dY"])
         A_, B_ = sets[0]["A"], sets[0]["B"]
 
-        def e2e_step():
-            dW.copy_(hW, non_blocking=True)
-            dXin.copy_(hX, non_blocking=True)
-            dG.copy_(hG, non_blocking=True)
-            q.quantize(dW, double_quant=True, out=wbuf, status=status)
-            q.linear_forward(dXin, wbuf, A_, B_, c, Y=Y, Zc=Zc, status=status)
-            q.linear_backward(dG, dXin, Zc, wbuf, A_, B_, c, dX=dX, dA=dA, dB=dB, status=status)
-            if world > 1:
-                grads.all_reduce()
-            hdA.copy_(dA, non_blocking=True)
-            hdB.copy_(dB, non_blocking=True)
+        # Two device input sets: the next step's inputs are copied from pinned
+        # host memory on a copy stream while this step computes; every step's
+        # copies and its D2H read of dA, dB are inside the timed region.
+        dbufs = [(dW, dXin, dG), (torch.empty_like(dW), torch.empty_like(dXin), torch.empty_like(dG))]
+        cs = torch.cuda.Stream(device=dev)
+        comp = torch.cuda.current_stream(dev)
+        ev_copied = [torch.cuda.Event(), torch.cuda.Event()]
+        ev_used = [torch.cuda.Event(), torch.cuda.Event()]
 
-        for _ in range(2):
-            e2e_step()
+        def issue_copy(i):
+            b = i % 2
+            cs.wait_event(ev_used[b])            # the step that last read these buffers
+            with torch.cuda.stream(cs):
+                for dst, src in zip(dbufs[b], (hW, hX, hG)):
+                    dst.copy_(src, non_blocking=True)
+                ev_copied[b].record(cs)
+
+        def e2e_run(n, start_ev=None):
+            if start_ev is not None:
+                start_ev.record(comp)
+                cs.wait_event(start_ev)
+            issue_copy(0)
+            for i in range(n):
+                b = i % 2
+                comp.wait_event(ev_copied[b])
+                w_, x_, g_ = dbufs[b]
+                q.quantize(w_, double_quant=True, out=wbuf, status=status)
+                q.linear_forward(x_, wbuf, A_, B_, c, Y=Y, Zc=Zc, status=status)
+                q.linear_backward(g_, x_, Zc, wbuf, A_, B_, c, dX=dX, dA=dA, dB=dB, status=status)
+                ev_used[b].record(comp)
+                if i + 1 < n:
+                    issue_copy(i + 1)
+                if world > 1:
+                    grads.all_reduce()
+                hdA.copy_(dA, non_blocking=True)
+                hdB.copy_(dB, non_blocking=True)
+
+        e2e_run(2)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         n_e2e = max(3, min(args.steps, 20))
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a0.record()
-        for _ in range(n_e2e):
-            e2e_step()
-        a1.record()
+        e2e_run(n_e2e, start_ev=a0)
+        a1.record(comp)
         torch.cuda.synchronize()
         ems = a0.elapsed_time(a1) / n_e2e
         if world > 1:

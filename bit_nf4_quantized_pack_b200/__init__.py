@@ -24,6 +24,7 @@ from . import _lib
 from ._lib import NF4StateC, QLoRAError, check, lib
 
 __all__ = ["NF4Weight", "quantize", "dequantize", "merge", "merge_requantize",
+           "quantize_shard_begin", "quantize_shard_end", "shard_workspace_size",
            "linear_forward", "linear_backward",
            "status_sync", "status_clear", "new_status", "QLoRAError", "lib"]
 
@@ -200,6 +201,52 @@ def quantize(W: torch.Tensor, double_quant: bool = True, *, out: NF4Weight | Non
           "qlora_nf4_quantize")
     _finish(status, own, "qlora_nf4_quantize")
     return w
+
+
+def shard_workspace_size(numel: int, block_begin: int, block_end: int, double_quant: bool) -> int:
+    return int(lib.qlora_nf4_quantize_shard_workspace_size(numel, block_begin, block_end,
+                                                           1 if double_quant else 0))
+
+
+def _dtype_code(W):
+    if W.dtype == torch.bfloat16:
+        return _lib.QLORA_DTYPE_BF16
+    if W.dtype == torch.float32:
+        return _lib.QLORA_DTYPE_F32
+    raise TypeError("W must be bfloat16 or float32")
+
+
+def quantize_shard_begin(W_shard: torch.Tensor, w: NF4Weight, block_begin: int, block_end: int, *,
+                         workspace: torch.Tensor | None, status: torch.Tensor | None = None) -> None:
+    """Phase 1 of a sharded quantization (qlora_nf4_quantize_shard_begin):
+    encode 64-blocks [block_begin, block_end) of the weight `w` describes;
+    W_shard holds exactly those elements (contiguous)."""
+    if not W_shard.is_contiguous():
+        raise ValueError("W_shard must be contiguous")
+    st = w.cstruct()
+    dev = w.packed.device
+    own = status is None
+    status = new_status(dev) if own else status
+    check(lib.qlora_nf4_quantize_shard_begin(
+        _ptr(W_shard) if W_shard.numel() else None, _dtype_code(W_shard), C.byref(st), block_begin,
+        block_end, _ptr(workspace), workspace.numel() if workspace is not None else 0,
+        _ptr(status), _stream()), "qlora_nf4_quantize_shard_begin")
+    _finish(status, own, "qlora_nf4_quantize_shard_begin")
+
+
+def quantize_shard_end(w: NF4Weight, block_begin: int, block_end: int, *,
+                       workspace: torch.Tensor | None, status: torch.Tensor | None = None) -> None:
+    """Phase 2 (qlora_nf4_quantize_shard_end): the workspace's first 2048 bytes
+    must hold the exponent bins summed over every shard."""
+    st = w.cstruct()
+    dev = w.packed.device
+    own = status is None
+    status = new_status(dev) if own else status
+    check(lib.qlora_nf4_quantize_shard_end(
+        C.byref(st), block_begin, block_end, _ptr(workspace),
+        workspace.numel() if workspace is not None else 0, _ptr(status), _stream()),
+        "qlora_nf4_quantize_shard_end")
+    _finish(status, own, "qlora_nf4_quantize_shard_end")
 
 
 def dequantize(w: NF4Weight, *, out: torch.Tensor | None = None,

@@ -53,6 +53,9 @@ SIGNATURES = {
     "qlora_nf4_quantize_workspace_size": (_SZ, [_I64, _I32]),
     "qlora_nf4_quantize": (_I32, [_VP, _I32, _PS, _VP, _SZ, _VP, _VP]),
     "qlora_nf4_quantize_noalloc": (_I32, [_VP, _I32, _PS, _VP, _VP]),
+    "qlora_nf4_quantize_shard_workspace_size": (_SZ, [_I64, _I64, _I64, _I32]),
+    "qlora_nf4_quantize_shard_begin": (_I32, [_VP, _I32, _PS, _I64, _I64, _VP, _SZ, _VP, _VP]),
+    "qlora_nf4_quantize_shard_end": (_I32, [_PS, _I64, _I64, _VP, _SZ, _VP, _VP]),
     "qlora_nf4_dequantize": (_I32, [_PS, _VP, _VP, _VP]),
     "qlora_linear_fwd_workspace_size": (_SZ, [_I64, _I64, _I64, _I32]),
     "qlora_linear_fwd": (_I32, [_I64, _I64, _I64, _I32, _VP, _PS, _VP, _VP, _F, _VP, _VP,

@@ -145,6 +145,73 @@ qlora_status qlora_nf4_quantize(const void* W, qlora_dtype dtype, const qlora_nf
   return cuda_status(e);
 }
 
+size_t qlora_nf4_quantize_shard_workspace_size(int64_t numel_total, int64_t block_begin,
+                                               int64_t block_end, int32_t double_quant) {
+  if (numel_total < 1 || block_begin < 0 || block_end < block_begin ||
+      block_end > qlora_nf4_n1(numel_total) || !double_quant)
+    return 0;
+  return qnf4::kQuantizeWsHead + static_cast<size_t>(block_end - block_begin) * 4;
+}
+
+namespace {
+qlora_status check_shard(const qlora_nf4_state* st, int64_t b0, int64_t b1) {
+  qlora_status v = check_state(st, true);
+  if (v != QLORA_OK) return v;
+  const int64_t n1 = qlora_nf4_n1(st->numel);
+  if (b0 < 0 || b1 < b0 || b1 > n1) return QLORA_ERR_INVALID_ARG;
+  // with double quantization a shard holds whole groups of 256 blocks (the
+  // last shard may end at n1)
+  if (st->double_quant && b1 > b0 &&
+      (b0 % qnf4::kDQBlock != 0 || (b1 != n1 && b1 % qnf4::kDQBlock != 0)))
+    return QLORA_ERR_INVALID_ARG;
+  return QLORA_OK;
+}
+}  // namespace
+
+qlora_status qlora_nf4_quantize_shard_begin(const void* W_shard, qlora_dtype dtype,
+                                            const qlora_nf4_state* st, int64_t block_begin,
+                                            int64_t block_end, void* ws, size_t ws_bytes,
+                                            int32_t* d_status, qlora_stream_t stream) {
+  NvtxRange nvtx_range("qlora_nf4_quantize_shard_begin");
+  qlora_status v = check_shard(st, block_begin, block_end);
+  if (v != QLORA_OK) return v;
+  if (dtype != QLORA_DTYPE_BF16 && dtype != QLORA_DTYPE_F32) return QLORA_ERR_INVALID_ARG;
+  const size_t need = qlora_nf4_quantize_shard_workspace_size(st->numel, block_begin, block_end,
+                                                              st->double_quant);
+  if (need > 0 && (!ws || ws_bytes < need || !aligned(ws, 16))) return QLORA_ERR_INVALID_ARG;
+  if (block_end == block_begin) {
+    // an empty shard contributes zero bins
+    if (st->double_quant)
+      return cuda_status(cudaMemsetAsync(ws, 0, qnf4::kQuantizeWsHead,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+    return QLORA_OK;
+  }
+  if (!W_shard || !aligned(W_shard, 16)) return QLORA_ERR_INVALID_ARG;
+  const int sms = sm_count();
+  if (sms <= 0) return QLORA_ERR_CUDA;
+  return cuda_status(qnf4::launch_quantize_shard_begin(
+      W_shard, dtype, st->numel, block_begin, block_end, st->packed, st->absmax,
+      st->double_quant != 0, ws, d_status, reinterpret_cast<cudaStream_t>(stream), sms,
+      st->codebook));
+}
+
+qlora_status qlora_nf4_quantize_shard_end(const qlora_nf4_state* st, int64_t block_begin,
+                                          int64_t block_end, const void* ws, size_t ws_bytes,
+                                          int32_t* d_status, qlora_stream_t stream) {
+  NvtxRange nvtx_range("qlora_nf4_quantize_shard_end");
+  (void)d_status;
+  qlora_status v = check_shard(st, block_begin, block_end);
+  if (v != QLORA_OK) return v;
+  if (!st->double_quant) return QLORA_OK;   // nothing happens after the bins
+  const size_t need = qlora_nf4_quantize_shard_workspace_size(st->numel, block_begin, block_end, 1);
+  if (!ws || ws_bytes < need || !aligned(ws, 16)) return QLORA_ERR_INVALID_ARG;
+  const int sms = sm_count();
+  if (sms <= 0) return QLORA_ERR_CUDA;
+  return cuda_status(qnf4::launch_quantize_shard_end(st->numel, block_begin, block_end, ws,
+                                                     st->code8, st->s2, st->offset,
+                                                     reinterpret_cast<cudaStream_t>(stream), sms));
+}
+
 qlora_status qlora_nf4_dequantize(const qlora_nf4_state* st, uint16_t* W_hat, int32_t* d_status,
                                   qlora_stream_t stream) {
   NvtxRange nvtx_range("qlora_nf4_dequantize");

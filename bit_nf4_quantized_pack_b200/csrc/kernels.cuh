@@ -88,6 +88,19 @@ cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* pa
                             void* ws, int32_t* d_status, cudaStream_t st, int num_sms,
                             int codebook = 0);
 size_t quantize_workspace_bytes(int64_t numel, bool dq);
+// Sharded quantization (blocks [b0, b1) of a tensor of numel_total elements;
+// W_shard points at element b0 * 64).  begin: packed bytes and, without DQ,
+// the scales go straight into the full-size state; with DQ the shard's
+// scales and the exponent bins of their sums go to `ws` (same layout as the
+// quantize workspace).  end: with the bins holding the sum over every shard,
+// the offset and the scale codes and s2 of the shard's groups.
+cudaError_t launch_quantize_shard_begin(const void* W_shard, int dtype, int64_t numel_total,
+                                        int64_t b0, int64_t b1, uint8_t* packed, float* absmax_out,
+                                        bool dq, void* ws, int32_t* d_status, cudaStream_t st,
+                                        int num_sms, int codebook);
+cudaError_t launch_quantize_shard_end(int64_t numel_total, int64_t b0, int64_t b1, const void* ws,
+                                      uint8_t* code8, float* s2, float* offset, cudaStream_t st,
+                                      int num_sms);
 
 // dequantize.cu
 cudaError_t launch_dequantize(const uint8_t* packed, int64_t numel, const float* absmax,

@@ -274,9 +274,14 @@ template <bool kBwd> constexpr int kFAccs = kFBM / (kBwd ? 256 : 128);
 constexpr int kFA = kFBM * 128;      // 512 x 64 bf16
 constexpr int kFBoxes = kFBM / 128;  // TMA boxes of 128 rows per activation tile
 constexpr int kFB = kFBN * 128;      // 128 x 64 bf16
-constexpr int kFDecWarps = kFBN / 32;   // one weight-tile row per decoder thread
+constexpr int kFDecWarps = kFBN / 32;   // one weight-tile row per decoder thread and K-step
+// Decoder groups of kFDecWarps warps take turns by K-step (group g decodes the
+// steps g, g + kFDecGroups, ...), so each warp has kFDecGroups K-steps of time
+// per row and its loads reach further ahead.
+constexpr int kFDecGroups = 2;
+constexpr int kFDecAll = kFDecWarps * kFDecGroups;
 constexpr int kFEpiWarps = 4;
-constexpr int kFThreads = (2 + kFDecWarps + kFEpiWarps) * 32;  // TMA, MMA, decoders, epilogue
+constexpr int kFThreads = (2 + kFDecAll + kFEpiWarps) * 32;  // TMA, MMA, decoders, epilogue
 constexpr size_t kFSmem = 1024 + kFAStages * kFA + kFBStages * kFB + 1024 + 512;
 static_assert(kFAccs<false> * kFAccCols<false> <= 512 && kFAccs<true> * kFAccCols<true> <= 512 &&
                   kFAccs<false> <= kFAccMax && kFBN == 128,
@@ -580,15 +585,17 @@ __global__ void __launch_bounds__(kFThreads, 1)
       umma_commit(drain);
       (void)mbar_wait(drain, 0);
     }
-  } else if (warp < 2 + kFDecWarps) {
+  } else if (warp < 2 + kFDecAll) {
     // ------------------------------ decoders -------------------------------
-    const int R = threadIdx.x - 64;            // weight-tile row 0..kFBN-1
+    const int grp = (warp - 2) / kFDecWarps;   // this warp's turn among the groups
+    const int R = threadIdx.x - 64 - grp * kFBN;   // weight-tile row 0..kFBN-1
     const float off = args.sv.code8 != nullptr ? __ldg(args.sv.offset) : 0.0f;
     const int nsteps = args.nk;                // decoded steps per tile
     bool ok = true;
     int tile = blockIdx.x, kk = 0;             // the step being decoded
+    advance(tile, kk, grp, nsteps);
     int ptile = tile, pkk = kk;                // the step being prefetched
-    uint32_t ib = 0;
+    uint32_t ib = static_cast<uint32_t>(grp);
     // One K-step: wait for a free weight stage, decode this thread's row.
     auto step = [&](const RowFetch& f) {
       const uint32_t s = ib % kFBStages, ph = (ib / kFBStages) & 1;
@@ -618,29 +625,29 @@ __global__ void __launch_bounds__(kFThreads, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&full_b[s]);
-      advance(tile, kk, 1, nsteps);
-      ++ib;
+      advance(tile, kk, kFDecGroups, nsteps);
+      ib += kFDecGroups;
     };
     // Three prefetch slots consumed and refilled in place (no register moves
     // that would wait on loads still in flight).
     RowFetch q0 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
-    advance(ptile, pkk, 1, nsteps);
+    advance(ptile, pkk, kFDecGroups, nsteps);
     RowFetch q1 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
-    advance(ptile, pkk, 1, nsteps);
+    advance(ptile, pkk, kFDecGroups, nsteps);
     RowFetch q2 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
-    advance(ptile, pkk, 1, nsteps);
+    advance(ptile, pkk, kFDecGroups, nsteps);
     while (ok && tile < num_tiles) {
       step(q0);
       q0 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
-      advance(ptile, pkk, 1, nsteps);
+      advance(ptile, pkk, kFDecGroups, nsteps);
       if (!ok || tile >= num_tiles) break;
       step(q1);
       q1 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
-      advance(ptile, pkk, 1, nsteps);
+      advance(ptile, pkk, kFDecGroups, nsteps);
       if (!ok || tile >= num_tiles) break;
       step(q2);
       q2 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
-      advance(ptile, pkk, 1, nsteps);
+      advance(ptile, pkk, kFDecGroups, nsteps);
     }
     if (!ok) *abort_flag = 1;
   } else {

@@ -495,6 +495,7 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const T* __restrict__ W
     __shared__ int last_cta;
     __shared__ int krange[2];
     __syncthreads();
+    if (offset_out == nullptr) return;   // a shard: the caller adds the bins of all shards
     if (threadIdx.x == 0) {
       __threadfence();
       last_cta = atomicAdd(done_ctas, 1u) == gridDim.x - 1;
@@ -587,6 +588,21 @@ __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict_
   }
 }
 
+// The exact mean of n1 first-level scales from exponent bins that already
+// hold every shard's sums (sharded quantization): one CTA.
+__global__ void __launch_bounds__(256) dq_mean_kernel(const unsigned long long* __restrict__ bins,
+                                                      int64_t n1, float* __restrict__ offset_out) {
+  __shared__ unsigned long long sb[256];
+  __shared__ int krange[2];
+  pdl_launch_dependents();
+  pdl_wait();
+  sb[threadIdx.x] = bins[threadIdx.x];
+  __syncthreads();
+  bins_key_range(sb, krange);
+  __syncthreads();
+  if (threadIdx.x == 0) *offset_out = __uint_as_float(exact_mean_bits(sb, krange[0], krange[1], n1));
+}
+
 // ---------------------------------------------------------------------------
 // Host launchers
 // ---------------------------------------------------------------------------
@@ -660,44 +676,23 @@ __global__ void __launch_bounds__(256) int4_encode_kernel(const T* __restrict__ 
   }
 }
 
-cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* packed,
-                            float* absmax_out, bool dq, uint8_t* code8, float* s2, float* offset,
-                            void* ws, int32_t* d_status, cudaStream_t st, int num_sms,
-                            int codebook) {
+namespace {
+
+// The NF4 encoder over `numel` elements of W: packed bytes, one fp32 scale per
+// 64-block into `scales`, and (dq) the scales' exponent bins; with
+// `offset_out` the last CTA also forms their exact mean there.
+cudaError_t launch_encoder(const void* W, int dtype, int64_t numel, uint8_t* packed, float* scales,
+                           bool dq, unsigned long long* bins, unsigned int* done_ctas,
+                           float* offset_out, int32_t* d_status, cudaStream_t st, int num_sms) {
   const int64_t n1 = (numel + kBlock - 1) / kBlock;
   const int threads = 256;
-  if (codebook == 1) {   // uniform INT4: no double quantization, no workspace
-    const dim3 grid(static_cast<unsigned>((n1 + 255) / 256));
-    ProfScope prof(kProfQuantize, st);
-    const cudaError_t e1 =
-        dtype == QLORA_DTYPE_BF16
-            ? launch_pdl(int4_encode_kernel<uint16_t>, grid, dim3(256), 0, st, 1,
-                         static_cast<const uint16_t*>(W), numel, packed, absmax_out, d_status)
-            : launch_pdl(int4_encode_kernel<float>, grid, dim3(256), 0, st, 1,
-                         static_cast<const float*>(W), numel, packed, absmax_out, d_status);
-    if (e1 != cudaSuccess) return e1;
-    return cudaGetLastError();
-  }
   const int64_t want = (n1 * 4 + threads - 1) / threads;
-  unsigned long long* bins = nullptr;
-  float* scales = absmax_out;
-  cudaError_t e = cudaSuccess;
-  unsigned int* done_ctas = nullptr;
-  if (dq) {
-    // workspace: 256 exponent bins, the finished-CTA counter, then the scales
-    bins = static_cast<unsigned long long*>(ws);
-    done_ctas = reinterpret_cast<unsigned int*>(static_cast<char*>(ws) + 2048);
-    scales = reinterpret_cast<float*>(static_cast<char*>(ws) + kQuantizeWsHead);
-    e = cudaMemsetAsync(ws, 0, kQuantizeWsHead, st);
-    if (e != cudaSuccess) return e;
-  }
-  {
   ProfScope prof(kProfQuantize, st);
   // one wave of resident CTAs (each loops over chunks); attributes and
   // occupancy per device
   static int per_sm[kMaxDevices][4];
   static DeviceOnce once;
-  e = once.run([&](int dev) {
+  cudaError_t e = once.run([&](int dev) {
     const int b16 = static_cast<int>(encode_smem_bytes<uint16_t>());
     const int b32 = static_cast<int>(encode_smem_bytes<float>());
     const void* fns[4] = {reinterpret_cast<const void*>(nf4_encode_kernel<uint16_t, false>),
@@ -727,31 +722,108 @@ cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* pa
     const size_t sm = encode_smem_bytes<uint16_t>();
     const uint16_t* w16 = static_cast<const uint16_t*>(W);
     e = dq ? launch_pdl(nf4_encode_kernel<uint16_t, true>, dim3(blocks), dim3(threads), sm, st, 1, w16,
-                        numel, n1, packed, scales, bins, done_ctas, offset, d_status)
+                        numel, n1, packed, scales, bins, done_ctas, offset_out, d_status)
            : launch_pdl(nf4_encode_kernel<uint16_t, false>, dim3(blocks), dim3(threads), sm, st, 1, w16,
-                        numel, n1, packed, scales, bins, done_ctas, offset, d_status);
+                        numel, n1, packed, scales, bins, done_ctas, offset_out, d_status);
   } else {
     const size_t sm = encode_smem_bytes<float>();
     const float* w32 = static_cast<const float*>(W);
     e = dq ? launch_pdl(nf4_encode_kernel<float, true>, dim3(blocks), dim3(threads), sm, st, 1, w32,
-                        numel, n1, packed, scales, bins, done_ctas, offset, d_status)
+                        numel, n1, packed, scales, bins, done_ctas, offset_out, d_status)
            : launch_pdl(nf4_encode_kernel<float, false>, dim3(blocks), dim3(threads), sm, st, 1, w32,
-                        numel, n1, packed, scales, bins, done_ctas, offset, d_status);
-  }
+                        numel, n1, packed, scales, bins, done_ctas, offset_out, d_status);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
-  if (e != cudaSuccess || !dq) return e;
+  return e;
+}
 
+// Scale codes and second-level scales of n1 centred scales (groups of 256
+// from the first), given the offset in device memory.
+cudaError_t launch_dq_encode(const float* scales, int64_t n1, const float* offset, uint8_t* code8,
+                             float* s2, cudaStream_t st, int num_sms) {
   const int64_t n2 = (n1 + kDQBlock - 1) / kDQBlock;
-  {
-    ProfScope prof(kProfQuantize, st);
-    const int64_t want_g = (n2 + 7) / 8;
-    const int64_t grid = want_g < num_sms * 8LL ? want_g : num_sms * 8LL;
-    e = launch_pdl(dq_encode_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, 1,
-                   static_cast<const float*>(scales), n1, static_cast<const float*>(offset), code8, s2);
-  }
+  ProfScope prof(kProfQuantize, st);
+  const int64_t want_g = (n2 + 7) / 8;
+  const int64_t grid = want_g < num_sms * 8LL ? want_g : num_sms * 8LL;
+  cudaError_t e = launch_pdl(dq_encode_kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st,
+                             1, scales, n1, offset, code8, s2);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+cudaError_t launch_int4(const void* W, int dtype, int64_t numel, uint8_t* packed, float* scales,
+                        int32_t* d_status, cudaStream_t st) {
+  const int64_t n1 = (numel + kBlock - 1) / kBlock;
+  const dim3 grid(static_cast<unsigned>((n1 + 255) / 256));
+  ProfScope prof(kProfQuantize, st);
+  const cudaError_t e1 =
+      dtype == QLORA_DTYPE_BF16
+          ? launch_pdl(int4_encode_kernel<uint16_t>, grid, dim3(256), 0, st, 1,
+                       static_cast<const uint16_t*>(W), numel, packed, scales, d_status)
+          : launch_pdl(int4_encode_kernel<float>, grid, dim3(256), 0, st, 1,
+                       static_cast<const float*>(W), numel, packed, scales, d_status);
+  if (e1 != cudaSuccess) return e1;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* packed,
+                            float* absmax_out, bool dq, uint8_t* code8, float* s2, float* offset,
+                            void* ws, int32_t* d_status, cudaStream_t st, int num_sms,
+                            int codebook) {
+  // uniform INT4: no double quantization, no workspace
+  if (codebook == 1) return launch_int4(W, dtype, numel, packed, absmax_out, d_status, st);
+  if (!dq)
+    return launch_encoder(W, dtype, numel, packed, absmax_out, false, nullptr, nullptr, nullptr,
+                          d_status, st, num_sms);
+  // workspace: 256 exponent bins, the finished-CTA counter, then the scales
+  const int64_t n1 = (numel + kBlock - 1) / kBlock;
+  unsigned long long* bins = static_cast<unsigned long long*>(ws);
+  unsigned int* done_ctas = reinterpret_cast<unsigned int*>(static_cast<char*>(ws) + 2048);
+  float* scales = reinterpret_cast<float*>(static_cast<char*>(ws) + kQuantizeWsHead);
+  cudaError_t e = cudaMemsetAsync(ws, 0, kQuantizeWsHead, st);
+  if (e != cudaSuccess) return e;
+  e = launch_encoder(W, dtype, numel, packed, scales, true, bins, done_ctas, offset, d_status, st,
+                     num_sms);
+  if (e != cudaSuccess) return e;
+  return launch_dq_encode(scales, n1, offset, code8, s2, st, num_sms);
+}
+
+cudaError_t launch_quantize_shard_begin(const void* W_shard, int dtype, int64_t numel_total,
+                                        int64_t b0, int64_t b1, uint8_t* packed, float* absmax_out,
+                                        bool dq, void* ws, int32_t* d_status, cudaStream_t st,
+                                        int num_sms, int codebook) {
+  const int64_t e_end = b1 * kBlock < numel_total ? b1 * kBlock : numel_total;
+  const int64_t numel = e_end - b0 * kBlock;
+  uint8_t* pk = packed + b0 * (kBlock / 2);
+  if (codebook == 1) return launch_int4(W_shard, dtype, numel, pk, absmax_out + b0, d_status, st);
+  if (!dq)
+    return launch_encoder(W_shard, dtype, numel, pk, absmax_out + b0, false, nullptr, nullptr,
+                          nullptr, d_status, st, num_sms);
+  unsigned long long* bins = static_cast<unsigned long long*>(ws);
+  float* scales = reinterpret_cast<float*>(static_cast<char*>(ws) + kQuantizeWsHead);
+  cudaError_t e = cudaMemsetAsync(ws, 0, kQuantizeWsHead, st);
+  if (e != cudaSuccess) return e;
+  return launch_encoder(W_shard, dtype, numel, pk, scales, true, bins, nullptr, nullptr, d_status,
+                        st, num_sms);
+}
+
+cudaError_t launch_quantize_shard_end(int64_t numel_total, int64_t b0, int64_t b1, const void* ws,
+                                      uint8_t* code8, float* s2, float* offset, cudaStream_t st,
+                                      int num_sms) {
+  const int64_t n1 = (numel_total + kBlock - 1) / kBlock;
+  const unsigned long long* bins = static_cast<const unsigned long long*>(ws);
+  const float* scales =
+      reinterpret_cast<const float*>(static_cast<const char*>(ws) + kQuantizeWsHead);
+  cudaError_t e;
+  {
+    ProfScope prof(kProfQuantize, st);
+    e = launch_pdl(dq_mean_kernel, dim3(1), dim3(256), 0, st, 1, bins, n1, offset);
+    if (e == cudaSuccess) e = cudaGetLastError();
+  }
+  if (e != cudaSuccess || b1 <= b0) return e;
+  return launch_dq_encode(scales, b1 - b0, offset, code8 + b0, s2 + b0 / kDQBlock, st, num_sms);
 }
 
 size_t quantize_workspace_bytes(int64_t numel, bool dq) {

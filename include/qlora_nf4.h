@@ -151,6 +151,49 @@ qlora_status qlora_nf4_quantize(const void* W, qlora_dtype dtype, const qlora_nf
                                 qlora_stream_t stream);
 
 /*
+ * Sharded quantization for data-parallel replicas (page "SFT（四）：QLoRA的
+ * 4-bit量化与LoRA微调原理", §26.1 为什么微批次设为 1: the effective batch spans
+ * devices, each holding the same frozen base).  Each of several processes
+ * encodes a contiguous range [block_begin, block_end) of the 64-blocks; the
+ * ranges together must cover 0 .. n1 exactly once.  The result, once the
+ * pieces are exchanged, is bit-identical to qlora_nf4_quantize of the whole
+ * tensor.
+ *
+ *   1. qlora_nf4_quantize_shard_begin: W_shard points at element
+ *      block_begin * 64 of the weight (the elements up to block_end * 64, or
+ *      to numel for the last block).  Writes the packed bytes of the range
+ *      into st->packed (at byte block_begin * 32) and, without double
+ *      quantization, the scales into st->absmax[block_begin ..].  With
+ *      double quantization the range's scales go to ws, and the first 2048
+ *      bytes of ws receive 256 unsigned 64-bit sums (exponent bins of the
+ *      range's scales).
+ *   2. The caller adds those 256 sums element-wise over every shard (an
+ *      integer all-reduce: exact, in any order) and writes the totals back
+ *      into the first 2048 bytes of each shard's ws.
+ *   3. qlora_nf4_quantize_shard_end (double quantization only; otherwise a
+ *      no-op): from the total bins, st->offset (the exact mean of all n1
+ *      scales, the same on every shard), and the scale codes and s2 of the
+ *      range's groups (st->code8[block_begin ..], st->s2[block_begin/256 ..]).
+ *   4. The caller gathers each shard's packed bytes, code8 and s2 (or
+ *      absmax) ranges into every replica.
+ * With double quantization block_begin must be a multiple of 256 and
+ * block_end a multiple of 256 or n1 (whole groups per shard), else
+ * INVALID_ARG.  An empty range (block_begin == block_end) is allowed anywhere
+ * (begin clears the bins; end forms only the offset).  st describes the whole tensor (numel = K·N); its
+ * buffers are full-size.  ws: at least qlora_nf4_quantize_shard_workspace_size
+ * bytes, the same buffer for begin and end (0 bytes without DQ).
+ */
+size_t qlora_nf4_quantize_shard_workspace_size(int64_t numel_total, int64_t block_begin,
+                                               int64_t block_end, int32_t double_quant);
+qlora_status qlora_nf4_quantize_shard_begin(const void* W_shard, qlora_dtype dtype,
+                                            const qlora_nf4_state* st, int64_t block_begin,
+                                            int64_t block_end, void* ws, size_t ws_bytes,
+                                            int32_t* d_status, qlora_stream_t stream);
+qlora_status qlora_nf4_quantize_shard_end(const qlora_nf4_state* st, int64_t block_begin,
+                                          int64_t block_end, const void* ws, size_t ws_bytes,
+                                          int32_t* d_status, qlora_stream_t stream);
+
+/*
  * Allocation-free NF4 quantization (no counterpart on the pages: it is a
  * property of this library, not of the method).  Same computation, arguments
  * and errors as qlora_nf4_quantize, without the workspace: some callers cannot

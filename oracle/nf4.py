@@ -272,8 +272,16 @@ def double_quantize(absmax, blocksize: int = DQ_BLOCKSIZE, chunk: int = 1 << 16)
     of c/s2 with ties to the smaller value.
     """
     a = np.asarray(absmax, dtype=np.float32).ravel()
+    return double_quantize_centred(a, exact_mean_f32(a), blocksize, chunk)
+
+
+def double_quantize_centred(absmax, offset, blocksize: int = DQ_BLOCKSIZE, chunk: int = 1 << 16):
+    """The encoding half of ``double_quantize`` for a given offset (the mean
+    of the whole tensor's scales): centre, then per group of 256 from the
+    first element an fp32 absmax s2 and the nearest 8-bit code of c/s2."""
+    a = np.asarray(absmax, dtype=np.float32).ravel()
+    offset = np.float32(offset)
     n1 = a.size
-    offset = exact_mean_f32(a)
     c = (a - offset).astype(np.float32)                   # fp32 subtraction, RN
     n2 = -(-n1 // blocksize)
     s2 = np.empty(n2, dtype=np.float32)
