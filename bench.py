@@ -486,6 +486,23 @@ def merge_bench(torch, q, dev, peaks):
     return {"shape": [Kq, Nq], "r": rq, "us": per * 1e6, "GB/s": gbs, "frac": gbs / peaks["hbm"]}
 
 
+def run_sweeps(args):
+    """The named sweeps alone on GPU 0 (one JSON line): for iterating on one
+    kernel family without the training step."""
+    import torch
+    import bit_nf4_quantized_pack_b200 as q
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    fns = {"gemv": gemv_sweep, "quantize": quantize_bench, "merge": merge_bench,
+           "layers": layers_bench}
+    out = {"sweeps": {}}
+    for name in args.sweep.split(","):
+        out["sweeps"][name] = fns[name](torch, q, dev, peaks)
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -500,11 +517,15 @@ def main():
     ap.add_argument("--shape", default="",
                     help="M,K,N for --case gemv (default 1,4096,11008); K,N for --case quantize")
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--sweep", default="",
+                    help="only these sweeps (comma list of gemv, quantize, merge, layers), no step")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
     if args.case:
         return run_case(args)
+    if args.sweep:
+        return run_sweeps(args)
 
     import torch
     import torch.distributed as dist

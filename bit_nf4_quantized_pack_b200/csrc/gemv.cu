@@ -56,8 +56,9 @@ constexpr int kGvMaxStages = 6;
 constexpr int kGvPk = kGvRows * 128;     // packed weights of a stage
 constexpr int kGvXb = 2 * 2048;          // 16 tokens x 128 k bf16, two swizzled 64-k halves
 constexpr int kGvCompute = 16;           // compute warps: 4 column blocks x 4 row slots
-constexpr int kGvThreads = (kGvCompute + 1) * 32;
-constexpr int kGvAhead = 4;              // stages of scale loads in flight per lane
+constexpr int kGvWarps = kGvCompute + 2; // + the TMA producer and the scale warp
+constexpr int kGvThreads = kGvWarps * 32;
+constexpr int kGvScaleWords = 4 * kGvRows;   // decode scales of one stage: 4 blocks x 128 rows
 constexpr int kGvSmemMax = 232448;       // 227 KB, the opt-in limit per CTA
 constexpr int kGvPLd = kGvCols + 4;      // fp32 words per token row of a CTA's sums
 // epilogue regions, carved from the ring once every stage is consumed
@@ -131,12 +132,6 @@ __device__ __forceinline__ GvScale gemv_scale_load(const ScaleView& sv, int64_t 
   return r;
 }
 
-__device__ __forceinline__ float gemv_scale_value(const ScaleView& sv, const GvScale& r, float off,
-                                                  const float* t8) {
-  if (sv.code8 == nullptr) return r.v;
-  return __fadd_rn(__fmul_rn(t8[r.q], r.v), off);
-}
-
 template <bool kM16>
 __global__ void __launch_bounds__(kGvThreads, 1)
     nf4_gemv_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmX,
@@ -147,10 +142,12 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   uint8_t* ring = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(gsm_raw + kGvTable) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sB = ring + args.nstages * args.stage_bytes;      // B: rp rows x 256 columns bf16
-  float* t8 = reinterpret_cast<float*>(sB + 512 * args.rp);
+  float* sc_ring = reinterpret_cast<float*>(sB + 512 * args.rp);   // [stage][4 blocks][128 rows]
+  float* t8 = sc_ring + kGvMaxStages * kGvScaleWords;
   uint64_t* full = reinterpret_cast<uint64_t*>(t8 + 256);
   uint64_t* empty = full + kGvMaxStages;
-  uint64_t* bfull = empty + kGvMaxStages;
+  uint64_t* sfull = empty + kGvMaxStages;
+  uint64_t* bfull = sfull + kGvMaxStages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   pdl_launch_dependents();
@@ -158,6 +155,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     for (int s = 0; s < kGvMaxStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kGvCompute);
+      mbar_init(&sfull[s], 1);
     }
     mbar_init(bfull, 1);
     fence_mbar_init();
@@ -166,7 +164,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   // the pair table is bf16(C[e >> 4]) | bf16(C[e & 15]) << 16, one copy per bank
   {
     const float cv = kCodeVals[16 * args.sv.codebook + (lane & 15)];
-    for (int e = warp; e < 256; e += kGvCompute + 1)
+    for (int e = warp; e < 256; e += kGvWarps)
       table[e * 64 + lane] =
           pack_bf16x2(__shfl_sync(0xFFFFFFFFu, cv, e >> 4), __shfl_sync(0xFFFFFFFFu, cv, e & 15));
   }
@@ -185,8 +183,8 @@ __global__ void __launch_bounds__(kGvThreads, 1)
 
   if (warp == kGvCompute) {
     // --------------------------------- producer ---------------------------------
+    pdl_wait();
     if (lane == 0) {
-      pdl_wait();
       if (!zc_only) tma_prefetch_desc(&tmP);
       tma_prefetch_desc(&tmX);
       tma_prefetch_desc(&tmA);
@@ -224,6 +222,53 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         if (last_parity[q] < 2 && !mbar_wait(&full[q], last_parity[q])) ok = false;
       if (!zc_only && !mbar_wait(bfull, 0)) ok = false;
     }
+  } else if (warp == kGvCompute + 1) {
+    // ------------------------------- scale warp -------------------------------
+    // a'[row][block] of every stage into sc_ring[stage][block][row]: lane l
+    // decodes block l & 3 for rows (l >> 2) + 8i, i < 16, and keeps the next
+    // stage's raw loads in flight while it decodes this one.
+    pdl_wait();
+    if (!zc_only) {
+      const int b = lane & 3, rl = lane >> 2;
+      const int blk = cg * 4 + b;
+      const bool colok = blk * 64 < N;
+      const int bpr = N / 64;
+      const bool dq = args.sv.code8 != nullptr;
+      const float off = dq ? __ldg(args.sv.offset) : 0.0f;
+      uint32_t qv[16];
+      float fv[16];
+      auto load = [&](int j) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int row = (st0 + j) * kGvRows + rl + 8 * i;
+          qv[i] = 0u;
+          fv[i] = 0.0f;
+          if (colok && row < K) {
+            const GvScale z = gemv_scale_load(args.sv, static_cast<int64_t>(row) * bpr + blk);
+            qv[i] = z.q;
+            fv[i] = z.v;
+          }
+        }
+      };
+      if (nst > 0) load(0);
+      int s = 0;
+      uint32_t ph = 0;
+      for (int j = 0; j < nst; ++j) {
+        float a[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          a[i] = dq ? __fadd_rn(__fmul_rn(t8[qv[i]], fv[i]), off) : fv[i];
+        if (j + 1 < nst) load(j + 1);
+        // the compute warps are done with this slot's previous stage
+        if (j >= args.nstages && !mbar_wait(&empty[s], ph ^ 1)) { ok = false; break; }
+        float* dst = sc_ring + s * kGvScaleWords + b * kGvRows + rl;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) dst[8 * i] = a[i];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sfull[s]);
+        if (++s == args.nstages) { s = 0; ph ^= 1; }
+      }
+    }
   } else {
     // ------------------------------ compute warps ------------------------------
     pdl_wait();
@@ -231,9 +276,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     const int blk = cg * 4 + b;                        // 64-column block
     const bool colok = !zc_only && blk * 64 < N;
     const int g = lane >> 2, t = lane & 3;
-    const int bpr = N / 64;
     const int kb = 16 * p;                             // rows kb.. and kb+64.. of a stage
-    const float off = (colok && args.sv.code8 != nullptr) ? __ldg(args.sv.offset) : 0.0f;
     const uint32_t tbase = smem_u32(gsm_raw);
     const uint32_t laneword = lane * 4;
     // Packed stage (128-byte swizzle: row R at R*128, 16-byte chunk c at
@@ -264,38 +307,24 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         zoff[i] = static_cast<uint32_t>(kGvPk + kGvXb + arow * args.rp2 * 2 + (((b + 4 * i) ^ sw) << 4));
     }
     const uint32_t ahalf = static_cast<uint32_t>(64 * args.rp2 * 2);   // A rows of the second step
+    // this lane's decode scales: a'[block b][rows kb + 2t, +1] and [kb + 2t + 8, +9]
+    const uint32_t soff = static_cast<uint32_t>((b * kGvRows + kb + 2 * t) * 4);
+    const uint32_t sc0 = smem_u32(sc_ring);
 
     // acc[f]: fragment rows = weight columns 8g+2f (g) and 8g+2f+1 (g+8),
     // columns = tokens 2t, 2t+1 (acc2: tokens 8+2t, 9+2t)
     float acc[4][4], acc2[4][4], zacc[2][4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int jj = 0; jj < 4; ++jj)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[j][i] = acc2[j][i] = 0.0f;
+      for (int i = 0; i < 4; ++i) acc[jj][i] = acc2[jj][i] = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 2; ++j)
+    for (int jj = 0; jj < 2; ++jj)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) zacc[j][i] = 0.0f;
-    // this lane's scale row inside a stage: kb + (lane & 15), second step for lanes 16-31
-    const int srow = kb + 64 * (lane >> 4) + (lane & 15);
-    auto scale_at = [&](int j) -> GvScale {
-      GvScale z;
-      z.q = 0u;
-      z.v = 0.0f;
-      const int row = (st0 + j) * kGvRows + srow;
-      if (colok && row < K) z = gemv_scale_load(args.sv, static_cast<int64_t>(row) * bpr + blk);
-      return z;
-    };
-    GvScale sring[kGvAhead];
-#pragma unroll
-    for (int u = 0; u < kGvAhead; ++u) {
-      sring[u].q = 0u;
-      sring[u].v = 0.0f;
-      if (u < nst) sring[u] = scale_at(u);
-    }
+      for (int i = 0; i < 4; ++i) zacc[jj][i] = 0.0f;
 
     // one 16-row step h (0: rows kb.., 1: rows kb+64..) of the stage at `sb`
-    auto step = [&](uint32_t sb, float sc, int h) {
+    auto step = [&](uint32_t sb, uint32_t ss, int h) {
       const uint32_t xs = sb + static_cast<uint32_t>(2048 * h);
       const uint32_t x0 = lds32(xs + xoff0), x1 = lds32(xs + xoff1);
       uint32_t y0 = 0u, y1 = 0u;
@@ -307,19 +336,18 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         const uint32_t ps = sb + static_cast<uint32_t>(8192 * h);
         const uint32_t w0 = lds32(ps + poff0), w8 = lds32(ps + poff0 + 1024);
         const uint32_t w1 = lds32(ps + poff1), w9 = lds32(ps + poff1 + 1024);
-        const float s0 = __shfl_sync(0xFFFFFFFFu, sc, 16 * h + 2 * t);
-        const float s1 = __shfl_sync(0xFFFFFFFFu, sc, 16 * h + 2 * t + 1);
-        const float s2 = __shfl_sync(0xFFFFFFFFu, sc, 16 * h + 2 * t + 8);
-        const float s3 = __shfl_sync(0xFFFFFFFFu, sc, 16 * h + 2 * t + 9);
+        float2 sa, sbv;
+        asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(sa.x), "=f"(sa.y) : "r"(ss + 256 * h));
+        asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(sbv.x), "=f"(sbv.y) : "r"(ss + 256 * h + 32));
         // B fragments: scaled activations of token g (and g + 8)
         const uint32_t bx0 =
-            pack_bf16x2(__uint_as_float(x0 << 16) * s0, __uint_as_float(x0 & 0xFFFF0000u) * s1);
+            pack_bf16x2(__uint_as_float(x0 << 16) * sa.x, __uint_as_float(x0 & 0xFFFF0000u) * sa.y);
         const uint32_t bx1 =
-            pack_bf16x2(__uint_as_float(x1 << 16) * s2, __uint_as_float(x1 & 0xFFFF0000u) * s3);
+            pack_bf16x2(__uint_as_float(x1 << 16) * sbv.x, __uint_as_float(x1 & 0xFFFF0000u) * sbv.y);
         uint32_t by0 = 0u, by1 = 0u;
         if (kM16) {
-          by0 = pack_bf16x2(__uint_as_float(y0 << 16) * s0, __uint_as_float(y0 & 0xFFFF0000u) * s1);
-          by1 = pack_bf16x2(__uint_as_float(y1 << 16) * s2, __uint_as_float(y1 & 0xFFFF0000u) * s3);
+          by0 = pack_bf16x2(__uint_as_float(y0 << 16) * sa.x, __uint_as_float(y0 & 0xFFFF0000u) * sa.y);
+          by1 = pack_bf16x2(__uint_as_float(y1 << 16) * sbv.x, __uint_as_float(y1 & 0xFFFF0000u) * sbv.y);
         }
         // bytes (row k nibble, row k+1 nibble) per column: even and odd columns
         const uint32_t lo_e = (w0 & 0xF0F0F0F0u) | ((w1 >> 4) & 0x0F0F0F0Fu);
@@ -342,33 +370,28 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       }
       // X·A: raw activations (tokens as rows) against A[k][8 jt + g]
       const uint32_t araw[4] = {x0, y0, x1, y1};
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        if (i < nzt) {
-          uint32_t zb0, zb1;
-          ldsm_x2_trans(sb + zoff[i] + ahalf * h, zb0, zb1);
-          mma_bf16_16816(zacc[i], araw, zb0, zb1);
+      if (nzt > 0) {
+        uint32_t zb0, zb1;
+        ldsm_x2_trans(sb + zoff[0] + ahalf * h, zb0, zb1);
+        mma_bf16_16816(zacc[0], araw, zb0, zb1);
+        if (nzt > 1) {
+          ldsm_x2_trans(sb + zoff[1] + ahalf * h, zb0, zb1);
+          mma_bf16_16816(zacc[1], araw, zb0, zb1);
         }
       }
     };
 
     int s = 0;
     uint32_t ph = 0;
-    for (int j0 = 0; j0 < nst && ok; j0 += kGvAhead) {
-#pragma unroll
-      for (int u = 0; u < kGvAhead; ++u) {
-        const int j = j0 + u;
-        if (j >= nst || !ok) break;
-        const float sc = colok ? gemv_scale_value(args.sv, sring[u], off, t8) : 0.0f;
-        if (j + kGvAhead < nst) sring[u] = scale_at(j + kGvAhead);
-        if (!mbar_wait(&full[s], ph)) { ok = false; break; }
-        const uint32_t sb = ring0 + static_cast<uint32_t>(s * args.stage_bytes);
-        step(sb, sc, 0);
-        step(sb, sc, 1);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-        if (++s == args.nstages) { s = 0; ph ^= 1; }
-      }
+    for (int j = 0; j < nst; ++j) {
+      if (!mbar_wait(&full[s], ph) || (colok && !mbar_wait(&sfull[s], ph))) { ok = false; break; }
+      const uint32_t sb = ring0 + static_cast<uint32_t>(s * args.stage_bytes);
+      const uint32_t ss = sc0 + static_cast<uint32_t>(s * kGvScaleWords * 4) + soff;
+      step(sb, ss, 0);
+      step(sb, ss, 1);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (++s == args.nstages) { s = 0; ph ^= 1; }
     }
     // every compute warp is past its last stage (and the producer has seen every
     // copy land) before the ring is reused for the sums
@@ -488,19 +511,67 @@ int pow2_at_least8(int v) {
   return p;
 }
 
+
+
+// Smem bytes besides the stage ring: the pair table (+ alignment slack), the
+// B tile, the decode-scale ring, T8 and the barriers.
+int gemv_fixed_smem(int rp) {
+  return kGvTable + 1024 + 512 * rp + kGvMaxStages * kGvScaleWords * 4 + 256 * 4 + 256;
+}
+
+// Clusters of 1 x S x 1 CTAs (one per SM at this kernel's shared memory)
+// that can be resident at once on this device, S = 1 .. 8; 0 if none.
+struct ClusterFit {
+  int n[9];
+};
+
+ClusterFit cluster_fit(int dev) {
+  static ClusterFit fit[kMaxDevices];
+  static DeviceOnce once;
+  const cudaError_t e = once.run([](int d) {
+    ClusterFit f{};
+    for (int S = 1; S <= 8; ++S) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(1, static_cast<unsigned>(S), 1);
+      cfg.blockDim = dim3(kGvThreads);
+      cfg.dynamicSmemBytes = static_cast<size_t>(kGvSmemMax);
+      cudaLaunchAttribute a[1];
+      a[0].id = cudaLaunchAttributeClusterDimension;
+      a[0].val.clusterDim.x = 1;
+      a[0].val.clusterDim.y = static_cast<unsigned>(S);
+      a[0].val.clusterDim.z = 1;
+      cfg.attrs = a;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, nf4_gemv_kernel<false>, &cfg) != cudaSuccess) n = 0;
+      f.n[S] = n;
+    }
+    (void)cudaGetLastError();
+    fit[d] = f;
+    return cudaSuccess;
+  });
+  ClusterFit none{};
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return none;
+  return fit[dev];
+}
+
 }  // namespace
 
-// K splits: stage-granular ranges, as many as keep every CTA of the launch on
-// its own SM (column groups x splits <= SMs), the fewest that reach the
-// shortest range.  The plan depends only on K, N and the SM count, so the
-// forward and the backward's recompute of Zc use the same splits.
+// K splits: stage-granular ranges.  Among the cluster sizes S whose G
+// clusters (one per 256-column group) are all resident at once (one wave),
+// take the one with the fewest stages per CTA (the fewest S on a tie).  The
+// plan depends only on K, N and the device, so the forward and the backward's
+// recompute of Zc use the same splits.
 GemvPlan gemv_plan(int64_t K, int64_t N, int num_sms) {
   GemvPlan pl;
   pl.G = static_cast<int>((N + kGvCols - 1) / kGvCols);
   const int nk = static_cast<int>((K + kGvRows - 1) / kGvRows);
+  int dev = 0;
+  const ClusterFit fit = cudaGetDevice(&dev) == cudaSuccess ? cluster_fit(dev) : ClusterFit{};
   int bestS = 1, best = nk;
   for (int S = 2; S <= 8 && S <= nk; ++S) {
-    if (static_cast<int64_t>(pl.G) * S > num_sms) break;
+    const int resident = fit.n[S] > 0 ? fit.n[S] : num_sms / S;
+    if (pl.G > resident) continue;
     const int per = (nk + S - 1) / S;
     if (per < best) {
       best = per;
@@ -535,7 +606,7 @@ cudaError_t launch_gemv(int64_t M, int64_t K, int64_t N, int r, const uint16_t* 
   ga.rp = rp;
   ga.rp2 = pow2_at_least8(rp);
   ga.stage_bytes = kGvPk + kGvXb + kGvRows * ga.rp2 * 2;
-  const int fixed = kGvTable + 1024 + 512 * rp + 256 * 4 + 256;
+  const int fixed = gemv_fixed_smem(rp);
   ga.nstages = (kGvSmemMax - fixed) / ga.stage_bytes;
   if (ga.nstages > kGvMaxStages) ga.nstages = kGvMaxStages;
   if (ga.nstages < 2 || ga.nstages * ga.stage_bytes < kGvEpilogueBytes) return cudaErrorInvalidValue;
