@@ -56,7 +56,8 @@ constexpr int kGvMaxStages = 6;
 constexpr int kGvPk = kGvRows * 128;     // packed weights of a stage
 constexpr int kGvXb = 2 * 2048;          // 16 tokens x 128 k bf16, two swizzled 64-k halves
 constexpr int kGvCompute = 16;           // compute warps: 4 column blocks x 4 row slots
-constexpr int kGvWarps = kGvCompute + 2; // + the TMA producer and the scale warp
+constexpr int kGvScaleWarps = 3;         // scale warps, taking stages in turn
+constexpr int kGvWarps = kGvCompute + 1 + kGvScaleWarps;   // + the TMA producer
 constexpr int kGvThreads = kGvWarps * 32;
 constexpr int kGvScaleWords = 4 * kGvRows;   // decode scales of one stage: 4 blocks x 128 rows
 constexpr int kGvSmemMax = 232448;       // 227 KB, the opt-in limit per CTA
@@ -222,12 +223,15 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         if (last_parity[q] < 2 && !mbar_wait(&full[q], last_parity[q])) ok = false;
       if (!zc_only && !mbar_wait(bfull, 0)) ok = false;
     }
-  } else if (warp == kGvCompute + 1) {
-    // ------------------------------- scale warp -------------------------------
-    // a'[row][block] of every stage into sc_ring[stage][block][row]: lane l
-    // decodes block l & 3 for rows (l >> 2) + 8i, i < 16, and keeps the next
-    // stage's raw loads in flight while it decodes this one.
+  } else if (warp > kGvCompute) {
+    // ------------------------------- scale warps ------------------------------
+    // a'[row][block] of every stage into sc_ring[stage][block][row].  Scale
+    // warp q takes the stages q, q + kGvScaleWarps, ...; lane l decodes block
+    // l & 3 for rows (l >> 2) + 8i, i < 16, and keeps its next stage's raw
+    // loads in flight while it decodes this one, kGvScaleWarps stages ahead
+    // of the compute warps.
     pdl_wait();
+    const int sq = warp - kGvCompute - 1;
     if (!zc_only) {
       const int b = lane & 3, rl = lane >> 2;
       const int blk = cg * 4 + b;
@@ -250,15 +254,15 @@ __global__ void __launch_bounds__(kGvThreads, 1)
           }
         }
       };
-      if (nst > 0) load(0);
-      int s = 0;
-      uint32_t ph = 0;
-      for (int j = 0; j < nst; ++j) {
+      if (sq < nst) load(sq);
+      for (int j = sq; j < nst; j += kGvScaleWarps) {
+        const int s = j % args.nstages;
+        const uint32_t ph = static_cast<uint32_t>((j / args.nstages) & 1);
         float a[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
           a[i] = dq ? __fadd_rn(__fmul_rn(t8[qv[i]], fv[i]), off) : fv[i];
-        if (j + 1 < nst) load(j + 1);
+        if (j + kGvScaleWarps < nst) load(j + kGvScaleWarps);
         // the compute warps are done with this slot's previous stage
         if (j >= args.nstages && !mbar_wait(&empty[s], ph ^ 1)) { ok = false; break; }
         float* dst = sc_ring + s * kGvScaleWords + b * kGvRows + rl;
@@ -266,7 +270,6 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         for (int i = 0; i < 16; ++i) dst[8 * i] = a[i];
         __syncwarp();
         if (lane == 0) mbar_arrive(&sfull[s]);
-        if (++s == args.nstages) { s = 0; ph ^= 1; }
       }
     }
   } else {

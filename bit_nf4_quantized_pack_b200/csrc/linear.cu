@@ -267,6 +267,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
 constexpr int kFAStages = 2;         // activation tiles (TMA)
 constexpr int kFBStages = 4;         // decoded weight tiles (decoder warps)
 constexpr int kFBM = 512, kFBN = 128;
+constexpr int kFPairM = 2 * kFBM;     // rows of a pair tile (two CTAs, 512 rows each)
 constexpr int kFAccMax = 4;          // accumulator release barriers
 // TMEM columns per accumulator and accumulators per tile of each direction
 template <bool kBwd> constexpr int kFAccCols = kBwd ? 256 : 128;
@@ -274,11 +275,15 @@ template <bool kBwd> constexpr int kFAccs = kFBM / (kBwd ? 256 : 128);
 constexpr int kFA = kFBM * 128;      // 512 x 64 bf16
 constexpr int kFBoxes = kFBM / 128;  // TMA boxes of 128 rows per activation tile
 constexpr int kFB = kFBN * 128;      // 128 x 64 bf16
-constexpr int kFDecWarps = kFBN / 32;   // one weight-tile row per decoder thread and K-step
+// The two CTAs of a cluster share each decoded weight tile: CTA rank q
+// decodes tile rows [64q, 64q + 64) and copies them into its partner's ring,
+// so each CTA decodes half of every tile.
+constexpr int kFHalfRows = kFBN / 2;
+constexpr int kFDecWarps = kFHalfRows / 32;   // one weight-tile row per decoder thread and K-step
 // Decoder groups of kFDecWarps warps take turns by K-step (group g decodes the
 // steps g, g + kFDecGroups, ...), so each warp has kFDecGroups K-steps of time
 // per row and its loads reach further ahead.
-constexpr int kFDecGroups = 2;
+constexpr int kFDecGroups = 4;
 constexpr int kFDecAll = kFDecWarps * kFDecGroups;
 constexpr int kFEpiWarps = 4;
 constexpr int kFThreads = (2 + kFDecAll + kFEpiWarps) * 32;  // TMA, MMA, decoders, epilogue
@@ -438,8 +443,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
       mbar_init(&empty_a[s], 1);
     }
     for (int s = 0; s < kFBStages; ++s) {
-      mbar_init(&full_b[s], kFDecWarps);
-      mbar_init(&empty_b[s], 1);
+      mbar_init(&full_b[s], kFDecWarps);   // + the partner's half as transaction bytes
+      mbar_init(&empty_b[s], 2);           // both CTAs' MMAs have read the stage
     }
     mbar_init(tfull, 1);
     for (int h = 0; h < kFAccMax; ++h) mbar_init(&tempty[h], kFEpiWarps);
@@ -479,7 +484,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
         return true;
       };
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m0 = (tile % args.m_tiles) * kFBM;
+        const int m0 = (tile % args.m_tiles) * kFPairM + kFBM * static_cast<int>(blockIdx.y);
         const int n0 = (tile / args.m_tiles) * kFBN;
         for (int kk = 0; kk < args.nk && ok; ++kk) {
           uint32_t s;
@@ -566,7 +571,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
           }
           if (!ok) break;
           umma_commit(&empty_a[sa]);
-          umma_commit(&empty_b[sb]);
+          umma_commit_mc(&empty_b[sb], 0x3);   // this CTA's and the partner's
         }
         if (!ok) break;
         // LoRA step
@@ -588,7 +593,12 @@ __global__ void __launch_bounds__(kFThreads, 1)
   } else if (warp < 2 + kFDecAll) {
     // ------------------------------ decoders -------------------------------
     const int grp = (warp - 2) / kFDecWarps;   // this warp's turn among the groups
-    const int R = threadIdx.x - 64 - grp * kFBN;   // weight-tile row 0..kFBN-1
+    const int rank = static_cast<int>(blockIdx.y);
+    const int Rl = threadIdx.x - 64 - grp * kFHalfRows;   // row within this CTA's half
+    const int R = kFHalfRows * rank + Rl;       // weight-tile row 0..kFBN-1
+    // the partner's ring and full barriers, where this warp's 32 rows go too
+    const uint32_t peer = static_cast<uint32_t>(rank ^ 1);
+    const uint32_t wrow0 = static_cast<uint32_t>(R - (Rl & 31)) * 128;   // first row of this warp
     const float off = args.sv.code8 != nullptr ? __ldg(args.sv.offset) : 0.0f;
     const int nsteps = args.nk;                // decoded steps per tile
     bool ok = true;
@@ -624,7 +634,18 @@ __global__ void __launch_bounds__(kFThreads, 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&full_b[s]);
+      if (lane == 0) {
+        // this warp's 32 rows (4 KB) into the partner's stage, then this CTA's
+        // own arrival; the first warp of the group also expects the partner's
+        // two 4 KB copies on this CTA's barrier
+        uint8_t* rows = sB + s * kFB + wrow0;
+        bulk_copy_to_peer(mapa_shared(smem_u32(rows), peer), rows, 32 * 128,
+                          mapa_shared(smem_u32(&full_b[s]), peer));
+        if (Rl < 32)
+          mbar_arrive_expect_tx(&full_b[s], kFHalfRows * 128);
+        else
+          mbar_arrive(&full_b[s]);
+      }
       advance(tile, kk, kFDecGroups, nsteps);
       ib += kFDecGroups;
     };
@@ -656,7 +677,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     uint32_t tc = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tc) {
-      const int m0 = (tile % args.m_tiles) * kFBM;
+      const int m0 = (tile % args.m_tiles) * kFPairM + kFBM * static_cast<int>(blockIdx.y);
       const int n0 = (tile / args.m_tiles) * kFBN;
       if (*abort_flag || !mbar_wait(tfull, tc & 1)) { ok = false; break; }
       tc_fence_after();
@@ -710,6 +731,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  // no CTA leaves while its partner may still copy into it or read from it
+  cluster_sync_all();
   if (*abort_flag && threadIdx.x == 0) raise_status(args.d_status, QLORA_ERR_TIMEOUT);
   if (warp == 1) {
     tc_fence_after();
@@ -952,7 +975,7 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
   fa.Nw = static_cast<int>(N);
   fa.nk = static_cast<int>(K / 64);
   fa.rsteps = rsteps_of(r);
-  fa.m_tiles = static_cast<int>((M + kFBM - 1) / kFBM);
+  fa.m_tiles = static_cast<int>((M + kFPairM - 1) / kFPairM);   // pair tiles of 1024 rows
   fa.n_tiles = static_cast<int>((N + kFBN - 1) / kFBN);
   fa.sv = sv;
   fa.packed = packed;
@@ -961,11 +984,12 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // persistent pairs of CTAs (a cluster of 1 x 2), one pair per two SMs
   const int tiles = fa.m_tiles * fa.n_tiles;
-  const int grid = tiles < sms ? tiles : sms;
+  const int grid = tiles < sms / 2 ? tiles : sms / 2;
   {
     ProfScope prof(kProfFusedFwd, st);
-    e = launch_pdl(fused_nf4_gemm_kernel<false>, dim3(grid), dim3(kFThreads), kFSmem, st, 1, tX, tZc,
+    e = launch_pdl(fused_nf4_gemm_kernel<false>, dim3(grid, 2), dim3(kFThreads), kFSmem, st, 2, tX, tZc,
                    tBl, fa);
   }
   if (e != cudaSuccess) return e;
@@ -1047,7 +1071,7 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   fa.Nw = static_cast<int>(N);
   fa.nk = static_cast<int>(N / 64);
   fa.rsteps = rsteps_of(r);
-  fa.m_tiles = static_cast<int>((M + kFBM - 1) / kFBM);
+  fa.m_tiles = static_cast<int>((M + kFPairM - 1) / kFPairM);   // pair tiles of 1024 rows
   fa.n_tiles = static_cast<int>((K + kFBN - 1) / kFBN);
   fa.sv = sv;
   fa.packed = packed;
@@ -1056,8 +1080,9 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // persistent pairs of CTAs (a cluster of 1 x 2), one pair per two SMs
   const int tiles = fa.m_tiles * fa.n_tiles;
-  const int grid = tiles < sms ? tiles : sms;
+  const int grid = tiles < sms / 2 ? tiles : sms / 2;
 
   // dX on the caller's stream first; dA and dB, which need only dZ, Zc, X and
   // G, on the side stream after dZ, so their CTAs take the SMs that dX's
@@ -1069,7 +1094,7 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   if (ss != nullptr && cudaEventRecord(ss->fork, st) == cudaSuccess) s2 = ss->s;
   {
     ProfScope prof(kProfFusedBwd, st);
-    e = launch_pdl(fused_nf4_gemm_kernel<true>, dim3(grid), dim3(kFThreads), kFSmem, st, 1, tG, tdZa,
+    e = launch_pdl(fused_nf4_gemm_kernel<true>, dim3(grid, 2), dim3(kFThreads), kFSmem, st, 2, tG, tdZa,
                    tAl, fa);
   }
   if (e == cudaSuccess) e = cudaGetLastError();

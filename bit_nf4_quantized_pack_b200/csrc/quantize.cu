@@ -512,6 +512,261 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const T* __restrict__ W
   }
 }
 
+// ---------------------------------------------------------------------------
+// bf16 encoder.  CTA = 8 compute warps + 1 producer warp.  Whole chunks of
+// 8192 elements (128 blocks) stream into a 4-stage ring by 1-D bulk copies;
+// two threads own one 64-block (32 elements each).  A warp copies its 2 KB
+// of a stage into registers and releases the stage at once (per-warp release
+// barrier, no CTA-wide barrier in the loop).  Per pair of elements the fast
+// path is: unpack, t = x/s, the bucket index and t - midpoint in packed f32x2
+// arithmetic, two 8-byte bucket loads from this lane's copy of the table, and
+// code = (codes below the bucket + 1) + (sign of t - midpoint).  The block's
+// absmax is a packed 16-bit integer max of the bf16 magnitudes (bits of |w|;
+// an exponent field of all ones means Inf or NaN).  Blocks whose scale would
+// make 1/s leave the normal range, and blocks with an element within 2^-17 of
+// its stored midpoint, take the exact path (encode32_exact).  Blocks past
+// the last whole chunk are left to the generic per-lane code (encode16).
+// ---------------------------------------------------------------------------
+constexpr int kBfChunkBlocks = 128;
+constexpr int kBfChunkElems = kBfChunkBlocks * kBlock;   // 8192
+constexpr int kBfStages = 3;
+constexpr int kBfComputeWarps = 8;
+constexpr int kBfThreads = (kBfComputeWarps + 1) * 32;
+constexpr size_t kBfSmem = static_cast<size_t>(kBfStages) * kBfChunkElems * 2 + 128;
+
+// Bucket entries for the packed path: per bucket and lane one 8-byte entry
+// (fp32 midpoint or 4.0, then codes below the bucket + 1); lane l reads its
+// own copy at byte 256 * bucket + 8 * l.
+__device__ __forceinline__ void build_buckets8(uint2* tab /*[33][32]*/) {
+  for (int i = threadIdx.x; i < kBuckets * 32; i += blockDim.x) {
+    const int b = i >> 5;
+    const double lo = (b - 16.5) / 16.0, hi = (b - 15.5) / 16.0;
+    int jlo = 0;
+    float mid = 4.0f;
+    for (int j = 0; j < 15; ++j) {
+      const double mj = 0.5 * (static_cast<double>(kNF4c[j]) + static_cast<double>(kNF4c[j + 1]));
+      if (mj < lo)
+        ++jlo;
+      else if (mj < hi)
+        mid = static_cast<float>(mj);
+    }
+    tab[i] = make_uint2(__float_as_uint(mid), static_cast<uint32_t>(jlo + 1));
+  }
+}
+
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+
+// Exact codes of 32 bf16 elements (read again from global memory: this path
+// is rare) for scale s: the careful bucket search with the fp64 check near
+// every midpoint, with s and the elements moved into the normal range of 1/s
+// when needed.
+__device__ __noinline__ void encode32_exact(const uint16_t* __restrict__ gsrc, float s,
+                                            const uint2* tab8, const double* mexact,
+                                            uint32_t* out /*[4]*/) {
+  float sc = 1.0f;
+  if (s < 1.17549435e-38f) sc = 18446744073709551616.0f;
+  if (s > 8.50705917e37f) sc = 5.42101086e-20f;
+  const float s_eff = s * sc;
+  float inv_s;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv_s) : "f"(s_eff));
+  for (int q = 0; q < 4; ++q) out[q] = 0u;
+  for (int e = 0; e < 32; ++e) {
+    const float x = bf16_bits_to_f32(__ldg(gsrc + e)) * sc;
+    const float t = x * inv_s;
+    int b = __float2int_rd(fmaf(t, 16.0f, 16.5f));
+    b = b < 0 ? 0 : (b > kBuckets - 1 ? kBuckets - 1 : b);
+    const uint2 ent = tab8[32 * b];
+    const int jlo = static_cast<int>(ent.y) - 1;
+    const float d = t - __uint_as_float(ent.x);
+    uint32_t code = static_cast<uint32_t>(jlo) + (d > 0.0f ? 1u : 0u);
+    if (fabsf(d) < kNearEps) code = exact_code(x, s_eff, jlo, mexact);
+    // element e: word e / 8, byte (e % 8) / 2, high nibble for even e
+    out[e >> 3] |= code << (8 * ((e & 7) >> 1) + ((e & 1) ? 0 : 4));
+  }
+}
+
+template <bool kDQ>
+__global__ void __launch_bounds__(kBfThreads) nf4_encode_bf16_kernel(
+    const uint16_t* __restrict__ W, int64_t numel, int64_t n1, uint8_t* __restrict__ packed,
+    float* __restrict__ scales, unsigned long long* __restrict__ bins,
+    unsigned int* __restrict__ done_ctas, float* __restrict__ offset_out, int32_t* d_status) {
+  extern __shared__ uint8_t esm_raw[];
+  uint16_t* ring = reinterpret_cast<uint16_t*>((reinterpret_cast<uintptr_t>(esm_raw) + 127) &
+                                               ~static_cast<uintptr_t>(127));
+  __shared__ uint2 tab8[kBuckets * 32];
+  __shared__ uint32_t tab4[kBuckets * 32];
+  __shared__ double mexact[15];
+  __shared__ unsigned long long sbins[kDQ ? 256 : 1];
+  __shared__ uint64_t full_bar[kBfStages];
+  __shared__ uint64_t empty_bar[kBfStages];
+  __shared__ int abort_flag;
+  __shared__ int last_cta;
+  __shared__ int krange[2];
+  pdl_launch_dependents();
+  build_buckets8(tab8);
+  build_buckets(tab4, mexact);
+  if (kDQ)
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = 0ull;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kBfStages; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], kBfComputeWarps);
+    }
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_wait();   // the tables above read no global memory
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t nchunks = numel / kBfChunkElems;
+  const int64_t my_n = nchunks > blockIdx.x ? (nchunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  constexpr uint32_t kChunkBytes = kBfChunkElems * 2;
+  BinCache bc;
+  bool bad = false;
+
+  if (warp == kBfComputeWarps) {
+    // ------------------------------ producer ------------------------------
+    if (lane == 0) {
+      uint32_t last_parity[kBfStages];
+      for (int s = 0; s < kBfStages; ++s) last_parity[s] = 2;
+      for (int64_t j = 0; j < my_n; ++j) {
+        const int s = static_cast<int>(j % kBfStages);
+        const uint32_t ph = static_cast<uint32_t>((j / kBfStages) & 1);
+        if (j >= kBfStages && !mbar_wait(&empty_bar[s], ph ^ 1)) { abort_flag = 1; break; }
+        const int64_t c = blockIdx.x + j * gridDim.x;
+        mbar_arrive_expect_tx(&full_bar[s], kChunkBytes);
+        bulk_load_1d(ring + s * kBfChunkElems, W + c * kBfChunkElems, kChunkBytes, &full_bar[s]);
+        last_parity[s] = ph;
+      }
+      // every copy issued has landed before the CTA can exit
+      for (int s = 0; s < kBfStages; ++s)
+        if (last_parity[s] < 2 && !mbar_wait(&full_bar[s], last_parity[s])) abort_flag = 1;
+    }
+  } else {
+    // ---------------------------- compute warps ----------------------------
+    const int half = lane & 1;
+    const int lb = (threadIdx.x >> 1);                  // block within the chunk
+    const uint32_t tb = smem_u32(tab8) + static_cast<uint32_t>(lane) * 8u - 0x4B000000u * 256u;
+    const uint64_t c16 = f2pack(8388624.0f, 8388624.0f);   // 2^23 + 16 in each lane of the pair
+    const uint64_t k16 = f2pack(16.0f, 16.0f);
+    for (int64_t j = 0; j < my_n; ++j) {
+      const int s = static_cast<int>(j % kBfStages);
+      const uint32_t ph = static_cast<uint32_t>((j / kBfStages) & 1);
+      if (!mbar_wait(&full_bar[s], ph)) { abort_flag = 1; break; }
+      const uint16_t* src = ring + s * kBfChunkElems + lb * kBlock + half * 32;
+      uint32_t w[16];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 q = *reinterpret_cast<const uint4*>(src + 8 * v);
+        w[4 * v] = q.x; w[4 * v + 1] = q.y; w[4 * v + 2] = q.z; w[4 * v + 3] = q.w;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[s]);
+      const int64_t c = blockIdx.x + j * gridDim.x;
+      const int64_t blk = c * kBfChunkBlocks + lb;
+      // absmax: largest bf16 magnitude of the block (the pair of threads)
+      uint32_t m2 = 0u;
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        asm("max.u16x2 %0, %0, %1;" : "+r"(m2) : "r"(w[i] & 0x7FFF7FFFu));
+      uint32_t amb = max(m2 & 0xFFFFu, m2 >> 16);
+      amb = max(amb, __shfl_xor_sync(0xFFFFFFFFu, amb, 1));
+      const bool finite = amb < 0x7F80u;
+      bad |= !finite;
+      const float s_ = (finite && amb != 0u) ? __uint_as_float(amb << 16) : 1.0f;
+      uint32_t out[4] = {0x77777777u, 0x77777777u, 0x77777777u, 0x77777777u};
+      if (finite) {
+        if (s_ < 1.17549435e-38f || s_ > 8.50705917e37f) {
+          encode32_exact(W + blk * kBlock + half * 32, s_, tab8, mexact, out);
+        } else {
+          float inv_s;
+          asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv_s) : "f"(s_));
+          const uint64_t inv2 = f2pack(inv_s, inv_s);
+          float dmin = 1.0f;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) out[q] = 0u;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint64_t x2 = f2pack(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+            uint64_t t2, y2;
+            asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(t2) : "l"(x2), "l"(inv2));
+            asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(y2) : "l"(t2), "l"(k16), "l"(c16));
+            float y0, y1;
+            f2unpack(y2, y0, y1);
+            uint32_t m0, j0, m1, j1;
+            asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(m0), "=r"(j0) : "r"(tb + __float_as_uint(y0) * 256u));
+            asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(m1), "=r"(j1) : "r"(tb + __float_as_uint(y1) * 256u));
+            uint64_t d2;
+            asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d2) : "l"(t2), "l"(f2pack(__uint_as_float(m0), __uint_as_float(m1))));
+            float d0, d1;
+            f2unpack(d2, d0, d1);
+            dmin = fminf(dmin, fminf(fabsf(d0), fabsf(d1)));
+            const uint32_t code0 = j0 + static_cast<uint32_t>(__float_as_int(d0) >> 31);
+            const uint32_t code1 = j1 + static_cast<uint32_t>(__float_as_int(d1) >> 31);
+            // elements 2i (high nibble) and 2i + 1 of byte i % 4 of word i / 4
+            out[i >> 2] += ((code0 << 4) | code1) << (8 * (i & 3));
+          }
+          if (dmin < kNearEps) encode32_exact(W + blk * kBlock + half * 32, s_, tab8, mexact, out);
+        }
+      }
+      *reinterpret_cast<uint4*>(packed + blk * (kBlock / 2) + half * 16) =
+          make_uint4(out[0], out[1], out[2], out[3]);
+      if (half == 0) {
+        scales[blk] = s_;
+        if (kDQ) bc.add(s_, sbins);
+      }
+    }
+  }
+  __syncthreads();
+  if (abort_flag && threadIdx.x == 0) raise_status(d_status, QLORA_ERR_TIMEOUT);
+  // blocks not covered by whole chunks: the generic path, 4 lanes per block
+  {
+    const int sub = lane & 3;
+    const unsigned gmask = 0xFu << (lane & 28);
+    const int64_t first = nchunks * kBfChunkBlocks;
+    const int64_t ngroups = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 2;
+    const bool aligned16 = (reinterpret_cast<uintptr_t>(W) & 15u) == 0;
+    for (int64_t blk = first + ((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 2);
+         blk < n1; blk += ngroups) {
+      const int64_t e0 = blk * kBlock + sub * kLaneElems;
+      const bool full = e0 + kLaneElems <= numel;
+      float x[kLaneElems];
+      load16<uint16_t>(W, e0, numel, full && aligned16, x);
+      encode16<kDQ>(x, blk, e0, sub, gmask, numel, full, tab4, mexact, packed, scales, bc, sbins, bad);
+    }
+  }
+  if (bad) raise_status(d_status, QLORA_ERR_NONFINITE);
+  if (kDQ) {
+    bc.flush(sbins);
+    __syncthreads();
+    for (int i = threadIdx.x; i < 256; i += blockDim.x)
+      if (sbins[i]) atomicAdd(&bins[i], sbins[i]);
+    __syncthreads();
+    if (offset_out == nullptr) return;   // a shard: the caller adds the bins of all shards
+    if (threadIdx.x == 0) {
+      __threadfence();
+      last_cta = atomicAdd(done_ctas, 1u) == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (last_cta) {
+      __threadfence();
+      for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = __ldcg(bins + i);
+      __syncthreads();
+      bins_key_range(sbins, krange);
+      __syncthreads();
+      if (threadIdx.x == 0) *offset_out = __uint_as_float(exact_mean_bits(sbins, krange[0], krange[1], n1));
+    }
+  }
+}
+
 // One warp per group of 256 centred scales (8 per lane, 8 groups per CTA).
 // The 255 distinct codebook values V_0 < ... < V_254 are: -|T|(127..1), 0,
 // |T|(1..127); the code of the nearest value to c/s2 (ties to the smaller
@@ -695,17 +950,19 @@ cudaError_t launch_encoder(const void* W, int dtype, int64_t numel, uint8_t* pac
   cudaError_t e = once.run([&](int dev) {
     const int b16 = static_cast<int>(encode_smem_bytes<uint16_t>());
     const int b32 = static_cast<int>(encode_smem_bytes<float>());
-    const void* fns[4] = {reinterpret_cast<const void*>(nf4_encode_kernel<uint16_t, false>),
-                          reinterpret_cast<const void*>(nf4_encode_kernel<uint16_t, true>),
+    (void)b16;
+    const void* fns[4] = {reinterpret_cast<const void*>(nf4_encode_bf16_kernel<false>),
+                          reinterpret_cast<const void*>(nf4_encode_bf16_kernel<true>),
                           reinterpret_cast<const void*>(nf4_encode_kernel<float, false>),
                           reinterpret_cast<const void*>(nf4_encode_kernel<float, true>)};
     for (int i = 0; i < 4; ++i) {
-      const int bytes = i < 2 ? b16 : b32;
+      const int bytes = i < 2 ? static_cast<int>(kBfSmem) : b32;
+      const int nthr = i < 2 ? kBfThreads : threads;
       cudaError_t r = cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
       if (r != cudaSuccess) return r;
       cudaFuncSetAttribute(fns[i], cudaFuncAttributePreferredSharedMemoryCarveout, 100);
       int nb = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fns[i], threads, bytes) != cudaSuccess || nb < 1)
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fns[i], nthr, bytes) != cudaSuccess || nb < 1)
         nb = 1;
       per_sm[dev][i] = nb;
     }
@@ -719,12 +976,21 @@ cudaError_t launch_encoder(const void* W, int dtype, int64_t numel, uint8_t* pac
   const int64_t cap = static_cast<int64_t>(num_sms) * per_sm[dev][kind];
   const int blocks = static_cast<int>(want < cap ? want : cap);
   if (dtype == QLORA_DTYPE_BF16) {
-    const size_t sm = encode_smem_bytes<uint16_t>();
+    // whole 8192-element chunks per CTA iteration; at least one CTA per SM
+    // for the ragged remainder
     const uint16_t* w16 = static_cast<const uint16_t*>(W);
-    e = dq ? launch_pdl(nf4_encode_kernel<uint16_t, true>, dim3(blocks), dim3(threads), sm, st, 1, w16,
-                        numel, n1, packed, scales, bins, done_ctas, offset_out, d_status)
-           : launch_pdl(nf4_encode_kernel<uint16_t, false>, dim3(blocks), dim3(threads), sm, st, 1, w16,
-                        numel, n1, packed, scales, bins, done_ctas, offset_out, d_status);
+    const int64_t chunks = numel / kBfChunkElems;
+    const int64_t cap16 = static_cast<int64_t>(num_sms) * per_sm[dev][kind];
+    int64_t g16 = chunks < cap16 ? chunks : cap16;
+    const int64_t rem_groups = (n1 - chunks * kBfChunkBlocks + kBfThreads / 4 - 1) / (kBfThreads / 4);
+    if (g16 < rem_groups) g16 = rem_groups < cap16 ? rem_groups : cap16;
+    if (g16 < 1) g16 = 1;
+    e = dq ? launch_pdl(nf4_encode_bf16_kernel<true>, dim3(static_cast<unsigned>(g16)), dim3(kBfThreads),
+                        kBfSmem, st, 1, w16, numel, n1, packed, scales, bins, done_ctas, offset_out,
+                        d_status)
+           : launch_pdl(nf4_encode_bf16_kernel<false>, dim3(static_cast<unsigned>(g16)), dim3(kBfThreads),
+                        kBfSmem, st, 1, w16, numel, n1, packed, scales, bins, done_ctas, offset_out,
+                        d_status);
   } else {
     const size_t sm = encode_smem_bytes<float>();
     const float* w32 = static_cast<const float*>(W);
