@@ -13,7 +13,7 @@ Configurations 1 and 2 are covered in test_gpu_linear.py.  Here:
 * config 5: the 65B MLP slice (8192 x 22016 and 22016 x 8192) with double
   quantization, M = 4096, r = 64: the whole scale state (every code8, s2 and
   the offset), the packed bytes of the sampled blocks, sampled columns of Y
-  and of dX, and all of dA and dB.
+  and of dX, all of dA and dB, and sampled rows of the merged weight.
 
 Every output is held to three bounds (tests/_gpu_util.py): the whole-matrix
 relative Frobenius error of 5e-3, and the worst row's and the worst 128 x 128
@@ -136,5 +136,19 @@ def test_config5_mlp_slice_with_double_quant():
             assert_close(f"{name} dX[:, {k}]", dXs[:, t], G64 @ wrow + dZ @ A64[k])
         assert_close(f"{name} dA", to_np(dA), X64.T @ dZ)
         assert_close(f"{name} dB", to_np(dB), c * (Z.T @ G64))
-        del Y, dX, Zc, wq
+        del Y, dX, Zc
+        # the merged weight at full size, on sampled rows: within one bf16 ulp
+        # of RN_bf16(W_hat + c A B), nearly all exact
+        from oracle.merge import merge_bf16, merge_exact
+        merged = q.merge(wq, At, Bt, c)
+        ms = to_np(merged[torch.from_numpy(ks).to(merged.device)])
+        for t, k in enumerate(ks):
+            wrow = decoded(W[k:k + 1, :], k * bpr + np.arange(bpr)).reshape(1, N)
+            ref = merge_bf16(wrow, A[k:k + 1], B, c)[0]
+            ex = merge_exact(wrow, A[k:k + 1], B, c)[0]
+            _, e = np.frexp(np.maximum(np.abs(ex), 1e-30))
+            diff = np.abs(ms[t] - ref)
+            assert np.all(diff <= np.ldexp(1.0, e - 8)), f"{name} merged row {k}"
+            assert np.mean(diff != 0) < 0.01, f"{name} merged row {k}"
+        del merged, wq
         torch.cuda.empty_cache()

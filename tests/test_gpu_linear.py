@@ -271,7 +271,11 @@ def test_full_size_projection_sampled_rows():
     assert_close("dB", to_np(dB), dBr)
 
 
-MERGE_CASES = [(64, 128, 8, True), (320, 384, 16, False), (256, 576, 64, True), (128, 64, 24, True)]
+# r % 8 == 0 runs the tensor-core tile kernel (128 x 256 tiles; 4160 x 2880
+# gives 396 tiles, several per CTA, with a ragged last row and column tile);
+# other ranks run the mma.sync kernel
+MERGE_CASES = [(64, 128, 8, True), (320, 384, 16, False), (256, 576, 64, True), (128, 64, 24, True),
+               (4160, 2880, 32, True), (1088, 1344, 64, False), (192, 320, 12, True), (64, 192, 3, False)]
 
 
 @pytest.mark.parametrize("K,N,r,dq", MERGE_CASES)
