@@ -38,15 +38,16 @@ __constant__ float kNF4g[32] = {QNF4_TABLE_VALUES, QNF4_INT4_VALUES};
 // (rows of 64 contiguous k') or MN-major (rows of 64 contiguous m'/n'), all
 // with the 128-byte swizzle.  blockIdx.x = 128-row tile, blockIdx.y = split.
 // ===========================================================================
-constexpr int kSkStages = 8;
-constexpr int kSkA = 16384, kSkB = 8192;
+constexpr int kSkW = 2;                  // 64-wide k' boxes per stage
+constexpr int kSkStages = 8 / kSkW;
+constexpr int kSkA = 16384 * kSkW, kSkB = 8192 * kSkW;
 constexpr int kSkThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr size_t kSkSmem = 1024 + kSkStages * (kSkA + kSkB) + 256;
 static_assert(kSkStages * 8 * 3 + 16 <= 256, "skinny barriers and flags fit the tail");
 
 struct SkinnyArgs {
   int Mp;            // rows of D
-  int nk;            // number of 64-wide k' blocks
+  int nk;            // number of k' blocks (64 * kSkW wide)
   int kb_per_split;  // k' blocks per split
   int splits;        // = cluster size along y (<= 8)
   int ncols;         // columns of D that are summed (the rank, or the padded rank)
@@ -114,16 +115,22 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       if (!mbar_wait(&empty[s], ph ^ 1)) { *abort_flag = 1; break; }
       const int kb = kb0 + i;
       mbar_arrive_expect_tx(&full[s], kSkA + kSkB);
-      if (kAmn) {
-        tma_load_2d(sA + s * kSkA, &tmA, &full[s], m0, kb * 64);
-        tma_load_2d(sA + s * kSkA + 8192, &tmA, &full[s], m0 + 64, kb * 64);
-      } else {
-        tma_load_2d(sA + s * kSkA, &tmA, &full[s], kb * 64, m0);
+#pragma unroll
+      for (int w = 0; w < kSkW; ++w) {
+        const int kx = (kb * kSkW + w) * 64;   // boxes past the end arrive as zero fill
+        uint8_t* a = sA + s * kSkA + w * 16384;
+        uint8_t* b = sB + s * kSkB + w * 8192;
+        if (kAmn) {
+          tma_load_2d(a, &tmA, &full[s], m0, kx);
+          tma_load_2d(a + 8192, &tmA, &full[s], m0 + 64, kx);
+        } else {
+          tma_load_2d(a, &tmA, &full[s], kx, m0);
+        }
+        if (kBmn)
+          tma_load_2d(b, &tmB, &full[s], 0, kx);
+        else
+          tma_load_2d(b, &tmB, &full[s], kx, 0);
       }
-      if (kBmn)
-        tma_load_2d(sB + s * kSkB, &tmB, &full[s], 0, kb * 64);
-      else
-        tma_load_2d(sB + s * kSkB, &tmB, &full[s], kb * 64, 0);
     }
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc = idesc_bf16_f32(128, 64, kAmn ? 1 : 0, kBmn ? 1 : 0);
@@ -133,12 +140,15 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       const uint32_t ph = (i / kSkStages) & 1;
       if (!mbar_wait(&full[s], ph)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t a0 = smem_u32(sA + s * kSkA), b0 = smem_u32(sB + s * kSkB);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint64_t ad = kAmn ? smem_desc(a0 + j * 2048, 8192, 1024) : smem_desc(a0 + j * 32, 16, 1024);
-        const uint64_t bd = kBmn ? smem_desc(b0 + j * 2048, 8192, 1024) : smem_desc(b0 + j * 32, 16, 1024);
-        umma_bf16(tmem, ad, bd, idesc, (i > 0 || j > 0) ? 1u : 0u);
+      for (int w = 0; w < kSkW; ++w) {
+        const uint32_t a0 = smem_u32(sA + s * kSkA + w * 16384), b0 = smem_u32(sB + s * kSkB + w * 8192);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint64_t ad = kAmn ? smem_desc(a0 + j * 2048, 8192, 1024) : smem_desc(a0 + j * 32, 16, 1024);
+          const uint64_t bd = kBmn ? smem_desc(b0 + j * 2048, 8192, 1024) : smem_desc(b0 + j * 32, 16, 1024);
+          umma_bf16(tmem, ad, bd, idesc, (i > 0 || w > 0 || j > 0) ? 1u : 0u);
+        }
       }
       umma_commit(&empty[s]);
     }
@@ -808,7 +818,7 @@ cudaError_t run_skinny(const CUtensorMap& ta, const CUtensorMap& tb, int Mp, int
                        cudaStream_t st, int nout = -1, uint16_t* out2 = nullptr, int ld2 = 0) {
   cudaError_t e = set_skinny_attr<kAmn, kBmn>();
   if (e != cudaSuccess) return e;
-  const int nk = (Kp + 63) / 64;
+  const int nk = (Kp + 64 * kSkW - 1) / (64 * kSkW);
   SkinnyArgs a;
   a.Mp = Mp;
   a.nk = nk;

@@ -38,23 +38,59 @@ __constant__ float kNF4c[16] = {QNF4_TABLE_VALUES};
 constexpr int kBuckets = 33;
 constexpr float kNearEps = 7.62939453125e-06f;   // 2^-17
 
-__device__ __forceinline__ void build_buckets(uint32_t* tab /*[33][32]*/, double* mexact) {
-  for (int i = threadIdx.x; i < kBuckets * 32; i += blockDim.x) {
-    const int b = i >> 5;
+// The buckets, formed at compile time: bucket b covers t in
+// [(b - 16.5)/16, (b - 15.5)/16); mid = the fp32 midpoint inside it (4.0 when
+// none), below = number of midpoints below it + 1; and the 15 midpoints in fp64.
+struct BucketTables {
+  float mid[kBuckets];
+  uint32_t below[kBuckets];
+  double mexact[15];
+};
+
+constexpr float kNF4host[16] = {QNF4_TABLE_VALUES};
+
+constexpr BucketTables make_bucket_tables() {
+  BucketTables t{};
+  for (int b = 0; b < kBuckets; ++b) {
     const double lo = (b - 16.5) / 16.0, hi = (b - 15.5) / 16.0;
     int jlo = 0;
     float mid = 4.0f;
     for (int j = 0; j < 15; ++j) {
-      const double mj = 0.5 * (static_cast<double>(kNF4c[j]) + static_cast<double>(kNF4c[j + 1]));
+      const double mj = 0.5 * (static_cast<double>(kNF4host[j]) + static_cast<double>(kNF4host[j + 1]));
       if (mj < lo)
         ++jlo;
       else if (mj < hi)
         mid = static_cast<float>(mj);
     }
-    tab[i] = (__float_as_uint(mid) & ~31u) | static_cast<uint32_t>(jlo + 1);
+    t.mid[b] = mid;
+    t.below[b] = static_cast<uint32_t>(jlo + 1);
   }
-  for (int j = threadIdx.x; j < 15; j += blockDim.x)
-    mexact[j] = 0.5 * (static_cast<double>(kNF4c[j]) + static_cast<double>(kNF4c[j + 1]));
+  for (int j = 0; j < 15; ++j)
+    t.mexact[j] = 0.5 * (static_cast<double>(kNF4host[j]) + static_cast<double>(kNF4host[j + 1]));
+  return t;
+}
+static_assert(make_bucket_tables().below[0] == 1 && make_bucket_tables().below[kBuckets - 1] == 16 &&
+                  make_bucket_tables().mid[16] == 4.0f,
+              "bucket table spot values");
+
+static __constant__ BucketTables kBucketTab = make_bucket_tables();
+
+// Per-lane copies of the bucket entries in shared memory (entry b of lane l at
+// index 32b + l; the 32 threads of a warp read one constant word at a time):
+// tab4 holds the midpoint with its low five bits replaced by `below`, tab8 the
+// pair (midpoint, below); either may be null.
+__device__ __forceinline__ void load_buckets(uint32_t* tab4, uint2* tab8, double* mexact) {
+  for (int i = threadIdx.x; i < kBuckets * 32; i += blockDim.x) {
+    const int b = i >> 5;
+    const uint32_t m = __float_as_uint(kBucketTab.mid[b]), j1 = kBucketTab.below[b];
+    if (tab4 != nullptr) tab4[i] = (m & ~31u) | j1;
+    if (tab8 != nullptr) tab8[i] = make_uint2(m, j1);
+  }
+  for (int j = threadIdx.x; j < 15; j += blockDim.x) mexact[j] = kBucketTab.mexact[j];
+}
+
+__device__ __forceinline__ void build_buckets(uint32_t* tab /*[33][32]*/, double* mexact) {
+  load_buckets(tab, nullptr, mexact);
 }
 
 // Exact decision for one element: code = jlo + (x > s*m_jlo) with the product
@@ -514,7 +550,7 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const T* __restrict__ W
 
 // ---------------------------------------------------------------------------
 // bf16 encoder.  CTA = 8 compute warps + 1 producer warp.  Whole chunks of
-// 8192 elements (128 blocks) stream into a 4-stage ring by 1-D bulk copies;
+// 8192 elements (128 blocks) stream into a 3-stage ring by 1-D bulk copies;
 // two threads own one 64-block (32 elements each).  A warp copies its 2 KB
 // of a stage into registers and releases the stage at once (per-warp release
 // barrier, no CTA-wide barrier in the loop).  Per pair of elements the fast
@@ -536,23 +572,7 @@ constexpr size_t kBfSmem = static_cast<size_t>(kBfStages) * kBfChunkElems * 2 + 
 
 // Bucket entries for the packed path: per bucket and lane one 8-byte entry
 // (fp32 midpoint or 4.0, then codes below the bucket + 1); lane l reads its
-// own copy at byte 256 * bucket + 8 * l.
-__device__ __forceinline__ void build_buckets8(uint2* tab /*[33][32]*/) {
-  for (int i = threadIdx.x; i < kBuckets * 32; i += blockDim.x) {
-    const int b = i >> 5;
-    const double lo = (b - 16.5) / 16.0, hi = (b - 15.5) / 16.0;
-    int jlo = 0;
-    float mid = 4.0f;
-    for (int j = 0; j < 15; ++j) {
-      const double mj = 0.5 * (static_cast<double>(kNF4c[j]) + static_cast<double>(kNF4c[j + 1]));
-      if (mj < lo)
-        ++jlo;
-      else if (mj < hi)
-        mid = static_cast<float>(mj);
-    }
-    tab[i] = make_uint2(__float_as_uint(mid), static_cast<uint32_t>(jlo + 1));
-  }
-}
+// own copy at byte 256 * bucket + 8 * l (load_buckets fills them).
 
 __device__ __forceinline__ uint64_t f2pack(float a, float b) {
   uint64_t r;
@@ -567,16 +587,15 @@ __device__ __forceinline__ void f2unpack(uint64_t v, float& a, float& b) {
 // is rare) for scale s: the careful bucket search with the fp64 check near
 // every midpoint, with s and the elements moved into the normal range of 1/s
 // when needed.
-__device__ __noinline__ void encode32_exact(const uint16_t* __restrict__ gsrc, float s,
-                                            const uint2* tab8, const double* mexact,
-                                            uint32_t* out /*[4]*/) {
+__device__ __noinline__ uint4 encode32_exact(const uint16_t* __restrict__ gsrc, float s,
+                                             const uint2* tab8, const double* mexact) {
   float sc = 1.0f;
   if (s < 1.17549435e-38f) sc = 18446744073709551616.0f;
   if (s > 8.50705917e37f) sc = 5.42101086e-20f;
   const float s_eff = s * sc;
   float inv_s;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv_s) : "f"(s_eff));
-  for (int q = 0; q < 4; ++q) out[q] = 0u;
+  uint32_t out[4] = {0u, 0u, 0u, 0u};
   for (int e = 0; e < 32; ++e) {
     const float x = bf16_bits_to_f32(__ldg(gsrc + e)) * sc;
     const float t = x * inv_s;
@@ -590,6 +609,7 @@ __device__ __noinline__ void encode32_exact(const uint16_t* __restrict__ gsrc, f
     // element e: word e / 8, byte (e % 8) / 2, high nibble for even e
     out[e >> 3] |= code << (8 * ((e & 7) >> 1) + ((e & 1) ? 0 : 4));
   }
+  return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
 template <bool kDQ>
@@ -610,8 +630,7 @@ __global__ void __launch_bounds__(kBfThreads) nf4_encode_bf16_kernel(
   __shared__ int last_cta;
   __shared__ int krange[2];
   pdl_launch_dependents();
-  build_buckets8(tab8);
-  build_buckets(tab4, mexact);
+  load_buckets(tab4, tab8, mexact);
   if (kDQ)
     for (int i = threadIdx.x; i < 256; i += blockDim.x) sbins[i] = 0ull;
   if (threadIdx.x == 0) {
@@ -662,10 +681,15 @@ __global__ void __launch_bounds__(kBfThreads) nf4_encode_bf16_kernel(
       const uint32_t ph = static_cast<uint32_t>((j / kBfStages) & 1);
       if (!mbar_wait(&full_bar[s], ph)) { abort_flag = 1; break; }
       const uint16_t* src = ring + s * kBfChunkElems + lb * kBlock + half * 32;
+      // The thread's 64 bytes are four 16-byte chunks; slot v reads chunk
+      // (v + rot) & 3, so that the 8 lanes of a quarter warp (4 blocks 128
+      // bytes apart) read 8 different bank groups.  Codes are formed in slot
+      // order and the packed words rotated back before the store.
+      const int rot = (lane >> 1) & 3;
       uint32_t w[16];
 #pragma unroll
       for (int v = 0; v < 4; ++v) {
-        const uint4 q = *reinterpret_cast<const uint4*>(src + 8 * v);
+        const uint4 q = *reinterpret_cast<const uint4*>(src + 8 * ((v + rot) & 3));
         w[4 * v] = q.x; w[4 * v + 1] = q.y; w[4 * v + 2] = q.z; w[4 * v + 3] = q.w;
       }
       __syncwarp();
@@ -685,7 +709,8 @@ __global__ void __launch_bounds__(kBfThreads) nf4_encode_bf16_kernel(
       uint32_t out[4] = {0x77777777u, 0x77777777u, 0x77777777u, 0x77777777u};
       if (finite) {
         if (s_ < 1.17549435e-38f || s_ > 8.50705917e37f) {
-          encode32_exact(W + blk * kBlock + half * 32, s_, tab8, mexact, out);
+          const uint4 ex = encode32_exact(W + blk * kBlock + half * 32, s_, tab8, mexact);
+          out[0] = ex.x; out[1] = ex.y; out[2] = ex.z; out[3] = ex.w;
         } else {
           float inv_s;
           asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv_s) : "f"(s_));
@@ -714,7 +739,16 @@ __global__ void __launch_bounds__(kBfThreads) nf4_encode_bf16_kernel(
             // elements 2i (high nibble) and 2i + 1 of byte i % 4 of word i / 4
             out[i >> 2] += ((code0 << 4) | code1) << (8 * (i & 3));
           }
-          if (dmin < kNearEps) encode32_exact(W + blk * kBlock + half * 32, s_, tab8, mexact, out);
+          // word v belongs to chunk (v + rot) & 3: rotate back in two steps
+          uint32_t o1[4];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) o1[v] = (rot & 1) ? out[(v + 3) & 3] : out[v];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) out[v] = (rot & 2) ? o1[(v + 2) & 3] : o1[v];
+          if (dmin < kNearEps) {
+            const uint4 ex = encode32_exact(W + blk * kBlock + half * 32, s_, tab8, mexact);
+            out[0] = ex.x; out[1] = ex.y; out[2] = ex.z; out[3] = ex.w;
+          }
         }
       }
       *reinterpret_cast<uint4*>(packed + blk * (kBlock / 2) + half * 16) =

@@ -239,10 +239,14 @@ qlora_status qlora_nf4_dequantize(const qlora_nf4_state* st, uint16_t* W_hat,
  *   W  : NF4 state of the K×N weight (numel must equal K·N)
  *   Y  : device bf16 M×N output
  *   Zc : device bf16 M×r output, bf16(c·X·A); pass it to qlora_linear_bwd.
- * The product is computed in fp32 on bf16 operands: Ŵ is decoded in tiles
- * to bf16 (each weight within one bf16 ulp of qlora_nf4_dequantize's output)
- * and never written to memory.  M <= 16 runs the HBM-bound GEMV path, larger
- * M the fused tensor-core path.
+ * The product is computed in fp32 on bf16 operands and Ŵ is never written to
+ * memory.  M > 16 runs the fused tensor-core path: Ŵ is decoded in tiles to
+ * bf16, each weight within one bf16 ulp of qlora_nf4_dequantize's output.
+ * M <= 16 runs the HBM-bound GEMV path, which folds each block's decode scale
+ * into the activation instead: every product is bf16(x·a')·bf16(C_j), one
+ * more bf16 rounding (relative <= 2^-9) than x·Ŵ carries; measured on the
+ * 4096 x 11008 and 11008 x 4096 decode shapes, Y is within 3.7e-3 relative
+ * Frobenius error of the fp64 result (the bf16 output rounding included).
  * Shapes: M >= 1, K % 64 == 0, N % 64 == 0, 1 <= r <= 64, else UNSUPPORTED.
  * A rank that is not a multiple of 8 is zero-padded to the next multiple of 8
  * inside the workspace (A, and the copy of Zc the tensor-core path reads), so
