@@ -46,6 +46,7 @@ _PS = C.POINTER(NF4StateC)
 SIGNATURES = {
     "qlora_abi_version": (_I32, []),
     "qlora_status_str": (C.c_char_p, [_I32]),
+    "qlora_last_cuda_error": (C.c_char_p, []),
     "qlora_nf4_n1": (_I64, [_I64]),
     "qlora_nf4_n2": (_I64, [_I64]),
     "qlora_status_sync": (_I32, [_VP, _VP, C.POINTER(C.c_int32)]),
@@ -96,7 +97,10 @@ lib = _load()
 class QLoRAError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {lib.qlora_status_str(status).decode()} (status {status})")
+        msg = f"{where}: {lib.qlora_status_str(status).decode()} (status {status})"
+        if status == QLORA_ERR_CUDA:
+            msg += f": {lib.qlora_last_cuda_error().decode()}"
+        super().__init__(msg)
 
 
 def check(status: int, where: str) -> None:

@@ -29,7 +29,14 @@ int sm_count() {
   return cached[dev];
 }
 
-qlora_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
+// The CUDA error behind this thread's latest QLORA_ERR_CUDA (qlora_last_cuda_error).
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+qlora_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return QLORA_OK;
+  t_last_cuda_error = e;
+  return QLORA_ERR_CUDA;
+}
 
 // An NVTX range around each compute entry point, so that a timeline tool
 // shows the library's calls (header-only NVTX: no cost without a tool).
@@ -86,6 +93,10 @@ extern "C" {
 
 int32_t qlora_abi_version(void) { return QLORA_NF4_ABI_VERSION; }
 
+const char* qlora_last_cuda_error(void) {
+  return t_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(t_last_cuda_error);
+}
+
 const char* qlora_status_str(qlora_status s) {
   switch (s) {
     case QLORA_OK: return "ok";
@@ -106,9 +117,10 @@ qlora_status qlora_status_sync(const int32_t* d_status, qlora_stream_t stream, i
   if (!d_status || !h_mask) return QLORA_ERR_INVALID_ARG;
   int32_t m = 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(&m, d_status, sizeof(m), cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return QLORA_ERR_CUDA;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return QLORA_ERR_CUDA;
+  qlora_status r = cuda_status(cudaMemcpyAsync(&m, d_status, sizeof(m), cudaMemcpyDeviceToHost, s));
+  if (r != QLORA_OK) return r;
+  r = cuda_status(cudaStreamSynchronize(s));
+  if (r != QLORA_OK) return r;
   *h_mask = m;
   for (int code = 1; code < 31; ++code)
     if (m & (1 << code)) return code;

@@ -234,73 +234,70 @@ __global__ void __launch_bounds__(kSkThreads, 1)
 // ===========================================================================
 // Fused NF4-decode GEMM (forward: kBwd = false, input gradient: kBwd = true)
 //
-// Output tile 512 (rows of X or G) x 128, K-step 64.  Each decoded weight tile
-// (128 x 64 bf16) is used by all 512 rows, which halves the decode work per
-// FLOP against a 256 x 256 tile.  The two directions issue it differently:
-//   forward   four tcgen05.mma of M = 128 (rows m0+128h .., h = 0..3) x
-//             N = 128 (the decoded tile as the MN-major B operand) per 16-wide
-//             K slice;
-//   backward  transposed: the decoded tile is the K-major A operand (M = 128
-//             output columns) and the dY rows the B operand, two products of
-//             N = 256 (rows m0+256h .., h = 0, 1) per K slice.  The tensor core
-//             then reads 96 KB of operands per K-step from shared memory
-//             instead of 128 KB (the weight tile is read twice, not four
-//             times); measured 9% faster for dX.  The same transposition of
-//             the forward measured slower than the untransposed form: 3% with
-//             its MN-major tile as the A operand, 6% with a K-major tile
-//             written by stmatrix .trans (two block scales per thread and
-//             K-step), so the forward keeps it.
+// Persistent pairs of CTAs on neighbouring SMs (a 1 x 2 thread-block cluster)
+// run CTA-pair tensor-core products (tcgen05.mma.cta_group::2, M = 256,
+// N = 256, K = 16), issued by CTA rank 0 for both: the A operand is split by
+// rows (128 per CTA) and the B operand by columns (128 per CTA), each half in
+// its own CTA's shared memory, and each CTA's TMEM receives its 128 rows of D
+// over all 256 columns.  So each CTA stages only half of each operand, and
+// the tensor core reads 8 KB of shared memory per CTA and 16-wide K slice
+// for a 128 x 256 x 16 product per SM.
+//   forward   pair tile 512 rows x 256 columns; CTA q holds rows
+//             m0 + 256q + [0, 256) (slices h = 0, 1 of 128 rows, the K-major
+//             A operand of accumulator h) and decodes columns n0 + 128q + [0,
+//             128) of every weight K-step (the MN-major B operand);
+//   backward  transposed: pair tile 256 output columns x 512 dY rows; CTA q
+//             decodes the weight rows n0 + 128q + [0, 128) (the K-major A
+//             operand: its output columns) and holds dY rows m0 + 256h + 128q +
+//             [0, 128) (its half of the B operand of accumulator h = 0, 1).
+// TMEM: two accumulators of 128 lanes x 256 fp32 columns per CTA (all 512).
 //
-// Shared memory holds two rings.  Activation tiles (512 x 64 bf16, K-major,
-// four TMA boxes) have 2 stages.  Decoded weight tiles have 4 stages; decoder
-// warps write them as 128 rows of 128 bytes, each row one NF4 block of 64
-// consecutive weights (row R at R*128, 16-byte chunk c at (c ^ (R & 7))*16,
-// the 128-byte swizzle pattern):
-//   forward   row R = 64*nb + k: weights (k0+k, n0+64nb .. +63) — an MN-major
-//             operand (atoms of 8 k-rows x 64 n; 8 KB between n-atoms);
-//   backward  row R: weights (n0+R, k0 .. k0+63) of W, i.e. row R of Ŵᵀ's
-//             K-major operand.
+// Shared memory holds two rings per CTA.  Activation tiles (256 x 64 bf16,
+// K-major, two TMA boxes of 128 rows) have 4 stages; TMA loads of both CTAs
+// complete on CTA 0's barrier (the cta_group::2 form of the copy), which CTA
+// 0's producer arms with both CTAs' bytes.  Decoded weight tiles have 4
+// stages; decoder warps write them as 128 rows of 128 bytes, each row one NF4
+// block of 64 consecutive weights (row R at R*128, 16-byte chunk c at
+// (c ^ (R & 7))*16, the 128-byte swizzle pattern):
+//   forward   row R = 64*nb + k: weights (k0+k, n0+128q+64nb .. +63) — an
+//             MN-major operand (atoms of 8 k-rows x 64 n; 8 KB between
+//             n-atoms);
+//   backward  row R: weights (n0+128q+R, k0 .. k0+63) of W, i.e. row R of
+//             Ŵᵀ's K-major operand.
 // Each decoder thread owns one row and loads its 32 packed bytes and its
-// block scale straight from global memory three K-steps ahead.
+// block scale straight from global memory K-steps ahead; both CTAs' decoder
+// warps arrive on CTA 0's barrier of the stage.  The MMA's commit releases
+// the stages and signals the accumulators in both CTAs (multicast), and both
+// CTAs' epilogue warps release an accumulator on CTA 0's barrier.
 //
 // After the last K-step of a tile, the LoRA step takes two activation stages:
 // Zc (or dZ) as the activation tile and B (or A) as the weight tile, both by
 // TMA with the rank padded to a multiple of 16 by TMA's zero fill; the decoder
-// warps skip it.  TMEM holds the accumulators in all 512 columns: forward four
-// of 128 lanes (rows) x 128 columns, backward two of 128 lanes (output
-// columns) x 256 columns (rows).  The epilogue releases each as soon as it has
-// read it, so the next tile's first MMAs into the first accumulators overlap
-// the drain of the last.  In the backward a warp's TMEM load gives each lane
-// one output column over 32 consecutive rows, so every store instruction
-// writes 32 adjacent bf16 of one output row.
+// warps skip it.  The epilogue releases each accumulator as soon as it has
+// read it, so the next tile's first MMAs overlap the drain of the last.  In
+// the backward a warp's TMEM load gives each lane one output column over 32
+// consecutive rows, so every store instruction writes 32 adjacent bf16 of one
+// output row.
 // ===========================================================================
-constexpr int kFAStages = 2;         // activation tiles (TMA)
-constexpr int kFBStages = 4;         // decoded weight tiles (decoder warps)
-constexpr int kFBM = 512, kFBN = 128;
-constexpr int kFPairM = 2 * kFBM;     // rows of a pair tile (two CTAs, 512 rows each)
-constexpr int kFAccMax = 4;          // accumulator release barriers
-// TMEM columns per accumulator and accumulators per tile of each direction
-template <bool kBwd> constexpr int kFAccCols = kBwd ? 256 : 128;
-template <bool kBwd> constexpr int kFAccs = kFBM / (kBwd ? 256 : 128);
-constexpr int kFA = kFBM * 128;      // 512 x 64 bf16
-constexpr int kFBoxes = kFBM / 128;  // TMA boxes of 128 rows per activation tile
-constexpr int kFB = kFBN * 128;      // 128 x 64 bf16
-// The two CTAs of a cluster share each decoded weight tile: CTA rank q
-// decodes tile rows [64q, 64q + 64) and copies them into its partner's ring,
-// so each CTA decodes half of every tile.
-constexpr int kFHalfRows = kFBN / 2;
-constexpr int kFDecWarps = kFHalfRows / 32;   // one weight-tile row per decoder thread and K-step
+constexpr int kFAStages = 4;          // activation tiles (TMA)
+constexpr int kFBStages = 4;          // decoded weight tiles (decoder warps)
+constexpr int kFBN = 128;             // decoded rows per CTA and K-step
+constexpr int kFSlices = 2;           // 128-row activation slices per CTA = accumulators
+constexpr int kFAccCols = 256;        // TMEM columns per accumulator (the pair MMA's N)
+constexpr int kFPairRows = 512;       // activation rows of a pair tile
+constexpr int kFPairCols = 256;       // output columns of a pair tile
+constexpr int kFA = kFSlices * 128 * 128;   // 256 x 64 bf16
+constexpr int kFB = kFBN * 128;             // 128 x 64 bf16
+constexpr int kFDecWarps = kFBN / 32;       // one weight-tile row per decoder thread and K-step
 // Decoder groups of kFDecWarps warps take turns by K-step (group g decodes the
 // steps g, g + kFDecGroups, ...), so each warp has kFDecGroups K-steps of time
 // per row and its loads reach further ahead.
-constexpr int kFDecGroups = 4;
+constexpr int kFDecGroups = 2;
 constexpr int kFDecAll = kFDecWarps * kFDecGroups;
 constexpr int kFEpiWarps = 4;
 constexpr int kFThreads = (2 + kFDecAll + kFEpiWarps) * 32;  // TMA, MMA, decoders, epilogue
 constexpr size_t kFSmem = 1024 + kFAStages * kFA + kFBStages * kFB + 1024 + 512;
-static_assert(kFAccs<false> * kFAccCols<false> <= 512 && kFAccs<true> * kFAccCols<true> <= 512 &&
-                  kFAccs<false> <= kFAccMax && kFBN == 128,
-              "accumulators fit TMEM");
+static_assert(kFSlices * kFAccCols == 512 && kFBN == 128, "accumulators fill TMEM");
 static_assert(kFSmem <= 232448, "fused kernel shared memory");
 
 struct FusedArgs {
@@ -369,8 +366,9 @@ struct RowFetch {
   bool valid;     // row inside the weight; false also for LoRA steps
 };
 
+// Row Rg (0 .. kFPairCols-1) of the pair's decoded tile at K-step kk.
 template <bool kBwd>
-__device__ __forceinline__ RowFetch fetch_row(const FusedArgs& a, int tile, int kk, int R,
+__device__ __forceinline__ RowFetch fetch_row(const FusedArgs& a, int tile, int kk, int Rg,
                                               int num_tiles) {
   RowFetch f;
   f.p0 = make_uint4(0, 0, 0, 0);
@@ -380,20 +378,20 @@ __device__ __forceinline__ RowFetch fetch_row(const FusedArgs& a, int tile, int 
   f.s2v = 1.0f;
   f.valid = false;
   if (tile >= num_tiles || kk >= a.nk) return f;
-  const int n0 = (tile / a.m_tiles) * kFBN;
+  const int n0 = (tile / a.m_tiles) * kFPairCols;
   const int64_t rowbytes = a.Nw / 2;
   const int64_t bpr = a.Nw / 64;
   int64_t blk;
   const uint8_t* src;
   if (!kBwd) {
-    const int nb = R >> 6, kr = R & 63;
+    const int nb = Rg >> 6, kr = Rg & 63;
     if (n0 + nb * 64 >= a.Nout) return f;
     const int64_t k = static_cast<int64_t>(kk) * 64 + kr;
     src = a.packed + k * rowbytes + n0 / 2 + nb * 32;
     blk = k * bpr + n0 / 64 + nb;
   } else {
-    if (n0 + R >= a.Nout) return f;
-    const int64_t kw = n0 + R;
+    if (n0 + Rg >= a.Nout) return f;
+    const int64_t kw = n0 + Rg;
     src = a.packed + kw * rowbytes + kk * 32;
     blk = kw * bpr + kk;
   }
@@ -415,12 +413,13 @@ __device__ __forceinline__ RowFetch fetch_row(const FusedArgs& a, int tile, int 
   return f;
 }
 
-// Advance an iteration cursor (tile, kk) by `n` steps of nsteps per tile.
-__device__ __forceinline__ void advance(int& tile, int& kk, int n, int nsteps) {
+// Advance an iteration cursor (tile, kk) by `n` steps of nsteps per tile;
+// consecutive tiles of one pair are `stride` apart.
+__device__ __forceinline__ void advance(int& tile, int& kk, int n, int nsteps, int stride) {
   kk += n;
   while (kk >= nsteps) {
     kk -= nsteps;
-    tile += gridDim.x;
+    tile += stride;
   }
 }
 
@@ -440,34 +439,41 @@ __global__ void __launch_bounds__(kFThreads, 1)
   uint64_t* full_b = empty_a + kFAStages;
   uint64_t* empty_b = full_b + kFBStages;
   uint64_t* tfull = empty_b + kFBStages;
-  uint64_t* tempty = tfull + 1;   // [kFAccMax]: one per accumulator
-  uint64_t* drain = tempty + kFAccMax;
+  uint64_t* tempty = tfull + 1;   // [kFSlices]: one per accumulator
+  uint64_t* drain = tempty + kFSlices;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the pair is the cluster (2 x 1 x 1): rank 0 issues the MMAs
+  const int rank = static_cast<int>(blockIdx.x & 1);
+  const int pair = static_cast<int>(blockIdx.x >> 1), npairs = static_cast<int>(gridDim.x >> 1);
   if (args.sv.code8 != nullptr) build_t8(t8);
   if (threadIdx.x == 0) {
+    // Only CTA 0's full_a, full_b and tempty are waited on; every CTA's
+    // empty_a, empty_b and tfull receive the pair MMA's multicast commits.
     for (int s = 0; s < kFAStages; ++s) {
-      mbar_init(&full_a[s], 1);
+      mbar_init(&full_a[s], 1);            // CTA 0's producer, plus both CTAs' bytes
       mbar_init(&empty_a[s], 1);
     }
     for (int s = 0; s < kFBStages; ++s) {
-      mbar_init(&full_b[s], kFDecWarps);   // + the partner's half as transaction bytes
-      mbar_init(&empty_b[s], 2);           // both CTAs' MMAs have read the stage
+      mbar_init(&full_b[s], 2 * kFDecWarps);   // both CTAs' decoder warps
+      mbar_init(&empty_b[s], 1);
     }
     mbar_init(tfull, 1);
-    for (int h = 0; h < kFAccMax; ++h) mbar_init(&tempty[h], kFEpiWarps);
+    for (int h = 0; h < kFSlices; ++h) mbar_init(&tempty[h], 2 * kFEpiWarps);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, 512);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_holder, 512);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  // the peer's barriers are initialised before any arrival reaches them
+  cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const int num_tiles = args.m_tiles * args.n_tiles;
@@ -485,61 +491,66 @@ __global__ void __launch_bounds__(kFThreads, 1)
 #pragma unroll
       for (int s = 0; s < kFAStages; ++s) last_parity[s] = 2;
       bool ok = true;
-      auto take = [&](uint32_t& s_out) -> bool {
+      // take the next slot; CTA 0 arms its full barrier with both CTAs' bytes
+      auto take = [&](uint32_t& s_out, uint32_t bytes) -> bool {
         const uint32_t s = ia % kFAStages, ph = (ia / kFAStages) & 1;
         if (*abort_flag || !mbar_wait(&empty_a[s], ph ^ 1)) return false;
+        if (rank == 0) mbar_arrive_expect_tx(&full_a[s], 2 * bytes);
         last_parity[s] = ph;
         s_out = s;
         ++ia;
         return true;
       };
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m0 = (tile % args.m_tiles) * kFPairM + kFBM * static_cast<int>(blockIdx.y);
-        const int n0 = (tile / args.m_tiles) * kFBN;
+      auto bar0 = [&](uint32_t s) -> uint32_t { return mapa_shared(smem_u32(&full_a[s]), 0); };
+      // the activation rows of slice h of this CTA
+      auto act_row = [&](int m0, int h) -> int {
+        return kBwd ? m0 + 256 * h + 128 * rank : m0 + 256 * rank + 128 * h;
+      };
+      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+        const int m0 = (tile % args.m_tiles) * kFPairRows;
+        const int n0 = (tile / args.m_tiles) * kFPairCols;
         for (int kk = 0; kk < args.nk && ok; ++kk) {
           uint32_t s;
-          if (!take(s)) { ok = false; break; }
+          if (!take(s, kFA)) { ok = false; break; }
           uint8_t* a = sA + s * kFA;
-          mbar_arrive_expect_tx(&full_a[s], kFA);
 #pragma unroll
-          for (int h = 0; h < kFBoxes; ++h)
-            tma_load_2d(a + h * 16384, &tmAct, &full_a[s], kk * 64, m0 + h * 128);
+          for (int h = 0; h < kFSlices; ++h)
+            tma_load_2d_pair(a + h * 16384, &tmAct, bar0(s), kk * 64, act_row(m0, h));
         }
         if (!ok) break;
         // LoRA step: Zc / dZ into one stage, B / A into the next
         uint32_t s1, s2;
-        if (!take(s1)) { ok = false; break; }
+        if (!take(s1, kFA)) { ok = false; break; }
         uint8_t* a = sA + s1 * kFA;
-        mbar_arrive_expect_tx(&full_a[s1], kFA);
 #pragma unroll
-        for (int h = 0; h < kFBoxes; ++h)
-          tma_load_2d(a + h * 16384, &tmLA, &full_a[s1], 0, m0 + h * 128);
-        if (!take(s2)) { ok = false; break; }
+        for (int h = 0; h < kFSlices; ++h)
+          tma_load_2d_pair(a + h * 16384, &tmLA, bar0(s1), 0, act_row(m0, h));
+        if (!take(s2, kFB)) { ok = false; break; }
         uint8_t* b = sA + s2 * kFA;
-        mbar_arrive_expect_tx(&full_a[s2], kFB);
         if (!kBwd) {
+          // B's columns of this CTA's half, two 64-column boxes (MN-major)
 #pragma unroll
           for (int nb = 0; nb < kFBN / 64; ++nb)
-            tma_load_2d(b + nb * 8192, &tmLB, &full_a[s2], n0 + nb * 64, 0);
+            tma_load_2d_pair(b + nb * 8192, &tmLB, bar0(s2), n0 + 128 * rank + nb * 64, 0);
         } else {
-          tma_load_2d(b, &tmLB, &full_a[s2], 0, n0);
+          // A's rows of this CTA's output columns (K-major)
+          tma_load_2d_pair(b, &tmLB, bar0(s2), 0, n0 + 128 * rank);
         }
       }
-      if (!ok) {
-        *abort_flag = 1;
-        // let copies already in flight land before the CTA can exit
+      if (!ok) *abort_flag = 1;
+      // CTA 0: let copies already in flight (its own and the peer's) land
+      // before either CTA can exit
+      if (rank == 0)
         for (int s = 0; s < kFAStages; ++s)
           if (last_parity[s] < 2) (void)mbar_wait(&full_a[s], last_parity[s]);
-      }
     }
   } else if (warp == 1) {
-    // ------------------------------ MMA issuer -----------------------------
-    if (lane == 0) {
+    // ------------------------- MMA issuer (CTA 0 only) ----------------------
+    if (lane == 0 && rank == 0) {
       // forward: D[m][n] += act[m][k] * Ŵtile[k][n] (tile MN-major, as B);
       // backward: D[n][m] += Ŵtile[n][k] * dY[m][k] (tile K-major, as A)
-      constexpr int kAcc = kFAccs<kBwd>, kCols = kFAccCols<kBwd>;
-      constexpr uint32_t idesc =
-          kBwd ? idesc_bf16_f32(kFBN, kCols, 0, 0) : idesc_bf16_f32(128, kFBN, 0, 1);
+      constexpr uint32_t idesc = kBwd ? idesc_bf16_f32(256, kFAccCols, 0, 0)
+                                      : idesc_bf16_f32(256, kFAccCols, 0, 1);
       uint32_t ia = 0, ib = 0, tc = 0;
       bool ok = true;
       auto wait_a = [&](uint32_t& s) -> bool {
@@ -548,18 +559,17 @@ __global__ void __launch_bounds__(kFThreads, 1)
         ++ia;
         return !*abort_flag && mbar_wait(&full_a[s], ph);
       };
-      auto wdesc = [&](uint32_t b0, int j) -> uint64_t {
-        return kBwd ? smem_desc(b0 + j * 32, 16, 1024) : smem_desc(b0 + j * 2048, 8192, 1024);
-      };
-      // one 16-wide K slice j of accumulator h (activation rows h*kCols ..)
-      auto mma = [&](int h, uint32_t a0, uint32_t b0, int j, uint32_t accum) {
-        const uint64_t adesc = smem_desc(a0 + h * (kCols * 128) + j * 32, 16, 1024);
+      // one 16-wide K slice j of accumulator h: `w0` the weight operand
+      // (decoded tile, or B / A in the LoRA step), `a0` the activation stage
+      auto mma = [&](int h, uint32_t a0, uint32_t w0, int j, uint32_t accum) {
+        const uint64_t adesc = smem_desc(a0 + h * 16384 + j * 32, 16, 1024);
         if (kBwd)
-          umma_bf16(tmem + h * kCols, wdesc(b0, j), adesc, idesc, accum);
+          umma_bf16_pair(tmem + h * kFAccCols, smem_desc(w0 + j * 32, 16, 1024), adesc, idesc, accum);
         else
-          umma_bf16(tmem + h * kCols, adesc, wdesc(b0, j), idesc, accum);
+          umma_bf16_pair(tmem + h * kFAccCols, adesc, smem_desc(w0 + j * 2048, 8192, 1024), idesc,
+                         accum);
       };
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tc) {
+      for (int tile = pair; tile < num_tiles && ok; tile += npairs, ++tc) {
         const uint32_t tph = (tc & 1) ^ 1;       // parity of the previous tile's release
         for (int kk = 0; kk < args.nk; ++kk) {
           uint32_t sa;
@@ -571,7 +581,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
           const uint32_t a0 = smem_u32(sA + sa * kFA), b0 = smem_u32(sB + sb * kFB);
           const uint32_t acc = kk > 0 ? 1u : 0u;
 #pragma unroll
-          for (int h = 0; h < kAcc; ++h) {
+          for (int h = 0; h < kFSlices; ++h) {
             if (kk == 0) {   // first K-step of a tile: wait until this accumulator is drained
               if (*abort_flag || !mbar_wait(&tempty[h], tph)) { ok = false; break; }
               tc_fence_after();
@@ -580,40 +590,36 @@ __global__ void __launch_bounds__(kFThreads, 1)
             for (int j = 0; j < 4; ++j) mma(h, a0, b0, j, (acc || j > 0) ? 1u : 0u);
           }
           if (!ok) break;
-          umma_commit(&empty_a[sa]);
-          umma_commit_mc(&empty_b[sb], 0x3);   // this CTA's and the partner's
+          umma_commit_pair_mc(&empty_a[sa], 0x3);
+          umma_commit_pair_mc(&empty_b[sb], 0x3);
         }
         if (!ok) break;
         // LoRA step
         uint32_t s1, s2;
         if (!wait_a(s1) || !wait_a(s2)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sA + s1 * kFA), b0 = smem_u32(sA + s2 * kFA);
+        const uint32_t a0 = smem_u32(sA + s1 * kFA), w0 = smem_u32(sA + s2 * kFA);
         for (int j = 0; j < args.rsteps; ++j)
 #pragma unroll
-          for (int h = 0; h < kAcc; ++h) mma(h, a0, b0, j, 1u);
-        umma_commit(&empty_a[s1]);
-        umma_commit(&empty_a[s2]);
-        umma_commit(tfull);
+          for (int h = 0; h < kFSlices; ++h) mma(h, a0, w0, j, 1u);
+        umma_commit_pair_mc(&empty_a[s1], 0x3);
+        umma_commit_pair_mc(&empty_a[s2], 0x3);
+        umma_commit_pair_mc(tfull, 0x3);
       }
       if (!ok) *abort_flag = 1;
-      umma_commit(drain);
+      umma_commit_pair_mc(drain, 0x1);
       (void)mbar_wait(drain, 0);
     }
   } else if (warp < 2 + kFDecAll) {
     // ------------------------------ decoders -------------------------------
     const int grp = (warp - 2) / kFDecWarps;   // this warp's turn among the groups
-    const int rank = static_cast<int>(blockIdx.y);
-    const int Rl = threadIdx.x - 64 - grp * kFHalfRows;   // row within this CTA's half
-    const int R = kFHalfRows * rank + Rl;       // weight-tile row 0..kFBN-1
-    // the partner's ring and full barriers, where this warp's 32 rows go too
-    const uint32_t peer = static_cast<uint32_t>(rank ^ 1);
-    const uint32_t wrow0 = static_cast<uint32_t>(R - (Rl & 31)) * 128;   // first row of this warp
+    const int R = threadIdx.x - 64 - grp * kFBN;   // row of this CTA's decoded tile
+    const int Rg = kFBN * rank + R;                // row of the pair's decoded tile
     const float off = args.sv.code8 != nullptr ? __ldg(args.sv.offset) : 0.0f;
     const int nsteps = args.nk;                // decoded steps per tile
     bool ok = true;
-    int tile = blockIdx.x, kk = 0;             // the step being decoded
-    advance(tile, kk, grp, nsteps);
+    int tile = pair, kk = 0;                   // the step being decoded
+    advance(tile, kk, grp, nsteps, npairs);
     int ptile = tile, pkk = kk;                // the step being prefetched
     uint32_t ib = static_cast<uint32_t>(grp);
     // One K-step: wait for a free weight stage, decode this thread's row.
@@ -642,43 +648,34 @@ __global__ void __launch_bounds__(kFThreads, 1)
           *reinterpret_cast<uint4*>(brow + ((static_cast<uint32_t>(c) ^ sw) << 4)) =
               make_uint4(0, 0, 0, 0);
       }
+      // the rows are visible to the tensor core (async proxy), then CTA 0's
+      // barrier of the stage counts this warp
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
-        // this warp's 32 rows (4 KB) into the partner's stage, then this CTA's
-        // own arrival; the first warp of the group also expects the partner's
-        // two 4 KB copies on this CTA's barrier
-        uint8_t* rows = sB + s * kFB + wrow0;
-        bulk_copy_to_peer(mapa_shared(smem_u32(rows), peer), rows, 32 * 128,
-                          mapa_shared(smem_u32(&full_b[s]), peer));
-        if (Rl < 32)
-          mbar_arrive_expect_tx(&full_b[s], kFHalfRows * 128);
-        else
-          mbar_arrive(&full_b[s]);
-      }
-      advance(tile, kk, kFDecGroups, nsteps);
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&full_b[s]), 0));
+      advance(tile, kk, kFDecGroups, nsteps, npairs);
       ib += kFDecGroups;
     };
     // Three prefetch slots consumed and refilled in place (no register moves
     // that would wait on loads still in flight).
-    RowFetch q0 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
-    advance(ptile, pkk, kFDecGroups, nsteps);
-    RowFetch q1 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
-    advance(ptile, pkk, kFDecGroups, nsteps);
-    RowFetch q2 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
-    advance(ptile, pkk, kFDecGroups, nsteps);
+    RowFetch q0 = fetch_row<kBwd>(args, ptile, pkk, Rg, num_tiles);
+    advance(ptile, pkk, kFDecGroups, nsteps, npairs);
+    RowFetch q1 = fetch_row<kBwd>(args, ptile, pkk, Rg, num_tiles);
+    advance(ptile, pkk, kFDecGroups, nsteps, npairs);
+    RowFetch q2 = fetch_row<kBwd>(args, ptile, pkk, Rg, num_tiles);
+    advance(ptile, pkk, kFDecGroups, nsteps, npairs);
     while (ok && tile < num_tiles) {
       step(q0);
-      q0 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
-      advance(ptile, pkk, kFDecGroups, nsteps);
+      q0 = fetch_row<kBwd>(args, ptile, pkk, Rg, num_tiles);
+      advance(ptile, pkk, kFDecGroups, nsteps, npairs);
       if (!ok || tile >= num_tiles) break;
       step(q1);
-      q1 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
-      advance(ptile, pkk, kFDecGroups, nsteps);
+      q1 = fetch_row<kBwd>(args, ptile, pkk, Rg, num_tiles);
+      advance(ptile, pkk, kFDecGroups, nsteps, npairs);
       if (!ok || tile >= num_tiles) break;
       step(q2);
-      q2 = fetch_row<kBwd>(args, ptile, pkk, R, num_tiles);
-      advance(ptile, pkk, kFDecGroups, nsteps);
+      q2 = fetch_row<kBwd>(args, ptile, pkk, Rg, num_tiles);
+      advance(ptile, pkk, kFDecGroups, nsteps, npairs);
     }
     if (!ok) *abort_flag = 1;
   } else {
@@ -686,24 +683,24 @@ __global__ void __launch_bounds__(kFThreads, 1)
     const int q = warp & 3;
     uint32_t tc = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++tc) {
-      const int m0 = (tile % args.m_tiles) * kFPairM + kFBM * static_cast<int>(blockIdx.y);
-      const int n0 = (tile / args.m_tiles) * kFBN;
+    const uint32_t tempty0 = mapa_shared(smem_u32(tempty), 0);   // CTA 0's release barriers
+    for (int tile = pair; tile < num_tiles && ok; tile += npairs, ++tc) {
+      const int m0 = (tile % args.m_tiles) * kFPairRows;
+      const int n0 = (tile / args.m_tiles) * kFPairCols;
       if (*abort_flag || !mbar_wait(tfull, tc & 1)) { ok = false; break; }
       tc_fence_after();
       const int64_t ld = args.Nout;
-      constexpr int kAcc = kFAccs<kBwd>, kCols = kFAccCols<kBwd>;
 #pragma unroll 1
-      for (int h = 0; h < kAcc; ++h) {
-        const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * kCols;
+      for (int h = 0; h < kFSlices; ++h) {
+        const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * kFAccCols;
 #pragma unroll 1
-        for (int c = 0; c < kCols / 32; ++c) {
+        for (int c = 0; c < kFAccCols / 32; ++c) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(tbase + c * 32, v);
           tmem_ld_wait();
           if (!kBwd) {
             // lane = output row, 32 consecutive output columns
-            const int row = m0 + h * 128 + q * 32 + lane;
+            const int row = m0 + 256 * rank + h * 128 + q * 32 + lane;
             const int col = n0 + c * 32;
             if (row < args.M && col < args.Nout) {
               uint4* dst = reinterpret_cast<uint4*>(args.out + row * ld + col);
@@ -717,8 +714,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
             }
           } else {
             // lane = output column, 32 consecutive output rows
-            const int col = n0 + q * 32 + lane;
-            const int row0 = m0 + h * kCols + c * 32;
+            const int col = n0 + 128 * rank + q * 32 + lane;
+            const int row0 = m0 + h * kFAccCols + c * 32;
             if (col < args.Nout && row0 < args.M) {
               uint16_t* dst = args.out + row0 * ld + col;
               const int nrows = args.M - row0;   // rows left in the output (>= 1)
@@ -733,7 +730,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[h]);
+        if (lane == 0) mbar_arrive_cluster(tempty0 + static_cast<uint32_t>(h) * 8u);
       }
     }
     if (!ok) *abort_flag = 1;
@@ -741,12 +738,13 @@ __global__ void __launch_bounds__(kFThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  // no CTA leaves while its partner may still copy into it or read from it
+  // neither CTA leaves while the pair MMA, the peer's copies or the peer's
+  // arrivals may still reach it
   cluster_sync_all();
   if (*abort_flag && threadIdx.x == 0) raise_status(args.d_status, QLORA_ERR_TIMEOUT);
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 
@@ -985,8 +983,8 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
   fa.Nw = static_cast<int>(N);
   fa.nk = static_cast<int>(K / 64);
   fa.rsteps = rsteps_of(r);
-  fa.m_tiles = static_cast<int>((M + kFPairM - 1) / kFPairM);   // pair tiles of 1024 rows
-  fa.n_tiles = static_cast<int>((N + kFBN - 1) / kFBN);
+  fa.m_tiles = static_cast<int>((M + kFPairRows - 1) / kFPairRows);   // pair tiles of 512 rows
+  fa.n_tiles = static_cast<int>((N + kFPairCols - 1) / kFPairCols);   // and 256 columns
   fa.sv = sv;
   fa.packed = packed;
   fa.out = Y;
@@ -994,13 +992,13 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // persistent pairs of CTAs (a cluster of 1 x 2), one pair per two SMs
+  // persistent pairs of CTAs (a cluster of 2 x 1), one pair per two SMs
   const int tiles = fa.m_tiles * fa.n_tiles;
   const int grid = tiles < sms / 2 ? tiles : sms / 2;
   {
     ProfScope prof(kProfFusedFwd, st);
-    e = launch_pdl(fused_nf4_gemm_kernel<false>, dim3(grid, 2), dim3(kFThreads), kFSmem, st, 2, tX, tZc,
-                   tBl, fa);
+    e = launch_pdl_pair(fused_nf4_gemm_kernel<false>, dim3(2 * grid), dim3(kFThreads), kFSmem, st, tX,
+                        tZc, tBl, fa);
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -1081,8 +1079,8 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   fa.Nw = static_cast<int>(N);
   fa.nk = static_cast<int>(N / 64);
   fa.rsteps = rsteps_of(r);
-  fa.m_tiles = static_cast<int>((M + kFPairM - 1) / kFPairM);   // pair tiles of 1024 rows
-  fa.n_tiles = static_cast<int>((K + kFBN - 1) / kFBN);
+  fa.m_tiles = static_cast<int>((M + kFPairRows - 1) / kFPairRows);   // pair tiles of 512 dY rows
+  fa.n_tiles = static_cast<int>((K + kFPairCols - 1) / kFPairCols);   // and 256 output columns
   fa.sv = sv;
   fa.packed = packed;
   fa.out = dX;
@@ -1090,7 +1088,7 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // persistent pairs of CTAs (a cluster of 1 x 2), one pair per two SMs
+  // persistent pairs of CTAs (a cluster of 2 x 1), one pair per two SMs
   const int tiles = fa.m_tiles * fa.n_tiles;
   const int grid = tiles < sms / 2 ? tiles : sms / 2;
 
@@ -1104,8 +1102,8 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   if (ss != nullptr && cudaEventRecord(ss->fork, st) == cudaSuccess) s2 = ss->s;
   {
     ProfScope prof(kProfFusedBwd, st);
-    e = launch_pdl(fused_nf4_gemm_kernel<true>, dim3(grid, 2), dim3(kFThreads), kFSmem, st, 2, tG, tdZa,
-                   tAl, fa);
+    e = launch_pdl_pair(fused_nf4_gemm_kernel<true>, dim3(2 * grid), dim3(kFThreads), kFSmem, st, tG,
+                        tdZa, tAl, fa);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
   if (s2 != st) {

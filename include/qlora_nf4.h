@@ -107,6 +107,11 @@ int32_t qlora_abi_version(void);
 /* Human-readable name of a status code (static string, never NULL). */
 const char* qlora_status_str(qlora_status s);
 
+/* For diagnostics: the description of the CUDA runtime error behind the
+ * calling thread's most recent QLORA_ERR_CUDA (a static string from the CUDA
+ * runtime, never NULL), or "no error" if this thread has had none. */
+const char* qlora_last_cuda_error(void);
+
 /* Element counts: n1 = ceil(numel/64), n2 = ceil(n1/256); 0 for numel < 1. */
 int64_t qlora_nf4_n1(int64_t numel);
 int64_t qlora_nf4_n2(int64_t numel);

@@ -51,6 +51,7 @@ def test_status_strings_and_counts(L):
     for code in range(7):
         assert lib.qlora_status_str(code)
     assert lib.qlora_status_str(99) == b"unknown status"
+    assert lib.qlora_last_cuda_error()          # a static string, never NULL
     assert lib.qlora_nf4_n1(1) == 1 and lib.qlora_nf4_n1(64) == 1 and lib.qlora_nf4_n1(65) == 2
     assert lib.qlora_nf4_n2(64 * 256) == 1 and lib.qlora_nf4_n2(64 * 256 + 1) == 2
     assert lib.qlora_nf4_n1(0) == 0 and lib.qlora_nf4_n2(0) == 0
