@@ -133,6 +133,19 @@ __device__ __forceinline__ GvScale gemv_scale_load(const ScaleView& sv, int64_t 
   return r;
 }
 
+// The value at `off` in the first S CTAs of the cluster, added in rank order
+// (all loads in flight before the first add).
+__device__ __forceinline__ float cluster_sum_in_order(uint32_t off, int S) {
+  float part[8];
+#pragma unroll
+  for (int sp = 0; sp < 8; ++sp) part[sp] = sp < S ? ld_dsmem_f32(off, static_cast<uint32_t>(sp)) : 0.0f;
+  float a = 0.0f;
+#pragma unroll
+  for (int sp = 0; sp < 8; ++sp)
+    if (sp < S) a += part[sp];
+  return a;
+}
+
 template <bool kM16>
 __global__ void __launch_bounds__(kGvThreads, 1)
     nf4_gemv_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmX,
@@ -161,16 +174,20 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     mbar_init(bfull, 1);
     fence_mbar_init();
   }
-  // tables of constants (no global memory another launch writes): entry e of
-  // the pair table is bf16(C[e >> 4]) | bf16(C[e & 15]) << 16, one copy per bank
-  {
+  __syncthreads();   // the barriers are initialised
+  if (warp != kGvCompute) {
+    // Tables of constants (no global memory another launch writes), built by
+    // every warp but the producer, which meanwhile starts the first copies:
+    // entry e of the pair table is bf16(C[e >> 4]) | bf16(C[e & 15]) << 16,
+    // one copy per bank; then T8.
+    const int wi = warp < kGvCompute ? warp : warp - 1;
     const float cv = kCodeVals[16 * args.sv.codebook + (lane & 15)];
-    for (int e = warp; e < 256; e += kGvWarps)
+    for (int e = wi; e < 256; e += kGvWarps - 1)
       table[e * 64 + lane] =
           pack_bf16x2(__shfl_sync(0xFFFFFFFFu, cv, e >> 4), __shfl_sync(0xFFFFFFFFu, cv, e & 15));
+    for (int u = wi * 32 + lane; u < 256; u += (kGvWarps - 1) * 32) t8[u] = kT8Table.v[u];
+    asm volatile("bar.sync 2, %0;" ::"n"((kGvWarps - 1) * 32) : "memory");
   }
-  for (int u = threadIdx.x; u < 256; u += blockDim.x) t8[u] = kT8Table.v[u];
-  __syncthreads();
 
   const int M = args.M, N = args.N, K = args.K;
   const int cg = blockIdx.x;                            // 256-column group
@@ -468,8 +485,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       uint16_t bits = 0;
       if (jr < r) {
         const uint32_t off = smem_u32(Zs + m * 64 + jr);
-        float a = 0.0f;
-        for (int sp = 0; sp < S; ++sp) a += ld_dsmem_f32(off, static_cast<uint32_t>(sp));
+        const float a = cluster_sum_in_order(off, S);
         bits = static_cast<uint16_t>(pack_bf16x2(args.c * a, 0.0f) & 0xFFFFu);
         zc = bf16_bits_to_f32(bits);
       }
@@ -487,8 +503,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         const int n = cg * kGvCols + cl;
         if (n >= N) continue;
         const uint32_t off = smem_u32(Ps + tok * kGvPLd + cl);
-        float y = 0.0f;
-        for (int sp = 0; sp < S; ++sp) y += ld_dsmem_f32(off, static_cast<uint32_t>(sp));
+        const float y = cluster_sum_in_order(off, S);
         float lora = 0.0f;
         for (int jr = 0; jr < r; ++jr)
           lora = fmaf(Zcs[tok * 64 + jr], bf16_bits_to_f32(Bs[jr * kGvCols + cl]), lora);
