@@ -352,6 +352,51 @@ __device__ __forceinline__ void bins_key_range(const unsigned long long* sb, int
   }
 }
 
+// floor(S / d) and S mod d for S < 2^126 and 0 < d < 2^62, without a
+// bit-serial division: three rounds of (double-precision quotient of the
+// remaining remainder, exact 128-bit correction of quotient and remainder);
+// each round shrinks the remainder by about 2^50, so the third leaves it
+// within one divisor of the final range, which the last steps settle exactly.
+__device__ __forceinline__ double u128_to_f64(unsigned __int128 v) {
+  return static_cast<double>(static_cast<uint64_t>(v >> 64)) * 18446744073709551616.0 +
+         static_cast<double>(static_cast<uint64_t>(v));
+}
+
+__device__ __forceinline__ unsigned __int128 f64_to_u128(double v) {   // v >= 0, < 2^127
+  const double hi = floor(v * 5.421010862427522e-20);                 // v / 2^64
+  const double lo = v - hi * 18446744073709551616.0;                    // exact
+  return (static_cast<unsigned __int128>(static_cast<uint64_t>(hi)) << 64) +
+         static_cast<unsigned __int128>(static_cast<uint64_t>(lo));
+}
+
+__device__ void divmod_u128_u64(unsigned __int128 S, uint64_t d, unsigned __int128& Q, uint64_t& R) {
+  const double dd = static_cast<double>(d);
+  unsigned __int128 q = 0;
+  __int128 r = static_cast<__int128>(S);
+  for (int round = 0; round < 3; ++round) {
+    const bool neg = r < 0;
+    const unsigned __int128 adj =
+        f64_to_u128(floor(u128_to_f64(static_cast<unsigned __int128>(neg ? -r : r)) / dd));
+    if (neg) {
+      q -= adj;
+      r += static_cast<__int128>(adj * d);
+    } else {
+      q += adj;
+      r -= static_cast<__int128>(adj * d);
+    }
+  }
+  for (int i = 0; i < 4 && r < 0; ++i) {
+    --q;
+    r += d;
+  }
+  for (int i = 0; i < 4 && r >= static_cast<__int128>(d); ++i) {
+    ++q;
+    r -= d;
+  }
+  Q = q;
+  R = static_cast<uint64_t>(r);
+}
+
 // ... and the sum divided by n1 with one rounding to fp32 (one thread).
 __device__ uint32_t exact_mean_bits(const unsigned long long* sb, int kmin, int kmax, int64_t n1) {
   const uint64_t d = static_cast<uint64_t>(n1);
@@ -360,8 +405,14 @@ __device__ uint32_t exact_mean_bits(const unsigned long long* sb, int kmin, int 
     unsigned __int128 S = 0;
     for (int key = kmin; key <= kmax; ++key)
       S += static_cast<unsigned __int128>(sb[key]) << (key - kmin);
-    const unsigned __int128 Q = S / d;
-    const uint64_t rem = static_cast<uint64_t>(S % d);
+    unsigned __int128 Q;
+    uint64_t rem;
+    if ((S >> 126) == 0 && (d >> 62) == 0) {
+      divmod_u128_u64(S, d, Q, rem);
+    } else {
+      Q = S / d;
+      rem = static_cast<uint64_t>(S % d);
+    }
     bits = round_q128_to_f32(Q, rem, d, kmin - 1 - 149);
   } else {
     constexpr int NL = 12;
@@ -801,6 +852,24 @@ __global__ void __launch_bounds__(kBfThreads) nf4_encode_bf16_kernel(
   }
 }
 
+// First guess of the index k (0..254, V_127 = 0) of the codebook value nearest
+// to c (x = |c| / s2 approximately).  The nonzero magnitudes come in decades:
+// decade f = 0..6 covers (10^(f-7), 10^(f-6)] with the 2^f values
+// 10^(f-7) * (1 + 9(m+1)/2^f), m = 0 .. 2^f - 1, at t = 2^f + m; so the decade
+// is ceil(log10 x) + 6 and m follows linearly.  `dec_scale[f]` = 10^(7-f).
+__device__ __forceinline__ int t8_index_guess(float c, float inv_s2, const float* dec_scale) {
+  const float x = fabsf(c) * inv_s2;
+  int t = 0;
+  if (x > 1e-7f) {
+    int f = static_cast<int>(ceilf(__log10f(x))) + 6;
+    f = min(max(f, 0), 6);
+    const float mr = (x * dec_scale[f] - 1.0f) * static_cast<float>(1 << f) * (1.0f / 9.0f) - 1.0f;
+    const int m = min(max(__float2int_rn(mr), -1), (1 << f) - 1);
+    t = min((1 << f) + m, 127);
+  }
+  return c >= 0.0f ? 127 + t : 127 - t;
+}
+
 // One warp per group of 256 centred scales (8 per lane, 8 groups per CTA).
 // The 255 distinct codebook values V_0 < ... < V_254 are: -|T|(127..1), 0,
 // |T|(1..127); the code of the nearest value to c/s2 (ties to the smaller
@@ -818,7 +887,13 @@ __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict_
   __shared__ float mag[128];
   __shared__ double mid[254];
   __shared__ float thr[8][256];
+  __shared__ float dec_scale[7];
   pdl_launch_dependents();
+  if (threadIdx.x < 7) {
+    float v = 1.0f;
+    for (int i = threadIdx.x; i < 7; ++i) v *= 10.0f;   // 10^(7 - f), exact in fp32
+    dec_scale[threadIdx.x] = v;
+  }
   for (int t = threadIdx.x; t < 128; t += blockDim.x) mag[t] = kT8Table.v[t];
   __syncthreads();
   for (int k = threadIdx.x; k < 254; k += blockDim.x) {
@@ -858,18 +933,28 @@ __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict_
       if (k < 254) T[k] = __double2float_rd(sd * mid[k]);
     }
     __syncwarp();
+    const float inv_s2 = 1.0f / sg;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int64_t i = g * kDQBlock + j * 32 + lane;
-      int lo = 0, hi = 254;           // the first k with T[k] >= c
-#pragma unroll
-      for (int it = 0; it < 8; ++it) {
-        const int md = min((lo + hi) >> 1, 253);   // < 254 whenever lo < hi
-        const bool less = T[md] < c[j];
-        lo = (lo < hi && less) ? md + 1 : lo;
-        hi = (lo < hi && !less) ? md : hi;
+      // the first k with T[k] >= c: from the first guess, step up while
+      // T[k] < c, then down while T[k-1] >= c (T is non-decreasing); a guess
+      // further off than a few steps falls back to the binary search
+      int k = t8_index_guess(c[j], inv_s2, dec_scale);
+      int steps = 0;
+      while (k < 254 && T[k] < c[j] && steps < 4) { ++k; ++steps; }
+      while (k > 0 && T[k - 1] >= c[j] && steps < 8) { --k; ++steps; }
+      if (steps >= 4 && !((k == 254 || T[k] >= c[j]) && (k == 0 || T[k - 1] < c[j]))) {
+        int lo = 0, hi = 254;
+#pragma unroll 1
+        for (int it = 0; it < 8; ++it) {
+          const int md = min((lo + hi) >> 1, 253);   // < 254 whenever lo < hi
+          const bool less = T[md] < c[j];
+          lo = (lo < hi && less) ? md + 1 : lo;
+          hi = (lo < hi && !less) ? md : hi;
+        }
+        k = lo;
       }
-      const int k = lo;
       if (i < n1)
         code8[i] = static_cast<uint8_t>(k < 127 ? (0x80u | static_cast<uint32_t>(127 - k))
                                                 : (k == 127 ? 0u : static_cast<uint32_t>(k - 127)));
