@@ -2,6 +2,7 @@
 // the block scales.  Page "QLoRA：冻结的 4-bit 权重怎样参与一次微调",
 // §NF4 保存的是索引而不是均匀整数值, §从 NF4 索引打包成字节,
 // §Double Quantization 压缩的是 Scale.
+#include <atomic>
 #include <cfloat>
 
 #include "common.cuh"
@@ -476,6 +477,39 @@ constexpr size_t encode_smem_bytes() {
 // iteration.  Whole chunks stream into a 4-stage shared-memory ring by 1-D
 // bulk copies; the remaining blocks (a partial last chunk, or everything when
 // W is not 16-byte aligned) are read directly from global memory.
+//
+// The workspace head (exponent bins, finished-CTA counter) is cleared by CTA 0
+// at the start of every call, which then publishes the call's token; every
+// CTA waits for that token before adding its bins (at its end, long after),
+// so no separate clearing step has to run before the kernel.
+__device__ __forceinline__ unsigned long long* ws_token(unsigned long long* bins) {
+  return reinterpret_cast<unsigned long long*>(reinterpret_cast<char*>(bins) + 2056);
+}
+
+__device__ __forceinline__ void ws_clear_and_publish(unsigned long long* bins, unsigned int* done_ctas,
+                                                     unsigned long long token) {
+  if (blockIdx.x != 0) return;
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) bins[i] = 0ull;
+  if (threadIdx.x == 0 && done_ctas != nullptr) *done_ctas = 0u;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(ws_token(bins)), "l"(token) : "memory");
+  }
+}
+
+// true once CTA 0 has cleared the head for this call (bounded wait)
+__device__ __forceinline__ bool ws_wait_published(unsigned long long* bins, unsigned long long token) {
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(ws_token(bins)) : "memory");
+    if (v == token) return true;
+    if (globaltimer_ns() - t0 > 2000000000ull) return false;
+    __nanosleep(64);
+  }
+}
+
 template <typename T, bool kDQ>
 __global__ void __launch_bounds__(256) nf4_encode_kernel(const T* __restrict__ W, int64_t numel,
                                                          int64_t n1, uint8_t* __restrict__ packed,
@@ -483,7 +517,7 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const T* __restrict__ W
                                                          unsigned long long* __restrict__ bins,
                                                          unsigned int* __restrict__ done_ctas,
                                                          float* __restrict__ offset_out,
-                                                         int32_t* d_status) {
+                                                         int32_t* d_status, unsigned long long token) {
   extern __shared__ uint8_t esm_raw[];
   T* ring = reinterpret_cast<T*>((reinterpret_cast<uintptr_t>(esm_raw) + 127) &
                                  ~static_cast<uintptr_t>(127));
@@ -493,6 +527,7 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const T* __restrict__ W
   __shared__ uint64_t full_bar[kEncStages];
   pdl_launch_dependents();
   pdl_wait();
+  if (kDQ) ws_clear_and_publish(bins, done_ctas, token);
   __shared__ int abort_flag;
   build_buckets(tab, mexact);
   if (kDQ)
@@ -573,9 +608,15 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const T* __restrict__ W
   if (bad) raise_status(d_status, QLORA_ERR_NONFINITE);
   if (kDQ) {
     if (sub == 0) bc.flush(sbins);
+    __shared__ int published;
+    if (threadIdx.x == 0) {
+      published = ws_wait_published(bins, token) ? 1 : 0;
+      if (!published) raise_status(d_status, QLORA_ERR_TIMEOUT);
+    }
     __syncthreads();
-    for (int i = threadIdx.x; i < 256; i += blockDim.x)
-      if (sbins[i]) atomicAdd(&bins[i], sbins[i]);
+    if (published)
+      for (int i = threadIdx.x; i < 256; i += blockDim.x)
+        if (sbins[i]) atomicAdd(&bins[i], sbins[i]);
     // The last CTA to finish forms the exact mean of all first-level scales
     // from the global bins (every other CTA's additions are visible to it:
     // each made them before its fenced increment of the counter).
@@ -667,7 +708,8 @@ template <bool kDQ>
 __global__ void __launch_bounds__(kBfThreads) nf4_encode_bf16_kernel(
     const uint16_t* __restrict__ W, int64_t numel, int64_t n1, uint8_t* __restrict__ packed,
     float* __restrict__ scales, unsigned long long* __restrict__ bins,
-    unsigned int* __restrict__ done_ctas, float* __restrict__ offset_out, int32_t* d_status) {
+    unsigned int* __restrict__ done_ctas, float* __restrict__ offset_out, int32_t* d_status,
+    unsigned long long token) {
   extern __shared__ uint8_t esm_raw[];
   uint16_t* ring = reinterpret_cast<uint16_t*>((reinterpret_cast<uintptr_t>(esm_raw) + 127) &
                                                ~static_cast<uintptr_t>(127));
@@ -694,6 +736,7 @@ __global__ void __launch_bounds__(kBfThreads) nf4_encode_bf16_kernel(
   }
   __syncthreads();
   pdl_wait();   // the tables above read no global memory
+  if (kDQ) ws_clear_and_publish(bins, done_ctas, token);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t nchunks = numel / kBfChunkElems;
@@ -804,9 +847,20 @@ __global__ void __launch_bounds__(kBfThreads) nf4_encode_bf16_kernel(
       }
       *reinterpret_cast<uint4*>(packed + blk * (kBlock / 2) + half * 16) =
           make_uint4(out[0], out[1], out[2], out[3]);
-      if (half == 0) {
-        scales[blk] = s_;
-        if (kDQ) bc.add(s_, sbins);
+      if (half == 0) scales[blk] = s_;
+      if (kDQ) {
+        // exponent bins of the warp's 16 block scales: lanes with one key
+        // sum their mantissas and one of them adds the sum to the CTA's bin
+        // (a few shared atomics per warp and chunk, instead of one per block
+        // on a handful of contended addresses)
+        const uint32_t u = __float_as_uint(s_);
+        const uint32_t E = (u >> 23) & 0xFFu;
+        const uint32_t key = half == 0 ? (E ? E : 1u) : 0x100u;   // odd lanes carry no scale
+        const uint32_t mant = half == 0 ? ((u & 0x7FFFFFu) | (E ? 0x800000u : 0u)) : 0u;
+        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, key);
+        const uint32_t sum = __reduce_add_sync(peers, mant);   // <= 16 * 2^24
+        if (key < 0x100u && lane == __ffs(static_cast<int>(peers)) - 1)
+          atomicAdd(&sbins[key], static_cast<unsigned long long>(sum));
       }
     }
   }
@@ -831,9 +885,15 @@ __global__ void __launch_bounds__(kBfThreads) nf4_encode_bf16_kernel(
   if (bad) raise_status(d_status, QLORA_ERR_NONFINITE);
   if (kDQ) {
     bc.flush(sbins);
+    __shared__ int published;
+    if (threadIdx.x == 0) {
+      published = ws_wait_published(bins, token) ? 1 : 0;
+      if (!published) raise_status(d_status, QLORA_ERR_TIMEOUT);
+    }
     __syncthreads();
-    for (int i = threadIdx.x; i < 256; i += blockDim.x)
-      if (sbins[i]) atomicAdd(&bins[i], sbins[i]);
+    if (published)
+      for (int i = threadIdx.x; i < 256; i += blockDim.x)
+        if (sbins[i]) atomicAdd(&bins[i], sbins[i]);
     __syncthreads();
     if (offset_out == nullptr) return;   // a shard: the caller adds the bins of all shards
     if (threadIdx.x == 0) {
@@ -1058,6 +1118,10 @@ namespace {
 cudaError_t launch_encoder(const void* W, int dtype, int64_t numel, uint8_t* packed, float* scales,
                            bool dq, unsigned long long* bins, unsigned int* done_ctas,
                            float* offset_out, int32_t* d_status, cudaStream_t st, int num_sms) {
+  // a token per call (never repeated within the process): the kernel's CTA 0
+  // publishes it once it has cleared the workspace head
+  static std::atomic<unsigned long long> next_token{0x9E3779B97F4A7C15ull};
+  const unsigned long long token = next_token.fetch_add(1ull);
   const int64_t n1 = (numel + kBlock - 1) / kBlock;
   const int threads = 256;
   const int64_t want = (n1 * 4 + threads - 1) / threads;
@@ -1106,17 +1170,17 @@ cudaError_t launch_encoder(const void* W, int dtype, int64_t numel, uint8_t* pac
     if (g16 < 1) g16 = 1;
     e = dq ? launch_pdl(nf4_encode_bf16_kernel<true>, dim3(static_cast<unsigned>(g16)), dim3(kBfThreads),
                         kBfSmem, st, 1, w16, numel, n1, packed, scales, bins, done_ctas, offset_out,
-                        d_status)
+                        d_status, token)
            : launch_pdl(nf4_encode_bf16_kernel<false>, dim3(static_cast<unsigned>(g16)), dim3(kBfThreads),
                         kBfSmem, st, 1, w16, numel, n1, packed, scales, bins, done_ctas, offset_out,
-                        d_status);
+                        d_status, token);
   } else {
     const size_t sm = encode_smem_bytes<float>();
     const float* w32 = static_cast<const float*>(W);
     e = dq ? launch_pdl(nf4_encode_kernel<float, true>, dim3(blocks), dim3(threads), sm, st, 1, w32,
-                        numel, n1, packed, scales, bins, done_ctas, offset_out, d_status)
+                        numel, n1, packed, scales, bins, done_ctas, offset_out, d_status, token)
            : launch_pdl(nf4_encode_kernel<float, false>, dim3(blocks), dim3(threads), sm, st, 1, w32,
-                        numel, n1, packed, scales, bins, done_ctas, offset_out, d_status);
+                        numel, n1, packed, scales, bins, done_ctas, offset_out, d_status, token);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
   return e;
@@ -1167,9 +1231,7 @@ cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* pa
   unsigned long long* bins = static_cast<unsigned long long*>(ws);
   unsigned int* done_ctas = reinterpret_cast<unsigned int*>(static_cast<char*>(ws) + 2048);
   float* scales = reinterpret_cast<float*>(static_cast<char*>(ws) + kQuantizeWsHead);
-  cudaError_t e = cudaMemsetAsync(ws, 0, kQuantizeWsHead, st);
-  if (e != cudaSuccess) return e;
-  e = launch_encoder(W, dtype, numel, packed, scales, true, bins, done_ctas, offset, d_status, st,
+  cudaError_t e = launch_encoder(W, dtype, numel, packed, scales, true, bins, done_ctas, offset, d_status, st,
                      num_sms);
   if (e != cudaSuccess) return e;
   return launch_dq_encode(scales, n1, offset, code8, s2, st, num_sms);
@@ -1188,8 +1250,6 @@ cudaError_t launch_quantize_shard_begin(const void* W_shard, int dtype, int64_t 
                           nullptr, d_status, st, num_sms);
   unsigned long long* bins = static_cast<unsigned long long*>(ws);
   float* scales = reinterpret_cast<float*>(static_cast<char*>(ws) + kQuantizeWsHead);
-  cudaError_t e = cudaMemsetAsync(ws, 0, kQuantizeWsHead, st);
-  if (e != cudaSuccess) return e;
   return launch_encoder(W_shard, dtype, numel, pk, scales, true, bins, nullptr, nullptr, d_status,
                         st, num_sms);
 }

@@ -145,7 +145,8 @@ qlora_status qlora_status_clear(int32_t* d_status, qlora_stream_t stream);
  *   st       : host struct; numel >= 1; its device buffers receive the result.
  *   ws       : device workspace of at least
  *              qlora_nf4_quantize_workspace_size(numel, double_quant) bytes
- *              (may be NULL when that size is 0).
+ *              (may be NULL when that size is 0); any contents on entry (the
+ *              call clears what it uses itself, on the device).
  * Device errors: QLORA_ERR_NONFINITE if any weight is NaN or ±Inf.
  * Host errors: INVALID_ARG (null/misaligned pointers, numel < 1, bad
  * blocksize, small workspace), UNSUPPORTED (numel > 2^40), CUDA.
@@ -205,7 +206,8 @@ qlora_status qlora_nf4_quantize_shard_end(const qlora_nf4_state* st, int64_t blo
  * allocate device memory when they quantize (runtimes that plan every device
  * buffer at start-up and forbid allocation in their steady state; plugins that
  * only receive tensor pointers from a host framework).  The scratch it needs
- * (2304 bytes of exponent bins and a counter, plus one fp32 per 64-block;
+ * (2304 bytes of exponent bins, a counter and a call token, plus one fp32 per
+ * 64-block;
  * about 4 MB at the limit) is a
  * fixed array inside the library, allocated on each GPU that loads this part
  * of the library and held until the process exits.
