@@ -357,10 +357,16 @@ __global__ void __launch_bounds__(kMtThreads, 1)
         const float sc = dq ? __fadd_rn(__fmul_rn(t8[code], s2v), off) : s2v;
         nonfinite |= !(fabsf(sc) <= FLT_MAX);
         // the row's table: entry e = bf16(C_e * sc)
+        // (the product of two fp32 values is exact in fp64; one rounding to bf16)
+        const double scd = static_cast<double>(sc);
         uint32_t w[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          w[j] = bf16_of_exact_product(Ctab[2 * j], sc) | (bf16_of_exact_product(Ctab[2 * j + 1], sc) << 16);
+        for (int j = 0; j < 8; ++j) {
+          unsigned short lo, hi;
+          asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(lo) : "d"(static_cast<double>(Ctab[2 * j]) * scd));
+          asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(hi) : "d"(static_cast<double>(Ctab[2 * j + 1]) * scd));
+          w[j] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+        }
         uint32_t H[4], L[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {

@@ -938,13 +938,32 @@ __device__ __forceinline__ int t8_index_guess(float c, float inv_s2, const float
 // c > s2 * m_k  <=>  c > RD_fp32(s2 * m_k); so each warp turns its group's
 // 254 midpoints into fp32 thresholds once and counts them by binary search.
 // k < 127 -> byte 0x80 | (127 - k), k = 127 -> 0x00, k > 127 -> byte k - 127.
+// The 254 midpoints between consecutive values of the sorted 255-value
+// codebook V (-|T|(127..1), 0, |T|(1..127)), in fp64, formed at compile time.
+struct T8Midpoints {
+  double m[254];
+};
+
+constexpr T8Midpoints make_t8_midpoints() {
+  T8Midpoints r{};
+  const T8Table t = make_t8_table();
+  auto V = [&t](int i) -> double {
+    return i < 127 ? -static_cast<double>(t.v[127 - i])
+                   : (i == 127 ? 0.0 : static_cast<double>(t.v[i - 127]));
+  };
+  for (int k = 0; k < 254; ++k) r.m[k] = 0.5 * (V(k) + V(k + 1));
+  return r;
+}
+
+// global (not constant) memory: each thread of a CTA reads a different entry
+static __device__ const T8Midpoints kT8Mid = make_t8_midpoints();
+
 __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict__ a, int64_t n1,
                                                         const float* __restrict__ offset_p,
                                                         uint8_t* __restrict__ code8,
                                                         float* __restrict__ s2) {
   // the exact mean (offset) was formed by the encoder's last CTA
   __shared__ float s_off;
-  __shared__ float mag[128];
   __shared__ double mid[254];
   __shared__ float thr[8][256];
   __shared__ float dec_scale[7];
@@ -954,17 +973,9 @@ __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict_
     for (int i = threadIdx.x; i < 7; ++i) v *= 10.0f;   // 10^(7 - f), exact in fp32
     dec_scale[threadIdx.x] = v;
   }
-  for (int t = threadIdx.x; t < 128; t += blockDim.x) mag[t] = kT8Table.v[t];
+  for (int k = threadIdx.x; k < 254; k += blockDim.x) mid[k] = kT8Mid.m[k];
   __syncthreads();
-  for (int k = threadIdx.x; k < 254; k += blockDim.x) {
-    auto V = [&](int i) -> double {
-      return i < 127 ? -static_cast<double>(mag[127 - i])
-                     : (i == 127 ? 0.0 : static_cast<double>(mag[i - 127]));
-    };
-    mid[k] = 0.5 * (V(k) + V(k + 1));
-  }
-  __syncthreads();
-  pdl_wait();   // the tables above read no global memory
+  pdl_wait();   // the tables above read only compile-time constants
   if (threadIdx.x == 0) s_off = *offset_p;
   __syncthreads();
   const float off = s_off;
