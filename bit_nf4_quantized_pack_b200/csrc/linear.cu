@@ -103,8 +103,12 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  pdl_launch_dependents();   // after this CTA holds its TMEM
+  // Wait for the preceding kernel first and only then let the next one
+  // launch: the fused kernel that follows a rank-r product then knows that
+  // every kernel before this one has completed, and reads its activations
+  // and weights at once, waiting only for this kernel's result.
   pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
@@ -478,7 +482,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
   const uint32_t tmem = *tmem_holder;
   const int num_tiles = args.m_tiles * args.n_tiles;
   pdl_launch_dependents();   // after this CTA holds its TMEM
-  pdl_wait();
+  // No wait for the preceding kernel here.  It is always this library's
+  // rank-r product (Zc, or dZ), which lets this kernel launch only after all
+  // kernels before it have completed: the activations, the weights and the
+  // output buffer are final or free, and only the LoRA step's Zc (dZ) comes
+  // from the preceding kernel; the producer waits before loading it.
 
   if (warp == 0) {
     // ------------------------------ TMA producer ---------------------------
@@ -506,6 +514,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
       auto act_row = [&](int m0, int h) -> int {
         return kBwd ? m0 + 256 * h + 128 * rank : m0 + 256 * rank + 128 * h;
       };
+      bool lora_ready = false;
       for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
         const int m0 = (tile % args.m_tiles) * kFPairRows;
         const int n0 = (tile / args.m_tiles) * kFPairCols;
@@ -519,6 +528,10 @@ __global__ void __launch_bounds__(kFThreads, 1)
         }
         if (!ok) break;
         // LoRA step: Zc / dZ into one stage, B / A into the next
+        if (!lora_ready) {
+          pdl_wait();   // Zc (dZ) is the preceding kernel's output
+          lora_ready = true;
+        }
         uint32_t s1, s2;
         if (!take(s1, kFA)) { ok = false; break; }
         uint8_t* a = sA + s1 * kFA;
