@@ -347,6 +347,15 @@ __device__ __forceinline__ void bins_key_range(const unsigned long long* sb, int
     uint32_t m = 0;
     for (int i = 0; i < 8; ++i) m |= (sb[threadIdx.x * 8 + i] != 0ull ? 1u : 0u) << i;
     const unsigned any = __ballot_sync(0xFFFFFFFFu, m != 0);
+    if (any == 0u) {
+      // no scale was binned (shards that covered no block): an empty range,
+      // which exact_mean_bits turns into a mean of 0
+      if (threadIdx.x == 0) {
+        range[0] = 1;
+        range[1] = 0;
+      }
+      return;
+    }
     const int lmin = __ffs(any) - 1, lmax = 31 - __clz(any);
     if (threadIdx.x == lmin) range[0] = threadIdx.x * 8 + (__ffs(m) - 1);
     if (threadIdx.x == lmax) range[1] = threadIdx.x * 8 + (31 - __clz(m));
@@ -486,11 +495,17 @@ __device__ __forceinline__ unsigned long long* ws_token(unsigned long long* bins
   return reinterpret_cast<unsigned long long*>(reinterpret_cast<char*>(bins) + 2056);
 }
 
+// The claimed-chunk counter of the bf16 encoder (chunks past its first wave).
+__device__ __forceinline__ unsigned long long* ws_chunk_counter(unsigned long long* bins) {
+  return reinterpret_cast<unsigned long long*>(reinterpret_cast<char*>(bins) + 2072);
+}
+
 __device__ __forceinline__ void ws_clear_and_publish(unsigned long long* bins, unsigned int* done_ctas,
                                                      unsigned long long token) {
   if (blockIdx.x != 0) return;
   for (int i = threadIdx.x; i < 256; i += blockDim.x) bins[i] = 0ull;
   if (threadIdx.x == 0 && done_ctas != nullptr) *done_ctas = 0u;
+  if (threadIdx.x == 0) *ws_chunk_counter(bins) = 0ull;
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
@@ -507,6 +522,23 @@ __device__ __forceinline__ bool ws_wait_published(unsigned long long* bins, unsi
     if (v == token) return true;
     if (globaltimer_ns() - t0 > 2000000000ull) return false;
     __nanosleep(64);
+  }
+}
+
+// The call's token again once the last CTA has stored the mean (the encoder
+// that also double-quantizes in the same launch).
+__device__ __forceinline__ unsigned long long* ws_mean_flag(unsigned long long* bins) {
+  return reinterpret_cast<unsigned long long*>(reinterpret_cast<char*>(bins) + 2064);
+}
+
+__device__ __forceinline__ bool ws_wait_mean(unsigned long long* bins, unsigned long long token) {
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(ws_mean_flag(bins)) : "memory");
+    if (v == token) return true;
+    if (globaltimer_ns() - t0 > 2000000000ull) return false;
+    __nanosleep(128);
   }
 }
 
@@ -641,6 +673,173 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const T* __restrict__ W
 }
 
 // ---------------------------------------------------------------------------
+// Double quantization of the scales: groups of 256 centred scales, one warp
+// per group.  The 255 distinct codebook values V_0 < ... < V_254 are: -|T|(127..1), 0,
+// |T|(1..127); the code of the nearest value to c/s2 (ties to the smaller
+// value) is the number k of midpoints m_k = (V_k + V_{k+1})/2 with
+// s2 * m_k < c.  s2 * m_k is exact in fp64, and for an fp32 c,
+// c > s2 * m_k  <=>  c > RD_fp32(s2 * m_k); so each warp turns its group's
+// 254 midpoints into fp32 thresholds T once, and the count k comes from a
+// cell table (below) and one comparison with T.
+// k < 127 -> byte 0x80 | (127 - k), k = 127 -> 0x00, k > 127 -> byte k - 127.
+// The 254 midpoints between consecutive values of the sorted 255-value
+// codebook V (-|T|(127..1), 0, |T|(1..127)), in fp64, formed at compile time.
+struct T8Midpoints {
+  double m[254];
+};
+
+constexpr T8Midpoints make_t8_midpoints() {
+  T8Midpoints r{};
+  const T8Table t = make_t8_table();
+  auto V = [&t](int i) -> double {
+    return i < 127 ? -static_cast<double>(t.v[127 - i])
+                   : (i == 127 ? 0.0 : static_cast<double>(t.v[i - 127]));
+  };
+  for (int k = 0; k < 254; ++k) r.m[k] = 0.5 * (V(k) + V(k + 1));
+  return r;
+}
+
+// Cells of x = c / s2 (as the fp32 product c * RN(1/s2), within 2^-23 of the
+// exact quotient, relative): the sign, the binade 2^-21 .. 2^0 (row 1 .. 22;
+// row 0 = |x| < 2^-21, below the smallest nonzero midpoint 5e-7) and the top
+// 6 mantissa bits (64 cells per row).  Widened by 2^-20 (relative) on both
+// sides, every cell holds at most one midpoint (checked at compile time: the
+// smallest gap between positive midpoints is 1.4%).  Entry k0 = the number of
+// midpoints certainly below any x of the cell, so the exact count is k0, or
+// k0 + 1 when T[k0] < c.  Positive cells follow the 127 negative midpoints;
+// negative cells count, by symmetry (m_{253-i} = -m_i), the midpoints above
+// -x.
+constexpr int kT8Rows = 23;
+constexpr int kT8CellBits = 6;
+constexpr int kT8SignCells = kT8Rows << kT8CellBits;   // cells per sign
+
+struct alignas(16) T8Cells {
+  uint8_t k0[2 * kT8SignCells];   // [0, kT8SignCells): x >= 0; then x < 0
+  int most_per_cell;              // compile-time check of the one-midpoint rule
+};
+
+constexpr T8Cells make_t8_cells() {
+  T8Cells r{};
+  const T8Midpoints mp = make_t8_midpoints();
+  const double widen = 1.0 / 1048576.0;   // 2^-20
+  int below = 0, upto = 0;                // positive midpoints < lo', <= hi'
+  r.most_per_cell = 0;
+  for (int row = 0; row < kT8Rows; ++row) {
+    double p2 = 1.0;                      // 2^(row - 22): the row's binade
+    for (int i = row; i < kT8Rows - 1; ++i) p2 *= 0.5;
+    for (int cell = 0; cell < (1 << kT8CellBits); ++cell) {
+      // row 0 (every cell alike): 0 <= |x| < 2^-21
+      const double lo = row == 0 ? 0.0 : p2 * (1.0 + cell / 64.0);
+      const double hi = row == 0 ? 2.0 * p2 : p2 * (1.0 + (cell + 1) / 64.0);
+      while (below < 127 && mp.m[127 + below] < lo * (1.0 - widen)) ++below;
+      while (upto < 127 && mp.m[127 + upto] <= hi * (1.0 + widen)) ++upto;
+      const int idx = (row << kT8CellBits) + cell;
+      r.k0[idx] = static_cast<uint8_t>(127 + below);
+      r.k0[kT8SignCells + idx] = static_cast<uint8_t>(127 - upto);
+      if (upto - below > r.most_per_cell) r.most_per_cell = upto - below;
+    }
+  }
+  return r;
+}
+static_assert(make_t8_cells().most_per_cell <= 1, "a T8 cell holds more than one midpoint");
+
+// global (not constant) memory: each thread of a CTA reads a different entry
+static __device__ const T8Midpoints kT8Mid = make_t8_midpoints();
+static __device__ const T8Cells kT8Cells = make_t8_cells();
+
+// The count of thresholds s2 * m_k below c by binary search (sd = s2, in
+// fp64, where each product is exact); the path of groups whose 1/s2 is not a
+// normal number.
+__device__ __noinline__ int t8_search(double cd, double sd, const double* mid) {
+  int lo = 0, hi = 254;
+#pragma unroll 1
+  for (int it = 0; it < 8; ++it) {
+    const int md = min((lo + hi) >> 1, 253);   // < 254 whenever lo < hi
+    const bool less = sd * mid[md] < cd;
+    lo = (lo < hi && less) ? md + 1 : lo;
+    hi = (lo < hi && !less) ? md : hi;
+  }
+  return lo;
+}
+
+// The code byte of one centred scale c (see above): x = c * inv_s2, its
+// cell's k0 from the table `cells` and one comparison of c with the exact
+// threshold s2 * m_{k0} in fp64 (sd = s2).  |x| >= 2 or not finite (inv_s2 =
+// infinity: see the caller) takes a binary search over the thresholds
+// instead.  Index k -> byte: k >= 127 -> k - 127, k < 127 -> 0x80 | (127 - k).
+__device__ __forceinline__ uint32_t t8_code_byte(float c, float inv_s2, double sd,
+                                                 const uint8_t* cells, const double* mid) {
+  const uint32_t xb = __float_as_uint(c * inv_s2);
+  const double cd = static_cast<double>(c);
+  // cells are (|x| bits >> 17) - (105 << 6): row 0 holds every |x| < 2^-21
+  const int r = max(static_cast<int>((xb & 0x7FFFFFFFu) >> 17) - (105 << kT8CellBits), 0);
+  int k;
+  if (r >= kT8SignCells) {
+    k = t8_search(cd, sd, mid);
+  } else {
+    const int k0 = cells[static_cast<int>(xb >> 31) * kT8SignCells + r];
+    k = k0 + ((k0 < 254 && sd * mid[min(k0, 253)] < cd) ? 1 : 0);
+  }
+  return static_cast<uint32_t>(k >= 127 ? k - 127 : 255 - k);
+}
+
+// Second-level scale and scale codes of group g (one warp; lane l holds
+// scales 4l..4l+3 and 128+4l..128+4l+3 of the group): c = a - offset,
+// s2 = max |c| (1 for an all-zero group), then each code from the cell table
+// and one threshold.  The scales are read through L2 (ld.global.cg): in the
+// encoder's own launch other CTAs wrote them.  `a` is 16-byte aligned.
+__device__ __forceinline__ void dq_encode_group(const float* a, int64_t n1, int64_t g, float off,
+                                                const double* mid, const uint8_t* cells,
+                                                uint8_t* __restrict__ code8, float* __restrict__ s2,
+                                                int lane) {
+  const int64_t base = g * kDQBlock;
+  const bool whole = base + kDQBlock <= n1;
+  float c[8];
+  if (whole) {
+    const float4 v0 = __ldcg(reinterpret_cast<const float4*>(a + base) + lane);
+    const float4 v1 = __ldcg(reinterpret_cast<const float4*>(a + base + 128) + lane);
+    c[0] = v0.x; c[1] = v0.y; c[2] = v0.z; c[3] = v0.w;
+    c[4] = v1.x; c[5] = v1.y; c[6] = v1.z; c[7] = v1.w;
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t i = base + (j >> 2) * 128 + 4 * lane + (j & 3);
+      c[j] = i < n1 ? __ldcg(a + i) : off;   // past the end: c = 0
+    }
+  }
+  float m = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    c[j] = __fsub_rn(c[j], off);
+    m = fmaxf(m, fabsf(c[j]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  const float sg = m > 0.0f ? m : 1.0f;
+  if (lane == 0) s2[g] = sg;
+  const double sd = static_cast<double>(sg);
+  // 1/s2 within 2^-24 (relative) while it is a normal number; outside
+  // 2^-128 <= s2 < 2^126 the group searches the thresholds instead (infinity)
+  const float inv_s2 = (sg >= 2.938735877e-39f && sg < 8.507059173e37f)
+                           ? 1.0f / sg : __int_as_float(0x7F800000);
+  uint32_t w[2] = {0u, 0u};
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    w[j >> 2] |= t8_code_byte(c[j], inv_s2, sd, cells, mid) << (8 * (j & 3));
+  uint8_t* dst = code8 + base + 4 * lane;
+  if (whole && (reinterpret_cast<uintptr_t>(code8 + base) & 3u) == 0) {
+    *reinterpret_cast<uint32_t*>(dst) = w[0];
+    *reinterpret_cast<uint32_t*>(dst + 128) = w[1];
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (base + (j >> 2) * 128 + 4 * lane + (j & 3) < n1)
+        dst[(j >> 2) * 128 + (j & 3)] = static_cast<uint8_t>(w[j >> 2] >> (8 * (j & 3)));
+  }
+}
+
+
+// ---------------------------------------------------------------------------
 // bf16 encoder.  CTA = 8 compute warps + 1 producer warp.  Whole chunks of
 // 8192 elements (128 blocks) stream into a 3-stage ring by 1-D bulk copies;
 // two threads own one 64-block (32 elements each).  A warp copies its 2 KB
@@ -656,11 +855,15 @@ __global__ void __launch_bounds__(256) nf4_encode_kernel(const T* __restrict__ W
 // the last whole chunk are left to the generic per-lane code (encode16).
 // ---------------------------------------------------------------------------
 constexpr int kBfChunkBlocks = 128;
+constexpr int kDqMidBytes = 2048;   // 254 fp64 midpoints, staged in the ring for the DQ stage
 constexpr int kBfChunkElems = kBfChunkBlocks * kBlock;   // 8192
 constexpr int kBfStages = 3;
 constexpr int kBfComputeWarps = 8;
 constexpr int kBfThreads = (kBfComputeWarps + 1) * 32;
 constexpr size_t kBfSmem = static_cast<size_t>(kBfStages) * kBfChunkElems * 2 + 128;
+static_assert(kDqMidBytes >= 254 * 8 && kDqMidBytes % 16 == 0 &&
+                  kDqMidBytes + 2 * kT8SignCells <= kBfStages * kBfChunkElems * 2,
+              "DQ stage tables fit the ring");
 
 // Bucket entries for the packed path: per bucket and lane one 8-byte entry
 // (fp32 midpoint or 4.0, then codes below the bucket + 1); lane l reads its
@@ -708,7 +911,8 @@ template <bool kDQ>
 __global__ void __launch_bounds__(kBfThreads) nf4_encode_bf16_kernel(
     const uint16_t* __restrict__ W, int64_t numel, int64_t n1, uint8_t* __restrict__ packed,
     float* __restrict__ scales, unsigned long long* __restrict__ bins,
-    unsigned int* __restrict__ done_ctas, float* __restrict__ offset_out, int32_t* d_status,
+    unsigned int* __restrict__ done_ctas, float* __restrict__ offset_out,
+    uint8_t* __restrict__ code8, float* __restrict__ s2, int32_t* d_status,
     unsigned long long token) {
   extern __shared__ uint8_t esm_raw[];
   uint16_t* ring = reinterpret_cast<uint16_t*>((reinterpret_cast<uintptr_t>(esm_raw) + 127) &
@@ -722,6 +926,7 @@ __global__ void __launch_bounds__(kBfThreads) nf4_encode_bf16_kernel(
   __shared__ int abort_flag;
   __shared__ int last_cta;
   __shared__ int krange[2];
+  __shared__ long long chunk_of[kBfStages];   // the chunk in each stage; -1: no more
   pdl_launch_dependents();
   load_buckets(tab4, tab8, mexact);
   if (kDQ)
@@ -740,21 +945,42 @@ __global__ void __launch_bounds__(kBfThreads) nf4_encode_bf16_kernel(
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t nchunks = numel / kBfChunkElems;
-  const int64_t my_n = nchunks > blockIdx.x ? (nchunks - 1 - blockIdx.x) / gridDim.x + 1 : 0;
   constexpr uint32_t kChunkBytes = kBfChunkElems * 2;
   BinCache bc;
   bool bad = false;
 
   if (warp == kBfComputeWarps) {
     // ------------------------------ producer ------------------------------
+    // Chunk j of this CTA: blockIdx.x + j * gridDim.x for the first
+    // kBfStages (and all of them without a workspace); then, with a workspace
+    // (kDQ), the next unclaimed chunk past those waves from the call's
+    // counter, so that CTAs that stream faster take more chunks.  The chunk
+    // goes to the compute warps with the stage; -1 (with a plain arrival)
+    // ends their loop.
     if (lane == 0) {
       uint32_t last_parity[kBfStages];
       for (int s = 0; s < kBfStages; ++s) last_parity[s] = 2;
-      for (int64_t j = 0; j < my_n; ++j) {
+      bool counter_ready = false;
+      for (int64_t j = 0;; ++j) {
         const int s = static_cast<int>(j % kBfStages);
         const uint32_t ph = static_cast<uint32_t>((j / kBfStages) & 1);
         if (j >= kBfStages && !mbar_wait(&empty_bar[s], ph ^ 1)) { abort_flag = 1; break; }
-        const int64_t c = blockIdx.x + j * gridDim.x;
+        int64_t c = blockIdx.x + j * static_cast<int64_t>(gridDim.x);
+        if (kDQ && j >= kBfStages) {
+          if (!counter_ready) {
+            counter_ready = ws_wait_published(bins, token);   // CTA 0 cleared the counter
+            if (!counter_ready) { abort_flag = 1; break; }
+          }
+          c = kBfStages * static_cast<int64_t>(gridDim.x) +
+              static_cast<int64_t>(atomicAdd(ws_chunk_counter(bins), 1ull));
+        }
+        if (c >= nchunks) {
+          chunk_of[s] = -1;
+          mbar_arrive(&full_bar[s]);
+          last_parity[s] = 2;   // the stage's last copy was consumed (the wait above)
+          break;
+        }
+        chunk_of[s] = c;
         mbar_arrive_expect_tx(&full_bar[s], kChunkBytes);
         bulk_load_1d(ring + s * kBfChunkElems, W + c * kBfChunkElems, kChunkBytes, &full_bar[s]);
         last_parity[s] = ph;
@@ -770,10 +996,12 @@ __global__ void __launch_bounds__(kBfThreads) nf4_encode_bf16_kernel(
     const uint32_t tb = smem_u32(tab8) + static_cast<uint32_t>(lane) * 8u - 0x4B000000u * 256u;
     const uint64_t c16 = f2pack(8388624.0f, 8388624.0f);   // 2^23 + 16 in each lane of the pair
     const uint64_t k16 = f2pack(16.0f, 16.0f);
-    for (int64_t j = 0; j < my_n; ++j) {
+    for (int64_t j = 0;; ++j) {
       const int s = static_cast<int>(j % kBfStages);
       const uint32_t ph = static_cast<uint32_t>((j / kBfStages) & 1);
       if (!mbar_wait(&full_bar[s], ph)) { abort_flag = 1; break; }
+      const int64_t c = *reinterpret_cast<volatile long long*>(&chunk_of[s]);
+      if (c < 0) break;
       const uint16_t* src = ring + s * kBfChunkElems + lb * kBlock + half * 32;
       // The thread's 64 bytes are four 16-byte chunks; slot v reads chunk
       // (v + rot) & 3, so that the 8 lanes of a quarter warp (4 blocks 128
@@ -788,7 +1016,6 @@ __global__ void __launch_bounds__(kBfThreads) nf4_encode_bf16_kernel(
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[s]);
-      const int64_t c = blockIdx.x + j * gridDim.x;
       const int64_t blk = c * kBfChunkBlocks + lb;
       // absmax: largest bf16 magnitude of the block (the pair of threads)
       uint32_t m2 = 0u;
@@ -849,18 +1076,24 @@ __global__ void __launch_bounds__(kBfThreads) nf4_encode_bf16_kernel(
           make_uint4(out[0], out[1], out[2], out[3]);
       if (half == 0) scales[blk] = s_;
       if (kDQ) {
-        // exponent bins of the warp's 16 block scales: lanes with one key
-        // sum their mantissas and one of them adds the sum to the CTA's bin
-        // (a few shared atomics per warp and chunk, instead of one per block
-        // on a handful of contended addresses)
+        // exponent bins of the warp's 16 block scales, summed exactly by two
+        // warp reductions.  Bin k counts units of 2^(k-150); a scale is a bf16
+        // magnitude m8 * 2^(key-134) (m8 its 8-bit significand), which is
+        // m8 << (16 + key - kb) units of bin kb.  With kb = the warp's largest
+        // key - 3 (at least 1), every scale within 16 binades of kb is an
+        // integer below 2^27 there, and the 16 of them sum below 2^31: one
+        // shared atomic per warp and chunk.  Scales further below go to their
+        // own bins, one atomic each.
         const uint32_t u = __float_as_uint(s_);
         const uint32_t E = (u >> 23) & 0xFFu;
-        const uint32_t key = half == 0 ? (E ? E : 1u) : 0x100u;   // odd lanes carry no scale
-        const uint32_t mant = half == 0 ? ((u & 0x7FFFFFu) | (E ? 0x800000u : 0u)) : 0u;
-        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, key);
-        const uint32_t sum = __reduce_add_sync(peers, mant);   // <= 16 * 2^24
-        if (key < 0x100u && lane == __ffs(static_cast<int>(peers)) - 1)
-          atomicAdd(&sbins[key], static_cast<unsigned long long>(sum));
+        const uint32_t key = half == 0 ? (E ? E : 1u) : 0u;   // odd lanes carry no scale
+        const uint32_t kmax = __reduce_max_sync(0xFFFFFFFFu, key);
+        const uint32_t kb = kmax > 4u ? kmax - 3u : 1u;
+        const uint32_t m8 = ((u >> 16) & 0x7Fu) | (E ? 0x80u : 0u);
+        const bool near = key + 16u >= kb;
+        const uint32_t sum = __reduce_add_sync(0xFFFFFFFFu, half == 0 && near ? m8 << (16u + key - kb) : 0u);
+        if (lane == 0) atomicAdd(&sbins[kb], static_cast<unsigned long long>(sum));
+        if (half == 0 && !near) atomicAdd(&sbins[key], static_cast<unsigned long long>(m8) << 16);
       }
     }
   }
@@ -886,6 +1119,7 @@ __global__ void __launch_bounds__(kBfThreads) nf4_encode_bf16_kernel(
   if (kDQ) {
     bc.flush(sbins);
     __shared__ int published;
+    __syncthreads();
     if (threadIdx.x == 0) {
       published = ws_wait_published(bins, token) ? 1 : 0;
       if (!published) raise_status(d_status, QLORA_ERR_TIMEOUT);
@@ -907,130 +1141,66 @@ __global__ void __launch_bounds__(kBfThreads) nf4_encode_bf16_kernel(
       __syncthreads();
       bins_key_range(sbins, krange);
       __syncthreads();
-      if (threadIdx.x == 0) *offset_out = __uint_as_float(exact_mean_bits(sbins, krange[0], krange[1], n1));
+      if (threadIdx.x == 0) {
+        *offset_out = __uint_as_float(exact_mean_bits(sbins, krange[0], krange[1], n1));
+        if (code8 != nullptr) {
+          __threadfence();
+          asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(ws_mean_flag(bins)), "l"(token)
+                       : "memory");
+        }
+      }
     }
+    if (code8 == nullptr) return;
+    // Double quantization in the same launch.  Every CTA of the grid is
+    // resident (one wave, sized by the occupancy of this kernel), so each
+    // waits for the last CTA's mean (bounded) and then encodes groups of 256
+    // scales, one warp per group.  The ring is free: every copy has landed
+    // and been read.
+    double* mid = reinterpret_cast<double*>(ring);
+    uint8_t* cells = reinterpret_cast<uint8_t*>(ring) + kDqMidBytes;
+    for (int k = threadIdx.x; k < 254; k += blockDim.x) mid[k] = kT8Mid.m[k];
+    for (int k = threadIdx.x; k < 2 * kT8SignCells / 16; k += blockDim.x)
+      reinterpret_cast<uint4*>(cells)[k] = reinterpret_cast<const uint4*>(kT8Cells.k0)[k];
+    __shared__ float s_mean;
+    if (threadIdx.x == 0) {
+      published = ws_wait_mean(bins, token) ? 1 : 0;
+      if (published)
+        s_mean = __ldcg(offset_out);
+      else
+        raise_status(d_status, QLORA_ERR_TIMEOUT);
+    }
+    __syncthreads();
+    if (!published) return;
+    const int nwarps = kBfComputeWarps + 1;
+    const int64_t n2 = (n1 + kDQBlock - 1) / kDQBlock;
+    for (int64_t g = static_cast<int64_t>(blockIdx.x) * nwarps + warp; g < n2;
+         g += static_cast<int64_t>(gridDim.x) * nwarps)
+      dq_encode_group(scales, n1, g, s_mean, mid, cells, code8, s2, lane);
   }
 }
 
-// First guess of the index k (0..254, V_127 = 0) of the codebook value nearest
-// to c (x = |c| / s2 approximately).  The nonzero magnitudes come in decades:
-// decade f = 0..6 covers (10^(f-7), 10^(f-6)] with the 2^f values
-// 10^(f-7) * (1 + 9(m+1)/2^f), m = 0 .. 2^f - 1, at t = 2^f + m; so the decade
-// is ceil(log10 x) + 6 and m follows linearly.  `dec_scale[f]` = 10^(7-f).
-__device__ __forceinline__ int t8_index_guess(float c, float inv_s2, const float* dec_scale) {
-  const float x = fabsf(c) * inv_s2;
-  int t = 0;
-  if (x > 1e-7f) {
-    int f = static_cast<int>(ceilf(__log10f(x))) + 6;
-    f = min(max(f, 0), 6);
-    const float mr = (x * dec_scale[f] - 1.0f) * static_cast<float>(1 << f) * (1.0f / 9.0f) - 1.0f;
-    const int m = min(max(__float2int_rn(mr), -1), (1 << f) - 1);
-    t = min((1 << f) + m, 127);
-  }
-  return c >= 0.0f ? 127 + t : 127 - t;
-}
-
-// One warp per group of 256 centred scales (8 per lane, 8 groups per CTA).
-// The 255 distinct codebook values V_0 < ... < V_254 are: -|T|(127..1), 0,
-// |T|(1..127); the code of the nearest value to c/s2 (ties to the smaller
-// value) is the number k of midpoints m_k = (V_k + V_{k+1})/2 with
-// s2 * m_k < c.  s2 * m_k is exact in fp64, and for an fp32 c,
-// c > s2 * m_k  <=>  c > RD_fp32(s2 * m_k); so each warp turns its group's
-// 254 midpoints into fp32 thresholds once and counts them by binary search.
-// k < 127 -> byte 0x80 | (127 - k), k = 127 -> 0x00, k > 127 -> byte k - 127.
-// The 254 midpoints between consecutive values of the sorted 255-value
-// codebook V (-|T|(127..1), 0, |T|(1..127)), in fp64, formed at compile time.
-struct T8Midpoints {
-  double m[254];
-};
-
-constexpr T8Midpoints make_t8_midpoints() {
-  T8Midpoints r{};
-  const T8Table t = make_t8_table();
-  auto V = [&t](int i) -> double {
-    return i < 127 ? -static_cast<double>(t.v[127 - i])
-                   : (i == 127 ? 0.0 : static_cast<double>(t.v[i - 127]));
-  };
-  for (int k = 0; k < 254; ++k) r.m[k] = 0.5 * (V(k) + V(k + 1));
-  return r;
-}
-
-// global (not constant) memory: each thread of a CTA reads a different entry
-static __device__ const T8Midpoints kT8Mid = make_t8_midpoints();
-
+// One warp per group of 256 scales, 8 groups per CTA (fp32 weights, and the
+// shards of a sharded quantization, whose mean is formed after all shards).
 __global__ void __launch_bounds__(256) dq_encode_kernel(const float* __restrict__ a, int64_t n1,
                                                         const float* __restrict__ offset_p,
                                                         uint8_t* __restrict__ code8,
                                                         float* __restrict__ s2) {
-  // the exact mean (offset) was formed by the encoder's last CTA
   __shared__ float s_off;
   __shared__ double mid[254];
-  __shared__ float thr[8][256];
-  __shared__ float dec_scale[7];
+  __shared__ __align__(16) uint8_t cells[2 * kT8SignCells];
   pdl_launch_dependents();
-  if (threadIdx.x < 7) {
-    float v = 1.0f;
-    for (int i = threadIdx.x; i < 7; ++i) v *= 10.0f;   // 10^(7 - f), exact in fp32
-    dec_scale[threadIdx.x] = v;
-  }
   for (int k = threadIdx.x; k < 254; k += blockDim.x) mid[k] = kT8Mid.m[k];
+  for (int k = threadIdx.x; k < 2 * kT8SignCells / 16; k += blockDim.x)
+    reinterpret_cast<uint4*>(cells)[k] = reinterpret_cast<const uint4*>(kT8Cells.k0)[k];
   __syncthreads();
   pdl_wait();   // the tables above read only compile-time constants
   if (threadIdx.x == 0) s_off = *offset_p;
   __syncthreads();
-  const float off = s_off;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  float* T = thr[warp];
   const int64_t n2 = (n1 + kDQBlock - 1) / kDQBlock;
   for (int64_t g = static_cast<int64_t>(blockIdx.x) * 8 + warp; g < n2;
-       g += static_cast<int64_t>(gridDim.x) * 8) {
-    float c[8];
-    float m = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int64_t i = g * kDQBlock + j * 32 + lane;
-      c[j] = i < n1 ? __fsub_rn(__ldg(a + i), off) : 0.0f;
-      m = fmaxf(m, fabsf(c[j]));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    const float sg = m > 0.0f ? m : 1.0f;
-    if (lane == 0) s2[g] = sg;
-    const double sd = static_cast<double>(sg);
-    __syncwarp();                     // previous group's searches are done with T
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int k = j * 32 + lane;
-      if (k < 254) T[k] = __double2float_rd(sd * mid[k]);
-    }
-    __syncwarp();
-    const float inv_s2 = 1.0f / sg;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int64_t i = g * kDQBlock + j * 32 + lane;
-      // the first k with T[k] >= c: from the first guess, step up while
-      // T[k] < c, then down while T[k-1] >= c (T is non-decreasing); a guess
-      // further off than a few steps falls back to the binary search
-      int k = t8_index_guess(c[j], inv_s2, dec_scale);
-      int steps = 0;
-      while (k < 254 && T[k] < c[j] && steps < 4) { ++k; ++steps; }
-      while (k > 0 && T[k - 1] >= c[j] && steps < 8) { --k; ++steps; }
-      if (steps >= 4 && !((k == 254 || T[k] >= c[j]) && (k == 0 || T[k - 1] < c[j]))) {
-        int lo = 0, hi = 254;
-#pragma unroll 1
-        for (int it = 0; it < 8; ++it) {
-          const int md = min((lo + hi) >> 1, 253);   // < 254 whenever lo < hi
-          const bool less = T[md] < c[j];
-          lo = (lo < hi && less) ? md + 1 : lo;
-          hi = (lo < hi && !less) ? md : hi;
-        }
-        k = lo;
-      }
-      if (i < n1)
-        code8[i] = static_cast<uint8_t>(k < 127 ? (0x80u | static_cast<uint32_t>(127 - k))
-                                                : (k == 127 ? 0u : static_cast<uint32_t>(k - 127)));
-    }
-  }
+       g += static_cast<int64_t>(gridDim.x) * 8)
+    dq_encode_group(a, n1, g, s_off, mid, cells, code8, s2, lane);
 }
 
 // The exact mean of n1 first-level scales from exponent bins that already
@@ -1128,7 +1298,8 @@ namespace {
 // `offset_out` the last CTA also forms their exact mean there.
 cudaError_t launch_encoder(const void* W, int dtype, int64_t numel, uint8_t* packed, float* scales,
                            bool dq, unsigned long long* bins, unsigned int* done_ctas,
-                           float* offset_out, int32_t* d_status, cudaStream_t st, int num_sms) {
+                           float* offset_out, uint8_t* code8, float* s2, int32_t* d_status,
+                           cudaStream_t st, int num_sms) {
   // a token per call (never repeated within the process): the kernel's CTA 0
   // publishes it once it has cleared the workspace head
   static std::atomic<unsigned long long> next_token{0x9E3779B97F4A7C15ull};
@@ -1181,10 +1352,10 @@ cudaError_t launch_encoder(const void* W, int dtype, int64_t numel, uint8_t* pac
     if (g16 < 1) g16 = 1;
     e = dq ? launch_pdl(nf4_encode_bf16_kernel<true>, dim3(static_cast<unsigned>(g16)), dim3(kBfThreads),
                         kBfSmem, st, 1, w16, numel, n1, packed, scales, bins, done_ctas, offset_out,
-                        d_status, token)
+                        code8, s2, d_status, token)
            : launch_pdl(nf4_encode_bf16_kernel<false>, dim3(static_cast<unsigned>(g16)), dim3(kBfThreads),
                         kBfSmem, st, 1, w16, numel, n1, packed, scales, bins, done_ctas, offset_out,
-                        d_status, token);
+                        code8, s2, d_status, token);
   } else {
     const size_t sm = encode_smem_bytes<float>();
     const float* w32 = static_cast<const float*>(W);
@@ -1236,15 +1407,19 @@ cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* pa
   if (codebook == 1) return launch_int4(W, dtype, numel, packed, absmax_out, d_status, st);
   if (!dq)
     return launch_encoder(W, dtype, numel, packed, absmax_out, false, nullptr, nullptr, nullptr,
-                          d_status, st, num_sms);
-  // workspace: 256 exponent bins, the finished-CTA counter, then the scales
+                          nullptr, nullptr, d_status, st, num_sms);
+  // workspace: 256 exponent bins, the finished-CTA counter, the call token and
+  // the mean's flag, then the scales
   const int64_t n1 = (numel + kBlock - 1) / kBlock;
   unsigned long long* bins = static_cast<unsigned long long*>(ws);
   unsigned int* done_ctas = reinterpret_cast<unsigned int*>(static_cast<char*>(ws) + 2048);
   float* scales = reinterpret_cast<float*>(static_cast<char*>(ws) + kQuantizeWsHead);
-  cudaError_t e = launch_encoder(W, dtype, numel, packed, scales, true, bins, done_ctas, offset, d_status, st,
-                     num_sms);
-  if (e != cudaSuccess) return e;
+  // bf16 weights: scale codes and second-level scales in the encoder's own
+  // launch; fp32 weights: a second launch
+  const bool fused = dtype == QLORA_DTYPE_BF16;
+  cudaError_t e = launch_encoder(W, dtype, numel, packed, scales, true, bins, done_ctas, offset,
+                                 fused ? code8 : nullptr, fused ? s2 : nullptr, d_status, st, num_sms);
+  if (e != cudaSuccess || fused) return e;
   return launch_dq_encode(scales, n1, offset, code8, s2, st, num_sms);
 }
 
@@ -1258,11 +1433,11 @@ cudaError_t launch_quantize_shard_begin(const void* W_shard, int dtype, int64_t 
   if (codebook == 1) return launch_int4(W_shard, dtype, numel, pk, absmax_out + b0, d_status, st);
   if (!dq)
     return launch_encoder(W_shard, dtype, numel, pk, absmax_out + b0, false, nullptr, nullptr,
-                          nullptr, d_status, st, num_sms);
+                          nullptr, nullptr, nullptr, d_status, st, num_sms);
   unsigned long long* bins = static_cast<unsigned long long*>(ws);
   float* scales = reinterpret_cast<float*>(static_cast<char*>(ws) + kQuantizeWsHead);
-  return launch_encoder(W_shard, dtype, numel, pk, scales, true, bins, nullptr, nullptr, d_status,
-                        st, num_sms);
+  return launch_encoder(W_shard, dtype, numel, pk, scales, true, bins, nullptr, nullptr, nullptr,
+                        nullptr, d_status, st, num_sms);
 }
 
 cudaError_t launch_quantize_shard_end(int64_t numel_total, int64_t b0, int64_t b1, const void* ws,

@@ -146,6 +146,30 @@ def test_full_size_65b_mlp_sampled():
         assert np.array_equal(packed[b * 32:(b + 1) * 32], payload), b
 
 
+@pytest.mark.parametrize("nblk", [128 * 3, 128 * 5 + 37])
+def test_double_quant_bf16_scales_spread_over_binades(nblk):
+    """bf16 weights whose block scales spread from bf16 subnormals to near the
+    largest bf16, mixed inside every group of 16 consecutive blocks: the
+    encoder's exponent bins then meet, within one warp, scales close to the
+    warp's largest and scales far below it.  Whole state, DQ offset
+    included, bit-exact against the oracle (whole 8192-element chunks plus a
+    ragged tail of blocks)."""
+    q = _q()
+    rng = np.random.default_rng(nblk)
+    e = rng.integers(-133, 127, nblk).astype(np.float64)
+    m = rng.integers(128, 256, nblk) / 128.0
+    sc = S.f32_to_bf16_values((m * 2.0 ** e).astype(np.float32))
+    sc[rng.random(nblk) < 0.5] = np.float32(0.0078125)   # a cluster of equal scales
+    w = np.zeros(64 * nblk, np.float32)
+    w[::64] = sc
+    w[1::64] = S.f32_to_bf16_values(-sc * np.float32(0.5))
+    w[2::64] = S.f32_to_bf16_values(sc * np.float32(0.3))
+    g = q.quantize(to_dev(w, torch.bfloat16), double_quant=True)
+    ow = OracleWeight(w, True)
+    assert_state_equal(g, ow)
+    assert np.array_equal(nf4.block_scales(w), sc)
+
+
 @pytest.mark.parametrize("scales", [
     [1.0, 1.0 + 2.0 ** -23],                        # exact tie -> even (1.0)
     [1.0 + 2.0 ** -23, 1.0 + 2.0 ** -22],           # exact tie -> even (upper)
