@@ -236,6 +236,158 @@ __global__ void __launch_bounds__(kSkThreads, 1)
 
 
 // ===========================================================================
+// Rank-r product on a few SMs beside the fused GEMM:  D = scale * A B with A
+// K-major (rows m, the activations or dY), the whole contraction per 128-row
+// tile in one CTA (no split), tiles blockIdx.x, + gridDim.x, ...  The fused
+// GEMM that follows leaves these SMs free (its grid is sized to the fewest
+// pairs that need no more waves of tiles), starts at once, and waits for D
+// only at its LoRA step.  Same roles as above: warp 0 TMA, warp 1 MMA into
+// one TMEM accumulator (128 x 64 fp32), warps 2..5 read it (released on
+// `tempty` per tile), scale, round to bf16 and store (mode 0 only).
+// ===========================================================================
+template <bool kBmn>
+__global__ void __launch_bounds__(kSkThreads, 1)
+    rank_rows_kernel(const __grid_constant__ CUtensorMap tmA,
+                     const __grid_constant__ CUtensorMap tmB, SkinnyArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kSkStages * kSkA;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kSkStages * kSkB);
+  uint64_t* empty = full + kSkStages;
+  uint64_t* done = empty + kSkStages;
+  uint64_t* tempty = done + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_tiles = (args.Mp + 127) / 128;
+  const int nkb = args.nk;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSkStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    mbar_init(tempty, 4);   // the four epilogue warps
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 64);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  // wait for the preceding kernel, then let the fused GEMM launch
+  pdl_wait();
+  pdl_launch_dependents();
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    int g = 0;   // stage uses over all tiles
+    bool ok = true;
+    for (int t = blockIdx.x; t < m_tiles && ok; t += gridDim.x) {
+      const int m0 = t * 128;
+      for (int i = 0; i < nkb; ++i, ++g) {
+        const int s = g % kSkStages;
+        const uint32_t ph = (g / kSkStages) & 1;
+        if (g >= kSkStages && !mbar_wait(&empty[s], ph ^ 1)) { ok = false; break; }
+        mbar_arrive_expect_tx(&full[s], kSkA + kSkB);
+#pragma unroll
+        for (int w = 0; w < kSkW; ++w) {
+          const int kx = (i * kSkW + w) * 64;   // boxes past the end arrive as zero fill
+          uint8_t* a = sA + s * kSkA + w * 16384;
+          uint8_t* b = sB + s * kSkB + w * 8192;
+          tma_load_2d(a, &tmA, &full[s], kx, m0);
+          if (kBmn)
+            tma_load_2d(b, &tmB, &full[s], 0, kx);
+          else
+            tma_load_2d(b, &tmB, &full[s], kx, 0);
+        }
+      }
+    }
+    if (!ok) *abort_flag = 1;
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc = idesc_bf16_f32(128, 64, 0, kBmn ? 1 : 0);
+    int g = 0, it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < m_tiles && ok; t += gridDim.x, ++it) {
+      // the epilogue has read the previous tile's accumulator
+      if (it > 0 && !mbar_wait(tempty, (it - 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      for (int i = 0; i < nkb; ++i, ++g) {
+        const int s = g % kSkStages;
+        const uint32_t ph = (g / kSkStages) & 1;
+        if (!mbar_wait(&full[s], ph)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int w = 0; w < kSkW; ++w) {
+          const uint32_t a0 = smem_u32(sA + s * kSkA + w * 16384), b0 = smem_u32(sB + s * kSkB + w * 8192);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint64_t ad = smem_desc(a0 + j * 32, 16, 1024);
+            const uint64_t bd = kBmn ? smem_desc(b0 + j * 2048, 8192, 1024) : smem_desc(b0 + j * 32, 16, 1024);
+            umma_bf16(tmem, ad, bd, idesc, (i > 0 || w > 0 || j > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(done);   // one phase per tile (also drains an aborted tile)
+    }
+    if (!ok) *abort_flag = 1;
+  } else if (warp >= 2) {
+    const int q = warp & 3;   // TMEM lanes 32q .. 32q + 31
+    const int nc = args.ncols;
+    int it = 0;
+    for (int t = blockIdx.x; t < m_tiles; t += gridDim.x, ++it) {
+      const bool okd = mbar_wait(done, it & 1);
+      tc_fence_after();
+      if (!okd) { *abort_flag = 1; break; }
+      const int grow = t * 128 + q * 32 + lane;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        if (c * 32 < nc) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c * 32, v);
+          tmem_ld_wait();
+          if (grow < args.Mp) {
+            uint16_t* o = static_cast<uint16_t*>(args.out) + static_cast<int64_t>(grow) * args.ld;
+            uint16_t* o2 = args.out2 != nullptr ? args.out2 + static_cast<int64_t>(grow) * args.ld2 : nullptr;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int cc = c * 32 + i;
+              if (cc < nc) {
+                // (0 + v) * scale: the split kernel's sum and rounding for one split
+                const uint16_t b = static_cast<uint16_t>(
+                    pack_bf16x2((0.0f + __uint_as_float(v[i])) * args.scale, 0.0f) & 0xFFFFu);
+                if (cc < args.nout) o[cc] = b;
+                if (o2 != nullptr) o2[cc] = b;
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) raise_status(args.d_status, QLORA_ERR_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
+  }
+}
+
+// ===========================================================================
 // Fused NF4-decode GEMM (forward: kBwd = false, input gradient: kBwd = true)
 //
 // Persistent pairs of CTAs on neighbouring SMs (a 1 x 2 thread-block cluster)
@@ -785,6 +937,11 @@ namespace {
 
 // K splits of a rank-r contraction: one CTA per SM (the kernel's shared
 // memory allows no second), so the grid is kept to a single wave.
+// The SM count that fixes split counts and the rank-r path, whatever the
+// device: results (the fp32 summation order of the rank-r products) depend on
+// the shape only.
+constexpr int g_ws_sms = 148;
+
 int skinny_splits(int Mp, int nk, int num_sms) {
   const int mt = (Mp + 127) / 128;
   int want = num_sms / mt;
@@ -853,6 +1010,70 @@ cudaError_t run_skinny(const CUtensorMap& ta, const CUtensorMap& tb, int Mp, int
   return cudaGetLastError();
 }
 
+template <bool B>
+cudaError_t set_rank_rows_attr() {
+  static DeviceOnce once;
+  return once.run([](int) {
+    return cudaFuncSetAttribute(rank_rows_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(kSkSmem));
+  });
+}
+
+// Pairs of the fused GEMM: the fewest that keep its number of waves of tiles
+// (so the SMs it leaves free cost it nothing).
+int fused_pairs(int tiles, int sms) {
+  const int most = sms / 2 > 0 ? sms / 2 : 1;
+  const int waves = (tiles + most - 1) / most;
+  const int pairs = waves > 0 ? (tiles + waves - 1) / waves : 1;
+  return pairs < 1 ? 1 : pairs;
+}
+
+// CTAs for the rank-r product of a Mp x Kc activation beside the fused GEMM
+// of `tiles` pair tiles, or 0 for the split kernel before it.  Decided for the
+// sizing SM count (not the device's), so the forward and the backward's
+// recompute make the same choice and form Zc alike: the SMs the fused GEMM
+// leaves free, when there are at least 8 of them and each streams at most
+// 2.5 MB (done long before the fused GEMM's first LoRA step).
+int rank_rows_ctas(int64_t Mp, int64_t Kc, int tiles) {
+  const int free_sms = g_ws_sms - 2 * fused_pairs(tiles, g_ws_sms);
+  if (free_sms < 8) return 0;
+  if (static_cast<double>(Mp) * static_cast<double>(Kc) * 2.0 > 2.5e6 * free_sms) return 0;
+  const int m_tiles = static_cast<int>((Mp + 127) / 128);
+  const int ctas = m_tiles < free_sms ? m_tiles : free_sms;
+  return (ctas + 1) & ~1;   // pairs of CTAs (a 2 x 1 cluster), for the fused pairs' placement
+}
+
+// D = scale * A(m',k') B(n',k') by rank_rows_kernel on `ctas` CTAs, mode 0
+// (bf16 out, and all ncols columns again into out2 when it is not null).
+template <bool kBmn>
+cudaError_t run_rank_rows(const CUtensorMap& ta, const CUtensorMap& tb, int Mp, int Kp, int ncols,
+                          float scale, void* out, int ld, int ctas, int32_t* d_status,
+                          cudaStream_t st, int nout = -1, uint16_t* out2 = nullptr, int ld2 = 0) {
+  cudaError_t e = set_rank_rows_attr<kBmn>();
+  if (e != cudaSuccess) return e;
+  SkinnyArgs a;
+  a.Mp = Mp;
+  a.nk = (Kp + 64 * kSkW - 1) / (64 * kSkW);
+  a.kb_per_split = a.nk;
+  a.splits = 1;
+  a.ncols = ncols;
+  a.nout = nout < 0 ? ncols : nout;
+  a.scale = scale;
+  a.mode = 0;
+  a.out = out;
+  a.ld = ld;
+  a.out2 = out2;
+  a.ld2 = ld2;
+  a.d_status = d_status;
+  {
+    ProfScope prof(kProfSkinny, st);
+    e = launch_pdl_pair(rank_rows_kernel<kBmn>, dim3(static_cast<unsigned>(ctas)),
+                        dim3(kSkThreads, 1, 1), kSkSmem, st, ta, tb, a);
+  }
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 template <bool kBwd>
 cudaError_t set_fused_attr() {
   static DeviceOnce once;
@@ -886,7 +1107,6 @@ cudaError_t launch_pad(const uint16_t* src, int64_t rows, int r, uint16_t* dst, 
 
 }  // namespace
 
-static int g_ws_sms = 148;  // sizing assumption for workspace queries (B200)
 
 // A library-owned stream per device for work that runs beside the caller's
 // stream, and the two events of one fork and join.  Created on first use
@@ -981,9 +1201,18 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
     if (!cur.ok) return cudaErrorInvalidValue;
   }
   {
-    const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
-    e = run_skinny<false, true>(tX, tAl, static_cast<int>(M), static_cast<int>(K), rp, c, 0, Zc, r,
-                                Sz, d_status, st, r, Zp, rp);
+    // beside the fused GEMM on the SMs it leaves free, or split-K before it
+    const int fwd_tiles = static_cast<int>(((M + kFPairRows - 1) / kFPairRows) *
+                                           ((N + kFPairCols - 1) / kFPairCols));
+    const int rows_ctas = rank_rows_ctas(M, K, fwd_tiles);
+    if (rows_ctas > 0) {
+      e = run_rank_rows<true>(tX, tAl, static_cast<int>(M), static_cast<int>(K), rp, c, Zc, r,
+                              rows_ctas, d_status, st, r, Zp, rp);
+    } else {
+      const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
+      e = run_skinny<false, true>(tX, tAl, static_cast<int>(M), static_cast<int>(K), rp, c, 0, Zc, r,
+                                  Sz, d_status, st, r, Zp, rp);
+    }
     if (e != cudaSuccess) return e;
   }
   e = set_fused_attr<false>();
@@ -1005,9 +1234,9 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // persistent pairs of CTAs (a cluster of 2 x 1), one pair per two SMs
-  const int tiles = fa.m_tiles * fa.n_tiles;
-  const int grid = tiles < sms / 2 ? tiles : sms / 2;
+  // persistent pairs of CTAs (a cluster of 2 x 1): the fewest pairs that
+  // keep the number of waves of tiles
+  const int grid = fused_pairs(fa.m_tiles * fa.n_tiles, sms);
   {
     ProfScope prof(kProfFusedFwd, st);
     e = launch_pdl_pair(fused_nf4_gemm_kernel<false>, dim3(2 * grid), dim3(kFThreads), kFSmem, st, tX,
@@ -1054,9 +1283,18 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
     CUtensorMap tXf, tAf;
     if (!make_tmap_2d(&tXf, X, kBF16, 2, M, K, K, 64, 128, kSW128)) return cudaErrorInvalidValue;
     if (!make_tmap_2d(&tAf, At, kBF16, 2, K, rp, rp, 64, 64, kSW128)) return cudaErrorInvalidValue;
-    const int Sf = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
-    e = run_skinny<false, true>(tXf, tAf, static_cast<int>(M), static_cast<int>(K), rp, c, 0, Zc_ws,
-                                rp, Sf, d_status, st);
+    // the forward's choice of kernel and split, so the same bits
+    const int fwd_tiles = static_cast<int>(((M + kFPairRows - 1) / kFPairRows) *
+                                           ((N + kFPairCols - 1) / kFPairCols));
+    const int rows_ctas = rank_rows_ctas(M, K, fwd_tiles);
+    if (rows_ctas > 0) {
+      e = run_rank_rows<true>(tXf, tAf, static_cast<int>(M), static_cast<int>(K), rp, c, Zc_ws, rp,
+                              rows_ctas, d_status, st);
+    } else {
+      const int Sf = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
+      e = run_skinny<false, true>(tXf, tAf, static_cast<int>(M), static_cast<int>(K), rp, c, 0, Zc_ws,
+                                  rp, Sf, d_status, st);
+    }
     if (e != cudaSuccess) return e;
     Zc = Zc_ws;
   } else if (pad) {
@@ -1070,8 +1308,17 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   // B's rows past r arrive as zero fill, so dZ's padding columns are zero
   if (!make_tmap_2d(&tG, dY, kBF16, 2, M, N, N, 64, 128, kSW128)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&tBk, B, kBF16, 2, r, N, N, 64, 64, kSW128)) return cudaErrorInvalidValue;
-  e = run_skinny<false, false>(tG, tBk, static_cast<int>(M), static_cast<int>(N), rp, c, 0, dZ, rp,
-                               Sz, d_status, st);
+  {
+    const int dx_tiles = static_cast<int>(((M + kFPairRows - 1) / kFPairRows) *
+                                          ((K + kFPairCols - 1) / kFPairCols));
+    const int rows_ctas = rank_rows_ctas(M, N, dx_tiles);
+    if (rows_ctas > 0)
+      e = run_rank_rows<false>(tG, tBk, static_cast<int>(M), static_cast<int>(N), rp, c, dZ, rp,
+                               rows_ctas, d_status, st);
+    else
+      e = run_skinny<false, false>(tG, tBk, static_cast<int>(M), static_cast<int>(N), rp, c, 0, dZ, rp,
+                                   Sz, d_status, st);
+  }
   if (e != cudaSuccess) return e;
   // dA = X^T dZ : A operand X^T (MN-major over K), B operand dZ (MN-major over r)
   if (!make_tmap_2d(&tXmn, X, kBF16, 2, M, K, K, 64, 64, kSW128)) return cudaErrorInvalidValue;
@@ -1101,9 +1348,9 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // persistent pairs of CTAs (a cluster of 2 x 1), one pair per two SMs
-  const int tiles = fa.m_tiles * fa.n_tiles;
-  const int grid = tiles < sms / 2 ? tiles : sms / 2;
+  // persistent pairs of CTAs (a cluster of 2 x 1): the fewest pairs that
+  // keep the number of waves of tiles
+  const int grid = fused_pairs(fa.m_tiles * fa.n_tiles, sms);
 
   // dX on the caller's stream first; dA and dB, which need only dZ, Zc, X and
   // G, on the side stream after dZ, so their CTAs take the SMs that dX's
