@@ -236,16 +236,17 @@ __global__ void __launch_bounds__(kSkThreads, 1)
 
 
 // ===========================================================================
-// Rank-r product on a few SMs beside the fused GEMM:  D = scale * A B with A
-// K-major (rows m, the activations or dY), the whole contraction per 128-row
-// tile in one CTA (no split), tiles blockIdx.x, + gridDim.x, ...  The fused
-// GEMM that follows leaves these SMs free (its grid is sized to the fewest
-// pairs that need no more waves of tiles), starts at once, and waits for D
-// only at its LoRA step.  Same roles as above: warp 0 TMA, warp 1 MMA into
+// Rank-r product on a few SMs beside the fused GEMM:  D = scale * A B (the
+// operand layouts and output modes of the split kernel above), the whole
+// contraction per 128-row tile in one CTA (no split), tiles blockIdx.x,
+// + gridDim.x, ...  The fused GEMM leaves these SMs free (its grid is sized
+// to the fewest pairs that need no more waves of tiles): Zc (dZ) here lets
+// it start at once and wait for the product only at its LoRA step, and dA,
+// dB here run beside dX.  Same roles as above: warp 0 TMA, warp 1 MMA into
 // one TMEM accumulator (128 x 64 fp32), warps 2..5 read it (released on
-// `tempty` per tile), scale, round to bf16 and store (mode 0 only).
+// `tempty` per tile), scale and store.
 // ===========================================================================
-template <bool kBmn>
+template <bool kAmn, bool kBmn>
 __global__ void __launch_bounds__(kSkThreads, 1)
     rank_rows_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB, SkinnyArgs args) {
@@ -304,7 +305,12 @@ __global__ void __launch_bounds__(kSkThreads, 1)
           const int kx = (i * kSkW + w) * 64;   // boxes past the end arrive as zero fill
           uint8_t* a = sA + s * kSkA + w * 16384;
           uint8_t* b = sB + s * kSkB + w * 8192;
-          tma_load_2d(a, &tmA, &full[s], kx, m0);
+          if (kAmn) {
+            tma_load_2d(a, &tmA, &full[s], m0, kx);
+            tma_load_2d(a + 8192, &tmA, &full[s], m0 + 64, kx);
+          } else {
+            tma_load_2d(a, &tmA, &full[s], kx, m0);
+          }
           if (kBmn)
             tma_load_2d(b, &tmB, &full[s], 0, kx);
           else
@@ -314,7 +320,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     }
     if (!ok) *abort_flag = 1;
   } else if (warp == 1 && lane == 0) {
-    constexpr uint32_t idesc = idesc_bf16_f32(128, 64, 0, kBmn ? 1 : 0);
+    constexpr uint32_t idesc = idesc_bf16_f32(128, 64, kAmn ? 1 : 0, kBmn ? 1 : 0);
     int g = 0, it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < m_tiles && ok; t += gridDim.x, ++it) {
@@ -331,7 +337,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
           const uint32_t a0 = smem_u32(sA + s * kSkA + w * 16384), b0 = smem_u32(sB + s * kSkB + w * 8192);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const uint64_t ad = smem_desc(a0 + j * 32, 16, 1024);
+            const uint64_t ad = kAmn ? smem_desc(a0 + j * 2048, 8192, 1024) : smem_desc(a0 + j * 32, 16, 1024);
             const uint64_t bd = kBmn ? smem_desc(b0 + j * 2048, 8192, 1024) : smem_desc(b0 + j * 32, 16, 1024);
             umma_bf16(tmem, ad, bd, idesc, (i > 0 || w > 0 || j > 0) ? 1u : 0u);
           }
@@ -356,7 +362,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
           uint32_t v[32];
           tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c * 32, v);
           tmem_ld_wait();
-          if (grow < args.Mp) {
+          if (grow < args.Mp && args.mode == 0) {
             uint16_t* o = static_cast<uint16_t*>(args.out) + static_cast<int64_t>(grow) * args.ld;
             uint16_t* o2 = args.out2 != nullptr ? args.out2 + static_cast<int64_t>(grow) * args.ld2 : nullptr;
 #pragma unroll
@@ -368,6 +374,20 @@ __global__ void __launch_bounds__(kSkThreads, 1)
                     pack_bf16x2((0.0f + __uint_as_float(v[i])) * args.scale, 0.0f) & 0xFFFFu);
                 if (cc < args.nout) o[cc] = b;
                 if (o2 != nullptr) o2[cc] = b;
+              }
+            }
+          } else if (grow < args.Mp) {
+            // fp32: mode 1 out[Mp][ld], mode 2 out[nout][Mp] (consecutive lanes, consecutive rows)
+            float* o = static_cast<float*>(args.out);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int cc = c * 32 + i;
+              if (cc < args.nout) {
+                const float x = (0.0f + __uint_as_float(v[i])) * args.scale;
+                if (args.mode == 1)
+                  o[static_cast<int64_t>(grow) * args.ld + cc] = x;
+                else
+                  o[static_cast<int64_t>(cc) * args.Mp + grow] = x;
               }
             }
           }
@@ -1010,11 +1030,11 @@ cudaError_t run_skinny(const CUtensorMap& ta, const CUtensorMap& tb, int Mp, int
   return cudaGetLastError();
 }
 
-template <bool B>
+template <bool A, bool B>
 cudaError_t set_rank_rows_attr() {
   static DeviceOnce once;
   return once.run([](int) {
-    return cudaFuncSetAttribute(rank_rows_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(rank_rows_kernel<A, B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(kSkSmem));
   });
 }
@@ -1028,29 +1048,33 @@ int fused_pairs(int tiles, int sms) {
   return pairs < 1 ? 1 : pairs;
 }
 
-// CTAs for the rank-r product of a Mp x Kc activation beside the fused GEMM
-// of `tiles` pair tiles, or 0 for the split kernel before it.  Decided for the
-// sizing SM count (not the device's), so the forward and the backward's
-// recompute make the same choice and form Zc alike: the SMs the fused GEMM
-// leaves free, when there are at least 8 of them and each streams at most
-// 2.5 MB (done long before the fused GEMM's first LoRA step).
-int rank_rows_ctas(int64_t Mp, int64_t Kc, int tiles) {
+// CTAs for rank-r products streaming `bytes` beside the fused GEMM of `tiles`
+// pair tiles, or 0 for the split kernel.  Decided for the sizing SM count
+// (not the device's), so the forward and the backward's recompute make the
+// same choice and form Zc alike: the SMs the fused GEMM leaves free (an even
+// number), when there are at least 8 of them and each streams at most
+// mb_per_sm MB (done long before the fused GEMM needs the product).
+int rank_rows_ctas(double bytes, int tiles, double mb_per_sm) {
   const int free_sms = g_ws_sms - 2 * fused_pairs(tiles, g_ws_sms);
   if (free_sms < 8) return 0;
-  if (static_cast<double>(Mp) * static_cast<double>(Kc) * 2.0 > 2.5e6 * free_sms) return 0;
-  const int m_tiles = static_cast<int>((Mp + 127) / 128);
-  const int ctas = m_tiles < free_sms ? m_tiles : free_sms;
-  return (ctas + 1) & ~1;   // pairs of CTAs (a 2 x 1 cluster), for the fused pairs' placement
+  if (bytes > mb_per_sm * 1e6 * free_sms) return 0;
+  return free_sms;
 }
 
-// D = scale * A(m',k') B(n',k') by rank_rows_kernel on `ctas` CTAs, mode 0
-// (bf16 out, and all ncols columns again into out2 when it is not null).
-template <bool kBmn>
+// D = scale * A(m',k') B(n',k') by rank_rows_kernel on `ctas` CTAs; modes as
+// for run_skinny (0: bf16 out, and all ncols columns again into out2 when it
+// is not null; 1: fp32 out[Mp][ld]; 2: fp32 out[nout][Mp]).
+template <bool kAmn, bool kBmn>
 cudaError_t run_rank_rows(const CUtensorMap& ta, const CUtensorMap& tb, int Mp, int Kp, int ncols,
-                          float scale, void* out, int ld, int ctas, int32_t* d_status,
+                          float scale, int mode, void* out, int ld, int ctas, int32_t* d_status,
                           cudaStream_t st, int nout = -1, uint16_t* out2 = nullptr, int ld2 = 0) {
-  cudaError_t e = set_rank_rows_attr<kBmn>();
+  cudaError_t e = set_rank_rows_attr<kAmn, kBmn>();
   if (e != cudaSuccess) return e;
+  // at most one CTA per tile, in pairs (a 2 x 1 cluster, so that the SMs left
+  // to the fused GEMM's pairs stay in pairs)
+  const int m_tiles = (Mp + 127) / 128;
+  if (ctas > m_tiles) ctas = m_tiles;
+  ctas = (ctas + 1) & ~1;
   SkinnyArgs a;
   a.Mp = Mp;
   a.nk = (Kp + 64 * kSkW - 1) / (64 * kSkW);
@@ -1059,7 +1083,7 @@ cudaError_t run_rank_rows(const CUtensorMap& ta, const CUtensorMap& tb, int Mp, 
   a.ncols = ncols;
   a.nout = nout < 0 ? ncols : nout;
   a.scale = scale;
-  a.mode = 0;
+  a.mode = mode;
   a.out = out;
   a.ld = ld;
   a.out2 = out2;
@@ -1067,7 +1091,7 @@ cudaError_t run_rank_rows(const CUtensorMap& ta, const CUtensorMap& tb, int Mp, 
   a.d_status = d_status;
   {
     ProfScope prof(kProfSkinny, st);
-    e = launch_pdl_pair(rank_rows_kernel<kBmn>, dim3(static_cast<unsigned>(ctas)),
+    e = launch_pdl_pair(rank_rows_kernel<kAmn, kBmn>, dim3(static_cast<unsigned>(ctas)),
                         dim3(kSkThreads, 1, 1), kSkSmem, st, ta, tb, a);
   }
   if (e != cudaSuccess) return e;
@@ -1204,10 +1228,10 @@ cudaError_t launch_linear_fwd(int64_t M, int64_t K, int64_t N, int r, const uint
     // beside the fused GEMM on the SMs it leaves free, or split-K before it
     const int fwd_tiles = static_cast<int>(((M + kFPairRows - 1) / kFPairRows) *
                                            ((N + kFPairCols - 1) / kFPairCols));
-    const int rows_ctas = rank_rows_ctas(M, K, fwd_tiles);
+    const int rows_ctas = rank_rows_ctas(2.0 * M * K, fwd_tiles, 2.5);
     if (rows_ctas > 0) {
-      e = run_rank_rows<true>(tX, tAl, static_cast<int>(M), static_cast<int>(K), rp, c, Zc, r,
-                              rows_ctas, d_status, st, r, Zp, rp);
+      e = run_rank_rows<false, true>(tX, tAl, static_cast<int>(M), static_cast<int>(K), rp, c, 0, Zc,
+                                     r, rows_ctas, d_status, st, r, Zp, rp);
     } else {
       const int Sz = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
       e = run_skinny<false, true>(tX, tAl, static_cast<int>(M), static_cast<int>(K), rp, c, 0, Zc, r,
@@ -1286,10 +1310,10 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
     // the forward's choice of kernel and split, so the same bits
     const int fwd_tiles = static_cast<int>(((M + kFPairRows - 1) / kFPairRows) *
                                            ((N + kFPairCols - 1) / kFPairCols));
-    const int rows_ctas = rank_rows_ctas(M, K, fwd_tiles);
+    const int rows_ctas = rank_rows_ctas(2.0 * M * K, fwd_tiles, 2.5);
     if (rows_ctas > 0) {
-      e = run_rank_rows<true>(tXf, tAf, static_cast<int>(M), static_cast<int>(K), rp, c, Zc_ws, rp,
-                              rows_ctas, d_status, st);
+      e = run_rank_rows<false, true>(tXf, tAf, static_cast<int>(M), static_cast<int>(K), rp, c, 0,
+                                     Zc_ws, rp, rows_ctas, d_status, st);
     } else {
       const int Sf = skinny_splits(static_cast<int>(M), static_cast<int>(K / 64), g_ws_sms);
       e = run_skinny<false, true>(tXf, tAf, static_cast<int>(M), static_cast<int>(K), rp, c, 0, Zc_ws,
@@ -1311,10 +1335,10 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
   {
     const int dx_tiles = static_cast<int>(((M + kFPairRows - 1) / kFPairRows) *
                                           ((K + kFPairCols - 1) / kFPairCols));
-    const int rows_ctas = rank_rows_ctas(M, N, dx_tiles);
+    const int rows_ctas = rank_rows_ctas(2.0 * M * N, dx_tiles, 2.5);
     if (rows_ctas > 0)
-      e = run_rank_rows<false>(tG, tBk, static_cast<int>(M), static_cast<int>(N), rp, c, dZ, rp,
-                               rows_ctas, d_status, st);
+      e = run_rank_rows<false, false>(tG, tBk, static_cast<int>(M), static_cast<int>(N), rp, c, 0, dZ,
+                                      rp, rows_ctas, d_status, st);
     else
       e = run_skinny<false, false>(tG, tBk, static_cast<int>(M), static_cast<int>(N), rp, c, 0, dZ, rp,
                                    Sz, d_status, st);
@@ -1374,12 +1398,22 @@ cudaError_t launch_linear_bwd(int64_t M, int64_t K, int64_t N, int r, const uint
       if (e == cudaSuccess) e = ew;
     }
   }
+  // dA, dB on the SMs dX leaves free when they can stream their 2 x M x
+  // (K + N) bytes there well within dX, else split-K
+  const int dx_tiles = fa.m_tiles * fa.n_tiles;
+  const int dadb_ctas = rank_rows_ctas(2.0 * M * (K + N), dx_tiles, 5.0);
   if (e == cudaSuccess)
-    e = run_skinny<true, true>(tXmn, tdZ, static_cast<int>(K), static_cast<int>(M), r, 1.0f, 1, dA,
-                               r, Sa, d_status, s2);
+    e = dadb_ctas > 0
+            ? run_rank_rows<true, true>(tXmn, tdZ, static_cast<int>(K), static_cast<int>(M), r, 1.0f, 1,
+                                        dA, r, dadb_ctas, d_status, s2)
+            : run_skinny<true, true>(tXmn, tdZ, static_cast<int>(K), static_cast<int>(M), r, 1.0f, 1, dA,
+                                     r, Sa, d_status, s2);
   if (e == cudaSuccess)
-    e = run_skinny<true, true>(tGmn, tZcmn, static_cast<int>(N), static_cast<int>(M), r, 1.0f, 2,
-                               dB, r, Sb, d_status, s2);
+    e = dadb_ctas > 0
+            ? run_rank_rows<true, true>(tGmn, tZcmn, static_cast<int>(N), static_cast<int>(M), r, 1.0f,
+                                        2, dB, r, dadb_ctas, d_status, s2)
+            : run_skinny<true, true>(tGmn, tZcmn, static_cast<int>(N), static_cast<int>(M), r, 1.0f, 2,
+                                     dB, r, Sb, d_status, s2);
   if (s2 != st) {
     // always join, so that nothing on st can run ahead of work already queued
     const cudaError_t ej = cudaEventRecord(ss->join, s2);
