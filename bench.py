@@ -41,7 +41,7 @@ ROTATE = 3          # input sets cycled per step: 3 x 96 MB of bf16 inputs > 2 x
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
 # fused kernel at M = K = N = 4096, mean of its forward and dX launches in one
 # ncu capture of the current kernel; None once the kernel changes.
-FUSED_TRAFFIC_BYTES = 0.5 * ((42683648 + 1685248) + (43897344 + 2266368))
+FUSED_TRAFFIC_BYTES = 0.5 * ((42661632 + 2432768) + (44022528 + 4504320))
 
 
 def flops_step(Mt=M, Kt=K, Nt=N, r=R):
