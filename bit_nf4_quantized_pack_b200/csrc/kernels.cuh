@@ -102,8 +102,9 @@ cudaError_t launch_bounded_wait_selftest(int32_t* d_status, uint64_t limit_ns, c
 
 // quantize.cu.  With double quantization the workspace holds, from its
 // start: 256 exponent bins of the scales (2 KB), the counter of finished
-// encoder CTAs, then (at kQuantizeWsHead) one fp32 scale per 64-block; the
-// first kQuantizeWsHead bytes are cleared by every call.
+// encoder CTAs, the call's token, the flag of its mean and the counter of
+// claimed chunks, then (at kQuantizeWsHead) one fp32 scale per 64-block; CTA
+// 0 of every call resets the head (any contents on entry).
 constexpr size_t kQuantizeWsHead = 2304;
 cudaError_t launch_quantize(const void* W, int dtype, int64_t numel, uint8_t* packed,
                             float* absmax_out, bool dq, uint8_t* code8, float* s2, float* offset,

@@ -495,7 +495,7 @@ __device__ __forceinline__ unsigned long long* ws_token(unsigned long long* bins
   return reinterpret_cast<unsigned long long*>(reinterpret_cast<char*>(bins) + 2056);
 }
 
-// The claimed-chunk counter of the bf16 encoder (chunks past its first wave).
+// The claimed-chunk counter of the bf16 encoder (chunks past its first waves).
 __device__ __forceinline__ unsigned long long* ws_chunk_counter(unsigned long long* bins) {
   return reinterpret_cast<unsigned long long*>(reinterpret_cast<char*>(bins) + 2072);
 }
