@@ -260,8 +260,13 @@ qlora_status qlora_nf4_dequantize(const qlora_nf4_state* st, uint16_t* W_hat,
  * that every row the tensor maps read starts on a 16-byte boundary; the padded
  * rank columns are zero and change no result.
  * ws: at least qlora_linear_fwd_workspace_size(M, K, N, r) bytes; that size is
- * 0 when r % 8 == 0 (every kernel of the forward adds its K splits inside a
- * thread-block cluster), and ws may then be null.
+ * 0 when r % 8 == 0 (the kernels of the forward keep their partial sums on
+ * chip: K splits added inside a thread-block cluster, or a whole contraction
+ * in one CTA), and ws may then be null.
+ * Work placement (no effect on the results): for M > 16 the fused GEMM runs
+ * on the fewest CTA pairs that keep its number of waves of tiles; when that
+ * leaves at least 8 SMs and Zc is small enough for them, Zc is formed there
+ * while the fused GEMM runs, else before it.
  */
 size_t qlora_linear_fwd_workspace_size(int64_t M, int64_t K, int64_t N, int32_t r);
 qlora_status qlora_linear_fwd(int64_t M, int64_t K, int64_t N, int32_t r,
@@ -290,8 +295,8 @@ qlora_status qlora_linear_fwd(int64_t M, int64_t K, int64_t N, int32_t r,
  * workspace convention as the forward.
  * Streams: dA and dB run on a stream the library owns (one per device,
  * created on first use), forked from `stream` after dZ and joined back into
- * it before the call returns, so that they use the SMs that dX's last
- * partial wave of tiles leaves idle.  To the caller the call is still one
+ * it before the call returns, so that they use the SMs that dX leaves free
+ * (as in the forward, dZ too runs there when it is small enough).  To the caller the call is still one
  * operation ordered on `stream` (later work on `stream` sees dX, dA and dB;
  * it can be captured in a CUDA graph), and the results are the same bits as
  * a run in order.  If the library stream cannot be created, or while
