@@ -576,8 +576,9 @@ def main():
     if sampler:
         sampler.start()
     # The step time: no event between launches (an event recorded between two
-    # launches keeps the second from starting while the first drains, which
-    # costs the step about 25 us); the library only counts its launches.
+    # launches keeps the second from starting while the first drains, and the
+    # rank-r kernels from running beside the fused GEMM: tens of microseconds
+    # per step); the library only counts its launches.
     q.lib.qlora_profile_reset()
     q.lib.qlora_profile_select(0)
     q.lib.qlora_profile_enable(1)
